@@ -1,0 +1,184 @@
+"""CPU oracle for the paged KV-cache decode step (fp64, plain C + numpy glue).
+
+TEST INFRASTRUCTURE ONLY: the test suite, ``__graft_entry__.smoke()`` and the
+benchmark's CPU-baseline leg are the only code that may import this package.
+The library under ``paged_kv_cache_420_b200`` never imports it, and it shares
+no code with that library; the seeded input generators in ``workloads`` are the
+only module both sides use.
+
+Functions follow the pages on vLLM's PagedAttention (block table, pos -> block
+and offset, attention read through the table, copy-on-write); the C source
+``pkv_oracle.c`` cites the passage for each.  Parity pins for every function
+are in ``tests/test_oracle_pins.py``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+from typing import Optional
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "pkv_oracle.c")
+_BUILD_DIR = os.path.join(_HERE, "_build")
+_LIB_PATH = os.path.join(_BUILD_DIR, "libpkv_oracle.so")
+_lib: Optional[ctypes.CDLL] = None
+
+
+def build(force: bool = False) -> str:
+    """Compiles the C oracle with gcc (-O2 -fopenmp) into oracle/_build/."""
+    os.makedirs(_BUILD_DIR, exist_ok=True)
+    if force or not os.path.exists(_LIB_PATH) or os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC):
+        tmp = _LIB_PATH + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-std=c11",
+                               "-Wall", "-Wextra", "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def _load() -> ctypes.CDLL:
+    global _lib
+    if _lib is None:
+        lib = ctypes.CDLL(build())
+        P = ctypes.c_void_p
+        I = ctypes.c_int
+        D = ctypes.c_double
+        lib.oracle_kv_write.argtypes = [P, P, P, P, P, I, I, I, I, I]
+        lib.oracle_copy_blocks.argtypes = [P, P, P, I, I, I, I, I]
+        lib.oracle_paged_attention.argtypes = [P, P, P, P, I, P, I, I, I, I, I, I, D, P]
+        lib.oracle_attention_partial.argtypes = [P, P, P, P, I, I, I, I, I, I, I, I, D, P, P, P]
+        lib.oracle_lse_merge.argtypes = [P, P, P, I, I, P]
+        lib.oracle_num_threads.argtypes = []
+        for f in (lib.oracle_kv_write, lib.oracle_copy_blocks, lib.oracle_paged_attention,
+                  lib.oracle_attention_partial, lib.oracle_lse_merge, lib.oracle_num_threads):
+            f.restype = ctypes.c_int
+        _lib = lib
+    return _lib
+
+
+def num_threads() -> int:
+    return int(_load().oracle_num_threads())
+
+
+# ---------------------------------------------------------------------------
+# array glue
+# ---------------------------------------------------------------------------
+
+def bits(x) -> np.ndarray:
+    """bf16 data (torch bf16 tensor, or uint16 bit patterns) -> contiguous uint16."""
+    if hasattr(x, "dtype") and str(x.dtype) == "torch.bfloat16":
+        import torch
+        return np.ascontiguousarray(x.detach().to("cpu").contiguous().view(torch.int16).numpy().view(np.uint16))
+    a = np.ascontiguousarray(x)
+    if a.dtype != np.uint16:
+        raise TypeError(f"expected bf16 bits (uint16), got {a.dtype}")
+    return a
+
+
+def bf16_bits_to_f64(b: np.ndarray) -> np.ndarray:
+    """Exact widening of bf16 bit patterns to float64."""
+    return (np.asarray(b, dtype=np.uint16).astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def _ptr(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _check(rc: int, what: str):
+    if rc == 1:
+        raise ValueError(f"oracle {what}: bad argument")
+    if rc == 2:
+        raise IndexError(f"oracle {what}: index out of range")
+    if rc:
+        raise RuntimeError(f"oracle {what}: status {rc}")
+
+
+# ---------------------------------------------------------------------------
+# the three operations
+# ---------------------------------------------------------------------------
+
+def kv_write(k_cache, v_cache, k, v, slot_mapping):
+    """Returns new (k_cache, v_cache) uint16 arrays [NB, Hkv, bs, d] after the
+    slot-mapped write of k, v [T, Hkv, d]."""
+    kc = bits(k_cache).copy()
+    vc = bits(v_cache).copy()
+    kb, vb = bits(k), bits(v)
+    slots = np.ascontiguousarray(slot_mapping, dtype=np.int64)
+    NB, Hkv, bs, d = kc.shape
+    T = slots.shape[0]
+    assert kb.shape == (T, Hkv, d) and vb.shape == (T, Hkv, d)
+    rc = _load().oracle_kv_write(_ptr(kc), _ptr(vc), _ptr(kb), _ptr(vb), _ptr(slots), T, NB, Hkv, bs, d)
+    _check(rc, "kv_write")
+    return kc, vc
+
+
+def copy_blocks(k_cache, v_cache, pairs):
+    """Returns new (k_cache, v_cache) after copying block src -> dst for every
+    (src, dst) in pairs [P, 2] (simultaneous semantics)."""
+    kc = bits(k_cache).copy()
+    vc = bits(v_cache).copy()
+    pr = np.ascontiguousarray(np.asarray(pairs, dtype=np.int32).reshape(-1, 2))
+    NB, Hkv, bs, d = kc.shape
+    rc = _load().oracle_copy_blocks(_ptr(kc), _ptr(vc), _ptr(pr), pr.shape[0], NB, Hkv, bs, d)
+    _check(rc, "copy_blocks")
+    return kc, vc
+
+
+def paged_attention(q, k_cache, v_cache, block_tables, context_lens, scale: float) -> np.ndarray:
+    """fp64 decode attention out[B, Hq, d] read through the block tables."""
+    qb = bits(q)
+    kc, vc = bits(k_cache), bits(v_cache)
+    tables = np.ascontiguousarray(block_tables, dtype=np.int32)
+    ctx = np.ascontiguousarray(context_lens, dtype=np.int32)
+    B, Hq, d = qb.shape
+    NB, Hkv, bs, d2 = kc.shape
+    assert d == d2 and tables.shape[0] == B and ctx.shape[0] == B
+    out = np.zeros((B, Hq, d), dtype=np.float64)
+    rc = _load().oracle_paged_attention(_ptr(qb), _ptr(kc), _ptr(vc), _ptr(tables), tables.shape[1],
+                                        _ptr(ctx), B, Hq, Hkv, d, bs, NB, float(np.float64(np.float32(scale))),
+                                        _ptr(out))
+    _check(rc, "paged_attention")
+    return out
+
+
+def attention_partial(q_row, k_cache, v_cache, table_row, num_q_heads: int, hq: int,
+                      t_begin: int, t_end: int, scale: float):
+    """(m, l, acc[d]) of one (sequence, query head) over tokens [t_begin, t_end)."""
+    qb = bits(q_row).reshape(-1)
+    kc, vc = bits(k_cache), bits(v_cache)
+    tr = np.ascontiguousarray(table_row, dtype=np.int32).reshape(-1)
+    NB, Hkv, bs, d = kc.shape
+    m = np.zeros(1)
+    l = np.zeros(1)
+    acc = np.zeros(d)
+    rc = _load().oracle_attention_partial(_ptr(qb), _ptr(kc), _ptr(vc), _ptr(tr), NB, num_q_heads, Hkv,
+                                          d, bs, hq, t_begin, t_end,
+                                          float(np.float64(np.float32(scale))), _ptr(m), _ptr(l), _ptr(acc))
+    _check(rc, "attention_partial")
+    return float(m[0]), float(l[0]), acc
+
+
+def lse_merge(m, l, acc) -> np.ndarray:
+    """Merges P partial results: m [P], l [P], acc [P, d] -> out [d]."""
+    m = np.ascontiguousarray(m, dtype=np.float64)
+    l = np.ascontiguousarray(l, dtype=np.float64)
+    acc = np.ascontiguousarray(acc, dtype=np.float64)
+    P, d = acc.shape
+    out = np.zeros(d)
+    rc = _load().oracle_lse_merge(_ptr(m), _ptr(l), _ptr(acc), P, d, _ptr(out))
+    _check(rc, "lse_merge")
+    return out
+
+
+def decode_step(w, attention: bool = True):
+    """Applies one whole step of a ``workloads.Workload`` on the CPU:
+    copy-on-write pairs, then the slot-mapped write, then attention.
+    Returns (k_cache_bits, v_cache_bits, out_f64 or None)."""
+    kc, vc = bits(w.k_cache), bits(w.v_cache)
+    if len(w.copy_pairs):
+        kc, vc = copy_blocks(kc, vc, w.copy_pairs)
+    kc, vc = kv_write(kc, vc, w.k_new, w.v_new, w.slot_mapping)
+    out = paged_attention(w.q, kc, vc, w.block_tables, w.context_lens, w.scale) if attention else None
+    return kc, vc, out

@@ -1,0 +1,243 @@
+/*
+ * pkv_oracle.c -- plain, slow CPU oracle for the paged KV-cache decode step.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only the test suite, the smoke check and the
+ * benchmark's CPU-baseline leg may load this code.  It shares no source,
+ * header, table or helper with the CUDA library, and neither side includes
+ * or links the other.
+ *
+ * What it computes, following the pages on vLLM's PagedAttention:
+ *   - KV cache split into fixed-size blocks of `bs` tokens, located through a
+ *     per-sequence block table (wkbse.com "加速 LLM 推理：深入了解 vllm 引擎",
+ *     section 3.1; intelliparadigm.com article 2012396, section 2.1).
+ *   - token position -> (logical block = pos / bs, offset = pos % bs)
+ *     (ruibaoantu.com article 3727998, section 1.1, the PagedAttention sketch).
+ *   - the paged attention kernel reads the same K/V through the table and
+ *     computes ordinary attention over it (wkbse.com section 3.1, third point
+ *     of the list), i.e. softmax(q K^T * scale) V.
+ *   - copy-on-write of a shared block (intelliparadigm.com section 2.1, item 2).
+ *
+ * Pool layout (the library's ABI; the oracle reads it through pool_row()):
+ *   cache[num_blocks][num_kv_heads][bs][d], bf16 bit patterns (uint16).
+ * Floating point: every product and sum in double; bf16 inputs are widened
+ * exactly (a bf16 is the top half of an IEEE binary32).
+ *
+ * Return codes: 0 ok, 1 bad argument, 2 index out of range.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+/* exact bf16 -> double */
+static double bf16_to_f64(uint16_t bits) {
+    uint32_t u = (uint32_t)bits << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return (double)f;
+}
+
+/* index of token row (block, head, offset) in a pool of layout
+ * [num_blocks][num_kv_heads][bs][d] (units of elements) */
+static size_t pool_row(int64_t block, int head, int offset, int num_kv_heads, int bs, int d) {
+    return (((size_t)block * (size_t)num_kv_heads + (size_t)head) * (size_t)bs + (size_t)offset) * (size_t)d;
+}
+
+int oracle_num_threads(void) {
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
+
+/*
+ * Write: for every new token t with slot_mapping[t] >= 0, block = slot / bs,
+ * offset = slot % bs, and for every kv head h the row
+ * cache[block][h][offset][:] becomes k[t][h][:] (same for v).  Tokens are
+ * applied in ascending t.  A negative slot marks padding and is skipped.
+ */
+int oracle_kv_write(uint16_t *k_cache, uint16_t *v_cache, const uint16_t *k, const uint16_t *v,
+                    const int64_t *slot_mapping, int num_tokens, int num_blocks, int num_kv_heads,
+                    int bs, int d) {
+    if (num_tokens < 0 || num_blocks <= 0 || num_kv_heads <= 0 || bs <= 0 || d <= 0) return 1;
+    for (int t = 0; t < num_tokens; ++t) {
+        int64_t slot = slot_mapping[t];
+        if (slot < 0) continue;
+        if (slot >= (int64_t)num_blocks * bs) return 2;
+        int64_t block = slot / bs;
+        int offset = (int)(slot % bs);
+        for (int h = 0; h < num_kv_heads; ++h) {
+            size_t dst = pool_row(block, h, offset, num_kv_heads, bs, d);
+            size_t src = ((size_t)t * num_kv_heads + h) * (size_t)d;
+            for (int i = 0; i < d; ++i) {
+                k_cache[dst + i] = k[src + i];
+                v_cache[dst + i] = v[src + i];
+            }
+        }
+    }
+    return 0;
+}
+
+/*
+ * Copy-on-write block copy: every pair (src, dst) makes block dst of both
+ * caches (all heads, all offsets) equal to block src.  The pairs act as if
+ * simultaneous: every source block is read before any destination is
+ * written.
+ */
+int oracle_copy_blocks(uint16_t *k_cache, uint16_t *v_cache, const int32_t *pairs, int num_pairs,
+                       int num_blocks, int num_kv_heads, int bs, int d) {
+    if (num_pairs < 0 || num_blocks <= 0) return 1;
+    size_t block_elems = (size_t)num_kv_heads * bs * d;
+    for (int p = 0; p < num_pairs; ++p) {
+        int32_t s = pairs[2 * p], t = pairs[2 * p + 1];
+        if (s < 0 || s >= num_blocks || t < 0 || t >= num_blocks) return 2;
+    }
+    if (num_pairs == 0) return 0;
+    uint16_t *snap_k = (uint16_t *)malloc(sizeof(uint16_t) * block_elems * num_pairs);
+    uint16_t *snap_v = (uint16_t *)malloc(sizeof(uint16_t) * block_elems * num_pairs);
+    if (!snap_k || !snap_v) { free(snap_k); free(snap_v); return 1; }
+    for (int p = 0; p < num_pairs; ++p) {
+        size_t src = (size_t)pairs[2 * p] * block_elems;
+        memcpy(snap_k + (size_t)p * block_elems, k_cache + src, sizeof(uint16_t) * block_elems);
+        memcpy(snap_v + (size_t)p * block_elems, v_cache + src, sizeof(uint16_t) * block_elems);
+    }
+    for (int p = 0; p < num_pairs; ++p) {
+        size_t dst = (size_t)pairs[2 * p + 1] * block_elems;
+        memcpy(k_cache + dst, snap_k + (size_t)p * block_elems, sizeof(uint16_t) * block_elems);
+        memcpy(v_cache + dst, snap_v + (size_t)p * block_elems, sizeof(uint16_t) * block_elems);
+    }
+    free(snap_k);
+    free(snap_v);
+    return 0;
+}
+
+/*
+ * Attention of one (sequence s, query head hq) over the token range
+ * [t_begin, t_end) of that sequence, returning the unnormalised pieces:
+ *   z_i   = scale * sum_c q[c] * K_i[c]                 (i in range)
+ *   m     = max_i z_i
+ *   l     = sum_i exp(z_i - m)
+ *   acc_c = sum_i exp(z_i - m) * V_i[c]
+ * where K_i, V_i are the rows of token i of the sequence, found through the
+ * block table: physical block = table[i / bs], offset = i % bs, kv head
+ * hkv = hq / (Hq / Hkv).  An empty range gives m = -inf, l = 0, acc = 0.
+ */
+static int attend_range(const uint16_t *q, const uint16_t *k_cache, const uint16_t *v_cache,
+                        const int32_t *table, int num_blocks, int Hq, int Hkv, int d, int bs,
+                        int hq, int t_begin, int t_end, double scale, double *m_out, double *l_out,
+                        double *acc) {
+    int g = Hq / Hkv;
+    int hkv = hq / g;
+    for (int c = 0; c < d; ++c) acc[c] = 0.0;
+    if (t_end <= t_begin) {
+        *m_out = -INFINITY;
+        *l_out = 0.0;
+        return 0;
+    }
+    int n = t_end - t_begin;
+    double *z = (double *)malloc(sizeof(double) * (size_t)n);
+    if (!z) return 1;
+    double m = -INFINITY;
+    for (int i = t_begin; i < t_end; ++i) {
+        int32_t block = table[i / bs];
+        if (block < 0 || block >= num_blocks) { free(z); return 2; }
+        const uint16_t *krow = k_cache + pool_row(block, hkv, i % bs, Hkv, bs, d);
+        double dot = 0.0;
+        for (int c = 0; c < d; ++c) dot += bf16_to_f64(q[c]) * bf16_to_f64(krow[c]);
+        z[i - t_begin] = scale * dot;
+        if (z[i - t_begin] > m) m = z[i - t_begin];
+    }
+    double l = 0.0;
+    for (int i = t_begin; i < t_end; ++i) {
+        int32_t block = table[i / bs];
+        const uint16_t *vrow = v_cache + pool_row(block, hkv, i % bs, Hkv, bs, d);
+        double w = exp(z[i - t_begin] - m);
+        l += w;
+        for (int c = 0; c < d; ++c) acc[c] += w * bf16_to_f64(vrow[c]);
+    }
+    free(z);
+    *m_out = m;
+    *l_out = l;
+    return 0;
+}
+
+/*
+ * Decode attention for a batch: out[s][hq][:] = softmax_i(z_i) . V_i over the
+ * context_lens[s] tokens of sequence s (z_i as in attend_range).  A sequence
+ * with context length 0 gets a zero output.  q is bf16 [B][Hq][d], tables are
+ * int32 [B][max_blocks_per_seq], out is double [B][Hq][d].
+ * (s, hq) pairs are independent and are spread over OpenMP threads; the
+ * arithmetic of each pair is the sequential sum above.
+ */
+int oracle_paged_attention(const uint16_t *q, const uint16_t *k_cache, const uint16_t *v_cache,
+                           const int32_t *block_tables, int max_blocks_per_seq,
+                           const int32_t *context_lens, int B, int Hq, int Hkv, int d, int bs,
+                           int num_blocks, double scale, double *out) {
+    if (B < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || d <= 0 || bs <= 0) return 1;
+    for (int s = 0; s < B; ++s) {
+        if (context_lens[s] < 0) return 1;
+        if ((int64_t)context_lens[s] > (int64_t)max_blocks_per_seq * bs) return 2;
+    }
+    int status = 0;
+#pragma omp parallel for schedule(dynamic, 1) collapse(2)
+    for (int s = 0; s < B; ++s) {
+        for (int hq = 0; hq < Hq; ++hq) {
+            double *o = out + ((size_t)s * Hq + hq) * (size_t)d;
+            double *acc = (double *)malloc(sizeof(double) * (size_t)d);
+            double m, l;
+            int rc = acc ? attend_range(q + ((size_t)s * Hq + hq) * (size_t)d, k_cache, v_cache,
+                                        block_tables + (size_t)s * max_blocks_per_seq, num_blocks,
+                                        Hq, Hkv, d, bs, hq, 0, context_lens[s], scale, &m, &l, acc)
+                         : 1;
+            if (rc) {
+#pragma omp atomic write
+                status = rc;
+            } else {
+                for (int c = 0; c < d; ++c) o[c] = (l > 0.0) ? acc[c] / l : 0.0;
+            }
+            free(acc);
+        }
+    }
+    return status;
+}
+
+/*
+ * Split-K pieces: for (s, hq) and token range [t_begin, t_end) return m, l and
+ * the unnormalised acc[d] of attend_range.
+ */
+int oracle_attention_partial(const uint16_t *q_row, const uint16_t *k_cache, const uint16_t *v_cache,
+                             const int32_t *table, int num_blocks, int Hq, int Hkv, int d, int bs,
+                             int hq, int t_begin, int t_end, double scale, double *m, double *l,
+                             double *acc) {
+    if (Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || t_begin < 0) return 1;
+    return attend_range(q_row, k_cache, v_cache, table, num_blocks, Hq, Hkv, d, bs, hq, t_begin,
+                        t_end, scale, m, l, acc);
+}
+
+/*
+ * Log-sum-exp merge of P partial results (m_p, l_p, acc_p[d]) of disjoint
+ * token ranges that together cover a context:
+ *   M = max_p m_p,  L = sum_p l_p e^{m_p - M},  out = sum_p acc_p e^{m_p - M} / L.
+ * Empty pieces (m = -inf) contribute nothing.  L = 0 gives a zero output.
+ */
+int oracle_lse_merge(const double *m, const double *l, const double *acc, int P, int d, double *out) {
+    if (P < 0 || d <= 0) return 1;
+    double M = -INFINITY;
+    for (int p = 0; p < P; ++p) if (m[p] > M) M = m[p];
+    double L = 0.0;
+    for (int c = 0; c < d; ++c) out[c] = 0.0;
+    if (M == -INFINITY) return 0;
+    for (int p = 0; p < P; ++p) {
+        if (m[p] == -INFINITY) continue;
+        double w = exp(m[p] - M);
+        L += l[p] * w;
+        for (int c = 0; c < d; ++c) out[c] += acc[(size_t)p * d + c] * w;
+    }
+    for (int c = 0; c < d; ++c) out[c] = (L > 0.0) ? out[c] / L : 0.0;
+    return 0;
+}

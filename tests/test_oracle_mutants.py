@@ -1,0 +1,81 @@
+"""The pins catch plausible oracle mistakes.
+
+Each case copies the oracle's C source to a temporary directory, plants one
+mistake by text substitution (a dropped term, a wrong sign, a wrong index or
+layout), builds it, swaps it in as the oracle's library and runs the pin
+tests.  At least one pin must fail for every planted mistake.  The committed
+oracle is never modified.
+"""
+import ctypes
+import os
+import subprocess
+
+import pytest
+
+import oracle
+from tests import test_oracle_pins as pins
+
+PIN_TESTS = [
+    pins.test_block_count_golden,
+    pins.test_write_roundtrip_and_untouched_rows,
+    pins.test_copy_blocks_simultaneous_semantics,
+    pins.test_copy_on_write_isolates_sharers,
+    lambda: pins.test_attention_equals_dense_library_softmax([5, 16, 31, 48, 100], 8, 2, 64, 16),
+    pins.test_attention_equals_torch_sdpa_gqa,
+    pins.test_uniform_attention_gives_mean_of_v,
+    pins.test_single_token_gives_its_value_row_exactly,
+    pins.test_gqa_head_mapping_is_contiguous_groups,
+    pins.test_two_token_closed_form_golden,
+    pins.test_context_len_zero_gives_zero_output,
+    lambda: pins.test_split_merge_equals_unsplit("ragged"),
+    pins.test_lse_merge_closed_form,
+]
+
+MUTANTS = {
+    "in-block offset": ("int offset = (int)(slot % bs);", "int offset = (int)((slot / bs) % bs);"),
+    "read offset": ("pool_row(block, hkv, i % bs, Hkv, bs, d);\n        double dot",
+                    "pool_row(block, hkv, (i + 1) % bs, Hkv, bs, d);\n        double dot"),
+    "gqa mapping": ("int hkv = hq / g;", "int hkv = hq % Hkv;"),
+    "dropped scale": ("z[i - t_begin] = scale * dot;", "z[i - t_begin] = dot;"),
+    "exp sign": ("double w = exp(z[i - t_begin] - m);", "double w = exp(m - z[i - t_begin]);"),
+    "pool layout": ("(((size_t)block * (size_t)num_kv_heads + (size_t)head) * (size_t)bs + (size_t)offset)",
+                    "(((size_t)block * (size_t)bs + (size_t)offset) * (size_t)num_kv_heads + (size_t)head)"),
+    "transposed k": ("bf16_to_f64(krow[c])", "bf16_to_f64(krow[d - 1 - c])"),
+    "sequential copy": ("memcpy(k_cache + dst, snap_k + (size_t)p * block_elems",
+                        "memcpy(k_cache + dst, k_cache + (size_t)pairs[2 * p] * block_elems"),
+    "missing normalisation": ("o[c] = (l > 0.0) ? acc[c] / l : 0.0;", "o[c] = (l > 0.0) ? acc[c] : 0.0;"),
+    "merge drops rescale": ("L += l[p] * w;", "L += l[p];"),
+    # the new token left out of the attended range (context_len - 1 tokens)
+    "context off by one": ("hq, 0, context_lens[s], scale", "hq, 0, context_lens[s] - 1, scale"),
+}
+
+
+def _build_mutant(tmp_path, old, new):
+    src = open(os.path.join(os.path.dirname(oracle.__file__), "pkv_oracle.c")).read()
+    assert src.count(old) >= 1, f"mutation anchor not found: {old!r}"
+    src = src.replace(old, new)
+    path = tmp_path / "mutant.c"
+    path.write_text(src)
+    so = tmp_path / "libmutant.so"
+    subprocess.check_call(["gcc", "-O1", "-fopenmp", "-fPIC", "-shared", "-std=c11", "-o", str(so), str(path), "-lm"])
+    return str(so)
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_pins_catch_planted_mistake(name, tmp_path, monkeypatch):
+    old, new = MUTANTS[name]
+    so = _build_mutant(tmp_path, old, new)
+    good = oracle._load()
+    lib = ctypes.CDLL(so)
+    for fn in ("oracle_kv_write", "oracle_copy_blocks", "oracle_paged_attention",
+               "oracle_attention_partial", "oracle_lse_merge", "oracle_num_threads"):
+        getattr(lib, fn).argtypes = getattr(good, fn).argtypes
+        getattr(lib, fn).restype = getattr(good, fn).restype
+    monkeypatch.setattr(oracle, "_lib", lib)
+    caught = []
+    for t in PIN_TESTS:
+        try:
+            t()
+        except (AssertionError, IndexError, ValueError) as e:
+            caught.append((getattr(t, "__name__", "lambda"), type(e).__name__))
+    assert caught, f"no pin caught the planted mistake {name!r}"

@@ -1,0 +1,101 @@
+"""Structure of the seeded synthetic workloads (host only, no arithmetic of the method)."""
+import numpy as np
+import pytest
+
+import workloads
+
+
+def _check_common(w):
+    B, bs = w.num_seqs, w.block_size
+    assert w.q.shape == (B, w.num_q_heads, w.head_dim)
+    assert w.k_new.shape == (B, w.num_kv_heads, w.head_dim)
+    assert w.k_cache.shape == (w.num_blocks, w.num_kv_heads, bs, w.head_dim)
+    assert w.block_tables.dtype == np.int32 and w.context_lens.dtype == np.int32
+    assert w.slot_mapping.dtype == np.int64
+    for s in range(B):
+        n = int(w.context_lens[s])
+        nb = (n + bs - 1) // bs
+        row = w.block_tables[s]
+        assert (row[:nb] >= 0).all() and (row[:nb] < w.num_blocks).all()
+        assert (row[nb:] == -1).all()
+        # the new token's slot is in the sequence's block for position n-1
+        assert w.slot_mapping[s] // bs == row[(n - 1) // bs]
+        assert w.slot_mapping[s] % bs == (n - 1) % bs
+    # no two sequences write the same slot
+    assert len(set(w.slot_mapping.tolist())) == B
+
+
+@pytest.mark.parametrize("name", ["tiny", "llama2-7b", "llama2-13b"])
+def test_private_blocks_are_disjoint(name):
+    w = workloads.make(name, seed=0, values_device="meta")
+    _check_common(w)
+    used = np.concatenate([w.block_tables[s][w.block_tables[s] >= 0] for s in range(w.num_seqs)])
+    assert len(np.unique(used)) == len(used)
+    if name != "tiny":
+        assert w.num_blocks == int(np.ceil(1.2 * len(used)))
+
+
+def test_tiny_matches_its_description():
+    w = workloads.make("tiny", seed=0, values_device="meta")
+    assert w.context_lens.tolist() == [1, 17, 33, 64]
+    assert (w.num_q_heads, w.num_kv_heads, w.head_dim, w.block_size, w.num_blocks) == (4, 4, 64, 16, 32)
+    assert abs(w.scale - 0.125) < 1e-9
+
+
+def test_13b_lengths_and_fragmentation():
+    w = workloads.make("llama2-13b", seed=0, values_device="meta")
+    assert w.num_seqs == 128 and w.num_q_heads == 40
+    assert w.context_lens.min() >= 16 and w.context_lens.max() <= 3072 + 512
+    # the fragmented free list does not hand out ids in order
+    first = w.block_tables[0][w.block_tables[0] >= 0]
+    assert not (np.diff(first) == 1).all()
+    w32 = workloads.make("llama2-13b", seed=0, values_device="meta", block_size=32)
+    assert w32.block_size == 32 and (w32.context_lens == w.context_lens).all()
+
+
+def test_gqa_prefix_sharing_structure():
+    w = workloads.make("llama3-8b-gqa-prefix", seed=0, values_device="meta")
+    _check_common(w)
+    assert (w.num_seqs, w.num_q_heads, w.num_kv_heads) == (256, 32, 8)
+    assert w.copy_pairs.shape == (8, 2)
+    t = w.block_tables
+    for g in range(32):
+        rows = t[g * 8:(g + 1) * 8]
+        long_rows = [r for s, r in zip(range(g * 8, g * 8 + 8), rows) if w.context_lens[s] > 1024]
+        for r in long_rows[1:]:
+            assert (r[:64] == long_rows[0][:64]).all()
+    for src, dst in w.copy_pairs:
+        s = int(np.nonzero((t == dst).any(axis=1))[0][0])
+        n = int(w.context_lens[s])
+        assert n <= 1024 and (n - 1) % 16 != 0
+        assert t[s][(n - 1) // 16] == dst
+        assert w.slot_mapping[s] // 16 == dst
+    srcs, dsts = set(w.copy_pairs[:, 0].tolist()), set(w.copy_pairs[:, 1].tolist())
+    assert not (srcs & dsts) and len(dsts) == 8
+
+
+def test_long_context_shape():
+    w = workloads.make("llama2-70b-long", seed=0, values_device="meta")
+    assert sorted(w.context_lens.tolist()) == sorted([32768, 65536, 98304, 131072] * 2)
+    assert w.partition_tokens == 512
+    w128 = workloads.make("llama2-70b-long", seed=0, values_device="meta", block_size=128)
+    assert w128.max_blocks_per_seq == 1024
+
+
+def test_values_are_seeded():
+    a = workloads.make("tiny", seed=7)
+    b = workloads.make("tiny", seed=7)
+    c = workloads.make("tiny", seed=8)
+    assert a.k_cache.equal(b.k_cache) and a.q.equal(b.q)
+    assert not a.q.equal(c.q)
+
+
+def test_poison_marks_only_unused_rows():
+    w = workloads.make("tiny", seed=1, poison=True)
+    kc = w.k_cache.float()
+    for s in range(w.num_seqs):
+        n = int(w.context_lens[s])
+        for pos in range(n - 1):
+            b = w.block_tables[s][pos // 16]
+            assert not kc[b, :, pos % 16].isnan().any()
+    assert kc.isnan().any()
