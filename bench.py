@@ -1,0 +1,475 @@
+#!/usr/bin/env python
+"""Benchmark of one paged-KV decode step on B200.
+
+A step is one pass of the whole hot path over one batch: copy-on-write block
+copies (when the workload has any), the slot-mapped write of one new token per
+sequence, and paged decode attention (plan + attention + split-K reduce
+kernels).  The default workload is the Llama-2-13B-shaped continuous batch
+(B 128, 40 MHA heads, d 128, block size 16, fragmented pool).
+
+Prints one JSON line.  `value` is algorithmic HBM GB/s of the whole step over
+all ranks (bytes that must move: unique K/V rows read, q, out, tables and
+lengths, the written rows and the copied blocks), measured with CUDA events on
+inputs already resident in HBM; `e2e` is the same metric with the per-step
+inputs copied from pinned host memory and the output copied back inside the
+timed region.  `roofline` reports the decode call alone against the measured
+HBM copy bandwidth.  `--impl reference` times the fp64 CPU oracle on the host
+cores instead (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+FALLBACK_HBM_GBS = 6650.0
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "decode_traffic.txt")
+DECODE_SOURCES = ["paged_kv_cache_420_b200/csrc/decode.cuh", "paged_kv_cache_420_b200/csrc/pkv_api.cu",
+                  "paged_kv_cache_420_b200/csrc/ptx.cuh"]
+
+
+# --------------------------------------------------------------------------
+# algorithmic bytes
+# --------------------------------------------------------------------------
+
+def decode_bytes(w) -> int:
+    """Bytes paged decode attention must move: every distinct (block, kv head,
+    offset) K and V row of valid tokens once, q and out, the table entries
+    read and the context lengths."""
+    bs = w.block_size
+    NB = w.num_blocks
+    used = np.zeros((NB, bs), dtype=bool)
+    for s in range(w.num_seqs):
+        n = int(w.context_lens[s])
+        nb = (n + bs - 1) // bs
+        full = nb - 1
+        if full > 0:
+            used[w.block_tables[s, :full]] = True
+        if nb > 0:
+            used[w.block_tables[s, nb - 1], : n - full * bs] = True
+    token_rows = int(used.sum())
+    kv = token_rows * w.num_kv_heads * w.head_dim * 2 * 2
+    qo = 2 * w.num_seqs * w.num_q_heads * w.head_dim * 2
+    tables = 4 * int(sum((int(n) + bs - 1) // bs for n in w.context_lens))
+    return kv + qo + tables + 4 * w.num_seqs
+
+
+def logical_decode_bytes(w) -> int:
+    """Same, but shared blocks counted once per sequence that reads them."""
+    kv = int(w.context_lens.astype(np.int64).sum()) * w.num_kv_heads * w.head_dim * 2 * 2
+    qo = 2 * w.num_seqs * w.num_q_heads * w.head_dim * 2
+    return kv + qo + 4 * int(sum((int(n) + w.block_size - 1) // w.block_size for n in w.context_lens)) + 4 * w.num_seqs
+
+
+def write_bytes(w) -> int:
+    return 2 * 2 * w.num_seqs * w.num_kv_heads * w.head_dim * 2 + 8 * w.num_seqs
+
+
+def copy_bytes(w) -> int:
+    blk = w.num_kv_heads * w.block_size * w.head_dim * 2
+    return 2 * 2 * len(w.copy_pairs) * blk
+
+
+def step_bytes(w) -> int:
+    return decode_bytes(w) + write_bytes(w) + copy_bytes(w)
+
+
+# --------------------------------------------------------------------------
+# environment helpers
+# --------------------------------------------------------------------------
+
+def measured_hbm_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def decode_source_hash() -> str:
+    h = hashlib.sha256()
+    for rel in DECODE_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload: str, bs: int):
+    """DRAM bytes per decode launch from a committed ncu summary, if it was
+    taken on the current decode sources."""
+    try:
+        with open(TRAFFIC_FILE) as f:
+            for line in f:
+                parts = line.split()
+                if len(parts) >= 4 and not line.startswith("#"):
+                    if parts[0] == decode_source_hash() and parts[1] == workload and parts[2] == f"bs{bs}":
+                        return int(float(parts[3]))
+    except FileNotFoundError:
+        pass
+    return None
+
+
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.dev}", f"--query-gpu={self.QUERY}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (FileNotFoundError, OSError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.text = ""
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.text, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                self.text, _ = self.proc.communicate()
+
+    def summary(self):
+        if not getattr(self, "text", ""):
+            return None
+        mhz, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.text.strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                mhz.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for name, val in zip(names, f[5:9]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        if not mhz:
+            return None
+        return {"sm_mhz": statistics.median(mhz), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(mhz)}
+
+
+# --------------------------------------------------------------------------
+# the timed arms
+# --------------------------------------------------------------------------
+
+def make_workload(args, rank: int, device):
+    bs = args.block_size
+    return workloads.make(args.workload, seed=args.seed + rank, values_device=device, block_size=bs)
+
+
+def partition_tokens(args, w) -> int:
+    return w.partition_tokens if args.partition_tokens < 0 else args.partition_tokens
+
+
+def launches_per_step(w, pt: int) -> int:
+    maxp = max(1, math.ceil(w.max_context_len / (pt if pt > 0 else 512)))
+    n = 1 + 1 + 1 + (1 if maxp > 1 else 0)  # write, plan, attention, reduce
+    if len(w.copy_pairs):
+        n += math.ceil(len(w.copy_pairs) / 1024)
+    return n
+
+
+def run_cuda(args, rank, world, dist):
+    import paged_kv_cache_420_b200 as pkv
+
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
+    torch.cuda.set_device(dev)
+    w = make_workload(args, rank, dev)
+    pt = partition_tokens(args, w)
+    slots = torch.from_numpy(w.slot_mapping).to(dev)
+    tables = torch.from_numpy(w.block_tables).to(dev)
+    ctx = torch.from_numpy(w.context_lens).to(dev)
+    out = torch.empty_like(w.q)
+    ws = torch.empty(pkv.decode_workspace_bytes(w.num_seqs, w.num_q_heads, w.num_kv_heads, w.head_dim,
+                                                w.max_context_len, pt), dtype=torch.uint8, device=dev)
+    kc, vc = w.k_cache, w.v_cache
+    stream = torch.cuda.current_stream()
+    ev_d = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+
+    def step(i=None):
+        if len(w.copy_pairs):
+            pkv.pkv_copy_blocks(w.copy_pairs, kc, vc, stream=stream)
+        pkv.pkv_write(w.k_new, w.v_new, slots, kc, vc, stream=stream)
+        if i is not None:
+            ev_d[i][0].record(stream)
+        pkv.paged_attn_decode(w.q, kc, vc, tables, ctx, w.scale, w.num_kv_heads, out, w.max_context_len, pt,
+                              workspace=ws, stream=stream)
+        if i is not None:
+            ev_d[i][1].record(stream)
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize()
+    err = pkv.get_device_error()
+    if err:
+        raise RuntimeError(f"device error word {err:#x} during warm-up")
+
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(dev.index) as clocks:
+        t0.record(stream)
+        for i in range(args.steps):
+            step(i)
+        t1.record(stream)
+        torch.cuda.synchronize()
+        if dist is not None:
+            dist.barrier()
+        # keep sampling a little if the timed region was shorter than one sample
+        if t0.elapsed_time(t1) < 450:
+            time.sleep(0.45)
+    ms_total = t0.elapsed_time(t1)
+    decode_ms = sum(a.elapsed_time(b) for a, b in ev_d) / args.steps
+    if pkv.get_device_error():
+        raise RuntimeError("device error word set during the timed region")
+
+    bytes_step = step_bytes(w)
+    dec_bytes = decode_bytes(w)
+    stats = torch.tensor([ms_total, float(bytes_step), float(w.num_seqs)], dtype=torch.float64, device=dev)
+    if dist is not None:
+        mx = stats.clone()
+        dist.all_reduce(mx, op=dist.ReduceOp.MAX)
+        sm = stats.clone()
+        dist.all_reduce(sm, op=dist.ReduceOp.SUM)
+        ms_max, bytes_all, seqs_all = float(mx[0]), float(sm[1]), float(sm[2])
+    else:
+        ms_max, bytes_all, seqs_all = ms_total, float(bytes_step), float(w.num_seqs)
+    sec = ms_max / 1e3
+    value = bytes_all * args.steps / sec / 1e9
+
+    # ---- end to end: per-step inputs from pinned host memory, output back
+    e2e = None
+    if not args.no_e2e:
+        host = {k: v.cpu().pin_memory() for k, v in dict(q=w.q, k_new=w.k_new, v_new=w.v_new, slots=slots,
+                                                           tables=tables, ctx=ctx).items()}
+        dbuf = {k: torch.empty_like(v, device=dev) for k, v in host.items()}
+        out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+        h2d = sum(v.numel() * v.element_size() for v in host.values())
+        d2h = out_h.numel() * out_h.element_size()
+        k_e2e = max(3, min(args.steps, 500))
+
+        def e2e_step():
+            for k in host:
+                dbuf[k].copy_(host[k], non_blocking=True)
+            if len(w.copy_pairs):
+                pkv.pkv_copy_blocks(w.copy_pairs, kc, vc, stream=stream)
+            pkv.pkv_write(dbuf["k_new"], dbuf["v_new"], dbuf["slots"], kc, vc, stream=stream)
+            pkv.paged_attn_decode(dbuf["q"], kc, vc, dbuf["tables"], dbuf["ctx"], w.scale, w.num_kv_heads, out,
+                                  w.max_context_len, pt, workspace=ws, stream=stream)
+            out_h.copy_(out, non_blocking=True)
+
+        for _ in range(3):
+            e2e_step()
+        torch.cuda.synchronize()
+        if dist is not None:
+            dist.barrier()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(k_e2e):
+            e2e_step()
+        b.record(stream)
+        torch.cuda.synchronize()
+        e_ms = torch.tensor([a.elapsed_time(b)], dtype=torch.float64, device=dev)
+        if dist is not None:
+            dist.all_reduce(e_ms, op=dist.ReduceOp.MAX)
+        e2e = {"value": round(bytes_all * k_e2e / (float(e_ms[0]) / 1e3) / 1e9, 2), "unit": "GB/s",
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "steps": k_e2e}
+
+    peak, peak_kind = measured_hbm_peak()
+    achieved = dec_bytes / (decode_ms / 1e3) / 1e9
+    line = {
+        "metric": "paged decode attn HBM GB/s (% of B200 peak) & tokens·layers/s at 13B shape",
+        "value": round(value, 2),
+        "unit": "GB/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_max / args.steps, 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic",
+        "config": {
+            "workload": f"{w.name}: {w.description}",
+            "num_seqs": w.num_seqs, "num_q_heads": w.num_q_heads, "num_kv_heads": w.num_kv_heads,
+            "head_dim": w.head_dim, "block_size": w.block_size, "kv_tokens": int(w.context_lens.sum()),
+            "partition_tokens": pt if pt > 0 else 512, "copy_pairs": int(len(w.copy_pairs)),
+            "seed": args.seed, "bytes_per_step": int(bytes_step),
+            "l2": "no flush: every step reads >1 GB of K/V (L2 is 126 MB)",
+            "parallelism": f"replicas x{world}, one independent batch per GPU",
+        },
+        "tokens_layers_per_s": round(seqs_all * args.steps / sec, 1),
+        "pct_of_hbm_peak": round(100 * value / world / peak, 2),
+        "roofline": {
+            "kernel": "paged_attn_decode (plan + attention + reduce kernels)",
+            "bound": "hbm", "achieved": round(achieved, 2), "peak": peak, "peak_kind": peak_kind,
+            "unit": "GB/s", "frac": round(achieved / peak, 4),
+            "algorithmic_bytes": int(dec_bytes), "logical_bytes": int(logical_decode_bytes(w)),
+            "decode_us": round(decode_ms * 1e3, 2),
+            "traffic": recorded_traffic(w.name, w.block_size),
+        },
+        "e2e": e2e,
+        "gpu_launches": launches_per_step(w, pt) * args.steps,
+        "clocks": clocks.summary(),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w, budget_s=args.cpu_budget)
+    return line
+
+
+def cpu_baseline(w, budget_s: float, label="oracle", pools=None):
+    """Times the fp64 CPU oracle's paged attention on the first sequences of
+    the workload until about `budget_s` seconds of CPU work are spent.  The
+    step's copy-on-write copies and write are applied to the pools once,
+    untimed (they are under 1% of the step's bytes)."""
+    import oracle
+
+    if pools is None:
+        pools = oracle_pools(w)
+    kc, vc = pools
+    done, elapsed, nbytes = 0, 0.0, 0
+    chunk = 1
+    while done < w.num_seqs and elapsed < budget_s:
+        idx = np.arange(done, min(w.num_seqs, done + chunk))
+        sub = _subset(w, idx)
+        t = time.perf_counter()
+        oracle.paged_attention(sub.q, kc, vc, sub.block_tables, sub.context_lens, sub.scale)
+        elapsed += time.perf_counter() - t
+        nbytes += decode_bytes(sub)
+        done += len(idx)
+        chunk = min(2 * chunk, 64)
+    return {"value": round(nbytes / elapsed / 1e9, 4), "unit": "GB/s", "cores": oracle.num_threads(),
+            "kind": label,
+            "sample": f"paged attention of the first {done} of {w.num_seqs} sequences (all heads), "
+                      f"{elapsed:.1f} s of fp64 C/OpenMP work",
+            "tokens_layers_per_s": round(done / elapsed, 2)}
+
+
+def oracle_pools(w):
+    """Pools after the step's copy-on-write copies and write, by the oracle."""
+    import oracle
+
+    kc, vc = oracle.bits(w.k_cache), oracle.bits(w.v_cache)
+    if len(w.copy_pairs):
+        kc, vc = oracle.copy_blocks(kc, vc, w.copy_pairs)
+    return oracle.kv_write(kc, vc, w.k_new, w.v_new, w.slot_mapping)
+
+
+def _subset(w, idx):
+    import copy as _copy
+    sub = _copy.copy(w)
+    ti = torch.from_numpy(np.asarray(idx, dtype=np.int64)).to(w.q.device)
+    sub.q, sub.k_new, sub.v_new = w.q[ti], w.k_new[ti], w.v_new[ti]
+    sub.block_tables = w.block_tables[idx]
+    sub.context_lens = w.context_lens[idx]
+    sub.slot_mapping = w.slot_mapping[idx]
+    sub.num_seqs = len(idx)
+    if len(w.copy_pairs):
+        dsts = set(int(b) for b in np.unique(sub.block_tables))
+        sub.copy_pairs = np.array([p for p in w.copy_pairs if int(p[1]) in dsts], np.int32).reshape(-1, 2)
+    return sub
+
+
+def run_reference(args, rank, world):
+    """The CPU oracle as the reference arm: rank 0 times it on the host cores,
+    one bounded sample of the workload per step."""
+    if rank != 0:
+        return None
+    w = workloads.make(args.workload, seed=args.seed, values_device="cpu", block_size=args.block_size)
+    per_step_budget = max(0.05, min(2.0, 150.0 / max(1, args.steps + args.warmup)))
+    pools = oracle_pools(w)
+    for _ in range(args.warmup):
+        cpu_baseline(w, per_step_budget, pools=pools)
+    vals, tls = [], []
+    t_all = time.perf_counter()
+    last = None
+    for _ in range(args.steps):
+        last = cpu_baseline(w, per_step_budget, label="oracle", pools=pools)
+        vals.append(last["value"])
+        tls.append(last["tokens_layers_per_s"])
+    t_all = time.perf_counter() - t_all
+    value = statistics.median(vals)
+    return {
+        "impl": "reference",
+        "metric": "paged decode attn HBM GB/s (% of B200 peak) & tokens·layers/s at 13B shape",
+        "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(1e3 * t_all / args.steps, 3), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": f"{w.name}: {w.description}", "block_size": w.block_size,
+                   "num_seqs": w.num_seqs, "seed": args.seed},
+        "tokens_layers_per_s": statistics.median(tls),
+        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": last["cores"], "kind": "oracle",
+                         "sample": last["sample"]},
+        "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["pkv", "reference"], default="pkv")
+    ap.add_argument("--workload", default="llama2-13b", choices=list(workloads.WORKLOADS))
+    ap.add_argument("--block-size", type=int, default=None)
+    ap.add_argument("--partition-tokens", type=int, default=-1, help="-1: the workload's choice, 0: library's")
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work for cpu_baseline")
+    args = ap.parse_args(argv)
+    args.warmup = max(args.warmup, 3)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    dist = None
+    if world > 1 and args.impl == "pkv":
+        import datetime
+
+        import torch.distributed as tdist
+        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", 0)))
+        tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+        dist = tdist
+    try:
+        if args.impl == "reference":
+            line = run_reference(args, rank, world)
+        else:
+            line = run_cuda(args, rank, world, dist)
+        if rank == 0 and line is not None:
+            print(json.dumps(line), flush=True)
+    finally:
+        if dist is not None:
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

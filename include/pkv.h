@@ -1,0 +1,174 @@
+/*
+ * pkv.h -- C ABI of libpkv.so, a B200 (sm_100a) library for the hot path of a
+ * paged KV cache: the slot-mapped write of new tokens, the copy-on-write block
+ * copy, and decode attention read through per-sequence block tables.
+ *
+ * Method (pages on vLLM's PagedAttention):
+ *   - The KV cache is split into fixed-size blocks of `block_size` tokens that
+ *     can sit anywhere in a preallocated physical pool; a per-sequence block
+ *     table maps logical block j to a physical block id, like a page table
+ *     (wkbse.com "加速 LLM 推理：深入了解 vllm 引擎", section 3.1;
+ *     intelliparadigm.com article 2012396, section 2.1, storage levels 1-2).
+ *   - Token position pos lives in logical block pos / block_size at offset
+ *     pos % block_size (ruibaoantu.com article 3727998, section 1.1 sketch).
+ *   - The attention kernel finds the physical blocks through the table and
+ *     reads the non-contiguous K/V from them (wkbse.com section 3.1).
+ *   - Shared blocks serve several sequences; a shared block is copied before a
+ *     sequence writes into it (copy-on-write, intelliparadigm.com section 2.1).
+ *
+ * Physical pool layout (both caches, bf16):
+ *     cache[num_blocks][num_kv_heads][block_size][head_dim]
+ * so one (block, head) tile of block_size x head_dim is contiguous and every
+ * token row is head_dim*2 bytes (a multiple of 16).  A slot names one token row
+ * of the pool: slot = physical_block * block_size + offset.
+ *
+ * Conventions shared by every call:
+ *   - Pointers are device pointers owned by the caller unless stated "host".
+ *     The library allocates no device memory; it keeps one 4-byte device error
+ *     word per GPU (a module global).
+ *   - All work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
+ *     stream) and returns before it finishes.
+ *   - Host validation covers shapes, null pointers and 16-byte alignment only;
+ *     the host never reads device arrays.  Data-dependent faults found on the
+ *     device (slot or block id outside the pool, context length outside the
+ *     table) set bits in the device error word, and the offending access is
+ *     skipped or clamped.  Read and clear it with pkv_get_device_error().
+ *   - Supported: head_dim in {64, 128}; block_size a multiple of 16 in
+ *     [16, 1024]; num_q_heads = g * num_kv_heads with 1 <= g <= 16.
+ */
+#ifndef PKV_H_
+#define PKV_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+struct CUstream_st;
+typedef struct CUstream_st *pkv_stream_t; /* same type as cudaStream_t */
+
+typedef enum pkv_status {
+    PKV_OK = 0,
+    PKV_EINVAL = 1,      /* bad size, null pointer, misaligned pointer, bad workspace */
+    PKV_ERANGE = 2,      /* host-visible index outside the pool (copy pairs) */
+    PKV_EALIAS = 3,      /* copy pairs: a destination repeats or is also a source */
+    PKV_ECUDA = 4,       /* a CUDA runtime/driver call failed (launch, tensor map) */
+    PKV_EDEVICE = 5,     /* pkv_get_device_error found a non-zero device error word */
+    PKV_EUNSUPPORTED = 6 /* valid request outside the supported shapes */
+} pkv_status;
+
+/* Bits of the device error word. */
+#define PKV_DEVERR_SLOT 0x1u     /* pkv_write: slot >= num_blocks * block_size (token skipped) */
+#define PKV_DEVERR_BLOCK 0x2u    /* decode: block table entry outside [0, num_blocks) (tile reads zeros) */
+#define PKV_DEVERR_CONTEXT 0x4u  /* decode: context_lens[s] < 0 or above the table / max_context_len (clamped) */
+#define PKV_DEVERR_TIMEOUT 0x8u  /* a bounded on-chip wait gave up (the call's results are invalid) */
+
+/* Describes one physical pool (k_cache and v_cache share it). */
+typedef struct pkv_pool {
+    int32_t num_blocks;
+    int32_t num_kv_heads;
+    int32_t block_size;
+    int32_t head_dim;
+} pkv_pool;
+
+/*
+ * pkv_write -- slot-mapped write of new tokens' K/V into their blocks.
+ * Follows: new tokens' KV go into a block of the sequence and the block table
+ * is updated (wkbse.com section 3.1, "flexible memory management"); the slot
+ * decodes as block = slot / block_size, offset = slot % block_size
+ * (ruibaoantu.com section 1.1).
+ *
+ *   k, v          bf16 [num_tokens][num_kv_heads][head_dim], contiguous, 16-B aligned
+ *   slot_mapping  int64 [num_tokens]; slot < 0 marks a padding token (skipped)
+ *   k_cache, v_cache  pool of layout above, 16-B aligned
+ * For every token t with slot >= 0 and every kv head h:
+ *   cache[slot / bs][h][slot % bs][:] = k[t][h][:]   (same for v), bit-exact.
+ * Two tokens with the same slot: which one lands is unspecified.
+ * Slots >= num_blocks * block_size set PKV_DEVERR_SLOT and are skipped.
+ * num_tokens == 0 is a no-op.
+ */
+pkv_status pkv_write(const void *k, const void *v, const int64_t *slot_mapping, int32_t num_tokens,
+                     void *k_cache, void *v_cache, pkv_pool pool, pkv_stream_t stream);
+
+/*
+ * pkv_copy_blocks -- copy-on-write block copy for shared prefixes
+ * (intelliparadigm.com section 2.1: COW for prefix sharing; a block holds a
+ * key region and a value region).
+ *
+ *   src_dst_pairs  HOST int32 [num_pairs][2] = (src, dst) physical block ids.
+ *                  The block manager that decides copy-on-write lives on the
+ *                  host, so the pairs are read there, validated completely and
+ *                  passed to the kernel by value (no device staging buffer).
+ * For every pair, block dst of both caches (all heads, all offsets) becomes a
+ * bit-exact copy of block src.  The pairs act as if simultaneous; to make that
+ * unambiguous a destination may appear only once and may not be any pair's
+ * source (PKV_EALIAS).  Ids outside [0, num_blocks) give PKV_ERANGE.  Nothing
+ * is enqueued when validation fails.  num_pairs == 0 is a no-op.
+ */
+pkv_status pkv_copy_blocks(const int32_t *src_dst_pairs, int32_t num_pairs, void *k_cache,
+                           void *v_cache, pkv_pool pool, pkv_stream_t stream);
+
+/*
+ * pkv_decode_workspace_bytes -- device scratch needed by paged_attn_decode for
+ * these sizes (a work list and the split-K partial results).  Returns 0 for
+ * invalid sizes.  partition_tokens as for paged_attn_decode (0 = library's
+ * choice).
+ */
+size_t pkv_decode_workspace_bytes(int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads,
+                                  int32_t head_dim, int32_t max_context_len,
+                                  int32_t partition_tokens);
+
+/*
+ * paged_attn_decode -- decode attention of one query token per sequence over
+ * its paged K/V (wkbse.com section 3.1: the custom kernel looks up the block
+ * table and reads the non-contiguous blocks; section 3.3: scale, softmax and
+ * weighted sum fused in one kernel).  For every sequence s and query head hq:
+ *   hkv   = hq / (num_q_heads / num_kv_heads)              (contiguous GQA groups)
+ *   z_i   = scale * <q[s][hq], K_i>,  i < context_lens[s]
+ *   out[s][hq] = sum_i softmax(z)_i * V_i
+ * where K_i, V_i are the rows of position i found through
+ * block_tables[s][i / block_size] at offset i % block_size.  Accumulation is
+ * fp32 with an online softmax; out is rounded to bf16 (nearest-even).
+ * Long contexts are split into partitions of partition_tokens tokens whose
+ * (max, sum, acc) are merged by a log-sum-exp reduce.
+ *
+ *   q             bf16 [num_seqs][num_q_heads][head_dim], 16-B aligned
+ *   k_cache, v_cache  pool (layout above); pool.num_kv_heads == num_kv_heads
+ *   block_tables  int32 [num_seqs][max_blocks_per_seq]; entries at and after
+ *                 ceil(context_len / block_size) are never read
+ *   context_lens  int32 [num_seqs]; 0 gives a zero output row
+ *   max_context_len  host upper bound of context_lens (sizes the workspace)
+ *   partition_tokens 0 = library's choice, else a multiple of 16 in [16, 65536]
+ *   out           bf16 [num_seqs][num_q_heads][head_dim], 16-B aligned
+ *   workspace     device scratch of at least pkv_decode_workspace_bytes(...)
+ *                 bytes, 256-B aligned; contents need no initialisation; one
+ *                 workspace must not be used by two calls that run concurrently
+ * Launches up to three kernels on `stream` (plan, attention, reduce).
+ */
+pkv_status paged_attn_decode(const void *q, const void *k_cache, const void *v_cache,
+                             const int32_t *block_tables, int32_t max_blocks_per_seq,
+                             const int32_t *context_lens, int32_t num_seqs, int32_t num_q_heads,
+                             float scale, int32_t num_kv_heads, void *out, pkv_pool pool,
+                             int32_t max_context_len, int32_t partition_tokens, void *workspace,
+                             size_t workspace_bytes, pkv_stream_t stream);
+
+/*
+ * pkv_get_device_error -- copies the current device's error word to
+ * *code_out and clears it, ordered after the work already on `stream`, and
+ * waits for it.  Returns PKV_EDEVICE when the word was non-zero.
+ */
+pkv_status pkv_get_device_error(int32_t *code_out, pkv_stream_t stream);
+
+/* Static description of a status code. */
+const char *pkv_status_string(pkv_status status);
+
+/* ABI version: major * 10000 + minor * 100 + patch. */
+int32_t pkv_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PKV_H_ */

@@ -1,0 +1,172 @@
+"""Python binding of libpkv.so: paged KV-cache write, copy-on-write block copy
+and paged decode attention on B200 (sm_100a).
+
+Argument marshalling only.  Every step of the path runs in the library's CUDA
+kernels; torch supplies device memory and streams.  There is no CPU fallback:
+if libpkv.so is missing or a call fails, an exception is raised.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import numpy as np
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libpkv.so")
+
+PKV_OK = 0
+STATUS_NAMES = {0: "PKV_OK", 1: "PKV_EINVAL", 2: "PKV_ERANGE", 3: "PKV_EALIAS", 4: "PKV_ECUDA",
+                5: "PKV_EDEVICE", 6: "PKV_EUNSUPPORTED"}
+DEVERR_SLOT, DEVERR_BLOCK, DEVERR_CONTEXT, DEVERR_TIMEOUT = 0x1, 0x2, 0x4, 0x8
+
+# Every symbol include/pkv.h declares.
+EXPORTED = ("pkv_write", "pkv_copy_blocks", "pkv_decode_workspace_bytes", "paged_attn_decode",
+            "pkv_get_device_error", "pkv_status_string", "pkv_version")
+
+
+class PkvError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {STATUS_NAMES.get(status, status)} ({status_string(status)})")
+
+
+class _Pool(ctypes.Structure):
+    _fields_ = [("num_blocks", ctypes.c_int32), ("num_kv_heads", ctypes.c_int32),
+                ("block_size", ctypes.c_int32), ("head_dim", ctypes.c_int32)]
+
+
+_lib: Optional[ctypes.CDLL] = None
+
+
+def load_library() -> ctypes.CDLL:
+    """Loads libpkv.so from this package directory (raises if it is absent)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is missing: build it with `python -m paged_kv_cache_420_b200.build`")
+        lib = ctypes.CDLL(LIB_PATH)
+        P, I32, I64, F, SZ = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t
+        lib.pkv_write.argtypes = [P, P, P, I32, P, P, _Pool, P]
+        lib.pkv_copy_blocks.argtypes = [P, I32, P, P, _Pool, P]
+        lib.pkv_decode_workspace_bytes.argtypes = [I32, I32, I32, I32, I32, I32]
+        lib.pkv_decode_workspace_bytes.restype = SZ
+        lib.paged_attn_decode.argtypes = [P, P, P, P, I32, P, I32, I32, F, I32, P, _Pool, I32, I32, P, SZ, P]
+        lib.pkv_get_device_error.argtypes = [ctypes.POINTER(I32), P]
+        lib.pkv_status_string.argtypes = [ctypes.c_int]
+        lib.pkv_status_string.restype = ctypes.c_char_p
+        lib.pkv_version.restype = I32
+        for f in ("pkv_write", "pkv_copy_blocks", "paged_attn_decode", "pkv_get_device_error"):
+            getattr(lib, f).restype = ctypes.c_int
+        _lib = lib
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return load_library().pkv_status_string(int(status)).decode()
+
+
+def version() -> int:
+    return int(load_library().pkv_version())
+
+
+def _check(status: int, what: str):
+    if status != PKV_OK:
+        raise PkvError(status, what)
+
+
+def _ptr(t) -> ctypes.c_void_p:
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _pool(k_cache: torch.Tensor) -> _Pool:
+    if k_cache.dim() != 4:
+        raise ValueError("cache must be [num_blocks, num_kv_heads, block_size, head_dim]")
+    nb, hkv, bs, d = k_cache.shape
+    return _Pool(nb, hkv, bs, d)
+
+
+def _need(t: torch.Tensor, name: str, dtype, cuda=True):
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if cuda and not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+
+
+def pkv_write(k: torch.Tensor, v: torch.Tensor, slot_mapping: torch.Tensor, k_cache: torch.Tensor,
+              v_cache: torch.Tensor, stream=None) -> None:
+    """cache[slot // bs][h][slot % bs] = k[t][h] (and v) for every token t with slot >= 0."""
+    for t, n in ((k, "k"), (v, "v"), (k_cache, "k_cache"), (v_cache, "v_cache")):
+        _need(t, n, torch.bfloat16)
+    _need(slot_mapping, "slot_mapping", torch.int64)
+    if v_cache.shape != k_cache.shape or k.shape != v.shape:
+        raise ValueError("k/v and k_cache/v_cache shapes must match")
+    T = slot_mapping.shape[0]
+    if k.shape != (T, k_cache.shape[1], k_cache.shape[3]):
+        raise ValueError(f"k must be [num_tokens, num_kv_heads, head_dim], got {tuple(k.shape)}")
+    st = load_library().pkv_write(_ptr(k), _ptr(v), _ptr(slot_mapping), T, _ptr(k_cache), _ptr(v_cache),
+                                  _pool(k_cache), _stream(stream))
+    _check(st, "pkv_write")
+
+
+def pkv_copy_blocks(src_dst_pairs, k_cache: torch.Tensor, v_cache: torch.Tensor, stream=None) -> None:
+    """Copies block src -> dst of both caches for every (src, dst) host pair."""
+    for t, n in ((k_cache, "k_cache"), (v_cache, "v_cache")):
+        _need(t, n, torch.bfloat16)
+    pairs = np.ascontiguousarray(np.asarray(src_dst_pairs, dtype=np.int32).reshape(-1, 2))
+    st = load_library().pkv_copy_blocks(pairs.ctypes.data_as(ctypes.c_void_p), pairs.shape[0], _ptr(k_cache),
+                                        _ptr(v_cache), _pool(k_cache), _stream(stream))
+    _check(st, "pkv_copy_blocks")
+
+
+def decode_workspace_bytes(num_seqs: int, num_q_heads: int, num_kv_heads: int, head_dim: int,
+                           max_context_len: int, partition_tokens: int = 0) -> int:
+    n = load_library().pkv_decode_workspace_bytes(num_seqs, num_q_heads, num_kv_heads, head_dim,
+                                                  max_context_len, partition_tokens)
+    if n == 0:
+        raise ValueError("invalid sizes for the decode workspace")
+    return int(n)
+
+
+def paged_attn_decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, block_tables: torch.Tensor,
+                      context_lens: torch.Tensor, scale: float, num_kv_heads: int, out: torch.Tensor,
+                      max_context_len: int, partition_tokens: int = 0,
+                      workspace: Optional[torch.Tensor] = None, stream=None) -> None:
+    """out[s][hq] = softmax(scale * q[s][hq] . K^T) V over the context_lens[s]
+    tokens of sequence s, read through block_tables[s]."""
+    for t, n in ((q, "q"), (k_cache, "k_cache"), (v_cache, "v_cache"), (out, "out")):
+        _need(t, n, torch.bfloat16)
+    _need(block_tables, "block_tables", torch.int32)
+    _need(context_lens, "context_lens", torch.int32)
+    B, Hq, D = q.shape
+    if out.shape != q.shape or v_cache.shape != k_cache.shape:
+        raise ValueError("out must match q, v_cache must match k_cache")
+    if block_tables.dim() != 2 or block_tables.shape[0] != B or context_lens.shape != (B,):
+        raise ValueError("block_tables must be [B, max_blocks_per_seq], context_lens [B]")
+    if workspace is None:
+        nbytes = decode_workspace_bytes(B, Hq, num_kv_heads, D, max_context_len, partition_tokens)
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=q.device)
+    st = load_library().paged_attn_decode(
+        _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables), block_tables.shape[1], _ptr(context_lens),
+        B, Hq, float(scale), int(num_kv_heads), _ptr(out), _pool(k_cache), int(max_context_len),
+        int(partition_tokens), _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(st, "paged_attn_decode")
+
+
+def get_device_error(stream=None) -> int:
+    """Reads and clears the device error word (waits for `stream`)."""
+    code = ctypes.c_int32(0)
+    st = load_library().pkv_get_device_error(ctypes.byref(code), _stream(stream))
+    if st not in (PKV_OK, 5):
+        raise PkvError(st, "pkv_get_device_error")
+    return int(code.value)

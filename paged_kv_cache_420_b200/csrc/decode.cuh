@@ -1,0 +1,762 @@
+// decode.cuh -- paged decode attention for sm_100a.
+//
+// Method (wkbse.com "加速 LLM 推理：深入了解 vllm 引擎", sections 3.1 and 3.3):
+// every sequence's query attends over its context, whose K/V rows are found
+// through the block table (logical block i / bs -> physical id, offset
+// i % bs); scale, softmax and the weighted sum of V are fused in one pass
+// (online softmax in fp32, exp2 with scale*log2(e) folded in).
+//
+// Work decomposition.  A unit (sequence s, kv head h) is cut into partitions
+// of PT tokens; an item = (s, h, partition).  A one-CTA planner kernel writes
+// the (s, partition) list in sequence-major order.  The attention kernel is
+// persistent: CTA c takes items c, c + gridDim.x, ...  Inside a CTA one
+// producer warp walks the items' 16-token stages and fills a ring of NS
+// shared-memory slots with TMA tensor loads (K and V tiles of 16 rows x D,
+// 128-byte swizzle) addressed through the block table; W consumer warps take
+// the stages round-robin, each keeping its own online-softmax state, and merge
+// their partial (m, l, acc) per item through shared memory.  A unit with one
+// partition writes bf16 out directly; otherwise the partition's (m, l, acc)
+// goes to the workspace and a reduce kernel merges them by log-sum-exp.
+//
+// Two consumer arithmetic paths:
+//  * GQA group g <= 2 (MHA): CUDA cores.  A lane owns D/32 elements of every
+//    row; q.k partial sums of the 16 tokens are reduced by a transposing
+//    butterfly of warp shuffles; p is broadcast by shuffles for the PV sum.
+//  * 3 <= g <= 16: the g query heads of one kv head form a dense tile, so
+//    QK^T and PV run on tensor cores (mma.sync m16n8k16 bf16, fp32 accumulate):
+//    S^T[16 tokens x 8 heads] = K_tile . Q^T, O^T[D x 8 heads] += V^T . P^T,
+//    with P^T moved from accumulator to operand layout by movmatrix.
+#pragma once
+
+#include "ptx.cuh"
+
+namespace pkv {
+
+constexpr int kStageTok = 16;       // tokens per pipeline stage (one TMA box height)
+constexpr int kConsumerWarps = 4;   // W
+constexpr int kDecodeThreads = (kConsumerWarps + 1) * 32;
+constexpr int kPlanThreads = 1024;
+constexpr int kReduceWarps = 4;
+constexpr uint64_t kWaitLimitNs = 2000000000ull;  // bounded on-chip waits: 2 s
+#define PKV_NEG_INF (-__int_as_float(0x7f800000))
+
+struct DecodeParams {
+    const __nv_bfloat16 *q;       // [B][Hq][D]
+    __nv_bfloat16 *out;           // [B][Hq][D]
+    const int32_t *block_tables;  // [B][MBS]
+    const int32_t *context_lens;  // [B]
+    int2 *entries;                // workspace: (seq, partition), sequence-major
+    int32_t *num_entries;         // workspace: number of entries
+    float2 *part_ml;              // workspace: [B][Hq][maxP] = (m in log2 units, l)
+    float *part_acc;              // workspace: [B][Hq][maxP][D]
+    int B, Hq, Hkv, g, MBS, bs, NB, max_ctx, PT, maxP;
+    int pool_rows;                // NB * Hkv * bs: first out-of-range TMA row
+    float scale_log2;             // scale * log2(e)
+};
+
+// Context length of sequence s, clamped to what the table and the workspace
+// can hold.  A value outside [0, cap] is reported (once, by the planner).
+__device__ __forceinline__ int clamped_context(const DecodeParams &p, int s, bool report) {
+    const int n = __ldg(p.context_lens + s);
+    const long long table_cap = (long long)p.MBS * p.bs;
+    const int cap = (int)min(table_cap, (long long)p.max_ctx);
+    if (n < 0 || n > cap) {
+        if (report) raise_error(PKV_DEVERR_CONTEXT);
+        return n < 0 ? 0 : cap;
+    }
+    return n;
+}
+
+// ------------------------------------------------------------- planner ----
+// Writes entries[] = (s, partition) for every sequence and partition, in
+// sequence-major order, and the count.  Zero-length sequences get a zero
+// output row here (they have no items).
+__global__ void __launch_bounds__(kPlanThreads) plan_kernel(DecodeParams p, int D) {
+    __shared__ int s_off[kPlanThreads + 1];
+    __shared__ int s_warp[kPlanThreads / 32];
+    __shared__ int s_carry, s_any_zero;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    // The attention kernel may start its prologue now; it waits for this
+    // grid's results with griddepcontrol.wait before reading them.
+    grid_launch_dependents();
+    if (tid == 0) { s_carry = 0; s_any_zero = 0; }
+    __syncthreads();
+    for (int base = 0; base < p.B; base += kPlanThreads) {
+        const int s = base + tid;
+        int parts = 0;
+        if (s < p.B) {
+            const int n = clamped_context(p, s, true);
+            parts = (n + p.PT - 1) / p.PT;
+            if (n == 0) s_any_zero = 1;
+        }
+        // block-wide inclusive scan of parts
+        int x = parts;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, x, o);
+            if (lane >= o) x += y;
+        }
+        if (lane == 31) s_warp[warp] = x;
+        __syncthreads();
+        if (warp == 0) {
+            int w = s_warp[lane];
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int y = __shfl_up_sync(0xffffffffu, w, o);
+                if (lane >= o) w += y;
+            }
+            s_warp[lane] = w;  // inclusive over warps
+        }
+        __syncthreads();
+        const int incl = x + (warp > 0 ? s_warp[warp - 1] : 0);
+        s_off[tid + 1] = incl;
+        if (tid == 0) s_off[0] = 0;
+        __syncthreads();
+        const int chunk_total = s_off[kPlanThreads];
+        const int carry = s_carry;
+        // cooperative fill: entry e of this chunk belongs to the last seq whose
+        // exclusive offset is <= e
+        for (int e = tid; e < chunk_total; e += kPlanThreads) {
+            int lo = 0, hi = kPlanThreads - 1;
+            while (lo < hi) {
+                const int mid = (lo + hi + 1) >> 1;
+                if (s_off[mid] <= e) lo = mid; else hi = mid - 1;
+            }
+            p.entries[carry + e] = make_int2(base + lo, e - s_off[lo]);
+        }
+        __syncthreads();
+        if (tid == 0) s_carry = carry + chunk_total;
+        __syncthreads();
+    }
+    if (tid == 0) *p.num_entries = s_carry;
+    if (s_any_zero) {
+        const int vec_per_seq = p.Hq * D / 8;
+        uint4 *out = reinterpret_cast<uint4 *>(p.out);
+        for (long long i = tid; i < (long long)p.B * vec_per_seq; i += kPlanThreads) {
+            const int s = (int)(i / vec_per_seq);
+            if (clamped_context(p, s, false) == 0) out[i] = make_uint4(0, 0, 0, 0);
+        }
+    }
+}
+
+// ------------------------------------------------------ attention kernel ----
+
+struct StageInfo {
+    int s, h, part, nparts;  // item
+    int k, npad;             // stage index within the item, stages padded to a multiple of W
+    int valid;               // valid tokens in this stage (0 = padding stage)
+    int ord;                 // CTA-local item ordinal (selects the q buffer); -1 ends the stream
+};
+
+template <int D, int GP, int NS>
+struct DecodeSmem {
+    static constexpr int kW = kConsumerWarps;
+    static constexpr int kHalfTile = kStageTok * 64 * 2;  // 16 rows x 64 elements = 2 KB
+    static constexpr int kTile = kStageTok * D * 2;       // one K (or V) stage tile
+    static constexpr int kStage = 2 * kTile;
+    static constexpr int kQBuf = 16 * D * 2;              // room for 16 query heads
+    static constexpr int kMergeStride = D + 4;            // floats, padded against bank conflicts
+    static constexpr int oTiles = 0;
+    static constexpr int oQ = oTiles + NS * kStage;
+    static constexpr int oMergeO = oQ + 2 * kQBuf;
+    static constexpr int oMergeM = oMergeO + kW * GP * kMergeStride * 4;
+    static constexpr int oMergeL = oMergeM + kW * GP * 4;
+    static constexpr int oBars = (oMergeL + kW * GP * 4 + 7) / 8 * 8;
+    static constexpr int kNumBars = 2 * NS + 6;  // full, empty, qfull[2], qempty[2], mfull, mempty
+    static constexpr int oInfo = oBars + kNumBars * 8;
+    static constexpr int oAbort = oInfo + NS * (int)sizeof(StageInfo);
+    static constexpr int kBytes = oAbort + 16;
+    static constexpr int kAlloc = kBytes + 1024;  // slack to align the base to 1024 B
+};
+
+// Bounded wait that also gives up when another warp has aborted.
+__device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity, volatile int *abort_flag) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_timer_ns();
+    for (uint32_t it = 1;; ++it) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((it & 255u) == 0) {
+            if (*abort_flag) return false;
+            if (global_timer_ns() - t0 > kWaitLimitNs) {
+                raise_error(PKV_DEVERR_TIMEOUT);
+                *abort_flag = 1;
+                return false;
+            }
+        }
+    }
+}
+
+// Byte address of element (row r, column c) of a stage tile in shared memory.
+// The tile is [D/64][16][64] bf16; each 128-byte line (one row of one half)
+// has its 16-byte chunks XOR-swizzled with (r & 7) by the TMA unit.
+__device__ __forceinline__ uint32_t tile_addr(uint32_t tile, int r, int c) {
+    const int half = c >> 6;
+    const int chunk = (c & 63) >> 3;
+    return tile + half * (kStageTok * 128) + r * 128 + ((chunk ^ (r & 7)) << 4) + ((c & 7) << 1);
+}
+
+// ----------------------------------------------- CUDA-core path (g <= 2) ----
+template <int D, int G>
+struct SimtState {
+    static constexpr int EPL = D / 32;  // elements per lane
+    float q[G][EPL];
+    float acc[G][EPL];
+    float m[G];
+    float l_part;  // this lane's share of l for head (lane / 16) (G = 2) or head 0
+
+    __device__ __forceinline__ void reset() {
+#pragma unroll
+        for (int j = 0; j < G; ++j) {
+            m[j] = PKV_NEG_INF;
+#pragma unroll
+            for (int e = 0; e < EPL; ++e) acc[j][e] = 0.f;
+        }
+        l_part = 0.f;
+    }
+
+    __device__ __forceinline__ void load_q(const __nv_bfloat16 *qs, int lane, float scale_log2) {
+#pragma unroll
+        for (int j = 0; j < G; ++j)
+#pragma unroll
+            for (int e = 0; e < EPL; e += 2) {
+                const uint32_t pr = *reinterpret_cast<const uint32_t *>(qs + j * D + lane * EPL + e);
+                q[j][e] = bf16lo_to_f32(pr) * scale_log2;
+                q[j][e + 1] = bf16hi_to_f32(pr) * scale_log2;
+            }
+    }
+
+    // Loads this lane's EPL elements of row r of a tile as fp32.
+    __device__ __forceinline__ void load_row(uint32_t tile, int r, int lane, float (&x)[EPL]) {
+        const uint32_t a = tile_addr(tile, r, lane * EPL);
+        if constexpr (EPL == 4) {
+            uint32_t w0, w1;
+            asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(w0), "=r"(w1) : "r"(a));
+            x[0] = bf16lo_to_f32(w0); x[1] = bf16hi_to_f32(w0);
+            x[2] = bf16lo_to_f32(w1); x[3] = bf16hi_to_f32(w1);
+        } else {
+            uint32_t w0;
+            asm volatile("ld.shared.u32 %0, [%1];" : "=r"(w0) : "r"(a));
+            x[0] = bf16lo_to_f32(w0); x[1] = bf16hi_to_f32(w0);
+        }
+    }
+
+    __device__ __forceinline__ void stage(uint32_t ktile, uint32_t vtile, int valid, int lane) {
+        constexpr int NV = 16 * G;
+        float v[NV];
+        // q.k partial sums: v[j*16 + r] for head j, token r
+#pragma unroll
+        for (int r = 0; r < 16; ++r) {
+            float x[EPL];
+            load_row(ktile, r, lane, x);
+#pragma unroll
+            for (int j = 0; j < G; ++j) {
+                float d = 0.f;
+#pragma unroll
+                for (int e = 0; e < EPL; ++e) d = fmaf(q[j][e], x[e], d);
+                v[j * 16 + r] = d;
+            }
+        }
+        // Transposing butterfly: after it, lane holds the full 32-lane sum of
+        // value index idx(lane): G = 1 -> token lane >> 1; G = 2 -> head
+        // lane >> 4, token lane & 15.
+        int n = NV;
+#pragma unroll
+        for (int mask = 16; mask >= 1; mask >>= 1) {
+            if (n > 1) {
+                const bool upper = (lane & mask) != 0;
+                n >>= 1;
+#pragma unroll
+                for (int i = 0; i < NV / 2; ++i) {
+                    if (i < n) {
+                        const float send = upper ? v[i] : v[i + n];
+                        const float keep = upper ? v[i + n] : v[i];
+                        v[i] = keep + __shfl_xor_sync(0xffffffffu, send, mask);
+                    }
+                }
+            } else {
+                v[0] += __shfl_xor_sync(0xffffffffu, v[0], mask);
+            }
+        }
+        const int my_tok = (G == 1) ? (lane >> 1) : (lane & 15);
+        const int my_head = (G == 1) ? 0 : (lane >> 4);
+        const float score = (my_tok < valid) ? v[0] : PKV_NEG_INF;
+        // stage max per head
+        float mx = score;
+        if (G == 1) {
+#pragma unroll
+            for (int o = 2; o < 32; o <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        } else {
+#pragma unroll
+            for (int o = 1; o < 16; o <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        }
+        float m_new[G], alpha[G];
+        if constexpr (G == 1) {
+            m_new[0] = fmaxf(m[0], mx);
+        } else {
+            const float other = __shfl_xor_sync(0xffffffffu, mx, 16);
+            m_new[0] = fmaxf(m[0], my_head == 0 ? mx : other);
+            m_new[1] = fmaxf(m[1], my_head == 0 ? other : mx);
+        }
+#pragma unroll
+        for (int j = 0; j < G; ++j) {
+            alpha[j] = exp2f(m[j] - m_new[j]);
+            m[j] = m_new[j];
+        }
+        // selects, not a lane-dependent register index
+        const float my_m = (G == 1 || my_head == 0) ? m_new[0] : m_new[G - 1];
+        const float my_alpha = (G == 1 || my_head == 0) ? alpha[0] : alpha[G - 1];
+        const float pr = exp2f(score - my_m);
+        l_part = l_part * my_alpha + pr;
+#pragma unroll
+        for (int j = 0; j < G; ++j)
+#pragma unroll
+            for (int e = 0; e < EPL; ++e) acc[j][e] *= alpha[j];
+        // PV: broadcast p of each valid token, accumulate its V row
+#pragma unroll
+        for (int r = 0; r < 16; ++r) {
+            if (r < valid) {
+                float x[EPL];
+                load_row(vtile, r, lane, x);
+#pragma unroll
+                for (int j = 0; j < G; ++j) {
+                    const int src = (G == 1) ? (2 * r) : (j * 16 + r);
+                    const float pj = __shfl_sync(0xffffffffu, pr, src);
+#pragma unroll
+                    for (int e = 0; e < EPL; ++e) acc[j][e] = fmaf(pj, x[e], acc[j][e]);
+                }
+            }
+        }
+    }
+
+    // Writes this warp's partial (m, l, acc) into the merge buffers.
+    __device__ __forceinline__ void store_partial(float *mO, float *mM, float *mL, int w, int lane, int stride,
+                                                  int GPn) {
+        float l = l_part;
+        if (G == 1) {
+#pragma unroll
+            for (int o = 2; o < 32; o <<= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
+        } else {
+#pragma unroll
+            for (int o = 1; o < 16; o <<= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
+        }
+#pragma unroll
+        for (int j = 0; j < G; ++j)
+#pragma unroll
+            for (int e = 0; e < EPL; ++e) mO[(w * GPn + j) * stride + lane * EPL + e] = acc[j][e];
+        if constexpr (G == 1) {
+            if (lane == 0) { mM[w * GPn] = m[0]; mL[w * GPn] = l; }
+        } else {
+            if (lane == 0) { mM[w * GPn] = m[0]; mL[w * GPn] = l; }
+            if (lane == 16) { mM[w * GPn + 1] = m[1]; mL[w * GPn + 1] = l; }
+        }
+    }
+};
+
+// ------------------------------------------- tensor-core path (3 <= g <= 16) --
+template <int D, int NT>
+struct MmaState {
+    static constexpr int KS = D / 16;  // k-steps of QK^T
+    static constexpr int MT = D / 16;  // m-tiles of O^T
+    uint32_t qb[NT][KS][2];            // B fragments of Q^T
+    float o[NT][MT][4];                // O^T accumulators
+    float m[NT][2];                    // running max of heads nt*8 + 2*(lane%4) + {0,1}
+    float l[NT][2];                    // this thread's share of the sums
+
+    __device__ __forceinline__ void reset() {
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+            for (int c = 0; c < 2; ++c) { m[nt][c] = PKV_NEG_INF; l[nt][c] = 0.f; }
+#pragma unroll
+            for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+                for (int c = 0; c < 4; ++c) o[nt][mt][c] = 0.f;
+        }
+    }
+
+    // B fragment of Q^T (k = head dim, n = head): b0 = Q[n][k0 + 2(l%4) + {0,1}],
+    // b1 = the same 8 columns further; heads >= g are zero.
+    __device__ __forceinline__ void load_q(const __nv_bfloat16 *qs, int lane, int g) {
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+            const int head = nt * 8 + (lane >> 2);
+#pragma unroll
+            for (int kk = 0; kk < KS; ++kk) {
+                const int col = kk * 16 + 2 * (lane & 3);
+                uint32_t b0 = 0, b1 = 0;
+                if (head < g) {
+                    b0 = *reinterpret_cast<const uint32_t *>(qs + head * D + col);
+                    b1 = *reinterpret_cast<const uint32_t *>(qs + head * D + col + 8);
+                }
+                qb[nt][kk][0] = b0;
+                qb[nt][kk][1] = b1;
+            }
+        }
+    }
+
+    __device__ __forceinline__ void stage(uint32_t ktile, uint32_t vtile, int valid, int lane, float scale_log2) {
+        // S^T[token][head] = K . Q^T
+        float s[NT][4];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int c = 0; c < 4; ++c) s[nt][c] = 0.f;
+        const int mi = lane >> 3, ri = lane & 7;
+#pragma unroll
+        for (int kk = 0; kk < KS; ++kk) {
+            // matrices: (rows 0-7, cols k0..+7), (rows 8-15, k0..), (rows 0-7, k0+8..), (rows 8-15, k0+8..)
+            const int row = ri + 8 * (mi & 1);
+            const int col = kk * 16 + 8 * (mi >> 1);
+            uint32_t a0, a1, a2, a3;
+            ldmatrix_x4(tile_addr(ktile, row, col), a0, a1, a2, a3);
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+                mma_bf16_16816(s[nt][0], s[nt][1], s[nt][2], s[nt][3], a0, a1, a2, a3, qb[nt][kk][0],
+                               qb[nt][kk][1]);
+        }
+        const int t0 = lane >> 2;  // tokens t0 and t0 + 8
+        const bool ok0 = t0 < valid, ok1 = t0 + 8 < valid;
+        uint32_t pb[NT][2];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+            float alpha[2], p[4];
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
+                const float z0 = ok0 ? s[nt][c] * scale_log2 : PKV_NEG_INF;
+                const float z1 = ok1 ? s[nt][c + 2] * scale_log2 : PKV_NEG_INF;
+                float mx = fmaxf(z0, z1);
+                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+                const float mn = fmaxf(m[nt][c], mx);
+                alpha[c] = exp2f(m[nt][c] - mn);
+                m[nt][c] = mn;
+                p[c] = exp2f(z0 - mn);
+                p[c + 2] = exp2f(z1 - mn);
+                l[nt][c] = l[nt][c] * alpha[c] + p[c] + p[c + 2];
+            }
+            // accumulator layout (token row, head pair) -> operand layout of P^T
+            pb[nt][0] = movmatrix_trans(pack_bf16x2(p[0], p[1]));
+            pb[nt][1] = movmatrix_trans(pack_bf16x2(p[2], p[3]));
+#pragma unroll
+            for (int mt = 0; mt < MT; ++mt) {
+                o[nt][mt][0] *= alpha[0];
+                o[nt][mt][1] *= alpha[1];
+                o[nt][mt][2] *= alpha[0];
+                o[nt][mt][3] *= alpha[1];
+            }
+        }
+        // token masks of this thread's V^T operand halves: tokens 2(l%4)+{0,1} and +8
+        uint32_t mask01 = 0xffffffffu, mask23 = 0xffffffffu;
+        if (valid < 16) {
+            const int j0 = 2 * (lane & 3);
+            mask01 = (j0 < valid ? 0x0000ffffu : 0u) | (j0 + 1 < valid ? 0xffff0000u : 0u);
+            mask23 = (j0 + 8 < valid ? 0x0000ffffu : 0u) | (j0 + 9 < valid ? 0xffff0000u : 0u);
+        }
+        // O^T[d][head] += V^T . P^T
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt) {
+            // matrices (stored rows = tokens): (tok 0-7, d0..+7), (tok 0-7, d0+8..), (tok 8-15, d0..), (tok 8-15, d0+8..)
+            const int row = ri + 8 * (mi >> 1);
+            const int col = mt * 16 + 8 * (mi & 1);
+            uint32_t a0, a1, a2, a3;
+            ldmatrix_x4_trans(tile_addr(vtile, row, col), a0, a1, a2, a3);
+            a0 &= mask01; a1 &= mask01; a2 &= mask23; a3 &= mask23;
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+                mma_bf16_16816(o[nt][mt][0], o[nt][mt][1], o[nt][mt][2], o[nt][mt][3], a0, a1, a2, a3,
+                               pb[nt][0], pb[nt][1]);
+        }
+    }
+
+    __device__ __forceinline__ void store_partial(float *mO, float *mM, float *mL, int w, int lane, int stride,
+                                                  int GPn, int g) {
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
+                float lsum = l[nt][c];
+                lsum += __shfl_xor_sync(0xffffffffu, lsum, 4);
+                lsum += __shfl_xor_sync(0xffffffffu, lsum, 8);
+                lsum += __shfl_xor_sync(0xffffffffu, lsum, 16);
+                const int head = nt * 8 + 2 * (lane & 3) + c;
+                if (head < g) {
+                    if (lane < 4) { mM[w * GPn + head] = m[nt][c]; mL[w * GPn + head] = lsum; }
+                    float *row = mO + (w * GPn + head) * stride;
+#pragma unroll
+                    for (int mt = 0; mt < MT; ++mt) {
+                        row[mt * 16 + (lane >> 2)] = o[nt][mt][c];
+                        row[mt * 16 + (lane >> 2) + 8] = o[nt][mt][c + 2];
+                    }
+                }
+            }
+        }
+    }
+};
+
+// PATH 0: CUDA cores with G = GSIMT heads per kv head; PATH 1: tensor cores
+// with NT n-tiles of 8 heads.
+template <int D, int PATH, int GSIMT, int NT, int NS>
+__global__ void __launch_bounds__(kDecodeThreads) paged_decode_kernel(const __grid_constant__ CUtensorMap tmap_k,
+                                                                      const __grid_constant__ CUtensorMap tmap_v,
+                                                                      const DecodeParams p) {
+    constexpr int W = kConsumerWarps;
+    constexpr int GP = PATH == 0 ? GSIMT : 8 * NT;
+    using L = DecodeSmem<D, GP, NS>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + L::oBars);
+    uint64_t *empty = full + NS;
+    uint64_t *qfull = empty + NS;
+    uint64_t *qempty = qfull + 2;
+    uint64_t *mfull = qempty + 2;
+    uint64_t *mempty = mfull + 1;
+    StageInfo *info = reinterpret_cast<StageInfo *>(smem + L::oInfo);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::oAbort);
+    const uint32_t tiles = smem_u32(smem + L::oTiles);
+    __nv_bfloat16 *qbuf = reinterpret_cast<__nv_bfloat16 *>(smem + L::oQ);
+    float *mO = reinterpret_cast<float *>(smem + L::oMergeO);
+    float *mM = reinterpret_cast<float *>(smem + L::oMergeM);
+    float *mL = reinterpret_cast<float *>(smem + L::oMergeL);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < NS; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); }
+        for (int i = 0; i < 2; ++i) { mbar_init(&qfull[i], 1); mbar_init(&qempty[i], W); }
+        mbar_init(mfull, W);
+        mbar_init(mempty, W);
+        *abort_flag = 0;
+        fence_mbar_init();
+        tma_prefetch_desc(&tmap_k);
+        tma_prefetch_desc(&tmap_v);
+    }
+    __syncthreads();
+    // Everything below reads data written by earlier kernels on the stream.
+    grid_dependency_wait();
+
+    if (warp == W) {
+        // ------------------------------------------------------ producer --
+        const int n_items = *reinterpret_cast<volatile int32_t *>(p.num_entries) * p.Hkv;
+        uint32_t gc = 0;
+        int ord = 0;
+        bool ok = true;
+        for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x, ++ord) {
+            const int e = it / p.Hkv;
+            const int h = it - e * p.Hkv;
+            const int2 sp = p.entries[e];
+            const int s = sp.x, part = sp.y;
+            const int n = clamped_context(p, s, false);
+            const int nparts = (n + p.PT - 1) / p.PT;
+            const int t0 = part * p.PT;
+            const int t1 = min(n, t0 + p.PT);
+            const int nst = (t1 - t0 + kStageTok - 1) / kStageTok;
+            const int npad = (nst + W - 1) / W * W;
+            if (lane == 0) {
+                const int qb = ord & 1;
+                ok = wait_or_abort(&qempty[qb], ((ord >> 1) & 1) ^ 1, abort_flag);
+                if (ok) {
+                    const uint32_t bytes = (uint32_t)(p.g * D * 2);
+                    mbar_arrive_expect_tx(&qfull[qb], bytes);
+                    bulk_load(qbuf + qb * (L::kQBuf / 2), p.q + ((size_t)s * p.Hq + (size_t)h * p.g) * D, bytes,
+                              &qfull[qb]);
+                }
+            }
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+            int blk_reg = -1;
+            for (int k = 0; k < npad && ok; ++k) {
+                if ((k & 31) == 0) {
+                    // lane l fetches the block id of stage k + l
+                    const int kk = k + lane;
+                    int blk = -1;
+                    if (kk < nst) {
+                        const int tok = t0 + kk * kStageTok;
+                        blk = __ldg(p.block_tables + (size_t)s * p.MBS + tok / p.bs);
+                        if (blk < 0 || blk >= p.NB) {
+                            raise_error(PKV_DEVERR_BLOCK);
+                            blk = -1;
+                        }
+                    }
+                    blk_reg = blk;
+                }
+                const int blk = __shfl_sync(0xffffffffu, blk_reg, k & 31);
+                if (lane == 0) {
+                    const uint32_t slot = gc % NS;
+                    ok = wait_or_abort(&empty[slot], ((gc / NS) & 1) ^ 1, abort_flag);
+                    if (ok) {
+                        const int tok = t0 + k * kStageTok;
+                        const int valid = k < nst ? min(kStageTok, t1 - tok) : 0;
+                        StageInfo si;
+                        si.s = s; si.h = h; si.part = part; si.nparts = nparts;
+                        si.k = k; si.npad = npad; si.valid = valid; si.ord = ord;
+                        info[slot] = si;
+                        if (valid > 0) {
+                            // rows of (block, head, offset): an invalid id reads the zero fill
+                            const int row = blk >= 0 ? (blk * p.Hkv + h) * p.bs + tok % p.bs : p.pool_rows;
+                            const uint32_t kt = tiles + slot * L::kStage;
+                            mbar_arrive_expect_tx(&full[slot], (uint32_t)L::kStage);
+#pragma unroll
+                            for (int hf = 0; hf < D / 64; ++hf) {
+                                tma_load_2d_u32(kt + hf * L::kHalfTile, &tmap_k, &full[slot], hf * 64, row);
+                                tma_load_2d_u32(kt + L::kTile + hf * L::kHalfTile, &tmap_v, &full[slot], hf * 64, row);
+                            }
+                        } else {
+                            mbar_arrive(&full[slot]);
+                        }
+                    }
+                }
+                ok = __shfl_sync(0xffffffffu, ok, 0);
+                ++gc;
+            }
+        }
+        // end-of-stream marker for every consumer warp
+        if (lane == 0) {
+            for (int w = 0; w < W && ok; ++w) {
+                const uint32_t slot = gc % NS;
+                ok = wait_or_abort(&empty[slot], ((gc / NS) & 1) ^ 1, abort_flag);
+                if (ok) {
+                    info[slot].ord = -1;
+                    mbar_arrive(&full[slot]);
+                }
+                ++gc;
+            }
+            // Drain: every TMA this CTA issued must have landed before exit.
+            // In a normal run the consumers already waited for all of them.
+            if (!ok) {
+                const uint32_t issued = gc;
+                for (uint32_t c = (issued > (uint32_t)NS ? issued - NS : 0); c < issued; ++c)
+                    mbar_wait_bounded(&full[c % NS], (c / NS) & 1, kWaitLimitNs);
+            }
+        }
+        grid_launch_dependents();
+    } else {
+        // ------------------------------------------------------ consumer --
+        const int w = warp;
+        uint32_t gc = w;
+        uint32_t mc = 0;  // merges done
+        float scale_log2 = p.scale_log2;
+        SimtState<D, (PATH == 0 ? GSIMT : 1)> st0;
+        MmaState<D, (PATH == 1 ? NT : 1)> st1;
+        while (true) {
+            const uint32_t slot = gc % NS;
+            if (!wait_or_abort(&full[slot], (gc / NS) & 1, abort_flag)) break;
+            const StageInfo si = info[slot];
+            if (si.ord < 0) break;
+            if (si.k == w) {
+                // first stage of this item for this warp: fresh state and q
+                const int qb = si.ord & 1;
+                if (!wait_or_abort(&qfull[qb], (si.ord >> 1) & 1, abort_flag)) break;
+                const __nv_bfloat16 *qs = qbuf + qb * (L::kQBuf / 2);
+                if constexpr (PATH == 0) { st0.reset(); st0.load_q(qs, lane, scale_log2); }
+                else { st1.reset(); st1.load_q(qs, lane, p.g); }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&qempty[qb]);
+            }
+            if (si.valid > 0) {
+                const uint32_t kt = tiles + slot * L::kStage;
+                if constexpr (PATH == 0) st0.stage(kt, kt + L::kTile, si.valid, lane);
+                else st1.stage(kt, kt + L::kTile, si.valid, lane, scale_log2);
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[slot]);
+            gc += W;
+            if (si.k + W >= si.npad) {
+                // this warp's last stage of the item: merge the W partials
+                if (!wait_or_abort(mempty, (mc & 1) ^ 1, abort_flag)) break;
+                if constexpr (PATH == 0) st0.store_partial(mO, mM, mL, w, lane, L::kMergeStride, GP);
+                else st1.store_partial(mO, mM, mL, w, lane, L::kMergeStride, GP, p.g);
+                __syncwarp();
+                if (lane == 0) mbar_arrive(mfull);
+                if (!wait_or_abort(mfull, mc & 1, abort_flag)) break;
+                const int g = p.g;
+                const size_t unit_head0 = (size_t)si.s * p.Hq + (size_t)si.h * g;
+                for (int idx = w * 32 + lane; idx < g * D; idx += W * 32) {
+                    const int j = idx / D, d = idx - j * D;
+                    float M = PKV_NEG_INF;
+#pragma unroll
+                    for (int u = 0; u < W; ++u) M = fmaxf(M, mM[u * GP + j]);
+                    float Lsum = 0.f, O = 0.f;
+#pragma unroll
+                    for (int u = 0; u < W; ++u) {
+                        const float mu = mM[u * GP + j];
+                        const float f = mu == PKV_NEG_INF ? 0.f : exp2f(mu - M);
+                        Lsum = fmaf(mL[u * GP + j], f, Lsum);
+                        O = fmaf(mO[(u * GP + j) * L::kMergeStride + d], f, O);
+                    }
+                    if (si.nparts == 1) {
+                        p.out[(unit_head0 + j) * D + d] = __float2bfloat16_rn(Lsum > 0.f ? O / Lsum : 0.f);
+                    } else {
+                        const size_t pi = (unit_head0 + j) * p.maxP + si.part;
+                        p.part_acc[pi * D + d] = O;
+                        if (d == 0) p.part_ml[pi] = make_float2(M, Lsum);
+                    }
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(mempty);
+                ++mc;
+            }
+        }
+        grid_launch_dependents();
+    }
+}
+
+// --------------------------------------------------------------- reduce ----
+// Log-sum-exp merge of the partitions of every (s, hq) with more than one
+// partition: M = max_p m_p, L = sum_p l_p 2^(m_p - M),
+// out = sum_p acc_p 2^(m_p - M) / L.  One CTA per (s, hq); warp w takes
+// partitions w, w + 4, ...; lanes own D/32 consecutive elements.
+template <int D>
+__global__ void __launch_bounds__(kReduceWarps * 32) splitk_reduce_kernel(const DecodeParams p) {
+    constexpr int EPL = D / 32;
+    __shared__ float s_o[kReduceWarps][D];
+    __shared__ float s_l[kReduceWarps];
+    grid_dependency_wait();
+    const int unit = blockIdx.x;  // s * Hq + hq
+    const int s = unit / p.Hq;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int n = clamped_context(p, s, false);
+    const int P = (n + p.PT - 1) / p.PT;
+    if (P <= 1) return;  // written directly by the attention kernel
+    const float2 *ml = p.part_ml + (size_t)unit * p.maxP;
+    float M = PKV_NEG_INF;
+    for (int i = lane; i < P; i += 32) M = fmaxf(M, ml[i].x);
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    float acc[EPL];
+#pragma unroll
+    for (int e = 0; e < EPL; ++e) acc[e] = 0.f;
+    float lsum = 0.f;
+    const float *base = p.part_acc + (size_t)unit * p.maxP * D + lane * EPL;
+#pragma unroll 4
+    for (int i = warp; i < P; i += kReduceWarps) {
+        const float2 mli = ml[i];
+        const float f = exp2f(mli.x - M);
+        lsum = fmaf(mli.y, f, lsum);
+        if constexpr (EPL == 4) {
+            const float4 a = *reinterpret_cast<const float4 *>(base + (size_t)i * D);
+            acc[0] = fmaf(a.x, f, acc[0]); acc[1] = fmaf(a.y, f, acc[1]);
+            acc[2] = fmaf(a.z, f, acc[2]); acc[3] = fmaf(a.w, f, acc[3]);
+        } else {
+            const float2 a = *reinterpret_cast<const float2 *>(base + (size_t)i * D);
+            acc[0] = fmaf(a.x, f, acc[0]); acc[1] = fmaf(a.y, f, acc[1]);
+        }
+    }
+#pragma unroll
+    for (int e = 0; e < EPL; ++e) s_o[warp][lane * EPL + e] = acc[e];
+    if (lane == 0) s_l[warp] = lsum;
+    __syncthreads();
+    if (warp == 0) {
+        float Lt = 0.f;
+#pragma unroll
+        for (int u = 0; u < kReduceWarps; ++u) Lt += s_l[u];
+        const float inv = Lt > 0.f ? 1.f / Lt : 0.f;
+#pragma unroll
+        for (int e = 0; e < EPL; ++e) {
+            float o = 0.f;
+#pragma unroll
+            for (int u = 0; u < kReduceWarps; ++u) o += s_o[u][lane * EPL + e];
+            p.out[(size_t)unit * D + lane * EPL + e] = __float2bfloat16_rn(o * inv);
+        }
+    }
+}
+
+}  // namespace pkv

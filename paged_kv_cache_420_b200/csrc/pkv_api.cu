@@ -1,0 +1,338 @@
+// pkv_api.cu -- host side of the C ABI declared in include/pkv.h: argument
+// validation, launch configuration, TMA descriptors and kernel launches.
+// The device code lives in the headers included below (one translation unit,
+// so the device error word is a single module global).
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "decode.cuh"
+#include "pkv.h"
+#include "write_copy.cuh"
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+constexpr int kDecodeStages = 8;  // NS: shared-memory ring slots per CTA
+
+bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+int current_device() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+    return dev;
+}
+
+int sm_count(int dev) {
+    static int cache[kMaxDevices] = {0};
+    if (dev < 0 || dev >= kMaxDevices) return 148;
+    if (cache[dev] == 0) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+        cache[dev] = n;
+    }
+    return cache[dev];
+}
+
+pkv_status check_pool(const pkv_pool &pool) {
+    if (pool.num_blocks <= 0 || pool.num_kv_heads <= 0 || pool.block_size <= 0 || pool.head_dim <= 0)
+        return PKV_EINVAL;
+    if (pool.head_dim != 64 && pool.head_dim != 128) return PKV_EUNSUPPORTED;
+    if (pool.block_size % 16 != 0 || pool.block_size > 1024) return PKV_EUNSUPPORTED;
+    const long long rows = (long long)pool.num_blocks * pool.num_kv_heads * pool.block_size;
+    if (rows >= (1ll << 31) - 1) return PKV_EUNSUPPORTED;  // TMA row coordinates are int32
+    return PKV_OK;
+}
+
+pkv_status launch_status() {
+    const cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? PKV_OK : PKV_ECUDA;
+}
+
+// ------------------------------------------------------------ TMA maps ----
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    });
+    return fn;
+}
+
+// The pool viewed as a 2-D tensor: rows = (block, head, offset), columns =
+// head_dim elements.  A box is 16 rows x 64 columns (128 B) with the 128-byte
+// swizzle, so a K or V stage tile of one (block, head) is D/64 boxes.
+bool encode_pool_map(CUtensorMap *map, const void *base, const pkv_pool &pool) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t rows = (cuuint64_t)pool.num_blocks * pool.num_kv_heads * pool.block_size;
+    cuuint64_t dims[2] = {(cuuint64_t)pool.head_dim, rows};
+    cuuint64_t strides[1] = {(cuuint64_t)pool.head_dim * 2};
+    cuuint32_t box[2] = {64, (cuuint32_t)pkv::kStageTok};
+    cuuint32_t estr[2] = {1, 1};
+    const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box,
+                          estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+// ----------------------------------------------------------- workspace ----
+
+struct WorkspaceLayout {
+    size_t off_count, off_entries, off_ml, off_acc, total;
+};
+
+size_t round256(size_t x) { return (x + 255) / 256 * 256; }
+
+int pick_partition_tokens(int32_t partition_tokens) {
+    return partition_tokens > 0 ? partition_tokens : 512;
+}
+
+bool workspace_layout(int32_t B, int32_t Hq, int32_t D, int32_t max_ctx, int32_t PT, WorkspaceLayout *w) {
+    if (B < 0 || Hq <= 0 || D <= 0 || max_ctx < 0 || PT <= 0) return false;
+    const long long maxP = std::max<long long>(1, ((long long)max_ctx + PT - 1) / PT);
+    size_t off = 0;
+    w->off_count = off;
+    off += 256;
+    w->off_entries = off;
+    off += round256((size_t)B * maxP * sizeof(int2));
+    w->off_ml = off;
+    if (maxP > 1) off += round256((size_t)B * Hq * maxP * sizeof(float2));
+    w->off_acc = off;
+    if (maxP > 1) off += round256((size_t)B * Hq * maxP * D * sizeof(float));
+    w->total = off;
+    return true;
+}
+
+// ---------------------------------------------------- decode dispatch ----
+
+template <int D, int PATH, int GS, int NT>
+pkv_status launch_decode(const pkv::DecodeParams &prm, const CUtensorMap &mk, const CUtensorMap &mv,
+                         cudaStream_t stream, int dev) {
+    using L = pkv::DecodeSmem<D, (PATH == 0 ? GS : 8 * NT), kDecodeStages>;
+    auto kernel = pkv::paged_decode_kernel<D, PATH, GS, NT, kDecodeStages>;
+    static int occ_cache[kMaxDevices] = {0};
+    int occ = (dev >= 0 && dev < kMaxDevices) ? occ_cache[dev] : 0;
+    if (occ == 0) {
+        if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc) != cudaSuccess)
+            return PKV_ECUDA;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kernel, pkv::kDecodeThreads, L::kAlloc) !=
+                cudaSuccess ||
+            occ <= 0)
+            return PKV_ECUDA;
+        if (dev >= 0 && dev < kMaxDevices) occ_cache[dev] = occ;
+    }
+    const long long items_upper = (long long)prm.B * prm.Hkv * prm.maxP;
+    const long long grid = std::max<long long>(1, std::min<long long>(items_upper, (long long)sm_count(dev) * occ));
+
+    cudaLaunchConfig_t cfg;
+    std::memset(&cfg, 0, sizeof cfg);
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3(pkv::kDecodeThreads);
+    cfg.dynamicSmemBytes = L::kAlloc;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, kernel, mk, mv, prm) != cudaSuccess) return PKV_ECUDA;
+    if (prm.maxP > 1) {
+        cudaLaunchConfig_t rc = cfg;
+        rc.gridDim = dim3((unsigned)((long long)prm.B * prm.Hq));
+        rc.blockDim = dim3(pkv::kReduceWarps * 32);
+        rc.dynamicSmemBytes = 0;
+        if (cudaLaunchKernelEx(&rc, pkv::splitk_reduce_kernel<D>, prm) != cudaSuccess) return PKV_ECUDA;
+    }
+    return launch_status();
+}
+
+template <int D>
+pkv_status dispatch_group(int g, const pkv::DecodeParams &prm, const CUtensorMap &mk, const CUtensorMap &mv,
+                          cudaStream_t stream, int dev) {
+    if (g == 1) return launch_decode<D, 0, 1, 1>(prm, mk, mv, stream, dev);
+    if (g == 2) return launch_decode<D, 0, 2, 1>(prm, mk, mv, stream, dev);
+    if (g <= 8) return launch_decode<D, 1, 1, 1>(prm, mk, mv, stream, dev);
+    return launch_decode<D, 1, 1, 2>(prm, mk, mv, stream, dev);
+}
+
+}  // namespace
+
+extern "C" {
+
+int32_t pkv_version(void) { return 10000; }
+
+const char *pkv_status_string(pkv_status s) {
+    switch (s) {
+        case PKV_OK: return "ok";
+        case PKV_EINVAL: return "invalid argument (size, null or misaligned pointer, workspace)";
+        case PKV_ERANGE: return "block id outside the pool";
+        case PKV_EALIAS: return "copy pairs alias (repeated destination, or destination that is a source)";
+        case PKV_ECUDA: return "CUDA call failed";
+        case PKV_EDEVICE: return "device error word set";
+        case PKV_EUNSUPPORTED: return "unsupported shape";
+    }
+    return "unknown status";
+}
+
+pkv_status pkv_write(const void *k, const void *v, const int64_t *slot_mapping, int32_t num_tokens, void *k_cache,
+                     void *v_cache, pkv_pool pool, pkv_stream_t stream) {
+    const pkv_status ps = check_pool(pool);
+    if (ps != PKV_OK) return ps;
+    if (num_tokens < 0) return PKV_EINVAL;
+    if (num_tokens == 0) return PKV_OK;
+    if (!k || !v || !slot_mapping || !k_cache || !v_cache) return PKV_EINVAL;
+    if (!aligned(k, 16) || !aligned(v, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) ||
+        !aligned(slot_mapping, 8))
+        return PKV_EINVAL;
+    pkv::WriteParams p;
+    p.k = static_cast<const uint4 *>(k);
+    p.v = static_cast<const uint4 *>(v);
+    p.slots = slot_mapping;
+    p.k_cache = static_cast<uint4 *>(k_cache);
+    p.v_cache = static_cast<uint4 *>(v_cache);
+    p.vpr = pool.head_dim / 8;
+    p.num_kv_heads = pool.num_kv_heads;
+    p.block_size = pool.block_size;
+    p.pool_slots = (int64_t)pool.num_blocks * pool.block_size;
+    p.total = (int64_t)num_tokens * 2 * pool.num_kv_heads * p.vpr;
+    const int dev = current_device();
+    const long long blocks = std::min<long long>((p.total + 255) / 256, (long long)sm_count(dev) * 16);
+    pkv::kv_write_kernel<<<(unsigned)std::max<long long>(blocks, 1), 256, 0, (cudaStream_t)stream>>>(p);
+    return launch_status();
+}
+
+pkv_status pkv_copy_blocks(const int32_t *src_dst_pairs, int32_t num_pairs, void *k_cache, void *v_cache,
+                           pkv_pool pool, pkv_stream_t stream) {
+    const pkv_status ps = check_pool(pool);
+    if (ps != PKV_OK) return ps;
+    if (num_pairs < 0) return PKV_EINVAL;
+    if (num_pairs == 0) return PKV_OK;
+    if (!src_dst_pairs || !k_cache || !v_cache) return PKV_EINVAL;
+    if (!aligned(k_cache, 16) || !aligned(v_cache, 16)) return PKV_EINVAL;
+    std::vector<int32_t> src(num_pairs), dst(num_pairs);
+    for (int i = 0; i < num_pairs; ++i) {
+        src[i] = src_dst_pairs[2 * i];
+        dst[i] = src_dst_pairs[2 * i + 1];
+        if (src[i] < 0 || src[i] >= pool.num_blocks || dst[i] < 0 || dst[i] >= pool.num_blocks) return PKV_ERANGE;
+    }
+    std::sort(src.begin(), src.end());
+    std::vector<int32_t> dsorted(dst);
+    std::sort(dsorted.begin(), dsorted.end());
+    for (int i = 1; i < num_pairs; ++i)
+        if (dsorted[i] == dsorted[i - 1]) return PKV_EALIAS;
+    for (int i = 0; i < num_pairs; ++i)
+        if (std::binary_search(src.begin(), src.end(), dsorted[i])) return PKV_EALIAS;
+
+    pkv::CopyParams p;
+    p.k_cache = static_cast<uint4 *>(k_cache);
+    p.v_cache = static_cast<uint4 *>(v_cache);
+    p.vec_per_block = (int64_t)pool.num_kv_heads * pool.block_size * pool.head_dim / 8;
+    const long long per_cta = pkv::kCopyThreads * pkv::kCopyVecPerThread;
+    const unsigned gx = (unsigned)((p.vec_per_block + per_cta - 1) / per_cta);
+    for (int base = 0; base < num_pairs; base += pkv::kMaxPairsPerLaunch) {
+        const int n = std::min(pkv::kMaxPairsPerLaunch, num_pairs - base);
+        p.num_pairs = n;
+        for (int i = 0; i < n; ++i)
+            p.pairs[i] = make_int2(src_dst_pairs[2 * (base + i)], src_dst_pairs[2 * (base + i) + 1]);
+        pkv::copy_blocks_kernel<<<dim3(gx, n), pkv::kCopyThreads, 0, (cudaStream_t)stream>>>(p);
+        const pkv_status st = launch_status();
+        if (st != PKV_OK) return st;
+    }
+    return PKV_OK;
+}
+
+size_t pkv_decode_workspace_bytes(int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                                  int32_t max_context_len, int32_t partition_tokens) {
+    if (num_kv_heads <= 0 || num_q_heads <= 0 || num_q_heads % num_kv_heads) return 0;
+    if (partition_tokens < 0 || partition_tokens % 16) return 0;
+    WorkspaceLayout w;
+    if (!workspace_layout(num_seqs, num_q_heads, head_dim, max_context_len, pick_partition_tokens(partition_tokens),
+                          &w))
+        return 0;
+    return w.total;
+}
+
+pkv_status paged_attn_decode(const void *q, const void *k_cache, const void *v_cache, const int32_t *block_tables,
+                             int32_t max_blocks_per_seq, const int32_t *context_lens, int32_t num_seqs,
+                             int32_t num_q_heads, float scale, int32_t num_kv_heads, void *out, pkv_pool pool,
+                             int32_t max_context_len, int32_t partition_tokens, void *workspace,
+                             size_t workspace_bytes, pkv_stream_t stream) {
+    const pkv_status ps = check_pool(pool);
+    if (ps != PKV_OK) return ps;
+    if (num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || max_blocks_per_seq <= 0 || max_context_len < 0)
+        return PKV_EINVAL;
+    if (num_kv_heads != pool.num_kv_heads || num_q_heads % num_kv_heads != 0) return PKV_EINVAL;
+    const int g = num_q_heads / num_kv_heads;
+    if (g > 16) return PKV_EUNSUPPORTED;
+    if (partition_tokens < 0 || partition_tokens % 16 != 0 || partition_tokens > 65536) return PKV_EINVAL;
+    if (num_seqs == 0) return PKV_OK;
+    if (!q || !k_cache || !v_cache || !block_tables || !context_lens || !out || !workspace) return PKV_EINVAL;
+    if (!aligned(q, 16) || !aligned(out, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) ||
+        !aligned(block_tables, 4) || !aligned(context_lens, 4) || !aligned(workspace, 256))
+        return PKV_EINVAL;
+    const int D = pool.head_dim;
+    const int PT = pick_partition_tokens(partition_tokens);
+    WorkspaceLayout wl;
+    if (!workspace_layout(num_seqs, num_q_heads, D, max_context_len, PT, &wl) || workspace_bytes < wl.total)
+        return PKV_EINVAL;
+
+    pkv::DecodeParams prm;
+    prm.q = static_cast<const __nv_bfloat16 *>(q);
+    prm.out = static_cast<__nv_bfloat16 *>(out);
+    prm.block_tables = block_tables;
+    prm.context_lens = context_lens;
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    prm.num_entries = reinterpret_cast<int32_t *>(ws + wl.off_count);
+    prm.entries = reinterpret_cast<int2 *>(ws + wl.off_entries);
+    prm.part_ml = reinterpret_cast<float2 *>(ws + wl.off_ml);
+    prm.part_acc = reinterpret_cast<float *>(ws + wl.off_acc);
+    prm.B = num_seqs;
+    prm.Hq = num_q_heads;
+    prm.Hkv = num_kv_heads;
+    prm.g = g;
+    prm.MBS = max_blocks_per_seq;
+    prm.bs = pool.block_size;
+    prm.NB = pool.num_blocks;
+    prm.max_ctx = max_context_len;
+    prm.PT = PT;
+    prm.maxP = (int)std::max<long long>(1, ((long long)max_context_len + PT - 1) / PT);
+    prm.pool_rows = pool.num_blocks * pool.num_kv_heads * pool.block_size;
+    prm.scale_log2 = scale * 1.4426950408889634f;
+
+    CUtensorMap mk, mv;
+    if (!encode_pool_map(&mk, k_cache, pool) || !encode_pool_map(&mv, v_cache, pool)) return PKV_ECUDA;
+
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    pkv::plan_kernel<<<1, pkv::kPlanThreads, 0, st>>>(prm, D);
+    pkv_status r = launch_status();
+    if (r != PKV_OK) return r;
+    const int dev = current_device();
+    return D == 128 ? dispatch_group<128>(g, prm, mk, mv, st, dev) : dispatch_group<64>(g, prm, mk, mv, st, dev);
+}
+
+pkv_status pkv_get_device_error(int32_t *code_out, pkv_stream_t stream) {
+    if (!code_out) return PKV_EINVAL;
+    void *dptr = nullptr;
+    if (cudaGetSymbolAddress(&dptr, pkv::g_device_error) != cudaSuccess) return PKV_ECUDA;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    unsigned int h = 0;
+    if (cudaMemcpyAsync(&h, dptr, sizeof h, cudaMemcpyDeviceToHost, st) != cudaSuccess) return PKV_ECUDA;
+    if (cudaMemsetAsync(dptr, 0, sizeof h, st) != cudaSuccess) return PKV_ECUDA;
+    if (cudaStreamSynchronize(st) != cudaSuccess) return PKV_ECUDA;
+    *code_out = (int32_t)h;
+    return h ? PKV_EDEVICE : PKV_OK;
+}
+
+}  // extern "C"

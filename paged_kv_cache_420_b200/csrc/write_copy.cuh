@@ -1,0 +1,93 @@
+// write_copy.cuh -- the slot-mapped KV write and the copy-on-write block copy.
+// Both are pure data movement in 16-byte vectors: bit-exact by construction.
+#pragma once
+
+#include "ptx.cuh"
+
+namespace pkv {
+
+// ---------------------------------------------------------------- write ----
+// One thread per 16-byte vector of one token row of K or V.  Thread order is
+// (token, K/V, head, vector), so a warp reads 512 contiguous bytes of k or v
+// and writes whole 256-byte (head_dim 128) rows of the pool.
+//   slot -> block = slot / bs, offset = slot % bs   (position -> block, offset
+//   rule of the PagedAttention sketch, ruibaoantu.com section 1.1)
+struct WriteParams {
+    const uint4 *k;        // [T][Hkv][D/8] vectors
+    const uint4 *v;
+    const int64_t *slots;  // [T]
+    uint4 *k_cache;        // [NB][Hkv][bs][D/8]
+    uint4 *v_cache;
+    int64_t total;         // T * 2 * Hkv * vpr
+    int64_t pool_slots;    // NB * bs
+    int num_kv_heads;
+    int block_size;
+    int vpr;               // vectors per row = D / 8
+};
+
+__global__ void __launch_bounds__(256) kv_write_kernel(WriteParams p) {
+    const int per_token = 2 * p.num_kv_heads * p.vpr;
+    const int per_kv = p.num_kv_heads * p.vpr;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < p.total;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t t = i / per_token;
+        const int rem = (int)(i - t * per_token);
+        const int is_v = rem >= per_kv;
+        const int j = rem - is_v * per_kv;  // head * vpr + vector
+        const int64_t slot = __ldg(p.slots + t);
+        if (slot < 0) continue;  // padding token
+        if (slot >= p.pool_slots) {
+            if (j == 0 && !is_v) raise_error(PKV_DEVERR_SLOT);
+            continue;
+        }
+        const int64_t block = slot / p.block_size;
+        const int offset = (int)(slot - block * p.block_size);
+        const int h = j / p.vpr;
+        const int c = j - h * p.vpr;
+        const uint4 val = __ldg((is_v ? p.v : p.k) + t * per_kv + j);
+        const int64_t dst = ((block * p.num_kv_heads + h) * p.block_size + offset) * p.vpr + c;
+        (is_v ? p.v_cache : p.k_cache)[dst] = val;
+    }
+}
+
+// ----------------------------------------------------------------- copy ----
+// Pairs travel by value in the kernel parameters (validated on the host).
+// grid.y = pair, grid.x = chunk of the block; each thread moves kVecPerThread
+// vectors of K and of V, loads first, then stores.
+constexpr int kMaxPairsPerLaunch = 1024;  // 8 KB of parameters
+constexpr int kCopyThreads = 256;
+constexpr int kCopyVecPerThread = 4;
+
+struct CopyParams {
+    uint4 *k_cache;
+    uint4 *v_cache;
+    int64_t vec_per_block;  // Hkv * bs * D / 8
+    int num_pairs;
+    int2 pairs[kMaxPairsPerLaunch];
+};
+
+__global__ void __launch_bounds__(kCopyThreads) copy_blocks_kernel(const __grid_constant__ CopyParams p) {
+    const int pair = blockIdx.y;
+    const int64_t src = (int64_t)p.pairs[pair].x * p.vec_per_block;
+    const int64_t dst = (int64_t)p.pairs[pair].y * p.vec_per_block;
+    const int64_t base = (int64_t)blockIdx.x * (kCopyThreads * kCopyVecPerThread) + threadIdx.x;
+    uint4 kv[kCopyVecPerThread], vv[kCopyVecPerThread];
+#pragma unroll
+    for (int u = 0; u < kCopyVecPerThread; ++u) {
+        const int64_t e = base + u * kCopyThreads;
+        if (e < p.vec_per_block) {
+            kv[u] = p.k_cache[src + e];
+            vv[u] = p.v_cache[src + e];
+        }
+    }
+#pragma unroll
+    for (int u = 0; u < kCopyVecPerThread; ++u) {
+        const int64_t e = base + u * kCopyThreads;
+        if (e < p.vec_per_block) {
+            p.k_cache[dst + e] = kv[u];
+            p.v_cache[dst + e] = vv[u];
+        }
+    }
+}
+
+}  // namespace pkv

@@ -1,0 +1,116 @@
+"""The C ABI library: it loads, exports every declared symbol, and its host
+validation rejects bad requests before any CUDA work (no GPU needed)."""
+import ctypes
+import os
+import re
+import subprocess
+
+import numpy as np
+import pytest
+
+import paged_kv_cache_420_b200 as pkv
+from paged_kv_cache_420_b200 import _Pool
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "pkv.h")
+
+EINVAL, ERANGE, EALIAS, EUNSUP = 1, 2, 3, 6
+FAKE = ctypes.c_void_p(0x10000)  # aligned, never dereferenced by the host checks below
+FAKE_ODD = ctypes.c_void_p(0x10008)  # 8-byte but not 16-byte aligned
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"^\s*[A-Za-z_][\w \*]*?\b([a-z_][a-z0-9_]*)\s*\(", text, flags=re.M)))
+
+
+def test_library_loads_and_exports_every_declared_symbol():
+    lib = pkv.load_library()
+    names = declared_functions()
+    assert set(names) == set(pkv.EXPORTED), names
+    nm = subprocess.run(["nm", "-D", "--defined-only", pkv.LIB_PATH], capture_output=True, text=True).stdout
+    for n in names:
+        assert hasattr(lib, n)
+        assert re.search(rf"\bT {n}$", nm, flags=re.M), n
+
+
+def test_status_strings_and_version():
+    assert pkv.version() == 10000
+    for code in range(7):
+        assert pkv.status_string(code)
+    assert pkv.status_string(99) == "unknown status"
+
+
+def _pool(nb=8, hkv=2, bs=16, d=128):
+    return _Pool(nb, hkv, bs, d)
+
+
+def test_write_validation():
+    lib = pkv.load_library()
+    ok = _pool()
+    assert lib.pkv_write(FAKE, FAKE, FAKE, 0, FAKE, FAKE, ok, None) == 0  # no tokens: no-op
+    assert lib.pkv_write(FAKE, FAKE, FAKE, -1, FAKE, FAKE, ok, None) == EINVAL
+    assert lib.pkv_write(None, FAKE, FAKE, 4, FAKE, FAKE, ok, None) == EINVAL
+    assert lib.pkv_write(FAKE_ODD, FAKE, FAKE, 4, FAKE, FAKE, ok, None) == EINVAL
+    assert lib.pkv_write(FAKE, FAKE, FAKE, 4, FAKE, FAKE, _pool(d=96), None) == EUNSUP
+    assert lib.pkv_write(FAKE, FAKE, FAKE, 4, FAKE, FAKE, _pool(bs=24), None) == EUNSUP
+    assert lib.pkv_write(FAKE, FAKE, FAKE, 4, FAKE, FAKE, _pool(nb=0), None) == EINVAL
+
+
+def _pairs(p):
+    a = np.ascontiguousarray(np.asarray(p, np.int32).reshape(-1, 2))
+    return a, a.ctypes.data_as(ctypes.c_void_p)
+
+
+def test_copy_pairs_validation():
+    lib = pkv.load_library()
+    pool = _pool(nb=8)
+    for pairs, code in [([[0, 8]], ERANGE), ([[-1, 2]], ERANGE), ([[0, 1], [2, 1]], EALIAS),
+                        ([[0, 1], [1, 2]], EALIAS), ([[3, 3]], EALIAS)]:
+        arr, ptr = _pairs(pairs)
+        assert lib.pkv_copy_blocks(ptr, arr.shape[0], FAKE, FAKE, pool, None) == code, pairs
+    arr, ptr = _pairs([[0, 1]])
+    assert lib.pkv_copy_blocks(ptr, 0, FAKE, FAKE, pool, None) == 0
+    assert lib.pkv_copy_blocks(ptr, 1, FAKE_ODD, FAKE, pool, None) == EINVAL
+    assert lib.pkv_copy_blocks(None, 1, FAKE, FAKE, pool, None) == EINVAL
+
+
+def _decode(lib, **kw):
+    a = dict(q=FAKE, kc=FAKE, vc=FAKE, tables=FAKE, mbs=4, ctx=FAKE, B=2, Hq=4, scale=0.1, Hkv=2, out=FAKE,
+             pool=_pool(hkv=2), max_ctx=64, pt=0, ws=FAKE, ws_bytes=1 << 30)
+    a.update(kw)
+    return lib.paged_attn_decode(a["q"], a["kc"], a["vc"], a["tables"], a["mbs"], a["ctx"], a["B"], a["Hq"],
+                                 a["scale"], a["Hkv"], a["out"], a["pool"], a["max_ctx"], a["pt"], a["ws"],
+                                 a["ws_bytes"], None)
+
+
+def test_decode_validation():
+    lib = pkv.load_library()
+    assert _decode(lib, B=0) == 0
+    assert _decode(lib, Hq=5) == EINVAL  # not a multiple of Hkv
+    assert _decode(lib, Hkv=4, Hq=8) == EINVAL  # disagrees with the pool
+    assert _decode(lib, Hq=2 * 17, pool=_pool(hkv=2)) == EUNSUP  # g = 17
+    assert _decode(lib, pt=24) == EINVAL
+    assert _decode(lib, pt=-16) == EINVAL
+    assert _decode(lib, q=FAKE_ODD) == EINVAL
+    assert _decode(lib, ws=ctypes.c_void_p(0x10010)) == EINVAL  # workspace not 256-B aligned
+    assert _decode(lib, ws_bytes=16) == EINVAL
+    assert _decode(lib, mbs=0) == EINVAL
+    assert _decode(lib, max_ctx=-1) == EINVAL
+    assert _decode(lib, out=None) == EINVAL
+    assert _decode(lib, pool=_pool(hkv=2, d=256)) == EUNSUP
+
+
+def test_workspace_size():
+    f = pkv.decode_workspace_bytes
+    # one partition per sequence: count + entries only
+    assert f(4, 4, 4, 64, 64, 512) == 256 + 256
+    # 3 partitions: partial (m, l) and accumulators appear
+    B, Hq, D, maxP = 8, 64, 128, 3
+    expect = 256 + (B * maxP * 8 + 255) // 256 * 256 + (B * Hq * maxP * 8 + 255) // 256 * 256 \
+        + (B * Hq * maxP * D * 4 + 255) // 256 * 256
+    assert f(B, Hq, 8, D, 1536, 512) == expect
+    assert f(B, Hq, 8, D, 1537, 512) > expect
+    with pytest.raises(ValueError):
+        f(2, 5, 2, 128, 64, 0)
