@@ -181,7 +181,10 @@ class ClockSampler:
 
 def make_workload(args, rank: int, device):
     bs = args.block_size
-    return workloads.make(args.workload, seed=args.seed + rank, values_device=device, block_size=bs)
+    w = workloads.make(args.workload, seed=args.seed + rank, values_device=device, block_size=bs)
+    if args.max_seqs and args.max_seqs < w.num_seqs:
+        w = workloads.subset(w, args.max_seqs)
+    return w
 
 
 def partition_tokens(args, w) -> int:
@@ -443,6 +446,7 @@ def main(argv=None):
     ap.add_argument("--block-size", type=int, default=None)
     ap.add_argument("--partition-tokens", type=int, default=-1, help="-1: the workload's choice, 0: library's")
     ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--max-seqs", type=int, default=0, help="time only the first N sequences (profiling)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work for cpu_baseline")

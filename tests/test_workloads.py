@@ -99,3 +99,17 @@ def test_poison_marks_only_unused_rows():
             b = w.block_tables[s][pos // 16]
             assert not kc[b, :, pos % 16].isnan().any()
     assert kc.isnan().any()
+
+
+def test_subset_renumbers_consistently():
+    import oracle
+    w = workloads.make("llama3-8b-gqa-prefix", seed=0, values_device="meta")
+    # structure only on meta; values on a small custom case below
+    sub = workloads.subset(workloads.make_custom([50, 70, 33], 4, 2, 64, 16, seed=3, share_prefix_tokens=32,
+                                                 group_size=3), 2)
+    full = workloads.make_custom([50, 70, 33], 4, 2, 64, 16, seed=3, share_prefix_tokens=32, group_size=3)
+    a = oracle.decode_step(sub)[2]
+    b = oracle.decode_step(full)[2][:2]
+    assert np.array_equal(a, b)
+    assert sub.num_blocks == len(np.unique(sub.block_tables[sub.block_tables >= 0]))
+    assert w.num_seqs == 256

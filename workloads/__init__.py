@@ -367,3 +367,27 @@ def make(name: str, seed: int = 0, values_device="cpu", poison: bool = False,
     if name not in _BUILDERS:
         raise KeyError(f"unknown workload {name!r}; choose from {WORKLOADS}")
     return _BUILDERS[name](seed, values_device, poison, block_size)
+
+
+def subset(w: Workload, num_seqs: int) -> Workload:
+    """The first ``num_seqs`` sequences of a workload, on a pool compacted to
+    the blocks they reference (and their copy-on-write sources), with tables,
+    slots and pairs renumbered.  For smaller profiling and test cases."""
+    n = min(int(num_seqs), w.num_seqs)
+    tables = w.block_tables[:n]
+    refd = set(int(b) for b in tables[tables >= 0].ravel())
+    pairs = [(int(s), int(d)) for s, d in w.copy_pairs if int(d) in refd]
+    used = sorted(refd | {s for s, _ in pairs})
+    new_id = {b: i for i, b in enumerate(used)}
+    remap = np.vectorize(lambda b: new_id[int(b)] if b >= 0 else -1, otypes=[np.int32])
+    new_tables = remap(tables) if tables.size else tables.copy()
+    bs = w.block_size
+    slots = np.array([new_id[int(s) // bs] * bs + int(s) % bs for s in w.slot_mapping[:n]], dtype=np.int64)
+    sel = torch.tensor(used, dtype=torch.long, device=w.k_cache.device)
+    return dataclasses.replace(
+        w, num_seqs=n, num_blocks=len(used), context_lens=w.context_lens[:n].copy(),
+        block_tables=new_tables.astype(np.int32), slot_mapping=slots,
+        copy_pairs=np.array([(new_id[s], new_id[d]) for s, d in pairs], dtype=np.int32).reshape(-1, 2),
+        q=w.q[:n].contiguous(), k_new=w.k_new[:n].contiguous(), v_new=w.v_new[:n].contiguous(),
+        k_cache=w.k_cache.index_select(0, sel).contiguous(), v_cache=w.v_cache.index_select(0, sel).contiguous(),
+        description=w.description + f" (first {n} sequences)")
