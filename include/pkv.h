@@ -25,7 +25,8 @@
  * Conventions shared by every call:
  *   - Pointers are device pointers owned by the caller unless stated "host".
  *     The library allocates no device memory; it keeps one 4-byte device error
- *     word per GPU (a module global).
+ *     word per GPU and the scratch array of paged_attn_decode_static_ws (both
+ *     module globals).
  *   - All work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
  *     stream) and returns before it finishes.
  *   - Host validation covers shapes, null pointers and 16-byte alignment only;
@@ -153,6 +154,41 @@ pkv_status paged_attn_decode(const void *q, const void *k_cache, const void *v_c
                              float scale, int32_t num_kv_heads, void *out, pkv_pool pool,
                              int32_t max_context_len, int32_t partition_tokens, void *workspace,
                              size_t workspace_bytes, pkv_stream_t stream);
+
+/*
+ * paged_attn_decode_static_ws -- paged_attn_decode for callers that cannot
+ * allocate device memory.  The pages have no counterpart of this call; it is
+ * a convenience of this library.
+ *
+ * Some callers have no way to obtain scratch memory: a plugin running inside
+ * a host engine that has reserved all device memory for its own pools and
+ * offers plugins no allocation hook, or a latency-critical path where a
+ * cudaMalloc (which can synchronise the device) is not acceptable.  This
+ * entry point takes the same arguments as paged_attn_decode except the
+ * workspace: its scratch is a file-scope device array of
+ * PKV_STATIC_WS_BYTES bytes inside libpkv.so.  Every GPU that loads the
+ * library holds that array until the process exits.  The call allocates
+ * nothing.
+ *
+ *   - A request whose pkv_decode_workspace_bytes(...) exceeds
+ *     PKV_STATIC_WS_BYTES returns PKV_EUNSUPPORTED and enqueues nothing;
+ *     invalid sizes return PKV_EINVAL as in paged_attn_decode.
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first call
+ *     before any stream capture.
+ *   - All calls on a device share the one array, and it keeps the previous
+ *     call's contents.  Nothing in it needs to start at zero (every call
+ *     rewrites what it reads).  Calls whose kernels overlap on the GPU (for
+ *     example on two streams) race on the array; order them on one stream.
+ */
+#define PKV_STATIC_WS_BYTES ((size_t)32 << 20)
+
+pkv_status paged_attn_decode_static_ws(const void *q, const void *k_cache, const void *v_cache,
+                                       const int32_t *block_tables, int32_t max_blocks_per_seq,
+                                       const int32_t *context_lens, int32_t num_seqs, int32_t num_q_heads,
+                                       float scale, int32_t num_kv_heads, void *out, pkv_pool pool,
+                                       int32_t max_context_len, int32_t partition_tokens,
+                                       pkv_stream_t stream);
 
 /*
  * pkv_get_device_error -- copies the current device's error word to

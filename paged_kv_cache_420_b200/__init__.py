@@ -24,7 +24,8 @@ DEVERR_SLOT, DEVERR_BLOCK, DEVERR_CONTEXT, DEVERR_TIMEOUT = 0x1, 0x2, 0x4, 0x8
 
 # Every symbol include/pkv.h declares.
 EXPORTED = ("pkv_write", "pkv_copy_blocks", "pkv_decode_workspace_bytes", "paged_attn_decode",
-            "pkv_get_device_error", "pkv_status_string", "pkv_version")
+            "paged_attn_decode_static_ws", "pkv_get_device_error", "pkv_status_string", "pkv_version")
+STATIC_WS_BYTES = 32 << 20  # PKV_STATIC_WS_BYTES
 
 
 class PkvError(RuntimeError):
@@ -170,3 +171,35 @@ def get_device_error(stream=None) -> int:
     if st not in (PKV_OK, 5):
         raise PkvError(st, "pkv_get_device_error")
     return int(code.value)
+
+
+def paged_attn_decode_static_ws(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+                                block_tables: torch.Tensor, context_lens: torch.Tensor, scale: float,
+                                num_kv_heads: int, out: torch.Tensor, max_context_len: int,
+                                partition_tokens: int = 0, stream=None) -> None:
+    """paged_attn_decode without a workspace argument, for callers that cannot
+    allocate device memory (for example a plugin whose host engine owns all
+    device memory).  Its scratch is a fixed device array of STATIC_WS_BYTES
+    inside libpkv.so, shared by every call on the device: calls that overlap
+    on the GPU race.  Requests that need more scratch raise PkvError
+    (PKV_EUNSUPPORTED); the first call on a device should come before any
+    stream capture."""
+    for t, n in ((q, "q"), (k_cache, "k_cache"), (v_cache, "v_cache"), (out, "out")):
+        _need(t, n, torch.bfloat16)
+    _need(block_tables, "block_tables", torch.int32)
+    _need(context_lens, "context_lens", torch.int32)
+    B, Hq, D = q.shape
+    if out.shape != q.shape or v_cache.shape != k_cache.shape:
+        raise ValueError("out must match q, v_cache must match k_cache")
+    if block_tables.dim() != 2 or block_tables.shape[0] != B or context_lens.shape != (B,):
+        raise ValueError("block_tables must be [B, max_blocks_per_seq], context_lens [B]")
+    lib = load_library()
+    f = lib.paged_attn_decode_static_ws
+    if f.argtypes is None:
+        P, I32, F = ctypes.c_void_p, ctypes.c_int32, ctypes.c_float
+        f.argtypes = [P, P, P, P, I32, P, I32, I32, F, I32, P, _Pool, I32, I32, P]
+        f.restype = ctypes.c_int
+    st = f(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables), block_tables.shape[1], _ptr(context_lens),
+           B, Hq, float(scale), int(num_kv_heads), _ptr(out), _pool(k_cache), int(max_context_len),
+           int(partition_tokens), _stream(stream))
+    _check(st, "paged_attn_decode_static_ws")

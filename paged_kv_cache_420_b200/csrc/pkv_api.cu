@@ -336,3 +336,41 @@ pkv_status pkv_get_device_error(int32_t *code_out, pkv_stream_t stream) {
 }
 
 }  // extern "C"
+
+// ------------------------------------------------- no-allocation variant ----
+// Scratch for paged_attn_decode_static_ws: a file-scope device array, so the
+// call needs no allocator.  Host code must not use the name as an address;
+// the device address is looked up once per device with cudaGetSymbolAddress.
+static __device__ __align__(256) unsigned char g_static_workspace[PKV_STATIC_WS_BYTES];
+
+namespace {
+std::mutex g_static_ws_mutex;
+void *g_static_ws_ptr[kMaxDevices] = {nullptr};
+}  // namespace
+
+extern "C" pkv_status paged_attn_decode_static_ws(const void *q, const void *k_cache, const void *v_cache,
+                                                  const int32_t *block_tables, int32_t max_blocks_per_seq,
+                                                  const int32_t *context_lens, int32_t num_seqs,
+                                                  int32_t num_q_heads, float scale, int32_t num_kv_heads,
+                                                  void *out, pkv_pool pool, int32_t max_context_len,
+                                                  int32_t partition_tokens, pkv_stream_t stream) {
+    const size_t need = pkv_decode_workspace_bytes(num_seqs, num_q_heads, num_kv_heads, pool.head_dim,
+                                                   max_context_len, partition_tokens);
+    if (need == 0) return PKV_EINVAL;
+    if (need > PKV_STATIC_WS_BYTES) return PKV_EUNSUPPORTED;
+    const int dev = current_device();
+    if (dev < 0 || dev >= kMaxDevices) return PKV_ECUDA;
+    void *ws = nullptr;
+    {
+        std::lock_guard<std::mutex> lock(g_static_ws_mutex);
+        if (g_static_ws_ptr[dev] == nullptr) {
+            void *p = nullptr;
+            if (cudaGetSymbolAddress(&p, g_static_workspace) != cudaSuccess || p == nullptr) return PKV_ECUDA;
+            g_static_ws_ptr[dev] = p;
+        }
+        ws = g_static_ws_ptr[dev];
+    }
+    return paged_attn_decode(q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens, num_seqs,
+                             num_q_heads, scale, num_kv_heads, out, pool, max_context_len, partition_tokens, ws,
+                             PKV_STATIC_WS_BYTES, stream);
+}
