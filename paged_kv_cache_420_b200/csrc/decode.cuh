@@ -9,7 +9,7 @@
 // Work decomposition.  A unit (sequence s, kv head h) is cut into partitions
 // of PT tokens; an item = (s, h, partition).  A one-CTA planner kernel writes
 // the (s, partition) list in sequence-major order.  The attention kernel is
-// persistent: CTA c takes items c, c + gridDim.x, ...  Inside a CTA one
+// persistent: CTAs claim items from a global counter in list order.  Inside a CTA one
 // producer warp walks the items' 16-token stages and fills a ring of NS
 // shared-memory slots with TMA tensor loads (K and V tiles of 16 rows x D,
 // 128-byte swizzle) addressed through the block table; W consumer warps take
@@ -32,8 +32,13 @@
 
 namespace pkv {
 
-constexpr int kStageTok = 16;       // tokens per pipeline stage (one TMA box height)
-constexpr int kConsumerWarps = 4;   // W
+#ifndef PKV_CONSUMER_WARPS
+#define PKV_CONSUMER_WARPS 4
+#endif
+
+constexpr int kStageTok = 16;                     // tokens per pipeline stage (one TMA box height)
+constexpr int kConsumerWarps = PKV_CONSUMER_WARPS;  // W
+static_assert(32 % kConsumerWarps == 0, "stage groups must tile the 32-entry table prefetch");
 constexpr int kDecodeThreads = (kConsumerWarps + 1) * 32;
 constexpr int kPlanThreads = 1024;
 constexpr int kReduceWarps = 4;
@@ -47,6 +52,7 @@ struct DecodeParams {
     const int32_t *context_lens;  // [B]
     int2 *entries;                // workspace: (seq, partition), sequence-major
     int32_t *num_entries;         // workspace: number of entries
+    int32_t *work_counter;        // workspace: next unclaimed item (zeroed by the planner)
     float2 *part_ml;              // workspace: [B][Hq][maxP] = (m in log2 units, l)
     float *part_acc;              // workspace: [B][Hq][maxP][D]
     int B, Hq, Hkv, g, MBS, bs, NB, max_ctx, PT, maxP;
@@ -69,8 +75,9 @@ __device__ __forceinline__ int clamped_context(const DecodeParams &p, int s, boo
 
 // ------------------------------------------------------------- planner ----
 // Writes entries[] = (s, partition) for every sequence and partition, in
-// sequence-major order, and the count.  Zero-length sequences get a zero
-// output row here (they have no items).
+// sequence-major order, and the count, and zeroes the attention kernel's work
+// counter.  Zero-length sequences get a zero output row here (they have no
+// items).
 __global__ void __launch_bounds__(kPlanThreads) plan_kernel(DecodeParams p, int D) {
     __shared__ int s_off[kPlanThreads + 1];
     __shared__ int s_warp[kPlanThreads / 32];
@@ -128,7 +135,10 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(DecodeParams p, int 
         if (tid == 0) s_carry = carry + chunk_total;
         __syncthreads();
     }
-    if (tid == 0) *p.num_entries = s_carry;
+    if (tid == 0) {
+        *p.num_entries = s_carry;
+        *p.work_counter = 0;
+    }
     if (s_any_zero) {
         const int vec_per_seq = p.Hq * D / 8;
         uint4 *out = reinterpret_cast<uint4 *>(p.out);
@@ -154,7 +164,7 @@ struct DecodeSmem {
     static constexpr int kHalfTile = kStageTok * 64 * 2;  // 16 rows x 64 elements = 2 KB
     static constexpr int kTile = kStageTok * D * 2;       // one K (or V) stage tile
     static constexpr int kStage = 2 * kTile;
-    static constexpr int kQBuf = 16 * D * 2;              // room for 16 query heads
+    static constexpr int kQBuf = GP * D * 2;              // the query heads of one kv head
     static constexpr int kMergeStride = D + 4;            // floats, padded against bank conflicts
     static constexpr int oTiles = 0;
     static constexpr int oQ = oTiles + NS * kStage;
@@ -396,11 +406,12 @@ struct MmaState {
 
     __device__ __forceinline__ void stage(uint32_t ktile, uint32_t vtile, int valid, int lane, float scale_log2) {
         // S^T[token][head] = K . Q^T
-        float s[NT][4];
+        // two independent accumulator chains (even / odd k-steps), summed after
+        float s[NT][4], s2[NT][4];
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-            for (int c = 0; c < 4; ++c) s[nt][c] = 0.f;
+            for (int c = 0; c < 4; ++c) { s[nt][c] = 0.f; s2[nt][c] = 0.f; }
         const int mi = lane >> 3, ri = lane & 7;
 #pragma unroll
         for (int kk = 0; kk < KS; ++kk) {
@@ -410,10 +421,15 @@ struct MmaState {
             uint32_t a0, a1, a2, a3;
             ldmatrix_x4(tile_addr(ktile, row, col), a0, a1, a2, a3);
 #pragma unroll
-            for (int nt = 0; nt < NT; ++nt)
-                mma_bf16_16816(s[nt][0], s[nt][1], s[nt][2], s[nt][3], a0, a1, a2, a3, qb[nt][kk][0],
-                               qb[nt][kk][1]);
+            for (int nt = 0; nt < NT; ++nt) {
+                float *acc = (kk & 1) ? s2[nt] : s[nt];
+                mma_bf16_16816(acc[0], acc[1], acc[2], acc[3], a0, a1, a2, a3, qb[nt][kk][0], qb[nt][kk][1]);
+            }
         }
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int c = 0; c < 4; ++c) s[nt][c] += s2[nt][c];
         const int t0 = lane >> 2;  // tokens t0 and t0 + 8
         const bool ok0 = t0 < valid, ok1 = t0 + 8 < valid;
         uint32_t pb[NT][2];
@@ -536,11 +552,18 @@ __global__ void __launch_bounds__(kDecodeThreads) paged_decode_kernel(const __gr
 
     if (warp == W) {
         // ------------------------------------------------------ producer --
+        // Items are claimed from a global counter (dynamic load balance); the
+        // claim of the next item is issued one item ahead so that its latency
+        // overlaps the current item's stage issue.
         const int n_items = *reinterpret_cast<volatile int32_t *>(p.num_entries) * p.Hkv;
         uint32_t gc = 0;
         int ord = 0;
         bool ok = true;
-        for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x, ++ord) {
+        int claimed = 0;
+        if (lane == 0) claimed = atomicAdd(p.work_counter, 1);
+        int it = __shfl_sync(0xffffffffu, claimed, 0);
+        for (; it < n_items && ok; ++ord) {
+            if (lane == 0) claimed = atomicAdd(p.work_counter, 1);
             const int e = it / p.Hkv;
             const int h = it - e * p.Hkv;
             const int2 sp = p.entries[e];
@@ -562,11 +585,14 @@ __global__ void __launch_bounds__(kDecodeThreads) paged_decode_kernel(const __gr
                 }
             }
             ok = __shfl_sync(0xffffffffu, ok, 0);
+            // Stages go out in groups of W, one per consumer warp: lane j < W
+            // issues stage k0 + j into slot (gc + j) % NS, so one pass of the
+            // warp issues W stages (waits, descriptors and TMA in lockstep).
             int blk_reg = -1;
-            for (int k = 0; k < npad && ok; ++k) {
-                if ((k & 31) == 0) {
-                    // lane l fetches the block id of stage k + l
-                    const int kk = k + lane;
+            for (int k0 = 0; k0 < npad && ok; k0 += W) {
+                if ((k0 & 31) == 0) {
+                    // lane l fetches the block id of stage k0 + l
+                    const int kk = k0 + lane;
                     int blk = -1;
                     if (kk < nst) {
                         const int tok = t0 + kk * kStageTok;
@@ -578,11 +604,14 @@ __global__ void __launch_bounds__(kDecodeThreads) paged_decode_kernel(const __gr
                     }
                     blk_reg = blk;
                 }
+                const int k = k0 + lane;
                 const int blk = __shfl_sync(0xffffffffu, blk_reg, k & 31);
-                if (lane == 0) {
-                    const uint32_t slot = gc % NS;
-                    ok = wait_or_abort(&empty[slot], ((gc / NS) & 1) ^ 1, abort_flag);
-                    if (ok) {
+                bool lane_ok = true;
+                if (lane < W) {
+                    const uint32_t g = gc + lane;
+                    const uint32_t slot = g % NS;
+                    lane_ok = wait_or_abort(&empty[slot], ((g / NS) & 1) ^ 1, abort_flag);
+                    if (lane_ok) {
                         const int tok = t0 + k * kStageTok;
                         const int valid = k < nst ? min(kStageTok, t1 - tok) : 0;
                         StageInfo si;
@@ -604,9 +633,10 @@ __global__ void __launch_bounds__(kDecodeThreads) paged_decode_kernel(const __gr
                         }
                     }
                 }
-                ok = __shfl_sync(0xffffffffu, ok, 0);
-                ++gc;
+                ok = __all_sync(0xffffffffu, lane_ok);
+                gc += W;
             }
+            it = __shfl_sync(0xffffffffu, claimed, 0);
         }
         // end-of-stream marker for every consumer warp
         if (lane == 0) {
@@ -667,23 +697,37 @@ __global__ void __launch_bounds__(kDecodeThreads) paged_decode_kernel(const __gr
                 __syncwarp();
                 if (lane == 0) mbar_arrive(mfull);
                 if (!wait_or_abort(mfull, mc & 1, abort_flag)) break;
+                // Combine: thread ct owns a contiguous run of the g*D outputs, so
+                // the per-head factors 2^(m_u - M) are computed once per run.
                 const int g = p.g;
                 const size_t unit_head0 = (size_t)si.s * p.Hq + (size_t)si.h * g;
-                for (int idx = w * 32 + lane; idx < g * D; idx += W * 32) {
-                    const int j = idx / D, d = idx - j * D;
-                    float M = PKV_NEG_INF;
+                const int total = g * D;
+                const int ept = (total + W * 32 - 1) / (W * 32);
+                const int e0 = (w * 32 + lane) * ept;
+                const int e1 = min(total, e0 + ept);
+                int jcur = -1;
+                float f[W], M = 0.f, Lsum = 0.f, invL = 0.f;
+                for (int e = e0; e < e1; ++e) {
+                    const int j = e / D, d = e - j * D;
+                    if (j != jcur) {
+                        jcur = j;
+                        M = PKV_NEG_INF;
 #pragma unroll
-                    for (int u = 0; u < W; ++u) M = fmaxf(M, mM[u * GP + j]);
-                    float Lsum = 0.f, O = 0.f;
+                        for (int u = 0; u < W; ++u) M = fmaxf(M, mM[u * GP + j]);
+                        Lsum = 0.f;
 #pragma unroll
-                    for (int u = 0; u < W; ++u) {
-                        const float mu = mM[u * GP + j];
-                        const float f = mu == PKV_NEG_INF ? 0.f : exp2f(mu - M);
-                        Lsum = fmaf(mL[u * GP + j], f, Lsum);
-                        O = fmaf(mO[(u * GP + j) * L::kMergeStride + d], f, O);
+                        for (int u = 0; u < W; ++u) {
+                            const float mu = mM[u * GP + j];
+                            f[u] = mu == PKV_NEG_INF ? 0.f : exp2f(mu - M);
+                            Lsum = fmaf(mL[u * GP + j], f[u], Lsum);
+                        }
+                        invL = Lsum > 0.f ? 1.f / Lsum : 0.f;
                     }
+                    float O = 0.f;
+#pragma unroll
+                    for (int u = 0; u < W; ++u) O = fmaf(mO[(u * GP + j) * L::kMergeStride + d], f[u], O);
                     if (si.nparts == 1) {
-                        p.out[(unit_head0 + j) * D + d] = __float2bfloat16_rn(Lsum > 0.f ? O / Lsum : 0.f);
+                        p.out[(unit_head0 + j) * D + d] = __float2bfloat16_rn(O * invL);
                     } else {
                         const size_t pi = (unit_head0 + j) * p.maxP + si.part;
                         p.part_acc[pi * D + d] = O;

@@ -19,7 +19,17 @@
 namespace {
 
 constexpr int kMaxDevices = 64;
-constexpr int kDecodeStages = 8;  // NS: shared-memory ring slots per CTA
+#ifndef PKV_STAGES_SIMT
+#define PKV_STAGES_SIMT 8
+#endif
+#ifndef PKV_STAGES_MMA
+#define PKV_STAGES_MMA 8
+#endif
+// NS: shared-memory ring slots per CTA (a multiple of the consumer warps)
+constexpr int kStagesSimt = PKV_STAGES_SIMT;
+constexpr int kStagesMma = PKV_STAGES_MMA;
+static_assert(kStagesSimt % pkv::kConsumerWarps == 0 && kStagesMma % pkv::kConsumerWarps == 0,
+              "ring slots must be a multiple of the consumer warps");
 
 bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 
@@ -120,8 +130,9 @@ bool workspace_layout(int32_t B, int32_t Hq, int32_t D, int32_t max_ctx, int32_t
 template <int D, int PATH, int GS, int NT>
 pkv_status launch_decode(const pkv::DecodeParams &prm, const CUtensorMap &mk, const CUtensorMap &mv,
                          cudaStream_t stream, int dev) {
-    using L = pkv::DecodeSmem<D, (PATH == 0 ? GS : 8 * NT), kDecodeStages>;
-    auto kernel = pkv::paged_decode_kernel<D, PATH, GS, NT, kDecodeStages>;
+    constexpr int NS = PATH == 0 ? kStagesSimt : kStagesMma;
+    using L = pkv::DecodeSmem<D, (PATH == 0 ? GS : 8 * NT), NS>;
+    auto kernel = pkv::paged_decode_kernel<D, PATH, GS, NT, NS>;
     static int occ_cache[kMaxDevices] = {0};
     int occ = (dev >= 0 && dev < kMaxDevices) ? occ_cache[dev] : 0;
     if (occ == 0) {
@@ -295,6 +306,7 @@ pkv_status paged_attn_decode(const void *q, const void *k_cache, const void *v_c
     prm.context_lens = context_lens;
     uint8_t *ws = static_cast<uint8_t *>(workspace);
     prm.num_entries = reinterpret_cast<int32_t *>(ws + wl.off_count);
+    prm.work_counter = reinterpret_cast<int32_t *>(ws + wl.off_count) + 1;
     prm.entries = reinterpret_cast<int2 *>(ws + wl.off_entries);
     prm.part_ml = reinterpret_cast<float2 *>(ws + wl.off_ml);
     prm.part_acc = reinterpret_cast<float *>(ws + wl.off_acc);
