@@ -179,6 +179,23 @@ class ClockSampler:
 # the timed arms
 # --------------------------------------------------------------------------
 
+def combine_ranks(dist, ms_total: float, bytes_step: int, seqs: int, device):
+    """Slowest rank's time, and all ranks' bytes and sequences per step."""
+    if dist is None:
+        return float(ms_total), float(bytes_step), float(seqs)
+    stats = torch.tensor([ms_total, float(bytes_step), float(seqs)], dtype=torch.float64, device=device)
+    mx = stats.clone()
+    dist.all_reduce(mx, op=dist.ReduceOp.MAX)
+    sm = stats.clone()
+    dist.all_reduce(sm, op=dist.ReduceOp.SUM)
+    return float(mx[0]), float(sm[1]), float(sm[2])
+
+
+def whole_job_gbs(bytes_all_ranks: float, steps: int, ms_max: float) -> float:
+    """GB/s of the whole job: every rank's bytes over the slowest rank's time."""
+    return bytes_all_ranks * steps / (ms_max / 1e3) / 1e9
+
+
 def make_workload(args, rank: int, device):
     bs = args.block_size
     w = workloads.make(args.workload, seed=args.seed + rank, values_device=device, block_size=bs)
@@ -191,8 +208,13 @@ def partition_tokens(args, w) -> int:
     return w.partition_tokens if args.partition_tokens < 0 else args.partition_tokens
 
 
+def library_partition_tokens(pt: int, max_context_len: int) -> int:
+    """The partition size the library uses for `pt` (0 = its own choice)."""
+    return pt if pt > 0 else (2048 if max_context_len > 16384 else 512)
+
+
 def launches_per_step(w, pt: int) -> int:
-    maxp = max(1, math.ceil(w.max_context_len / (pt if pt > 0 else 512)))
+    maxp = max(1, math.ceil(w.max_context_len / library_partition_tokens(pt, w.max_context_len)))
     n = 1 + 1 + 1 + (1 if maxp > 1 else 0)  # write, plan, attention, reduce
     if len(w.copy_pairs):
         n += math.ceil(len(w.copy_pairs) / 1024)
@@ -256,55 +278,74 @@ def run_cuda(args, rank, world, dist):
 
     bytes_step = step_bytes(w)
     dec_bytes = decode_bytes(w)
-    stats = torch.tensor([ms_total, float(bytes_step), float(w.num_seqs)], dtype=torch.float64, device=dev)
-    if dist is not None:
-        mx = stats.clone()
-        dist.all_reduce(mx, op=dist.ReduceOp.MAX)
-        sm = stats.clone()
-        dist.all_reduce(sm, op=dist.ReduceOp.SUM)
-        ms_max, bytes_all, seqs_all = float(mx[0]), float(sm[1]), float(sm[2])
-    else:
-        ms_max, bytes_all, seqs_all = ms_total, float(bytes_step), float(w.num_seqs)
+    ms_max, bytes_all, seqs_all = combine_ranks(dist, ms_total, bytes_step, w.num_seqs, dev)
     sec = ms_max / 1e3
-    value = bytes_all * args.steps / sec / 1e9
+    value = whole_job_gbs(bytes_all, args.steps, ms_max)
 
     # ---- end to end: per-step inputs from pinned host memory, output back
     e2e = None
     if not args.no_e2e:
+        # Per step: the step's inputs are copied from pinned host memory and the
+        # output back, inside the timed region.  Copies run on a second stream,
+        # double-buffered, so step i+1's inputs and step i-1's output move
+        # while step i computes (the kernels themselves stay in stream order).
         host = {k: v.cpu().pin_memory() for k, v in dict(q=w.q, k_new=w.k_new, v_new=w.v_new, slots=slots,
                                                            tables=tables, ctx=ctx).items()}
-        dbuf = {k: torch.empty_like(v, device=dev) for k, v in host.items()}
-        out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+        dbuf = [{k: torch.empty_like(v, device=dev) for k, v in host.items()} for _ in range(2)]
+        dout = [torch.empty_like(out) for _ in range(2)]
+        out_h = [torch.empty(out.shape, dtype=out.dtype).pin_memory() for _ in range(2)]
         h2d = sum(v.numel() * v.element_size() for v in host.values())
-        d2h = out_h.numel() * out_h.element_size()
-        k_e2e = max(3, min(args.steps, 500))
+        d2h = out_h[0].numel() * out_h[0].element_size()
+        k_e2e = max(3, min(args.steps, 1000))
+        copy = torch.cuda.Stream(device=dev)
+        ev_in = [torch.cuda.Event() for _ in range(2)]
+        ev_done = [torch.cuda.Event() for _ in range(2)]
 
-        def e2e_step():
-            for k in host:
-                dbuf[k].copy_(host[k], non_blocking=True)
-            if len(w.copy_pairs):
-                pkv.pkv_copy_blocks(w.copy_pairs, kc, vc, stream=stream)
-            pkv.pkv_write(dbuf["k_new"], dbuf["v_new"], dbuf["slots"], kc, vc, stream=stream)
-            pkv.paged_attn_decode(dbuf["q"], kc, vc, dbuf["tables"], dbuf["ctx"], w.scale, w.num_kv_heads, out,
-                                  w.max_context_len, pt, workspace=ws, stream=stream)
-            out_h.copy_(out, non_blocking=True)
+        def h2d(i):
+            b = i % 2
+            if i >= 2:  # buffer b was read by step i-2
+                copy.wait_event(ev_done[b])
+            with torch.cuda.stream(copy):
+                for k in host:
+                    dbuf[b][k].copy_(host[k], non_blocking=True)
+                ev_in[b].record(copy)
 
-        for _ in range(3):
-            e2e_step()
+        def e2e_run(n):
+            h2d(0)
+            for i in range(n):
+                b = i % 2
+                if i + 1 < n:
+                    h2d(i + 1)  # the next step's inputs move while this step computes
+                stream.wait_event(ev_in[b])
+                if len(w.copy_pairs):
+                    pkv.pkv_copy_blocks(w.copy_pairs, kc, vc, stream=stream)
+                pkv.pkv_write(dbuf[b]["k_new"], dbuf[b]["v_new"], dbuf[b]["slots"], kc, vc, stream=stream)
+                pkv.paged_attn_decode(dbuf[b]["q"], kc, vc, dbuf[b]["tables"], dbuf[b]["ctx"], w.scale,
+                                      w.num_kv_heads, dout[b], w.max_context_len, pt, workspace=ws, stream=stream)
+                ev_done[b].record(stream)
+                copy.wait_event(ev_done[b])
+                with torch.cuda.stream(copy):
+                    out_h[b].copy_(dout[b], non_blocking=True)
+
+        e2e_run(4)
         torch.cuda.synchronize()
         if dist is not None:
             dist.barrier()
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record(stream)
-        for _ in range(k_e2e):
-            e2e_step()
-        b.record(stream)
+        a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(copy)
+        stream.wait_stream(copy)
+        e2e_run(k_e2e)
+        copy.wait_stream(stream)
+        b_.record(copy)
         torch.cuda.synchronize()
-        e_ms = torch.tensor([a.elapsed_time(b)], dtype=torch.float64, device=dev)
+        if not torch.equal(out_h[(k_e2e - 1) % 2].to(dev), out):
+            raise RuntimeError("end-to-end output differs from the device-resident run")
+        e_ms = torch.tensor([a.elapsed_time(b_)], dtype=torch.float64, device=dev)
         if dist is not None:
             dist.all_reduce(e_ms, op=dist.ReduceOp.MAX)
         e2e = {"value": round(bytes_all * k_e2e / (float(e_ms[0]) / 1e3) / 1e9, 2), "unit": "GB/s",
-               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "steps": k_e2e}
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "steps": k_e2e,
+               "overlap": "copies on a second stream, double-buffered"}
 
     peak, peak_kind = measured_hbm_peak()
     achieved = dec_bytes / (decode_ms / 1e3) / 1e9
@@ -325,7 +366,7 @@ def run_cuda(args, rank, world, dist):
             "workload": f"{w.name}: {w.description}",
             "num_seqs": w.num_seqs, "num_q_heads": w.num_q_heads, "num_kv_heads": w.num_kv_heads,
             "head_dim": w.head_dim, "block_size": w.block_size, "kv_tokens": int(w.context_lens.sum()),
-            "partition_tokens": pt if pt > 0 else 512, "copy_pairs": int(len(w.copy_pairs)),
+            "partition_tokens": library_partition_tokens(pt, w.max_context_len), "copy_pairs": int(len(w.copy_pairs)),
             "seed": args.seed, "bytes_per_step": int(bytes_step),
             "l2": "no flush: every step reads >1 GB of K/V (L2 is 126 MB)",
             "parallelism": f"replicas x{world}, one independent batch per GPU",
@@ -361,8 +402,9 @@ def cpu_baseline(w, budget_s: float, label="oracle", pools=None):
     kc, vc = pools
     done, elapsed, nbytes = 0, 0.0, 0
     chunk = 1
-    while done < w.num_seqs and elapsed < budget_s:
-        idx = np.arange(done, min(w.num_seqs, done + chunk))
+    while elapsed < budget_s:
+        start = done % w.num_seqs
+        idx = np.arange(start, min(w.num_seqs, start + chunk))
         sub = _subset(w, idx)
         t = time.perf_counter()
         oracle.paged_attention(sub.q, kc, vc, sub.block_tables, sub.context_lens, sub.scale)
@@ -370,10 +412,11 @@ def cpu_baseline(w, budget_s: float, label="oracle", pools=None):
         nbytes += decode_bytes(sub)
         done += len(idx)
         chunk = min(2 * chunk, 64)
+    passes = done / w.num_seqs
     return {"value": round(nbytes / elapsed / 1e9, 4), "unit": "GB/s", "cores": oracle.num_threads(),
             "kind": label,
-            "sample": f"paged attention of the first {done} of {w.num_seqs} sequences (all heads), "
-                      f"{elapsed:.1f} s of fp64 C/OpenMP work",
+            "sample": f"paged attention of {done} sequences ({passes:.2f} passes over the {w.num_seqs}-sequence "
+                      f"batch, all heads), {elapsed:.1f} s of fp64 C/OpenMP work",
             "tokens_layers_per_s": round(done / elapsed, 2)}
 
 
@@ -439,7 +482,7 @@ def run_reference(args, rank, world):
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--steps", type=int, default=5000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["pkv", "reference"], default="pkv")
     ap.add_argument("--workload", default="llama2-13b", choices=list(workloads.WORKLOADS))

@@ -65,6 +65,7 @@ typedef enum pkv_status {
 #define PKV_DEVERR_BLOCK 0x2u    /* decode: block table entry outside [0, num_blocks) (tile reads zeros) */
 #define PKV_DEVERR_CONTEXT 0x4u  /* decode: context_lens[s] < 0 or above the table / max_context_len (clamped) */
 #define PKV_DEVERR_TIMEOUT 0x8u  /* a bounded on-chip wait gave up (the call's results are invalid) */
+#define PKV_DEVERR_LAYOUT 0x10u  /* decode: shared memory window not 1 KB-aligned (results invalid) */
 
 /* Describes one physical pool (k_cache and v_cache share it). */
 typedef struct pkv_pool {
@@ -141,7 +142,8 @@ size_t pkv_decode_workspace_bytes(int32_t num_seqs, int32_t num_q_heads, int32_t
  *                 ceil(context_len / block_size) are never read
  *   context_lens  int32 [num_seqs]; 0 gives a zero output row
  *   max_context_len  host upper bound of context_lens (sizes the workspace)
- *   partition_tokens 0 = library's choice, else a multiple of 16 in [16, 65536]
+ *   partition_tokens 0 = library's choice (512 tokens, or 2048 when
+ *                 max_context_len > 16384), else a multiple of 16 in [16, 65536]
  *   out           bf16 [num_seqs][num_q_heads][head_dim], 16-B aligned
  *   workspace     device scratch of at least pkv_decode_workspace_bytes(...)
  *                 bytes, 256-B aligned; contents need no initialisation; one

@@ -20,7 +20,7 @@ LIB_PATH = os.path.join(_HERE, "libpkv.so")
 PKV_OK = 0
 STATUS_NAMES = {0: "PKV_OK", 1: "PKV_EINVAL", 2: "PKV_ERANGE", 3: "PKV_EALIAS", 4: "PKV_ECUDA",
                 5: "PKV_EDEVICE", 6: "PKV_EUNSUPPORTED"}
-DEVERR_SLOT, DEVERR_BLOCK, DEVERR_CONTEXT, DEVERR_TIMEOUT = 0x1, 0x2, 0x4, 0x8
+DEVERR_SLOT, DEVERR_BLOCK, DEVERR_CONTEXT, DEVERR_TIMEOUT, DEVERR_LAYOUT = 0x1, 0x2, 0x4, 0x8, 0x10
 
 # Every symbol include/pkv.h declares.
 EXPORTED = ("pkv_write", "pkv_copy_blocks", "pkv_decode_workspace_bytes", "paged_attn_decode",

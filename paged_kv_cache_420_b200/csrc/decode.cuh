@@ -176,7 +176,7 @@ struct DecodeSmem {
     static constexpr int oInfo = oBars + kNumBars * 8;
     static constexpr int oAbort = oInfo + NS * (int)sizeof(StageInfo);
     static constexpr int kBytes = oAbort + 16;
-    static constexpr int kAlloc = kBytes + 1024;  // slack to align the base to 1024 B
+    static constexpr int kAlloc = kBytes;  // the dynamic window is 1 KB-aligned (checked in the kernel)
 };
 
 // Bounded wait that also gives up when another warp has aborted.
@@ -511,16 +511,27 @@ struct MmaState {
 };
 
 // PATH 0: CUDA cores with G = GSIMT heads per kv head; PATH 1: tensor cores
-// with NT n-tiles of 8 heads.
-template <int D, int PATH, int GSIMT, int NT, int NS>
+// with query heads padded to GPAD in {4, 8, 16} (n-tiles of 8: GPAD/8 rounded up).
+template <int D, int PATH, int GSIMT, int GPAD, int NS>
 __global__ void __launch_bounds__(kDecodeThreads) paged_decode_kernel(const __grid_constant__ CUtensorMap tmap_k,
                                                                       const __grid_constant__ CUtensorMap tmap_v,
                                                                       const DecodeParams p) {
     constexpr int W = kConsumerWarps;
-    constexpr int GP = PATH == 0 ? GSIMT : 8 * NT;
+    constexpr int GP = PATH == 0 ? GSIMT : GPAD;
+    constexpr int NT = (GPAD + 7) / 8;
     using L = DecodeSmem<D, GP, NS>;
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    // 1024-B alignment: the 128-byte swizzle pattern repeats every 1 KB.
+    // Everything below indexes the shared array itself, so accesses stay in
+    // the shared window (ld.shared / st.shared, not generic loads).
+    // The dynamic window starts 1 KB-aligned when the kernel has no static
+    // shared variables (none here); the allocation has no slack for
+    // realignment, so a misaligned base is reported and the CTA does nothing.
+    if ((smem_u32(smem_raw) & 1023u) != 0) {
+        if (threadIdx.x == 0) raise_error(PKV_DEVERR_LAYOUT);
+        return;
+    }
+    uint8_t *smem = smem_raw;
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + L::oBars);
     uint64_t *empty = full + NS;
     uint64_t *qfull = empty + NS;
@@ -697,41 +708,37 @@ __global__ void __launch_bounds__(kDecodeThreads) paged_decode_kernel(const __gr
                 __syncwarp();
                 if (lane == 0) mbar_arrive(mfull);
                 if (!wait_or_abort(mfull, mc & 1, abort_flag)) break;
-                // Combine: thread ct owns a contiguous run of the g*D outputs, so
-                // the per-head factors 2^(m_u - M) are computed once per run.
+                // Combine: warp w takes heads w, w + W, ...; lane handles the
+                // elements lane, lane + 32, ... of the head (consecutive lanes on
+                // consecutive words: no bank conflicts), and the per-head factors
+                // 2^(m_u - M) are computed once per head.
                 const int g = p.g;
                 const size_t unit_head0 = (size_t)si.s * p.Hq + (size_t)si.h * g;
-                const int total = g * D;
-                const int ept = (total + W * 32 - 1) / (W * 32);
-                const int e0 = (w * 32 + lane) * ept;
-                const int e1 = min(total, e0 + ept);
-                int jcur = -1;
-                float f[W], M = 0.f, Lsum = 0.f, invL = 0.f;
-                for (int e = e0; e < e1; ++e) {
-                    const int j = e / D, d = e - j * D;
-                    if (j != jcur) {
-                        jcur = j;
-                        M = PKV_NEG_INF;
+                for (int j = w; j < g; j += W) {
+                    float M = PKV_NEG_INF;
 #pragma unroll
-                        for (int u = 0; u < W; ++u) M = fmaxf(M, mM[u * GP + j]);
-                        Lsum = 0.f;
+                    for (int u = 0; u < W; ++u) M = fmaxf(M, mM[u * GP + j]);
+                    float f[W], Lsum = 0.f;
 #pragma unroll
-                        for (int u = 0; u < W; ++u) {
-                            const float mu = mM[u * GP + j];
-                            f[u] = mu == PKV_NEG_INF ? 0.f : exp2f(mu - M);
-                            Lsum = fmaf(mL[u * GP + j], f[u], Lsum);
-                        }
-                        invL = Lsum > 0.f ? 1.f / Lsum : 0.f;
+                    for (int u = 0; u < W; ++u) {
+                        const float mu = mM[u * GP + j];
+                        f[u] = mu == PKV_NEG_INF ? 0.f : exp2f(mu - M);
+                        Lsum = fmaf(mL[u * GP + j], f[u], Lsum);
                     }
-                    float O = 0.f;
+                    const float invL = Lsum > 0.f ? 1.f / Lsum : 0.f;
 #pragma unroll
-                    for (int u = 0; u < W; ++u) O = fmaf(mO[(u * GP + j) * L::kMergeStride + d], f[u], O);
-                    if (si.nparts == 1) {
-                        p.out[(unit_head0 + j) * D + d] = __float2bfloat16_rn(O * invL);
-                    } else {
-                        const size_t pi = (unit_head0 + j) * p.maxP + si.part;
-                        p.part_acc[pi * D + d] = O;
-                        if (d == 0) p.part_ml[pi] = make_float2(M, Lsum);
+                    for (int i = 0; i < D / 32; ++i) {
+                        const int d = lane + 32 * i;
+                        float O = 0.f;
+#pragma unroll
+                        for (int u = 0; u < W; ++u) O = fmaf(mO[(u * GP + j) * L::kMergeStride + d], f[u], O);
+                        if (si.nparts == 1) {
+                            p.out[(unit_head0 + j) * D + d] = __float2bfloat16_rn(O * invL);
+                        } else {
+                            const size_t pi = (unit_head0 + j) * p.maxP + si.part;
+                            p.part_acc[pi * D + d] = O;
+                            if (d == 0) p.part_ml[pi] = make_float2(M, Lsum);
+                        }
                     }
                 }
                 __syncwarp();

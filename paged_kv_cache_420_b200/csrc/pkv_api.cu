@@ -105,8 +105,12 @@ struct WorkspaceLayout {
 
 size_t round256(size_t x) { return (x + 255) / 256 * 256; }
 
-int pick_partition_tokens(int32_t partition_tokens) {
-    return partition_tokens > 0 ? partition_tokens : 512;
+// Library's choice of split-K partition: 512 tokens up to 16K-token contexts
+// (short items keep a ragged batch balanced over the persistent CTAs), 2048
+// beyond (fewer partitions per sequence: less per-item and reduce overhead).
+int pick_partition_tokens(int32_t partition_tokens, int32_t max_context_len) {
+    if (partition_tokens > 0) return partition_tokens;
+    return max_context_len > 16384 ? 2048 : 512;
 }
 
 bool workspace_layout(int32_t B, int32_t Hq, int32_t D, int32_t max_ctx, int32_t PT, WorkspaceLayout *w) {
@@ -127,12 +131,12 @@ bool workspace_layout(int32_t B, int32_t Hq, int32_t D, int32_t max_ctx, int32_t
 
 // ---------------------------------------------------- decode dispatch ----
 
-template <int D, int PATH, int GS, int NT>
+template <int D, int PATH, int GS, int GPAD>
 pkv_status launch_decode(const pkv::DecodeParams &prm, const CUtensorMap &mk, const CUtensorMap &mv,
                          cudaStream_t stream, int dev) {
     constexpr int NS = PATH == 0 ? kStagesSimt : kStagesMma;
-    using L = pkv::DecodeSmem<D, (PATH == 0 ? GS : 8 * NT), NS>;
-    auto kernel = pkv::paged_decode_kernel<D, PATH, GS, NT, NS>;
+    using L = pkv::DecodeSmem<D, (PATH == 0 ? GS : GPAD), NS>;
+    auto kernel = pkv::paged_decode_kernel<D, PATH, GS, GPAD, NS>;
     static int occ_cache[kMaxDevices] = {0};
     int occ = (dev >= 0 && dev < kMaxDevices) ? occ_cache[dev] : 0;
     if (occ == 0) {
@@ -174,8 +178,9 @@ pkv_status dispatch_group(int g, const pkv::DecodeParams &prm, const CUtensorMap
                           cudaStream_t stream, int dev) {
     if (g == 1) return launch_decode<D, 0, 1, 1>(prm, mk, mv, stream, dev);
     if (g == 2) return launch_decode<D, 0, 2, 1>(prm, mk, mv, stream, dev);
-    if (g <= 8) return launch_decode<D, 1, 1, 1>(prm, mk, mv, stream, dev);
-    return launch_decode<D, 1, 1, 2>(prm, mk, mv, stream, dev);
+    if (g <= 4) return launch_decode<D, 1, 1, 4>(prm, mk, mv, stream, dev);
+    if (g <= 8) return launch_decode<D, 1, 1, 8>(prm, mk, mv, stream, dev);
+    return launch_decode<D, 1, 1, 16>(prm, mk, mv, stream, dev);
 }
 
 }  // namespace
@@ -269,8 +274,8 @@ size_t pkv_decode_workspace_bytes(int32_t num_seqs, int32_t num_q_heads, int32_t
     if (num_kv_heads <= 0 || num_q_heads <= 0 || num_q_heads % num_kv_heads) return 0;
     if (partition_tokens < 0 || partition_tokens % 16) return 0;
     WorkspaceLayout w;
-    if (!workspace_layout(num_seqs, num_q_heads, head_dim, max_context_len, pick_partition_tokens(partition_tokens),
-                          &w))
+    if (!workspace_layout(num_seqs, num_q_heads, head_dim, max_context_len,
+                          pick_partition_tokens(partition_tokens, max_context_len), &w))
         return 0;
     return w.total;
 }
@@ -294,7 +299,7 @@ pkv_status paged_attn_decode(const void *q, const void *k_cache, const void *v_c
         !aligned(block_tables, 4) || !aligned(context_lens, 4) || !aligned(workspace, 256))
         return PKV_EINVAL;
     const int D = pool.head_dim;
-    const int PT = pick_partition_tokens(partition_tokens);
+    const int PT = pick_partition_tokens(partition_tokens, max_context_len);
     WorkspaceLayout wl;
     if (!workspace_layout(num_seqs, num_q_heads, D, max_context_len, PT, &wl) || workspace_bytes < wl.total)
         return PKV_EINVAL;
