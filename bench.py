@@ -301,7 +301,7 @@ def run_cuda(args, rank, world, dist):
         ev_in = [torch.cuda.Event() for _ in range(2)]
         ev_done = [torch.cuda.Event() for _ in range(2)]
 
-        def h2d(i):
+        def upload(i):
             b = i % 2
             if i >= 2:  # buffer b was read by step i-2
                 copy.wait_event(ev_done[b])
@@ -311,11 +311,11 @@ def run_cuda(args, rank, world, dist):
                 ev_in[b].record(copy)
 
         def e2e_run(n):
-            h2d(0)
+            upload(0)
             for i in range(n):
                 b = i % 2
                 if i + 1 < n:
-                    h2d(i + 1)  # the next step's inputs move while this step computes
+                    upload(i + 1)  # the next step's inputs move while this step computes
                 stream.wait_event(ev_in[b])
                 if len(w.copy_pairs):
                     pkv.pkv_copy_blocks(w.copy_pairs, kc, vc, stream=stream)
