@@ -43,6 +43,11 @@ constexpr int kDecodeThreads = (kConsumerWarps + 1) * 32;
 constexpr int kPlanThreads = 1024;
 constexpr int kReduceWarps = 4;
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // bounded on-chip waits: 2 s
+// Online softmax keeps a reference max m per head and raises it only when a
+// stage's max exceeds it by more than this (log2 units), so most stages skip
+// the rescale of acc and l.  Weights 2^(s - m) then stay below 2^8: exact
+// enough in fp32, and the final out = acc / l does not depend on m.
+constexpr float kRescaleSlack = 8.0f;
 #define PKV_NEG_INF (-__int_as_float(0x7f800000))
 
 struct DecodeParams {
@@ -253,17 +258,20 @@ struct SimtState {
     __device__ __forceinline__ void stage(uint32_t ktile, uint32_t vtile, int valid, int lane) {
         constexpr int NV = 16 * G;
         float v[NV];
-        // q.k partial sums: v[j*16 + r] for head j, token r
+        // q.k partial sums v[j*16 + r] for head j, token r; tokens r and r+1
+        // share one packed fp32x2 FMA per element.
 #pragma unroll
-        for (int r = 0; r < 16; ++r) {
-            float x[EPL];
-            load_row(ktile, r, lane, x);
+        for (int r = 0; r < 16; r += 2) {
+            float x0[EPL], x1[EPL];
+            load_row(ktile, r, lane, x0);
+            load_row(ktile, r + 1, lane, x1);
 #pragma unroll
             for (int j = 0; j < G; ++j) {
-                float d = 0.f;
+                float d0 = 0.f, d1 = 0.f;
 #pragma unroll
-                for (int e = 0; e < EPL; ++e) d = fmaf(q[j][e], x[e], d);
-                v[j * 16 + r] = d;
+                for (int e = 0; e < EPL; ++e) fma_f32x2(d0, d1, q[j][e], q[j][e], x0[e], x1[e]);
+                v[j * 16 + r] = d0;
+                v[j * 16 + r + 1] = d1;
             }
         }
         // Transposing butterfly: after it, lane holds the full 32-lane sum of
@@ -290,38 +298,29 @@ struct SimtState {
         const int my_tok = (G == 1) ? (lane >> 1) : (lane & 15);
         const int my_head = (G == 1) ? 0 : (lane >> 4);
         const float score = (my_tok < valid) ? v[0] : PKV_NEG_INF;
-        // stage max per head
-        float mx = score;
-        if (G == 1) {
-#pragma unroll
-            for (int o = 2; o < 32; o <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-        } else {
-#pragma unroll
-            for (int o = 1; o < 16; o <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-        }
-        float m_new[G], alpha[G];
+        // stage max per head (one warp reduction each), lazy rescale
+        float mx[G];
         if constexpr (G == 1) {
-            m_new[0] = fmaxf(m[0], mx);
+            mx[0] = warp_max_f32(score);
         } else {
-            const float other = __shfl_xor_sync(0xffffffffu, mx, 16);
-            m_new[0] = fmaxf(m[0], my_head == 0 ? mx : other);
-            m_new[1] = fmaxf(m[1], my_head == 0 ? other : mx);
+            mx[0] = warp_max_f32(my_head == 0 ? score : PKV_NEG_INF);
+            mx[1] = warp_max_f32(my_head == 1 ? score : PKV_NEG_INF);
         }
 #pragma unroll
         for (int j = 0; j < G; ++j) {
-            alpha[j] = exp2f(m[j] - m_new[j]);
-            m[j] = m_new[j];
+            if (mx[j] > m[j] + kRescaleSlack) {  // warp-uniform, rare after the first stage
+                const float alpha = exp2f(m[j] - mx[j]);
+                m[j] = mx[j];
+#pragma unroll
+                for (int e = 0; e < EPL; ++e) acc[j][e] *= alpha;
+                if (G == 1 || my_head == j) l_part *= alpha;
+            }
         }
-        // selects, not a lane-dependent register index
-        const float my_m = (G == 1 || my_head == 0) ? m_new[0] : m_new[G - 1];
-        const float my_alpha = (G == 1 || my_head == 0) ? alpha[0] : alpha[G - 1];
+        const float my_m = (G == 1 || my_head == 0) ? m[0] : m[G - 1];
         const float pr = exp2f(score - my_m);
-        l_part = l_part * my_alpha + pr;
-#pragma unroll
-        for (int j = 0; j < G; ++j)
-#pragma unroll
-            for (int e = 0; e < EPL; ++e) acc[j][e] *= alpha[j];
-        // PV: broadcast p of each valid token, accumulate its V row
+        l_part += pr;
+        // PV: broadcast p of each valid token, accumulate its V row (packed
+        // fp32x2 FMA over element pairs)
 #pragma unroll
         for (int r = 0; r < 16; ++r) {
             if (r < valid) {
@@ -332,7 +331,7 @@ struct SimtState {
                     const int src = (G == 1) ? (2 * r) : (j * 16 + r);
                     const float pj = __shfl_sync(0xffffffffu, pr, src);
 #pragma unroll
-                    for (int e = 0; e < EPL; ++e) acc[j][e] = fmaf(pj, x[e], acc[j][e]);
+                    for (int e = 0; e < EPL; e += 2) fma_f32x2(acc[j][e], acc[j][e + 1], pj, pj, x[e], x[e + 1]);
                 }
             }
         }
@@ -435,31 +434,39 @@ struct MmaState {
         uint32_t pb[NT][2];
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
-            float alpha[2], p[4];
+            float alpha[2], p[4], z[4];
+            bool raise = false;
 #pragma unroll
             for (int c = 0; c < 2; ++c) {
-                const float z0 = ok0 ? s[nt][c] * scale_log2 : PKV_NEG_INF;
-                const float z1 = ok1 ? s[nt][c + 2] * scale_log2 : PKV_NEG_INF;
-                float mx = fmaxf(z0, z1);
+                z[c] = ok0 ? s[nt][c] * scale_log2 : PKV_NEG_INF;
+                z[c + 2] = ok1 ? s[nt][c + 2] * scale_log2 : PKV_NEG_INF;
+                float mx = fmaxf(z[c], z[c + 2]);
                 mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
                 mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
                 mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
-                const float mn = fmaxf(m[nt][c], mx);
-                alpha[c] = exp2f(m[nt][c] - mn);
-                m[nt][c] = mn;
-                p[c] = exp2f(z0 - mn);
-                p[c + 2] = exp2f(z1 - mn);
+                // lazy rescale: raise the reference max only when exceeded by the slack
+                const bool up = mx > m[nt][c] + kRescaleSlack;
+                alpha[c] = up ? exp2f(m[nt][c] - mx) : 1.f;
+                if (up) m[nt][c] = mx;
+                raise |= up;
+            }
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
+                p[c] = exp2f(z[c] - m[nt][c]);
+                p[c + 2] = exp2f(z[c + 2] - m[nt][c]);
                 l[nt][c] = l[nt][c] * alpha[c] + p[c] + p[c + 2];
             }
             // accumulator layout (token row, head pair) -> operand layout of P^T
             pb[nt][0] = movmatrix_trans(pack_bf16x2(p[0], p[1]));
             pb[nt][1] = movmatrix_trans(pack_bf16x2(p[2], p[3]));
+            if (__any_sync(0xffffffffu, raise)) {
 #pragma unroll
-            for (int mt = 0; mt < MT; ++mt) {
-                o[nt][mt][0] *= alpha[0];
-                o[nt][mt][1] *= alpha[1];
-                o[nt][mt][2] *= alpha[0];
-                o[nt][mt][3] *= alpha[1];
+                for (int mt = 0; mt < MT; ++mt) {
+                    o[nt][mt][0] *= alpha[0];
+                    o[nt][mt][1] *= alpha[1];
+                    o[nt][mt][2] *= alpha[0];
+                    o[nt][mt][3] *= alpha[1];
+                }
             }
         }
         // token masks of this thread's V^T operand halves: tokens 2(l%4)+{0,1} and +8

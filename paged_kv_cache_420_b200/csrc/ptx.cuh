@@ -145,6 +145,25 @@ __device__ __forceinline__ void mma_bf16_16816(float &d0, float &d1, float &d2, 
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
+// Warp-wide maximum of a float (sm_100a); NaN inputs are ignored.
+__device__ __forceinline__ float warp_max_f32(float v) {
+    float r;
+    asm volatile("redux.sync.max.f32 %0, %1, 0xffffffff;" : "=f"(r) : "f"(v));
+    return r;
+}
+
+// Packed fp32 pair FMA (sm_100a): (a0, a1) += (b0 * c0, b1 * c1).
+__device__ __forceinline__ void fma_f32x2(float &a0, float &a1, float b0, float b1, float c0, float c1) {
+    asm("{\n\t.reg .b64 pa, pb, pc;\n\t"
+        "mov.b64 pa, {%0, %1};\n\t"
+        "mov.b64 pb, {%2, %3};\n\t"
+        "mov.b64 pc, {%4, %5};\n\t"
+        "fma.rn.f32x2 pa, pb, pc, pa;\n\t"
+        "mov.b64 {%0, %1}, pa;\n\t}"
+        : "+f"(a0), "+f"(a1)
+        : "f"(b0), "f"(b1), "f"(c0), "f"(c1));
+}
+
 // ------------------------------------------------------------------ bf16 --
 
 // A bf16 is the upper half of an fp32, so widening is a shift / mask.
