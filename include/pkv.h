@@ -199,6 +199,19 @@ pkv_status paged_attn_decode_static_ws(const void *q, const void *k_cache, const
  */
 pkv_status pkv_get_device_error(int32_t *code_out, pkv_stream_t stream);
 
+/*
+ * pkv_selftest_bounded_wait -- diagnostic of this library (the pages have no
+ * counterpart).  Runs, in one CTA, the bounded on-chip wait that the attention
+ * kernel uses for its pipeline barriers, against barriers that nothing ever
+ * arrives on: one warp gives up after limit_ns nanoseconds (0 < limit_ns <=
+ * 1e9), sets PKV_DEVERR_TIMEOUT and the CTA's abort flag, and a second warp,
+ * waiting with the kernel's 2 s limit, must then give up early.  Writes to
+ * result_dev (device int32[3]): [0] first wait completed (expected 0),
+ * [1] second wait completed (expected 0), [2] microseconds the second warp
+ * waited.  No fault and no hang: both waits end by themselves.
+ */
+pkv_status pkv_selftest_bounded_wait(int64_t limit_ns, int32_t *result_dev, pkv_stream_t stream);
+
 /* Static description of a status code. */
 const char *pkv_status_string(pkv_status status);
 

@@ -24,7 +24,8 @@ DEVERR_SLOT, DEVERR_BLOCK, DEVERR_CONTEXT, DEVERR_TIMEOUT, DEVERR_LAYOUT = 0x1, 
 
 # Every symbol include/pkv.h declares.
 EXPORTED = ("pkv_write", "pkv_copy_blocks", "pkv_decode_workspace_bytes", "paged_attn_decode",
-            "paged_attn_decode_static_ws", "pkv_get_device_error", "pkv_status_string", "pkv_version")
+            "paged_attn_decode_static_ws", "pkv_get_device_error", "pkv_selftest_bounded_wait", "pkv_status_string",
+            "pkv_version")
 STATIC_WS_BYTES = 32 << 20  # PKV_STATIC_WS_BYTES
 
 
@@ -203,3 +204,17 @@ def paged_attn_decode_static_ws(q: torch.Tensor, k_cache: torch.Tensor, v_cache:
            B, Hq, float(scale), int(num_kv_heads), _ptr(out), _pool(k_cache), int(max_context_len),
            int(partition_tokens), _stream(stream))
     _check(st, "paged_attn_decode_static_ws")
+
+
+def selftest_bounded_wait(limit_ns: int, stream=None) -> torch.Tensor:
+    """Runs the library's bounded on-chip wait against barriers that never
+    complete (see pkv_selftest_bounded_wait).  Returns the device int32[3]
+    result; the device error word then holds DEVERR_TIMEOUT."""
+    lib = load_library()
+    f = lib.pkv_selftest_bounded_wait
+    if f.argtypes is None:
+        f.argtypes = [ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p]
+        f.restype = ctypes.c_int
+    res = torch.full((3,), -1, dtype=torch.int32, device="cuda")
+    _check(f(int(limit_ns), _ptr(res), _stream(stream)), "pkv_selftest_bounded_wait")
+    return res

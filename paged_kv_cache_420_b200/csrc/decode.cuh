@@ -185,14 +185,15 @@ struct DecodeSmem {
 };
 
 // Bounded wait that also gives up when another warp has aborted.
-__device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity, volatile int *abort_flag) {
+__device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
+                                              uint64_t limit_ns = kWaitLimitNs) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_timer_ns();
     for (uint32_t it = 1;; ++it) {
         if (mbar_try_wait(bar, parity)) return true;
         if ((it & 255u) == 0) {
             if (*abort_flag) return false;
-            if (global_timer_ns() - t0 > kWaitLimitNs) {
+            if (global_timer_ns() - t0 > limit_ns) {
                 raise_error(PKV_DEVERR_TIMEOUT);
                 *abort_flag = 1;
                 return false;
@@ -813,6 +814,35 @@ __global__ void __launch_bounds__(kReduceWarps * 32) splitk_reduce_kernel(const 
 #pragma unroll
             for (int u = 0; u < kReduceWarps; ++u) o += s_o[u][lane * EPL + e];
             p.out[(size_t)unit * D + lane * EPL + e] = __float2bfloat16_rn(o * inv);
+        }
+    }
+}
+
+// ------------------------------------------------------------- self-test --
+// Exercises the bounded waits of the attention kernel without a fault: warp 0
+// waits on a barrier that nothing arrives on and gives up after limit_ns
+// (setting PKV_DEVERR_TIMEOUT and the CTA's abort flag); warp 1 waits on
+// another such barrier with the 2 s default limit and must return early
+// because of the abort flag.  out[0] = warp 0's result, out[1] = warp 1's,
+// out[2] = warp 1's wait time in microseconds.
+__global__ void __launch_bounds__(64) selftest_wait_kernel(uint64_t limit_ns, int32_t *out) {
+    __shared__ uint64_t bars[2];
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        mbar_init(&bars[0], 1);
+        mbar_init(&bars[1], 1);
+        abort_flag = 0;
+        fence_mbar_init();
+    }
+    __syncthreads();
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (lane == 0) {
+        if (warp == 0) {
+            out[0] = wait_or_abort(&bars[0], 0, &abort_flag, limit_ns) ? 1 : 0;
+        } else {
+            const uint64_t t0 = global_timer_ns();
+            out[1] = wait_or_abort(&bars[1], 0, &abort_flag) ? 1 : 0;
+            out[2] = (int32_t)((global_timer_ns() - t0) / 1000);
         }
     }
 }

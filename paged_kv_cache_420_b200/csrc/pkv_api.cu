@@ -352,6 +352,12 @@ pkv_status pkv_get_device_error(int32_t *code_out, pkv_stream_t stream) {
     return h ? PKV_EDEVICE : PKV_OK;
 }
 
+pkv_status pkv_selftest_bounded_wait(int64_t limit_ns, int32_t *result_dev, pkv_stream_t stream) {
+    if (limit_ns <= 0 || limit_ns > 1000000000ll || !result_dev || !aligned(result_dev, 4)) return PKV_EINVAL;
+    pkv::selftest_wait_kernel<<<1, 64, 0, reinterpret_cast<cudaStream_t>(stream)>>>((uint64_t)limit_ns, result_dev);
+    return launch_status();
+}
+
 }  // extern "C"
 
 // ------------------------------------------------- no-allocation variant ----
