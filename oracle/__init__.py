@@ -50,9 +50,11 @@ def _load() -> ctypes.CDLL:
         lib.oracle_paged_attention.argtypes = [P, P, P, P, I, P, I, I, I, I, I, I, D, P]
         lib.oracle_attention_partial.argtypes = [P, P, P, P, I, I, I, I, I, I, I, I, D, P, P, P]
         lib.oracle_lse_merge.argtypes = [P, P, P, I, I, P]
+        lib.oracle_paged_prefill.argtypes = [P, P, P, P, I, P, P, I, I, I, I, I, I, D, P]
         lib.oracle_num_threads.argtypes = []
         for f in (lib.oracle_kv_write, lib.oracle_copy_blocks, lib.oracle_paged_attention,
-                  lib.oracle_attention_partial, lib.oracle_lse_merge, lib.oracle_num_threads):
+                  lib.oracle_attention_partial, lib.oracle_lse_merge, lib.oracle_num_threads,
+                  lib.oracle_paged_prefill):
             f.restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -140,6 +142,26 @@ def paged_attention(q, k_cache, v_cache, block_tables, context_lens, scale: floa
                                         _ptr(ctx), B, Hq, Hkv, d, bs, NB, float(np.float64(np.float32(scale))),
                                         _ptr(out))
     _check(rc, "paged_attention")
+    return out
+
+
+def paged_prefill(q, k_cache, v_cache, block_tables, context_lens, query_start, scale: float) -> np.ndarray:
+    """fp64 chunked-prefill attention out[T, Hq, d]: query row i of sequence
+    s's chunk is at position ctx_s - q_len_s + i and sees positions [0, pos]."""
+    qb = bits(q)
+    kc, vc = bits(k_cache), bits(v_cache)
+    tables = np.ascontiguousarray(block_tables, dtype=np.int32)
+    ctx = np.ascontiguousarray(context_lens, dtype=np.int32)
+    qsl = np.ascontiguousarray(query_start, dtype=np.int32)
+    T, Hq, d = qb.shape
+    NB, Hkv, bs, d2 = kc.shape
+    B = ctx.shape[0]
+    assert d == d2 and qsl.shape == (B + 1,) and int(qsl[-1]) == T
+    out = np.zeros((T, Hq, d), dtype=np.float64)
+    rc = _load().oracle_paged_prefill(_ptr(qb), _ptr(kc), _ptr(vc), _ptr(tables), tables.shape[1], _ptr(ctx),
+                                      _ptr(qsl), B, Hq, Hkv, d, bs, NB, float(np.float64(np.float32(scale))),
+                                      _ptr(out))
+    _check(rc, "paged_prefill")
     return out
 
 

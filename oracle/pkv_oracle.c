@@ -241,3 +241,50 @@ int oracle_lse_merge(const double *m, const double *l, const double *acc, int P,
     for (int c = 0; c < d; ++c) out[c] = (L > 0.0) ? out[c] / L : 0.0;
     return 0;
 }
+
+/*
+ * Chunked prefill (multi-token query, wkbse.com section 3.1 attention read
+ * through the block table, with the causal rule of autoregressive decoding:
+ * a token sees itself and the tokens before it).  Sequence s holds
+ * context_lens[s] tokens in the cache, the last q_len = query_start[s+1] -
+ * query_start[s] of which are the new chunk; query row i of the chunk is at
+ * position pos = context_lens[s] - q_len + i and attends to positions
+ * [0, pos].  q and out are [T][Hq][d] with T = query_start[B]; out in double.
+ */
+int oracle_paged_prefill(const uint16_t *q, const uint16_t *k_cache, const uint16_t *v_cache,
+                         const int32_t *block_tables, int max_blocks_per_seq, const int32_t *context_lens,
+                         const int32_t *query_start, int B, int Hq, int Hkv, int d, int bs, int num_blocks,
+                         double scale, double *out) {
+    if (B < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || d <= 0 || bs <= 0) return 1;
+    for (int s = 0; s < B; ++s) {
+        int q_len = query_start[s + 1] - query_start[s];
+        if (q_len < 0 || q_len > context_lens[s]) return 1;
+        if ((int64_t)context_lens[s] > (int64_t)max_blocks_per_seq * bs) return 2;
+    }
+    int T = query_start[B];
+    int status = 0;
+#pragma omp parallel for schedule(dynamic, 1) collapse(2)
+    for (int t = 0; t < T; ++t) {
+        for (int hq = 0; hq < Hq; ++hq) {
+            int s = 0;
+            while (query_start[s + 1] <= t) ++s;
+            int q_len = query_start[s + 1] - query_start[s];
+            int pos = context_lens[s] - q_len + (t - query_start[s]);
+            double *o = out + ((size_t)t * Hq + hq) * (size_t)d;
+            double *acc = (double *)malloc(sizeof(double) * (size_t)d);
+            double m, l;
+            int rc = acc ? attend_range(q + ((size_t)t * Hq + hq) * (size_t)d, k_cache, v_cache,
+                                        block_tables + (size_t)s * max_blocks_per_seq, num_blocks, Hq, Hkv, d,
+                                        bs, hq, 0, pos + 1, scale, &m, &l, acc)
+                         : 1;
+            if (rc) {
+#pragma omp atomic write
+                status = rc;
+            } else {
+                for (int c = 0; c < d; ++c) o[c] = (l > 0.0) ? acc[c] / l : 0.0;
+            }
+            free(acc);
+        }
+    }
+    return status;
+}

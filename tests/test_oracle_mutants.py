@@ -14,6 +14,7 @@ import pytest
 
 import oracle
 from tests import test_oracle_pins as pins
+from tests import test_oracle_prefill as prefill_pins
 
 PIN_TESTS = [
     pins.test_block_count_golden,
@@ -29,6 +30,8 @@ PIN_TESTS = [
     pins.test_context_len_zero_gives_zero_output,
     lambda: pins.test_split_merge_equals_unsplit("ragged"),
     pins.test_lse_merge_closed_form,
+    lambda: prefill_pins.test_prefill_equals_sdpa_with_bottom_right_causal_mask([31, 17, 0, 64], [1, 20, 48, 3],
+                                                                                 6, 3, 64, 16),
 ]
 
 MUTANTS = {
@@ -45,6 +48,11 @@ MUTANTS = {
                         "memcpy(k_cache + dst, k_cache + (size_t)pairs[2 * p] * block_elems"),
     "missing normalisation": ("o[c] = (l > 0.0) ? acc[c] / l : 0.0;", "o[c] = (l > 0.0) ? acc[c] : 0.0;"),
     "merge drops rescale": ("L += l[p] * w;", "L += l[p];"),
+    # prefill: a query also sees the next position, or misses its own
+    "prefill causal bound +1": ("bs, hq, 0, pos + 1, scale", "bs, hq, 0, pos + 2 > context_lens[s] ? context_lens[s] : pos + 2, scale"),
+    "prefill causal bound -1": ("bs, hq, 0, pos + 1, scale", "bs, hq, 0, pos, scale"),
+    "prefill query position": ("int pos = context_lens[s] - q_len + (t - query_start[s]);",
+                               "int pos = (t - query_start[s]);"),
     # the new token left out of the attended range (context_len - 1 tokens)
     "context off by one": ("hq, 0, context_lens[s], scale", "hq, 0, context_lens[s] - 1, scale"),
 }
@@ -68,7 +76,7 @@ def test_pins_catch_planted_mistake(name, tmp_path, monkeypatch):
     good = oracle._load()
     lib = ctypes.CDLL(so)
     for fn in ("oracle_kv_write", "oracle_copy_blocks", "oracle_paged_attention",
-               "oracle_attention_partial", "oracle_lse_merge", "oracle_num_threads"):
+               "oracle_attention_partial", "oracle_lse_merge", "oracle_num_threads", "oracle_paged_prefill"):
         getattr(lib, fn).argtypes = getattr(good, fn).argtypes
         getattr(lib, fn).restype = getattr(good, fn).restype
     monkeypatch.setattr(oracle, "_lib", lib)

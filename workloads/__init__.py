@@ -391,3 +391,121 @@ def subset(w: Workload, num_seqs: int) -> Workload:
         q=w.q[:n].contiguous(), k_new=w.k_new[:n].contiguous(), v_new=w.v_new[:n].contiguous(),
         k_cache=w.k_cache.index_select(0, sel).contiguous(), v_cache=w.v_cache.index_select(0, sel).contiguous(),
         description=w.description + f" (first {n} sequences)")
+
+
+# --------------------------------------------------------------------------
+# chunked prefill: several new tokens per sequence
+# --------------------------------------------------------------------------
+
+@dataclasses.dataclass
+class PrefillWorkload:
+    """State before one prefill chunk and its inputs: sequence s already holds
+    prefix_lens[s] tokens; its chunk of q_len_s = query_start[s+1] -
+    query_start[s] new tokens is written at positions prefix..ctx-1 (slot
+    mapping) and then attends causally.  context_lens counts the chunk."""
+    name: str
+    seed: int
+    num_seqs: int
+    num_q_heads: int
+    num_kv_heads: int
+    head_dim: int
+    block_size: int
+    num_blocks: int
+    max_blocks_per_seq: int
+    scale: float
+    context_lens: np.ndarray  # int32 [B]
+    query_start: np.ndarray  # int32 [B + 1]
+    block_tables: np.ndarray  # int32 [B, MBS]
+    slot_mapping: np.ndarray  # int64 [T]
+    q: torch.Tensor  # bf16 [T, Hq, D]
+    k_new: torch.Tensor  # bf16 [T, Hkv, D]
+    v_new: torch.Tensor  # bf16 [T, Hkv, D]
+    k_cache: torch.Tensor
+    v_cache: torch.Tensor
+    description: str = ""
+
+    @property
+    def num_tokens(self) -> int:
+        return int(self.query_start[-1])
+
+    @property
+    def max_context_len(self) -> int:
+        return int(self.context_lens.max()) if self.num_seqs else 0
+
+    @property
+    def max_query_len(self) -> int:
+        return int(np.diff(self.query_start).max()) if self.num_seqs else 0
+
+
+def make_prefill_custom(prefix_lens: Sequence[int], chunk_lens: Sequence[int], num_q_heads: int,
+                        num_kv_heads: int, head_dim: int, block_size: int, seed: int = 0,
+                        pool_factor: float = 1.2, values_device="cpu", poison=False,
+                        name: str = "prefill-custom", description: str = "") -> PrefillWorkload:
+    rng = np.random.default_rng(seed)
+    bs = block_size
+    prefix = [int(x) for x in prefix_lens]
+    chunk = [int(x) for x in chunk_lens]
+    ctx = [p + c for p, c in zip(prefix, chunk)]
+    need = sum(_nblocks(c, bs) for c in ctx) + 1
+    NB = max(int(math.ceil(pool_factor * need)), 1)
+    free = [int(x) for x in rng.permutation(NB)]
+    per_seq = _pop_tables(ctx, bs, free)
+    mbs = max([len(b) for b in per_seq] + [1])
+    tables = _tables_array(per_seq, mbs)
+    qsl = np.zeros(len(ctx) + 1, dtype=np.int32)
+    qsl[1:] = np.cumsum(chunk)
+    T = int(qsl[-1])
+    slots = np.empty(T, dtype=np.int64)
+    for s, (p0, c) in enumerate(zip(prefix, chunk)):
+        for i in range(c):
+            pos = p0 + i
+            slots[qsl[s] + i] = int(tables[s, pos // bs]) * bs + pos % bs
+    gen = None
+    if str(values_device) != "meta":
+        gen = torch.Generator(device=values_device)
+        gen.manual_seed(int(seed))
+    Hq, Hkv, D = num_q_heads, num_kv_heads, head_dim
+    q = _normal_bf16((T, Hq, D), gen, values_device)
+    k_new = _normal_bf16((T, Hkv, D), gen, values_device)
+    v_new = _normal_bf16((T, Hkv, D), gen, values_device)
+    k_cache = _normal_bf16((NB, Hkv, bs, D), gen, values_device)
+    v_cache = _normal_bf16((NB, Hkv, bs, D), gen, values_device)
+    if poison and gen is not None:
+        live = np.zeros((NB, bs), dtype=bool)
+        for s in range(len(ctx)):
+            for pos in range(prefix[s]):
+                live[per_seq[s][pos // bs], pos % bs] = True
+        dead = torch.from_numpy(~live).to(values_device)
+        nan = torch.tensor(BF16_NAN_BITS, dtype=torch.int16).view(torch.bfloat16).to(values_device)
+        mask = dead[:, None, :, None].expand(NB, Hkv, bs, D)
+        k_cache = torch.where(mask, nan, k_cache)
+        v_cache = torch.where(mask, nan, v_cache)
+    return PrefillWorkload(name=name, seed=seed, num_seqs=len(ctx), num_q_heads=Hq, num_kv_heads=Hkv,
+                           head_dim=D, block_size=bs, num_blocks=NB, max_blocks_per_seq=mbs,
+                           scale=float(np.float32(1.0 / math.sqrt(D))),
+                           context_lens=np.asarray(ctx, dtype=np.int32), query_start=qsl, block_tables=tables,
+                           slot_mapping=slots, q=q, k_new=k_new, v_new=v_new, k_cache=k_cache,
+                           v_cache=v_cache, description=description or f"prefix={prefix} chunk={chunk}")
+
+
+PREFILL_WORKLOADS = ("llama2-13b-prefill", "llama3-8b-prefill")
+
+
+def make_prefill(name: str, seed: int = 0, values_device="cpu", poison: bool = False,
+                 block_size: Optional[int] = None) -> PrefillWorkload:
+    """Chunked-prefill workloads: 8 sequences, each with an already cached
+    prefix of U[0, L] tokens and a new 512-token chunk (Llama-2-13B: 40 MHA
+    heads, L = 3072; Llama-3-8B: 32 q / 8 kv heads, L = 7680)."""
+    rng = np.random.default_rng(seed)
+    bs = 16 if block_size is None else block_size
+    if name == "llama2-13b-prefill":
+        Hq, Hkv, L = 40, 40, 3072
+    elif name == "llama3-8b-prefill":
+        Hq, Hkv, L = 32, 8, 7680
+    else:
+        raise KeyError(f"unknown prefill workload {name!r}; choose from {PREFILL_WORKLOADS}")
+    prefix = [int(x) for x in rng.integers(0, L, size=8, endpoint=True)]
+    return make_prefill_custom(prefix, [512] * 8, Hq, Hkv, 128, bs, seed=seed, values_device=values_device,
+                               poison=poison, name=name,
+                               description=f"B8, {Hq}q/{Hkv}kv heads, d128, bs{bs}, cached prefix U[0,{L}], "
+                                           "512-token chunk each")
