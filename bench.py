@@ -390,6 +390,93 @@ def run_cuda(args, rank, world, dist):
     return line
 
 
+def prefill_flops(w) -> float:
+    """QK^T and PV multiply-adds of causal chunked prefill: every (query row,
+    query head) attends to pos + 1 keys, 2 flops per element of each."""
+    keys = 0
+    for s in range(w.num_seqs):
+        ql = int(w.query_start[s + 1] - w.query_start[s])
+        n = int(w.context_lens[s])
+        keys += ql * (n - ql) + ql * (ql + 1) // 2
+    return 4.0 * w.head_dim * w.num_q_heads * keys
+
+
+def measured_tensor_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["bf16_tflops"]), "measured"
+    except Exception:
+        return 1590.0, "fallback"
+
+
+def run_prefill_cuda(args, rank, world, dist):
+    """One step = slot-mapped write of every chunk token + chunked-prefill
+    attention; metric TFLOP/s of the attention (causal flops)."""
+    import paged_kv_cache_420_b200 as pkv
+
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
+    torch.cuda.set_device(dev)
+    w = workloads.make_prefill(args.workload, seed=args.seed + rank, values_device=dev, block_size=args.block_size)
+    slots = torch.from_numpy(w.slot_mapping).to(dev)
+    tables = torch.from_numpy(w.block_tables).to(dev)
+    ctx = torch.from_numpy(w.context_lens).to(dev)
+    qs = torch.from_numpy(w.query_start).to(dev)
+    out = torch.empty_like(w.q)
+    ws = torch.empty(pkv.prefill_workspace_bytes(w.num_seqs, w.num_q_heads, w.num_kv_heads, w.max_query_len),
+                     dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+
+    def step(i=None):
+        pkv.pkv_write(w.k_new, w.v_new, slots, w.k_cache, w.v_cache, stream=stream)
+        if i is not None:
+            ev[i][0].record(stream)
+        pkv.paged_attn_prefill(w.q, w.k_cache, w.v_cache, tables, ctx, qs, w.scale, w.num_kv_heads, out,
+                               w.max_query_len, w.max_context_len, workspace=ws, stream=stream)
+        if i is not None:
+            ev[i][1].record(stream)
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(dev.index) as clocks:
+        t0.record(stream)
+        for i in range(args.steps):
+            step(i)
+        t1.record(stream)
+        torch.cuda.synchronize()
+        if dist is not None:
+            dist.barrier()
+        if t0.elapsed_time(t1) < 450:
+            time.sleep(0.45)
+    if pkv.get_device_error():
+        raise RuntimeError("device error word set during the timed region")
+    flops = prefill_flops(w)
+    ms_max, flops_all, tok_all = combine_ranks(dist, t0.elapsed_time(t1), int(flops), w.num_tokens, dev)
+    attn_ms = sum(a.elapsed_time(b) for a, b in ev) / args.steps
+    peak, kind = measured_tensor_peak()
+    achieved = flops / (attn_ms / 1e3) / 1e12
+    return {
+        "metric": "paged chunked-prefill attention TFLOP/s",
+        "value": round(flops_all * args.steps / (ms_max / 1e3) / 1e12, 2), "unit": "TFLOP/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_max / args.steps, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": f"{w.name}: {w.description}", "num_seqs": w.num_seqs,
+                   "query_tokens": w.num_tokens, "kv_tokens": int(w.context_lens.sum()),
+                   "block_size": w.block_size, "seed": args.seed},
+        "tokens_per_s": round(tok_all * args.steps / (ms_max / 1e3), 1),
+        "roofline": {"kernel": "paged_attn_prefill (plan + attention kernels)", "bound": "tensor",
+                     "achieved": round(achieved, 2), "peak": peak, "peak_kind": kind, "unit": "TFLOP/s",
+                     "frac": round(achieved / peak, 4), "algorithmic_flops": flops,
+                     "prefill_us": round(attn_ms * 1e3, 2), "traffic": None},
+        "e2e": None, "gpu_launches": 3 * args.steps, "clocks": clocks.summary(),
+    }
+
+
 def cpu_baseline(w, budget_s: float, label="oracle", pools=None):
     """Times the fp64 CPU oracle's paged attention on the first sequences of
     the workload until about `budget_s` seconds of CPU work are spent.  The
@@ -445,11 +532,55 @@ def _subset(w, idx):
     return sub
 
 
+def run_prefill_reference(args, world):
+    """The CPU oracle's chunked prefill on the host cores: each step is a
+    bounded sample of query rows (whole sequences' chunks, cycling)."""
+    import oracle
+
+    w = workloads.make_prefill(args.workload, seed=args.seed, values_device="cpu", block_size=args.block_size)
+    kc, vc = oracle.kv_write(w.k_cache, w.v_cache, w.k_new, w.v_new, w.slot_mapping)
+    budget = max(0.05, min(2.0, 150.0 / max(1, args.steps + args.warmup)))
+    qb = oracle.bits(w.q)
+    vals, t_all, rows_done, flops_done, spent, seq = [], 0.0, 0, 0.0, 0.0, 0
+    for i in range(args.warmup + args.steps):
+        spent_step, fl = 0.0, 0.0
+        while spent_step < budget:
+            s = seq % w.num_seqs
+            a, b = int(w.query_start[s]), int(w.query_start[s + 1])
+            rows = np.arange(a, min(b, a + 16))  # 16 query rows of the chunk
+            pos = w.context_lens[s] - (b - rows)
+            ctx = (pos + 1).astype(np.int32)
+            t = time.perf_counter()
+            oracle.paged_prefill(qb[rows], kc, vc, w.block_tables[[s] * len(rows)], ctx,
+                                 np.arange(len(rows) + 1, dtype=np.int32), w.scale)
+            spent_step += time.perf_counter() - t
+            fl += 4.0 * w.head_dim * w.num_q_heads * float(ctx.sum())
+            seq += 1
+            if i >= args.warmup:
+                rows_done += len(rows)
+        if i >= args.warmup:
+            vals.append(fl / spent_step / 1e12)
+            t_all += spent_step
+    value = statistics.median(vals)
+    return {
+        "impl": "reference", "metric": "paged chunked-prefill attention TFLOP/s", "value": value,
+        "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(1e3 * t_all / args.steps, 3), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": f"{w.name}: {w.description}", "seed": args.seed},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": oracle.num_threads(), "kind": "oracle",
+                         "sample": f"{rows_done} query rows (16 per sequence, cycling), all heads"},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
 def run_reference(args, rank, world):
     """The CPU oracle as the reference arm: rank 0 times it on the host cores,
     one bounded sample of the workload per step."""
     if rank != 0:
         return None
+    if args.workload in workloads.PREFILL_WORKLOADS:
+        return run_prefill_reference(args, world)
     w = workloads.make(args.workload, seed=args.seed, values_device="cpu", block_size=args.block_size)
     per_step_budget = max(0.05, min(2.0, 150.0 / max(1, args.steps + args.warmup)))
     pools = oracle_pools(w)
@@ -485,7 +616,8 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=5000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["pkv", "reference"], default="pkv")
-    ap.add_argument("--workload", default="llama2-13b", choices=list(workloads.WORKLOADS))
+    ap.add_argument("--workload", default="llama2-13b",
+                    choices=list(workloads.WORKLOADS) + list(workloads.PREFILL_WORKLOADS))
     ap.add_argument("--block-size", type=int, default=None)
     ap.add_argument("--partition-tokens", type=int, default=-1, help="-1: the workload's choice, 0: library's")
     ap.add_argument("--seed", type=int, default=0)
@@ -509,6 +641,8 @@ def main(argv=None):
     try:
         if args.impl == "reference":
             line = run_reference(args, rank, world)
+        elif args.workload in workloads.PREFILL_WORKLOADS:
+            line = run_prefill_cuda(args, rank, world, dist)
         else:
             line = run_cuda(args, rank, world, dist)
         if rank == 0 and line is not None:

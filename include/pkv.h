@@ -193,6 +193,41 @@ pkv_status paged_attn_decode_static_ws(const void *q, const void *k_cache, const
                                        pkv_stream_t stream);
 
 /*
+ * pkv_prefill_workspace_bytes -- device scratch needed by paged_attn_prefill
+ * (its work list).  Returns 0 for invalid sizes.
+ */
+size_t pkv_prefill_workspace_bytes(int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads,
+                                   int32_t max_query_len);
+
+/*
+ * paged_attn_prefill -- chunked-prefill attention: several new query tokens per
+ * sequence, each attending causally to the sequence's cached context read
+ * through the block table (wkbse.com section 3.1; a token sees itself and the
+ * tokens before it).  The chunk's own K/V must already be in the cache
+ * (pkv_write of its tokens' slots).  For sequence s with q_len =
+ * query_start[s+1] - query_start[s] and ctx = context_lens[s] (counting the
+ * chunk), query row t = query_start[s] + i is at position pos = ctx - q_len + i
+ * and, for every query head hq (kv head hq / (num_q_heads / num_kv_heads)):
+ *   out[t][hq] = sum_{j <= pos} softmax_j(scale * <q[t][hq], K_j>) V_j
+ * in fp32 with bf16 (nearest-even) output.  decode is the case q_len = 1.
+ *
+ *   q, out        bf16 [T][num_q_heads][head_dim], T = query_start[num_seqs], 16-B aligned
+ *   query_start   int32 [num_seqs + 1], non-decreasing, query_start[0] = 0
+ *   context_lens  int32 [num_seqs]; q_len <= context_len
+ *   max_query_len / max_context_len  host upper bounds (size the work list)
+ *   workspace     at least pkv_prefill_workspace_bytes(...), 256-B aligned
+ * A query length above its context or the bounds sets PKV_DEVERR_CONTEXT and is
+ * clamped (rows past the clamp are not written).  Launches a plan kernel and
+ * the attention kernel on `stream`.
+ */
+pkv_status paged_attn_prefill(const void *q, const void *k_cache, const void *v_cache,
+                              const int32_t *block_tables, int32_t max_blocks_per_seq,
+                              const int32_t *context_lens, const int32_t *query_start, int32_t num_seqs,
+                              int32_t num_q_heads, float scale, int32_t num_kv_heads, void *out,
+                              pkv_pool pool, int32_t max_query_len, int32_t max_context_len,
+                              void *workspace, size_t workspace_bytes, pkv_stream_t stream);
+
+/*
  * pkv_get_device_error -- copies the current device's error word to
  * *code_out and clears it, ordered after the work already on `stream`, and
  * waits for it.  Returns PKV_EDEVICE when the word was non-zero.

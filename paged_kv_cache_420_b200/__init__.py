@@ -24,8 +24,8 @@ DEVERR_SLOT, DEVERR_BLOCK, DEVERR_CONTEXT, DEVERR_TIMEOUT, DEVERR_LAYOUT = 0x1, 
 
 # Every symbol include/pkv.h declares.
 EXPORTED = ("pkv_write", "pkv_copy_blocks", "pkv_decode_workspace_bytes", "paged_attn_decode",
-            "paged_attn_decode_static_ws", "pkv_get_device_error", "pkv_selftest_bounded_wait", "pkv_status_string",
-            "pkv_version")
+            "paged_attn_decode_static_ws", "pkv_prefill_workspace_bytes", "paged_attn_prefill",
+            "pkv_get_device_error", "pkv_selftest_bounded_wait", "pkv_status_string", "pkv_version")
 STATIC_WS_BYTES = 32 << 20  # PKV_STATIC_WS_BYTES
 
 
@@ -218,3 +218,44 @@ def selftest_bounded_wait(limit_ns: int, stream=None) -> torch.Tensor:
     res = torch.full((3,), -1, dtype=torch.int32, device="cuda")
     _check(f(int(limit_ns), _ptr(res), _stream(stream)), "pkv_selftest_bounded_wait")
     return res
+
+
+def prefill_workspace_bytes(num_seqs: int, num_q_heads: int, num_kv_heads: int, max_query_len: int) -> int:
+    lib = load_library()
+    f = lib.pkv_prefill_workspace_bytes
+    f.argtypes = [ctypes.c_int32] * 4
+    f.restype = ctypes.c_size_t
+    n = f(num_seqs, num_q_heads, num_kv_heads, max_query_len)
+    if n == 0:
+        raise ValueError("invalid sizes for the prefill workspace")
+    return int(n)
+
+
+def paged_attn_prefill(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, block_tables: torch.Tensor,
+                       context_lens: torch.Tensor, query_start: torch.Tensor, scale: float, num_kv_heads: int,
+                       out: torch.Tensor, max_query_len: int, max_context_len: int,
+                       workspace: Optional[torch.Tensor] = None, stream=None) -> None:
+    """Chunked-prefill attention: query row i of sequence s's chunk (rows
+    query_start[s]..query_start[s+1]-1) sits at position ctx - q_len + i and
+    attends to positions [0, pos] read through block_tables[s]."""
+    for t, n in ((q, "q"), (k_cache, "k_cache"), (v_cache, "v_cache"), (out, "out")):
+        _need(t, n, torch.bfloat16)
+    for t, n in ((block_tables, "block_tables"), (context_lens, "context_lens"), (query_start, "query_start")):
+        _need(t, n, torch.int32)
+    T, Hq, D = q.shape
+    B = context_lens.shape[0]
+    if out.shape != q.shape or query_start.shape != (B + 1,) or block_tables.shape[0] != B:
+        raise ValueError("shape mismatch among q/out, query_start [B+1], block_tables [B, MBS]")
+    if workspace is None:
+        workspace = torch.empty(prefill_workspace_bytes(B, Hq, num_kv_heads, max_query_len), dtype=torch.uint8,
+                                device=q.device)
+    lib = load_library()
+    f = lib.paged_attn_prefill
+    if f.argtypes is None:
+        P, I32, F, SZ = ctypes.c_void_p, ctypes.c_int32, ctypes.c_float, ctypes.c_size_t
+        f.argtypes = [P, P, P, P, I32, P, P, I32, I32, F, I32, P, _Pool, I32, I32, P, SZ, P]
+        f.restype = ctypes.c_int
+    st = f(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables), block_tables.shape[1], _ptr(context_lens),
+           _ptr(query_start), B, Hq, float(scale), int(num_kv_heads), _ptr(out), _pool(k_cache), int(max_query_len),
+           int(max_context_len), _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(st, "paged_attn_prefill")

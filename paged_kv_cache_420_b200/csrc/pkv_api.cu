@@ -14,6 +14,7 @@
 
 #include "decode.cuh"
 #include "pkv.h"
+#include "prefill.cuh"
 #include "write_copy.cuh"
 
 namespace {
@@ -183,6 +184,54 @@ pkv_status dispatch_group(int g, const pkv::DecodeParams &prm, const CUtensorMap
     return launch_decode<D, 1, 1, 16>(prm, mk, mv, stream, dev);
 }
 
+// -------------------------------------------------------- prefill ----
+
+int prefill_query_tile(int g) { return pkv::kPrefillRows / g; }
+
+bool prefill_layout(int32_t B, int32_t g, int32_t max_q, size_t *off_entries, size_t *total) {
+    if (B < 0 || g <= 0 || max_q < 0) return false;
+    const int QT = prefill_query_tile(g);
+    const long long max_tiles = std::max<long long>(1, ((long long)max_q + QT - 1) / QT);
+    *off_entries = 256;
+    *total = 256 + round256((size_t)B * max_tiles * sizeof(int2));
+    return true;
+}
+
+template <int D>
+pkv_status launch_prefill(const pkv::PrefillParams &prm, const CUtensorMap &mk, const CUtensorMap &mv,
+                          cudaStream_t stream, int dev) {
+    constexpr int NS = 8;
+    using L = pkv::PrefillSmem<D, NS>;
+    auto kernel = pkv::paged_prefill_kernel<D, NS>;
+    static int occ_cache[kMaxDevices] = {0};
+    int occ = (dev >= 0 && dev < kMaxDevices) ? occ_cache[dev] : 0;
+    if (occ == 0) {
+        if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kBytes) != cudaSuccess)
+            return PKV_ECUDA;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kernel, pkv::kDecodeThreads, L::kBytes) !=
+                cudaSuccess ||
+            occ <= 0)
+            return PKV_ECUDA;
+        if (dev >= 0 && dev < kMaxDevices) occ_cache[dev] = occ;
+    }
+    const long long tiles = std::max<long long>(1, ((long long)prm.max_q + prm.QT - 1) / prm.QT);
+    const long long items_upper = (long long)prm.B * tiles * prm.Hkv;
+    const long long grid = std::max<long long>(1, std::min<long long>(items_upper, (long long)sm_count(dev) * occ));
+    cudaLaunchConfig_t cfg;
+    std::memset(&cfg, 0, sizeof cfg);
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3(pkv::kDecodeThreads);
+    cfg.dynamicSmemBytes = L::kBytes;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, kernel, mk, mv, prm) != cudaSuccess) return PKV_ECUDA;
+    return launch_status();
+}
+
 }  // namespace
 
 extern "C" {
@@ -337,6 +386,68 @@ pkv_status paged_attn_decode(const void *q, const void *k_cache, const void *v_c
     if (r != PKV_OK) return r;
     const int dev = current_device();
     return D == 128 ? dispatch_group<128>(g, prm, mk, mv, st, dev) : dispatch_group<64>(g, prm, mk, mv, st, dev);
+}
+
+size_t pkv_prefill_workspace_bytes(int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads,
+                                   int32_t max_query_len) {
+    if (num_kv_heads <= 0 || num_q_heads <= 0 || num_q_heads % num_kv_heads) return 0;
+    size_t off, total;
+    if (!prefill_layout(num_seqs, num_q_heads / num_kv_heads, max_query_len, &off, &total)) return 0;
+    return total;
+}
+
+pkv_status paged_attn_prefill(const void *q, const void *k_cache, const void *v_cache, const int32_t *block_tables,
+                              int32_t max_blocks_per_seq, const int32_t *context_lens, const int32_t *query_start,
+                              int32_t num_seqs, int32_t num_q_heads, float scale, int32_t num_kv_heads, void *out,
+                              pkv_pool pool, int32_t max_query_len, int32_t max_context_len, void *workspace,
+                              size_t workspace_bytes, pkv_stream_t stream) {
+    const pkv_status ps = check_pool(pool);
+    if (ps != PKV_OK) return ps;
+    if (num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || max_blocks_per_seq <= 0 || max_context_len < 0 ||
+        max_query_len < 0)
+        return PKV_EINVAL;
+    if (num_kv_heads != pool.num_kv_heads || num_q_heads % num_kv_heads != 0) return PKV_EINVAL;
+    const int g = num_q_heads / num_kv_heads;
+    if (g > 16) return PKV_EUNSUPPORTED;
+    if (num_seqs == 0 || max_query_len == 0) return PKV_OK;
+    if (!q || !k_cache || !v_cache || !block_tables || !context_lens || !query_start || !out || !workspace)
+        return PKV_EINVAL;
+    if (!aligned(q, 16) || !aligned(out, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) ||
+        !aligned(block_tables, 4) || !aligned(context_lens, 4) || !aligned(query_start, 4) || !aligned(workspace, 256))
+        return PKV_EINVAL;
+    size_t off_entries, total;
+    if (!prefill_layout(num_seqs, g, max_query_len, &off_entries, &total) || workspace_bytes < total)
+        return PKV_EINVAL;
+    pkv::PrefillParams prm;
+    prm.q = static_cast<const __nv_bfloat16 *>(q);
+    prm.out = static_cast<__nv_bfloat16 *>(out);
+    prm.block_tables = block_tables;
+    prm.context_lens = context_lens;
+    prm.query_start = query_start;
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    prm.num_entries = reinterpret_cast<int32_t *>(ws);
+    prm.work_counter = reinterpret_cast<int32_t *>(ws) + 1;
+    prm.entries = reinterpret_cast<int2 *>(ws + off_entries);
+    prm.B = num_seqs;
+    prm.Hq = num_q_heads;
+    prm.Hkv = num_kv_heads;
+    prm.g = g;
+    prm.MBS = max_blocks_per_seq;
+    prm.bs = pool.block_size;
+    prm.NB = pool.num_blocks;
+    prm.max_ctx = max_context_len;
+    prm.max_q = max_query_len;
+    prm.QT = prefill_query_tile(g);
+    prm.pool_rows = pool.num_blocks * pool.num_kv_heads * pool.block_size;
+    prm.scale_log2 = scale * 1.4426950408889634f;
+    CUtensorMap mk, mv;
+    if (!encode_pool_map(&mk, k_cache, pool) || !encode_pool_map(&mv, v_cache, pool)) return PKV_ECUDA;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    pkv::plan_prefill_kernel<<<1, pkv::kPlanThreads, 0, st>>>(prm);
+    const pkv_status r = launch_status();
+    if (r != PKV_OK) return r;
+    const int dev = current_device();
+    return pool.head_dim == 128 ? launch_prefill<128>(prm, mk, mv, st, dev) : launch_prefill<64>(prm, mk, mv, st, dev);
 }
 
 pkv_status pkv_get_device_error(int32_t *code_out, pkv_stream_t stream) {

@@ -1,0 +1,85 @@
+"""GPU parity of chunked-prefill paged attention against the fp64 oracle.
+
+Cases span query tiles (64 rows = tokens x GQA group), chunks shorter and
+longer than a tile, prefixes that are empty or end mid-block, every GQA group
+size 1..16 (including ones that do not divide a tile), both head dims,
+several block sizes and poisoned unused pool rows.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import paged_kv_cache_420_b200 as pkv
+import workloads
+from tests._gpu_util import assert_attention_close, bits_equal, no_device_error
+
+pytestmark = pytest.mark.gpu
+
+
+def run_prefill(w):
+    for name in ("q", "k_new", "v_new", "k_cache", "v_cache"):
+        setattr(w, name, getattr(w, name).to("cuda").contiguous())
+    kc, vc = w.k_cache.clone(), w.v_cache.clone()
+    pkv.pkv_write(w.k_new, w.v_new, torch.from_numpy(w.slot_mapping).cuda(), kc, vc)
+    out = torch.full_like(w.q, float("nan"))
+    pkv.paged_attn_prefill(w.q, kc, vc, torch.from_numpy(w.block_tables).cuda(),
+                           torch.from_numpy(w.context_lens).cuda(), torch.from_numpy(w.query_start).cuda(),
+                           w.scale, w.num_kv_heads, out, w.max_query_len, w.max_context_len)
+    torch.cuda.synchronize()
+    return kc, vc, out
+
+
+CASES = [
+    # prefix lens, chunk lens, Hq, Hkv, D, bs
+    ([0, 5, 40], [7, 16, 33], 4, 4, 64, 16),
+    ([0, 100, 17], [64, 65, 130], 8, 8, 128, 16),        # MHA, tiles of 64 tokens
+    ([300, 0, 33], [200, 129, 1], 32, 8, 128, 16),       # g = 4: 16-token tiles
+    ([1000, 7], [100, 63], 64, 8, 128, 128),             # g = 8, bs 128
+    ([50, 0], [31, 17], 12, 4, 64, 32),                  # g = 3: 21-token tiles (one padding row)
+    ([17, 260], [40, 9], 32, 2, 128, 16),                # g = 16
+    ([0], [256], 2, 1, 128, 16),                         # g = 2, whole-sequence prefill
+    ([2000, 15, 16], [1, 1, 1], 8, 4, 128, 16),          # single-token chunks (= decode)
+]
+
+
+@pytest.mark.parametrize("prefix,chunk,Hq,Hkv,D,bs", CASES)
+@pytest.mark.parametrize("poison", [False, True])
+def test_prefill_parity(prefix, chunk, Hq, Hkv, D, bs, poison):
+    w = workloads.make_prefill_custom(prefix, chunk, Hq, Hkv, D, bs, seed=sum(prefix) + Hq + D, poison=poison)
+    kc, vc, out = run_prefill(w)
+    okc, ovc = oracle.kv_write(w.k_cache, w.v_cache, w.k_new, w.v_new, w.slot_mapping)
+    assert bits_equal(kc, okc)
+    ref = oracle.paged_prefill(w.q, okc, ovc, w.block_tables, w.context_lens, w.query_start, w.scale)
+    assert_attention_close(out, ref, f"prefix={prefix} chunk={chunk} g={Hq // Hkv} D={D} bs={bs}")
+    no_device_error()
+
+
+def test_prefill_single_token_equals_decode_kernel():
+    w = workloads.make_prefill_custom([300, 1000, 0], [1, 1, 1], 32, 8, 128, 16, seed=9)
+    kc, vc, out = run_prefill(w)
+    dec = torch.empty_like(out)
+    pkv.paged_attn_decode(w.q, kc, vc, torch.from_numpy(w.block_tables).cuda(),
+                          torch.from_numpy(w.context_lens).cuda(), w.scale, w.num_kv_heads, dec, w.max_context_len)
+    torch.cuda.synchronize()
+    assert (out.float() - dec.float()).abs().max().item() <= 2e-2
+
+
+@pytest.mark.parametrize("name", workloads.PREFILL_WORKLOADS)
+def test_named_prefill_workload_full_size(name):
+    w = workloads.make_prefill(name, seed=0, values_device="cuda")
+    kc0, vc0 = w.k_cache.cpu(), w.v_cache.cpu()
+    kc, vc, out = run_prefill(w)
+    no_device_error()
+    assert torch.isfinite(out.float()).all()
+    okc, ovc = oracle.kv_write(kc0, vc0, w.k_new, w.v_new, w.slot_mapping)
+    assert bits_equal(kc, okc) and bits_equal(vc, ovc)
+    # sampled rows: the first and last 32 query rows of two sequences
+    rows = np.concatenate([np.arange(s0, s0 + 32) for s0 in (int(w.query_start[1]), int(w.query_start[6]) - 32)])
+    sub_q = w.q[torch.from_numpy(rows).cuda()]
+    # oracle on single-row chunks with the rows' own context lengths
+    seq_of = np.searchsorted(w.query_start, rows, side="right") - 1
+    ctx = (w.context_lens[seq_of] - (w.query_start[seq_of + 1] - rows) + 1).astype(np.int32)
+    qs = np.arange(len(rows) + 1, dtype=np.int32)
+    ref = oracle.paged_prefill(sub_q, okc, ovc, w.block_tables[seq_of], ctx, qs, w.scale)
+    assert_attention_close(out[torch.from_numpy(rows).cuda()], ref, name)
