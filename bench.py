@@ -38,8 +38,7 @@ import workloads  # noqa: E402
 
 FALLBACK_HBM_GBS = 6650.0
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "decode_traffic.txt")
-DECODE_SOURCES = ["paged_kv_cache_420_b200/csrc/decode.cuh", "paged_kv_cache_420_b200/csrc/pkv_api.cu",
-                  "paged_kv_cache_420_b200/csrc/ptx.cuh"]
+DECODE_SOURCES = ["paged_kv_cache_420_b200/csrc/decode.cuh", "paged_kv_cache_420_b200/csrc/ptx.cuh"]
 
 
 # --------------------------------------------------------------------------
