@@ -211,20 +211,23 @@ size_t pkv_prefill_workspace_bytes(int32_t num_seqs, int32_t num_q_heads, int32_
  *   out[t][hq] = sum_{j <= pos} softmax_j(scale * <q[t][hq], K_j>) V_j
  * in fp32 with bf16 (nearest-even) output.  decode is the case q_len = 1.
  *
- *   q, out        bf16 [T][num_q_heads][head_dim], T = query_start[num_seqs], 16-B aligned
+ *   q, out        bf16 [num_tokens][num_q_heads][head_dim], 16-B aligned; query_start[num_seqs]
+ *                 <= num_tokens (rows past query_start[num_seqs] are neither read as queries nor written)
  *   query_start   int32 [num_seqs + 1], non-decreasing, query_start[0] = 0
  *   context_lens  int32 [num_seqs]; q_len <= context_len
  *   max_query_len / max_context_len  host upper bounds (size the work list)
  *   workspace     at least pkv_prefill_workspace_bytes(...), 256-B aligned
  * A query length above its context or the bounds sets PKV_DEVERR_CONTEXT and is
  * clamped (rows past the clamp are not written).  Launches a plan kernel and
- * the attention kernel on `stream`.
+ * the attention kernel on `stream`.  The attention kernel runs on the
+ * tcgen05 tensor cores: tiles of 128 query rows (query token x head of the GQA
+ * group), 64-key blocks, accumulators in tensor memory; one CTA per SM.
  */
 pkv_status paged_attn_prefill(const void *q, const void *k_cache, const void *v_cache,
                               const int32_t *block_tables, int32_t max_blocks_per_seq,
                               const int32_t *context_lens, const int32_t *query_start, int32_t num_seqs,
-                              int32_t num_q_heads, float scale, int32_t num_kv_heads, void *out,
-                              pkv_pool pool, int32_t max_query_len, int32_t max_context_len,
+                              int32_t num_tokens, int32_t num_q_heads, float scale, int32_t num_kv_heads,
+                              void *out, pkv_pool pool, int32_t max_query_len, int32_t max_context_len,
                               void *workspace, size_t workspace_bytes, pkv_stream_t stream);
 
 /*

@@ -253,9 +253,10 @@ def paged_attn_prefill(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Te
     f = lib.paged_attn_prefill
     if f.argtypes is None:
         P, I32, F, SZ = ctypes.c_void_p, ctypes.c_int32, ctypes.c_float, ctypes.c_size_t
-        f.argtypes = [P, P, P, P, I32, P, P, I32, I32, F, I32, P, _Pool, I32, I32, P, SZ, P]
+        f.argtypes = [P, P, P, P, I32, P, P, I32, I32, I32, F, I32, P, _Pool, I32, I32, P, SZ, P]
         f.restype = ctypes.c_int
     st = f(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables), block_tables.shape[1], _ptr(context_lens),
-           _ptr(query_start), B, Hq, float(scale), int(num_kv_heads), _ptr(out), _pool(k_cache), int(max_query_len),
-           int(max_context_len), _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream))
+           _ptr(query_start), B, T, Hq, float(scale), int(num_kv_heads), _ptr(out), _pool(k_cache),
+           int(max_query_len), int(max_context_len), _ptr(workspace), workspace.numel() * workspace.element_size(),
+           _stream(stream))
     _check(st, "paged_attn_prefill")

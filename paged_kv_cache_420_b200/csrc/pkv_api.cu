@@ -15,6 +15,7 @@
 #include "decode.cuh"
 #include "pkv.h"
 #include "prefill.cuh"
+#include "prefill_tc.cuh"
 #include "write_copy.cuh"
 
 namespace {
@@ -93,6 +94,22 @@ bool encode_pool_map(CUtensorMap *map, const void *base, const pkv_pool &pool) {
     cuuint32_t box[2] = {64, (cuuint32_t)pkv::kStageTok};
     cuuint32_t estr[2] = {1, 1};
     const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box,
+                          estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+// The query tensor [T][Hq][D] viewed as 3-D (columns, heads, tokens); a box is
+// 64 columns x g heads x QT tokens, so one tcgen05 prefill tile (rows = token x
+// head of the group) lands as [QT][g][64] with the 128-byte swizzle.
+bool encode_query_map(CUtensorMap *map, const void *base, int T, int Hq, int D, int g, int QT) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)Hq, (cuuint64_t)T};
+    cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)Hq * D * 2};
+    cuuint32_t box[3] = {64, (cuuint32_t)g, (cuuint32_t)QT};
+    cuuint32_t estr[3] = {1, 1, 1};
+    const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box,
                           estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
@@ -195,6 +212,38 @@ bool prefill_layout(int32_t B, int32_t g, int32_t max_q, size_t *off_entries, si
     *off_entries = 256;
     *total = 256 + round256((size_t)B * max_tiles * sizeof(int2));
     return true;
+}
+
+template <int D>
+pkv_status launch_prefill_tc(const pkv::PrefillParams &prm, const CUtensorMap &mk, const CUtensorMap &mv,
+                             const CUtensorMap &mq, cudaStream_t stream, int dev) {
+    constexpr int NKV = D == 128 ? 3 : 4;
+    using L = pkv::TcSmem<D, NKV>;
+    auto kernel = pkv::paged_prefill_tc_kernel<D, NKV>;
+    static bool attr_set[kMaxDevices] = {false};
+    if (dev >= 0 && dev < kMaxDevices && !attr_set[dev]) {
+        if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kBytes) != cudaSuccess)
+            return PKV_ECUDA;
+        attr_set[dev] = true;
+    }
+    const long long tiles = std::max<long long>(1, ((long long)prm.max_q + prm.QT - 1) / prm.QT);
+    const long long items_upper = (long long)prm.B * tiles * prm.Hkv;
+    // a CTA holds 512 tensor-memory columns at head dim 128 (one per SM), 256 at 64
+    const long long per_sm = pkv::TcTmem<D>::kCols == 512 ? 1 : 2;
+    const long long grid = std::max<long long>(1, std::min<long long>(items_upper, per_sm * sm_count(dev)));
+    cudaLaunchConfig_t cfg;
+    std::memset(&cfg, 0, sizeof cfg);
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3(pkv::kTcThreads);
+    cfg.dynamicSmemBytes = L::kBytes;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, kernel, mk, mv, mq, prm) != cudaSuccess) return PKV_ECUDA;
+    return launch_status();
 }
 
 template <int D>
@@ -398,18 +447,18 @@ size_t pkv_prefill_workspace_bytes(int32_t num_seqs, int32_t num_q_heads, int32_
 
 pkv_status paged_attn_prefill(const void *q, const void *k_cache, const void *v_cache, const int32_t *block_tables,
                               int32_t max_blocks_per_seq, const int32_t *context_lens, const int32_t *query_start,
-                              int32_t num_seqs, int32_t num_q_heads, float scale, int32_t num_kv_heads, void *out,
-                              pkv_pool pool, int32_t max_query_len, int32_t max_context_len, void *workspace,
-                              size_t workspace_bytes, pkv_stream_t stream) {
+                              int32_t num_seqs, int32_t num_tokens, int32_t num_q_heads, float scale,
+                              int32_t num_kv_heads, void *out, pkv_pool pool, int32_t max_query_len,
+                              int32_t max_context_len, void *workspace, size_t workspace_bytes, pkv_stream_t stream) {
     const pkv_status ps = check_pool(pool);
     if (ps != PKV_OK) return ps;
-    if (num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || max_blocks_per_seq <= 0 || max_context_len < 0 ||
-        max_query_len < 0)
+    if (num_seqs < 0 || num_tokens < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || max_blocks_per_seq <= 0 ||
+        max_context_len < 0 || max_query_len < 0)
         return PKV_EINVAL;
     if (num_kv_heads != pool.num_kv_heads || num_q_heads % num_kv_heads != 0) return PKV_EINVAL;
     const int g = num_q_heads / num_kv_heads;
     if (g > 16) return PKV_EUNSUPPORTED;
-    if (num_seqs == 0 || max_query_len == 0) return PKV_OK;
+    if (num_seqs == 0 || max_query_len == 0 || num_tokens == 0) return PKV_OK;
     if (!q || !k_cache || !v_cache || !block_tables || !context_lens || !query_start || !out || !workspace)
         return PKV_EINVAL;
     if (!aligned(q, 16) || !aligned(out, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) ||
@@ -437,17 +486,31 @@ pkv_status paged_attn_prefill(const void *q, const void *k_cache, const void *v_
     prm.NB = pool.num_blocks;
     prm.max_ctx = max_context_len;
     prm.max_q = max_query_len;
+#ifdef PKV_PREFILL_MMA_SYNC
     prm.QT = prefill_query_tile(g);
+#else
+    prm.QT = pkv::kTcRows / g;
+#endif
+    prm.T = num_tokens;
     prm.pool_rows = pool.num_blocks * pool.num_kv_heads * pool.block_size;
     prm.scale_log2 = scale * 1.4426950408889634f;
     CUtensorMap mk, mv;
     if (!encode_pool_map(&mk, k_cache, pool) || !encode_pool_map(&mv, v_cache, pool)) return PKV_ECUDA;
+#ifndef PKV_PREFILL_MMA_SYNC
+    CUtensorMap mq;
+    if (!encode_query_map(&mq, q, num_tokens, num_q_heads, pool.head_dim, g, prm.QT)) return PKV_ECUDA;
+#endif
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     pkv::plan_prefill_kernel<<<1, pkv::kPlanThreads, 0, st>>>(prm);
     const pkv_status r = launch_status();
     if (r != PKV_OK) return r;
     const int dev = current_device();
+#ifdef PKV_PREFILL_MMA_SYNC
     return pool.head_dim == 128 ? launch_prefill<128>(prm, mk, mv, st, dev) : launch_prefill<64>(prm, mk, mv, st, dev);
+#else
+    return pool.head_dim == 128 ? launch_prefill_tc<128>(prm, mk, mv, mq, st, dev)
+                                : launch_prefill_tc<64>(prm, mk, mv, mq, st, dev);
+#endif
 }
 
 pkv_status pkv_get_device_error(int32_t *code_out, pkv_stream_t stream) {

@@ -35,7 +35,7 @@ struct PrefillParams {
     int2 *entries;                // workspace: (seq, query tile)
     int32_t *num_entries;
     int32_t *work_counter;
-    int B, Hq, Hkv, g, MBS, bs, NB, max_ctx, max_q, QT;
+    int B, Hq, Hkv, g, MBS, bs, NB, max_ctx, max_q, QT, T;
     int pool_rows;
     float scale_log2;
 };
@@ -51,8 +51,11 @@ __device__ __forceinline__ void prefill_lengths(const PrefillParams &p, int s, b
                                                 int &prefix) {
     int ctx = __ldg(p.context_lens + s);
     const long long cap = min((long long)p.MBS * p.bs, (long long)p.max_ctx);
-    int ql = __ldg(p.query_start + s + 1) - __ldg(p.query_start + s);
+    const int q_begin = __ldg(p.query_start + s);
+    int ql = __ldg(p.query_start + s + 1) - q_begin;
     bool bad = false;
+    if (q_begin < 0 || q_begin > p.T) { bad = true; ql = 0; }
+    else if (ql > p.T - q_begin) { bad = true; ql = p.T - q_begin; }
     if (ctx < 0 || ctx > cap) { bad = true; ctx = ctx < 0 ? 0 : (int)cap; }
     if (ql < 0 || ql > p.max_q || ql > ctx) { bad = true; ql = max(0, min(min(ql, p.max_q), ctx)); }
     if (bad && report) raise_error(PKV_DEVERR_CONTEXT);

@@ -145,6 +145,12 @@ __device__ __forceinline__ void mma_bf16_16816(float &d0, float &d1, float &d2, 
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
+// Orders this thread's generic-proxy shared-memory writes before later
+// async-proxy reads (TMA, tensor core) of the same CTA.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 // Warp-wide maximum of a float (sm_100a); NaN inputs are ignored.
 __device__ __forceinline__ float warp_max_f32(float v) {
     float r;

@@ -1,9 +1,10 @@
 """GPU parity of chunked-prefill paged attention against the fp64 oracle.
 
-Cases span query tiles (64 rows = tokens x GQA group), chunks shorter and
-longer than a tile, prefixes that are empty or end mid-block, every GQA group
-size 1..16 (including ones that do not divide a tile), both head dims,
-several block sizes and poisoned unused pool rows.
+Cases span query tiles (128 rows = tokens x GQA group), chunks shorter and
+longer than a tile, prefixes that are empty or end mid-block, key counts that
+end inside a 16-key stage, GQA group sizes 1..16 (including ones that do not
+divide a tile, leaving padding rows), both head dims, several block sizes and
+poisoned unused pool rows.
 """
 import numpy as np
 import pytest
@@ -33,13 +34,16 @@ def run_prefill(w):
 CASES = [
     # prefix lens, chunk lens, Hq, Hkv, D, bs
     ([0, 5, 40], [7, 16, 33], 4, 4, 64, 16),
-    ([0, 100, 17], [64, 65, 130], 8, 8, 128, 16),        # MHA, tiles of 64 tokens
-    ([300, 0, 33], [200, 129, 1], 32, 8, 128, 16),       # g = 4: 16-token tiles
+    ([0, 100, 17], [64, 65, 130], 8, 8, 128, 16),        # MHA, 128-token tiles
+    ([300, 0, 33], [200, 129, 1], 32, 8, 128, 16),       # g = 4: 32-token tiles
     ([1000, 7], [100, 63], 64, 8, 128, 128),             # g = 8, bs 128
-    ([50, 0], [31, 17], 12, 4, 64, 32),                  # g = 3: 21-token tiles (one padding row)
+    ([50, 0], [31, 17], 12, 4, 64, 32),                  # g = 3: 42-token tiles (two padding rows)
     ([17, 260], [40, 9], 32, 2, 128, 16),                # g = 16
     ([0], [256], 2, 1, 128, 16),                         # g = 2, whole-sequence prefill
     ([2000, 15, 16], [1, 1, 1], 8, 4, 128, 16),          # single-token chunks (= decode)
+    ([0, 513], [384, 300], 8, 8, 64, 16),                # MHA head dim 64, several 128-token tiles
+    ([70], [200], 20, 4, 128, 32),                       # g = 5: 25-token tiles, 3 padding rows
+    ([129, 1], [777, 64], 14, 2, 128, 16),               # g = 7: 18-token tiles, long chunk
 ]
 
 
