@@ -215,13 +215,15 @@ size_t pkv_prefill_workspace_bytes(int32_t num_seqs, int32_t num_q_heads, int32_
  *                 <= num_tokens (rows past query_start[num_seqs] are neither read as queries nor written)
  *   query_start   int32 [num_seqs + 1], non-decreasing, query_start[0] = 0
  *   context_lens  int32 [num_seqs]; q_len <= context_len
+ *   scale         finite and > 0 (else PKV_EINVAL)
  *   max_query_len / max_context_len  host upper bounds (size the work list)
  *   workspace     at least pkv_prefill_workspace_bytes(...), 256-B aligned
  * A query length above its context or the bounds sets PKV_DEVERR_CONTEXT and is
  * clamped (rows past the clamp are not written).  Launches a plan kernel and
  * the attention kernel on `stream`.  The attention kernel runs on the
  * tcgen05 tensor cores: tiles of 128 query rows (query token x head of the GQA
- * group), 64-key blocks, accumulators in tensor memory; one CTA per SM.
+ * group), 64-key blocks, accumulators in tensor memory; two persistent CTAs
+ * per SM, each holding 256 columns of tensor memory.
  */
 pkv_status paged_attn_prefill(const void *q, const void *k_cache, const void *v_cache,
                               const int32_t *block_tables, int32_t max_blocks_per_seq,

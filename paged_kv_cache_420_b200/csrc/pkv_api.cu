@@ -8,6 +8,7 @@
 
 #include <algorithm>
 #include <cstdint>
+#include <cmath>
 #include <cstring>
 #include <mutex>
 #include <vector>
@@ -217,9 +218,8 @@ bool prefill_layout(int32_t B, int32_t g, int32_t max_q, size_t *off_entries, si
 template <int D>
 pkv_status launch_prefill_tc(const pkv::PrefillParams &prm, const CUtensorMap &mk, const CUtensorMap &mv,
                              const CUtensorMap &mq, cudaStream_t stream, int dev) {
-    constexpr int NKV = D == 128 ? 3 : 4;
-    using L = pkv::TcSmem<D, NKV>;
-    auto kernel = pkv::paged_prefill_tc_kernel<D, NKV>;
+    using L = pkv::TcSmem<D>;
+    auto kernel = pkv::paged_prefill_tc_kernel<D>;
     static bool attr_set[kMaxDevices] = {false};
     if (dev >= 0 && dev < kMaxDevices && !attr_set[dev]) {
         if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kBytes) != cudaSuccess)
@@ -228,9 +228,9 @@ pkv_status launch_prefill_tc(const pkv::PrefillParams &prm, const CUtensorMap &m
     }
     const long long tiles = std::max<long long>(1, ((long long)prm.max_q + prm.QT - 1) / prm.QT);
     const long long items_upper = (long long)prm.B * tiles * prm.Hkv;
-    // a CTA holds 512 tensor-memory columns at head dim 128 (one per SM), 256 at 64
-    const long long per_sm = pkv::TcTmem<D>::kCols == 512 ? 1 : 2;
-    const long long grid = std::max<long long>(1, std::min<long long>(items_upper, per_sm * sm_count(dev)));
+    // persistent: two CTAs per SM, each holding half of tensor memory
+    const long long grid = std::max<long long>(
+        1, std::min<long long>(items_upper, (long long)pkv::kTcCtasPerSm * sm_count(dev)));
     cudaLaunchConfig_t cfg;
     std::memset(&cfg, 0, sizeof cfg);
     cfg.gridDim = dim3((unsigned)grid);
@@ -458,6 +458,7 @@ pkv_status paged_attn_prefill(const void *q, const void *k_cache, const void *v_
     if (num_kv_heads != pool.num_kv_heads || num_q_heads % num_kv_heads != 0) return PKV_EINVAL;
     const int g = num_q_heads / num_kv_heads;
     if (g > 16) return PKV_EUNSUPPORTED;
+    if (!(scale > 0.f) || !std::isfinite(scale)) return PKV_EINVAL;
     if (num_seqs == 0 || max_query_len == 0 || num_tokens == 0) return PKV_OK;
     if (!q || !k_cache || !v_cache || !block_tables || !context_lens || !query_start || !out || !workspace)
         return PKV_EINVAL;

@@ -7,23 +7,28 @@
 // 引擎", section 3.1).  An item is (sequence, kv head, tile of 128 query rows),
 // a row being (query token, head of the GQA group).
 //
-// One CTA per SM, warp-specialised (192 threads):
-//   warp 0       producer: the item's Q tile (128 x D bf16) by a 3-D TMA load
-//                into a double buffer, and 64-key K/V blocks of the paged cache
-//                (4 stages of 16 keys, addressed through the block table) into
-//                a ring; all 128-byte swizzled.
+// Two CTAs per SM (each holds half of tensor memory and ~97 KB of shared
+// memory), warp-specialised (192 threads):
+//   warp 0       producer: the item's Q tile (128 x D bf16) by a 3-D TMA load,
+//                and 64-key K and V blocks of the paged cache (4 stages of 16
+//                keys each, addressed through the block table) into separate
+//                K and V rings; all 128-byte swizzled.  A K slot is released
+//                when its S product completes, a V slot when its PV product
+//                does, so the next K block streams in while P V still runs.
 //   warp 1       MMA issuer (one thread) and tensor-memory owner:
 //                S_j = Q K_j^T  (tcgen05.mma kind::f16, M 128, N 64, K-major
-//                smem operands, fp32 into one of two TMEM S buffers), then
+//                smem operands, fp32 into the TMEM S buffer), then
 //                O += P_j V_j   (A = P_j in TMEM, B = V_j MN-major in smem,
 //                N = D), each followed by tcgen05.commit onto an mbarrier.
-//   warps 2-5    softmax: thread r owns row r (TMEM lane r).  It loads S_j,
-//                applies the causal mask and scale, keeps the row's running
-//                max (raised lazily, as in decode) and sum, writes P_j as bf16
-//                into TMEM, rescales its O row when the max was raised (after
-//                the previous PV product has completed), and at the end of the
-//                item normalises O and stores the row.
-// S_{j+1} runs on the tensor cores while the softmax works on S_j.
+//   warps 2-5    softmax: thread r owns row r (TMEM lane r).  It loads S_j
+//                (releasing the S buffer at once), masks the diagonal block,
+//                keeps the row's running max in scaled log2 units (raised
+//                lazily, as in decode) and sum, writes P_j as bf16 into one of
+//                two TMEM P buffers, rescales its O row when the max was raised
+//                (after the previous PV product has completed), and at the end
+//                of the item normalises O and stores the row.
+// S_{j+1} runs on the tensor cores while the softmax works on S_j, and the
+// other CTA on the SM fills the gaps of this one.
 #pragma once
 
 #include "prefill.cuh"
@@ -33,35 +38,36 @@ namespace pkv {
 constexpr int kTcRows = 128;          // M: query rows per item
 constexpr int kTcKeys = 64;           // N: keys per block (4 stages of 16)
 constexpr int kTcThreads = 6 * 32;
-constexpr uint32_t kTmemS = 0;        // two S buffers: columns [0, 64) and [64, 128)
-constexpr uint32_t kTmemP = 128;      // two P buffers (bf16 pairs): [128, 160) and [160, 192)
-
-// O follows the P buffers; the allocation is the next power of two (head dim
-// 64 takes half of tensor memory, so two CTAs may share an SM).
-template <int D>
-struct TcTmem {
-    static constexpr uint32_t kO = D == 64 ? 192 : 256;
-    static constexpr uint32_t kCols = D == 64 ? 256 : 512;
-};
+constexpr int kTcCtasPerSm = 2;
+// Tensor memory of one CTA (256 of the SM's 512 columns):
+constexpr uint32_t kTmemCols = 256;
+constexpr uint32_t kTmemS = 0;        // S: fp32, columns [0, 64)
+constexpr uint32_t kTmemP = 64;       // two P buffers (bf16 pairs): [64, 96) and [96, 128)
+constexpr uint32_t kTmemO = 128;      // O: fp32, [128, 128 + D)
 
 struct TcItem {
     int s, h, tile, q_len, prefix, q0, n_keys, n_blocks;
 };
 
-template <int D, int NKV>
+// Shared memory of one CTA: NQ query buffers, NK-slot K and V rings.
+template <int D>
 struct TcSmem {
     static constexpr int kHalves = D / 64;
+    static constexpr int NQ = D == 128 ? 1 : 2;
+    static constexpr int NK = D == 128 ? 2 : 4;
     static constexpr int kQHalf = kTcRows * 128;          // 16 KB: 128 rows x 64 columns
     static constexpr int kQBuf = kHalves * kQHalf;
     static constexpr int kKVHalf = kTcKeys * 128;         // 8 KB: 64 keys x 64 columns
-    static constexpr int kSlot = 2 * kHalves * kKVHalf;   // K halves then V halves
+    static constexpr int kSlot = kHalves * kKVHalf;       // one K (or V) block
     static constexpr int oQ = 0;
-    static constexpr int oKV = 2 * kQBuf;
-    static constexpr int oBars = oKV + NKV * kSlot;
-    // full[NKV], empty[NKV], qfull[2], qempty[2], sfull[2], sfree[2], pfull[2], odone, drain
-    static constexpr int kNumBars = 2 * NKV + 12;
+    static constexpr int oK = NQ * kQBuf;
+    static constexpr int oV = oK + NK * kSlot;
+    static constexpr int oBars = oV + NK * kSlot;
+    // kfull, kempty, vfull, vempty [NK]; qfull, qempty [NQ]; sfull, sfree,
+    // pfull[2], odone, drain
+    static constexpr int kNumBars = 4 * NK + 2 * NQ + 6;
     static constexpr int oItem = oBars + kNumBars * 8;
-    static constexpr int oTmemSlot = oItem + 2 * (int)sizeof(TcItem);
+    static constexpr int oTmemSlot = oItem + NQ * (int)sizeof(TcItem);
     static constexpr int oAbort = oTmemSlot + 16;
     static constexpr int kBytes = oAbort + 16;
 };
@@ -150,6 +156,92 @@ __device__ __forceinline__ void tma_load_3d_u32(uint32_t smem_dst, const CUtenso
         : "memory");
 }
 
+// 2^x on the special-function unit, flushing subnormal results to zero (a
+// probability below 2^-126 of the row maximum contributes nothing in bf16).
+__device__ __forceinline__ float ex2_ftz(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// Packed pair (a0, a1) = (b0 * c + d, b1 * c + d).
+__device__ __forceinline__ void ffma2_bcast(float &a0, float &a1, float b0, float b1, float c, float d) {
+    asm("{\n\t.reg .b64 pa, pb, pc, pd;\n\t"
+        "mov.b64 pb, {%2, %3};\n\t"
+        "mov.b64 pc, {%4, %4};\n\t"
+        "mov.b64 pd, {%5, %5};\n\t"
+        "fma.rn.f32x2 pa, pb, pc, pd;\n\t"
+        "mov.b64 {%0, %1}, pa;\n\t}"
+        : "=f"(a0), "=f"(a1)
+        : "f"(b0), "f"(b1), "f"(c), "f"(d));
+}
+
+// Packed pair (d0, d1) = (a0 * b0 + c0, a1 * b1 + c1).
+__device__ __forceinline__ void ffma2(float &d0, float &d1, float a0, float a1, float b0, float b1, float c0,
+                                      float c1) {
+    asm("{\n\t.reg .b64 pa, pb, pc, pd;\n\t"
+        "mov.b64 pa, {%2, %3};\n\t"
+        "mov.b64 pb, {%4, %5};\n\t"
+        "mov.b64 pc, {%6, %7};\n\t"
+        "fma.rn.f32x2 pd, pa, pb, pc;\n\t"
+        "mov.b64 {%0, %1}, pd;\n\t}"
+        : "=f"(d0), "=f"(d1)
+        : "f"(a0), "f"(a1), "f"(b0), "f"(b1), "f"(c0), "f"(c1));
+}
+
+__device__ __forceinline__ float fmax3f(float a, float b, float c) {
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
+// 2^x for a pair, x <= 64, on the FMA and integer pipes instead of the
+// special-function unit (which the softmax otherwise saturates):
+//   x = j + f, j = round(x) (by adding 1.5 * 2^23, which leaves j in the low
+//   mantissa bits), f = x - j in [-0.5, 0.5] exactly;
+//   2^f ~ c0 + f (c1 + f (c2 + f c3)), the relative-error minimax cubic on
+//   [-0.5, 0.5] (Remez exchange; fit_exp2_poly.py beside this file), max
+//   relative error 7.5e-5, far below bf16's 2^-9;
+//   2^j is added to the exponent field.
+// x is clamped to -126 first, so masked scores (-inf) give 2^-126 and the
+// exponent field cannot underflow.
+constexpr float kExp2C0 = 0.9999280571937561f;
+constexpr float kExp2C1 = 0.6932609677314758f;
+constexpr float kExp2C2 = 0.2426111251115799f;
+constexpr float kExp2C3 = 0.0551716685295105f;
+constexpr float kRoundMagic = 12582912.0f;  // 1.5 * 2^23
+
+__device__ __forceinline__ void exp2_poly2(float x0, float x1, float &y0, float &y1) {
+    x0 = fmaxf(x0, -126.f);
+    x1 = fmaxf(x1, -126.f);
+    float t0, t1, j0, j1, f0, f1, p0, p1;
+    ffma2(t0, t1, x0, x1, 1.f, 1.f, kRoundMagic, kRoundMagic);     // t = x + M (round to integer)
+    ffma2(j0, j1, t0, t1, 1.f, 1.f, -kRoundMagic, -kRoundMagic);   // j = t - M
+    ffma2(f0, f1, j0, j1, -1.f, -1.f, x0, x1);                     // f = x - j
+    ffma2(p0, p1, f0, f1, kExp2C3, kExp2C3, kExp2C2, kExp2C2);
+    ffma2(p0, p1, p0, p1, f0, f1, kExp2C1, kExp2C1);
+    ffma2(p0, p1, p0, p1, f0, f1, kExp2C0, kExp2C0);
+    y0 = __uint_as_float(__float_as_uint(p0) + (__float_as_uint(t0) << 23));
+    y1 = __uint_as_float(__float_as_uint(p1) + (__float_as_uint(t1) << 23));
+}
+
+// Every kExpEmuEvery-th pair of scores takes exp2_poly2 (0: none).
+#ifndef PKV_TC_EXP_EMU
+#define PKV_TC_EXP_EMU 0
+#endif
+constexpr int kExpEmuEvery = PKV_TC_EXP_EMU;
+
+// Packed pair (a0, a1) += (b0, b1).
+__device__ __forceinline__ void fadd2(float &a0, float &a1, float b0, float b1) {
+    asm("{\n\t.reg .b64 pa, pb;\n\t"
+        "mov.b64 pa, {%0, %1};\n\t"
+        "mov.b64 pb, {%2, %3};\n\t"
+        "add.rn.f32x2 pa, pa, pb;\n\t"
+        "mov.b64 {%0, %1}, pa;\n\t}"
+        : "+f"(a0), "+f"(a1)
+        : "f"(b0), "f"(b1));
+}
+
 // Item geometry shared by the three roles.
 __device__ __forceinline__ TcItem tc_item(const PrefillParams &p, int it) {
     TcItem t;
@@ -166,12 +258,12 @@ __device__ __forceinline__ TcItem tc_item(const PrefillParams &p, int it) {
     return t;
 }
 
-template <int D, int NKV>
-__global__ void __launch_bounds__(kTcThreads, 1) paged_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmap_k,
-                                                                         const __grid_constant__ CUtensorMap tmap_v,
-                                                                         const __grid_constant__ CUtensorMap tmap_q,
-                                                                         const PrefillParams p) {
-    using L = TcSmem<D, NKV>;
+template <int D>
+__global__ void __launch_bounds__(kTcThreads, kTcCtasPerSm)
+    paged_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v,
+                            const __grid_constant__ CUtensorMap tmap_q, const PrefillParams p) {
+    using L = TcSmem<D>;
+    constexpr int NQ = L::NQ, NK = L::NK;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     if ((smem_u32(smem_raw) & 1023u) != 0) {
         if (threadIdx.x == 0) raise_error(PKV_DEVERR_LAYOUT);
@@ -179,11 +271,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) paged_prefill_tc_kernel(const _
     }
     uint8_t *smem = smem_raw;
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L::oBars);
-    uint64_t *full = bars, *empty = bars + NKV;
-    uint64_t *qfull = bars + 2 * NKV, *qempty = qfull + 2;
-    uint64_t *sfull = qempty + 2, *sfree = sfull + 2, *pfull = sfree + 2, *odone = pfull + 2, *drain = odone + 1;
-    constexpr uint32_t kTmemO = TcTmem<D>::kO;
-    constexpr uint32_t kTmemCols = TcTmem<D>::kCols;
+    uint64_t *kfull = bars, *kempty = bars + NK, *vfull = bars + 2 * NK, *vempty = bars + 3 * NK;
+    uint64_t *qfull = bars + 4 * NK, *qempty = qfull + NQ;
+    uint64_t *sfull = qempty + NQ, *sfree = sfull + 1, *pfull = sfree + 1, *odone = pfull + 2, *drain = odone + 1;
     TcItem *items = reinterpret_cast<TcItem *>(smem + L::oItem);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::oTmemSlot);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::oAbort);
@@ -191,16 +281,22 @@ __global__ void __launch_bounds__(kTcThreads, 1) paged_prefill_tc_kernel(const _
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     if (threadIdx.x == 0) {
-        for (int i = 0; i < NKV; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); }
-        for (int i = 0; i < 2; ++i) {
+        for (int i = 0; i < NK; ++i) {
+            mbar_init(&kfull[i], 1);
+            mbar_init(&kempty[i], 1);
+            mbar_init(&vfull[i], 1);
+            mbar_init(&vempty[i], 1);
+        }
+        for (int i = 0; i < NQ; ++i) {
             mbar_init(&qfull[i], 1);
             // released by the MMA's commit (Q read) and by every softmax
             // thread once it has taken the item description
             mbar_init(&qempty[i], 1 + kTcRows);
-            mbar_init(&sfull[i], 1);
-            mbar_init(&sfree[i], kTcRows);
-            mbar_init(&pfull[i], kTcRows);
         }
+        mbar_init(sfull, 1);
+        mbar_init(sfree, kTcRows);
+        mbar_init(&pfull[0], kTcRows);
+        mbar_init(&pfull[1], kTcRows);
         mbar_init(odone, 1);
         mbar_init(drain, 1);
         *abort_flag = 0;
@@ -210,7 +306,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) paged_prefill_tc_kernel(const _
         tma_prefetch_desc(&tmap_q);
     }
     // Q buffers start as zeros: rows a tile does not fill stay finite.
-    for (int i = threadIdx.x; i < 2 * L::kQBuf / 16; i += kTcThreads)
+    for (int i = threadIdx.x; i < NQ * L::kQBuf / 16; i += kTcThreads)
         reinterpret_cast<uint4 *>(smem + L::oQ)[i] = make_uint4(0, 0, 0, 0);
     fence_proxy_async_smem();
     if (warp == 1) {
@@ -227,16 +323,16 @@ __global__ void __launch_bounds__(kTcThreads, 1) paged_prefill_tc_kernel(const _
 
     if (warp == 0) {
         // ------------------------------------------------------ producer --
-        uint32_t gs = 0;  // KV slots filled
-        int q_issued = -1;  // ord of the last Q tile load
+        uint32_t gk = 0, gv = 0;  // K and V blocks issued
+        int q_issued = -1;        // ord of the last Q tile load
         bool ok = true;
         int claimed = 0;
         if (lane == 0) claimed = atomicAdd(p.work_counter, 1);
         int it = __shfl_sync(0xffffffffu, claimed, 0);
         for (int ord = 0; ok; ++ord) {
-            const int qb = ord & 1;
+            const int qb = ord % NQ;
             if (lane == 0) {
-                ok = wait_or_abort(&qempty[qb], ((ord >> 1) & 1) ^ 1, abort_flag);
+                ok = wait_or_abort(&qempty[qb], ((ord / NQ) & 1) ^ 1, abort_flag);
                 if (ok) {
                     TcItem t;
                     if (it < n_items) t = tc_item(p, it);
@@ -260,101 +356,104 @@ __global__ void __launch_bounds__(kTcThreads, 1) paged_prefill_tc_kernel(const _
             if (lane == 0) claimed = atomicAdd(p.work_counter, 1);
             const TcItem t = tc_item(p, it);
             for (int j = 0; j < t.n_blocks && ok; ++j) {
-                const uint32_t slot = gs % NKV;
-                if (lane == 0) {
-                    ok = wait_or_abort(&empty[slot], ((gs / NKV) & 1) ^ 1, abort_flag);
-                    if (ok) mbar_arrive_expect_tx(&full[slot], (uint32_t)L::kSlot);
+                // lane < 4: stage of 16 keys within the block; stages past the
+                // keys read rows beyond the pool (zero fill)
+                int row = p.pool_rows;
+                const int tok = j * kTcKeys + (lane & 3) * kStageTok;
+                if (lane < 4 && tok < t.n_keys) {
+                    const int blk = __ldg(p.block_tables + (size_t)t.s * p.MBS + tok / p.bs);
+                    if (blk >= 0 && blk < p.NB) row = (blk * p.Hkv + t.h) * p.bs + tok % p.bs;
+                    else raise_error(PKV_DEVERR_BLOCK);
                 }
-                ok = __shfl_sync(0xffffffffu, ok, 0);
-                __syncwarp();
-                if (ok && lane < 4) {
-                    // lane = stage of 16 keys within the block; stages past the
-                    // keys read rows beyond the pool (zero fill)
-                    const int tok = j * kTcKeys + lane * kStageTok;
-                    int row = p.pool_rows;
-                    if (tok < t.n_keys) {
-                        const int blk = __ldg(p.block_tables + (size_t)t.s * p.MBS + tok / p.bs);
-                        if (blk >= 0 && blk < p.NB) row = (blk * p.Hkv + t.h) * p.bs + tok % p.bs;
-                        else raise_error(PKV_DEVERR_BLOCK);
-                    }
-                    const uint32_t kdst = sbase + L::oKV + slot * L::kSlot + lane * (kStageTok * 128);
 #pragma unroll
-                    for (int hf = 0; hf < L::kHalves; ++hf) {
-                        tma_load_2d_u32(kdst + hf * L::kKVHalf, &tmap_k, &full[slot], hf * 64, row);
-                        tma_load_2d_u32(kdst + (L::kHalves + hf) * L::kKVHalf, &tmap_v, &full[slot], hf * 64, row);
+                for (int kv = 0; kv < 2 && ok; ++kv) {
+                    const uint32_t g = kv ? gv : gk;
+                    const uint32_t slot = g % NK;
+                    uint64_t *fb = kv ? &vfull[slot] : &kfull[slot];
+                    if (lane == 0) {
+                        ok = wait_or_abort(kv ? &vempty[slot] : &kempty[slot], ((g / NK) & 1) ^ 1, abort_flag);
+                        if (ok) mbar_arrive_expect_tx(fb, (uint32_t)L::kSlot);
+                    }
+                    ok = __shfl_sync(0xffffffffu, ok, 0);
+                    if (ok && lane < 4) {
+                        const uint32_t dst = sbase + (kv ? L::oV : L::oK) + slot * L::kSlot + lane * (kStageTok * 128);
+#pragma unroll
+                        for (int hf = 0; hf < L::kHalves; ++hf)
+                            tma_load_2d_u32(dst + hf * L::kKVHalf, kv ? &tmap_v : &tmap_k, fb, hf * 64, row);
+                    }
+                    if (ok) {
+                        if (kv) ++gv;
+                        else ++gk;
                     }
                 }
-                if (ok) ++gs;
             }
             it = __shfl_sync(0xffffffffu, claimed, 0);
         }
         // After an abort, loads this CTA issued must land before it exits.
         if (lane == 0 && *abort_flag) {
-            for (uint32_t c = (gs > (uint32_t)NKV ? gs - NKV : 0); c < gs; ++c)
-                mbar_wait_bounded(&full[c % NKV], (c / NKV) & 1, kWaitLimitNs);
-            if (q_issued >= 0) mbar_wait_bounded(&qfull[q_issued & 1], (q_issued >> 1) & 1, kWaitLimitNs);
+            for (uint32_t c = (gk > (uint32_t)NK ? gk - NK : 0); c < gk; ++c)
+                mbar_wait_bounded(&kfull[c % NK], (c / NK) & 1, kWaitLimitNs);
+            for (uint32_t c = (gv > (uint32_t)NK ? gv - NK : 0); c < gv; ++c)
+                mbar_wait_bounded(&vfull[c % NK], (c / NK) & 1, kWaitLimitNs);
+            if (q_issued >= 0) mbar_wait_bounded(&qfull[q_issued % NQ], ((q_issued / NQ) & 1), kWaitLimitNs);
         }
     } else if (warp == 1) {
         // ---------------------------------------------------------- MMA --
-        uint32_t gs = 0, gb = 0;  // KV slots consumed, blocks processed
+        uint32_t gb = 0;  // blocks processed (K and V slots advance with it)
         bool ok = true;
         const uint32_t idesc_s = umma_idesc_bf16(kTcRows, kTcKeys, false);
         const uint32_t idesc_o = umma_idesc_bf16(kTcRows, D, true);
         for (int ord = 0; ok; ++ord) {
-            const int qb = ord & 1;
-            ok = wait_or_abort(&qfull[qb], (ord >> 1) & 1, abort_flag);
-            ok = __all_sync(0xffffffffu, ok);
+            const int qb = ord % NQ;
+            ok = __all_sync(0xffffffffu, wait_or_abort(&qfull[qb], (ord / NQ) & 1, abort_flag));
             if (!ok) break;
             const int nb = items[qb].n_blocks;
             if (nb < 0) break;
             tc_fence_after();
             const uint32_t qaddr = sbase + L::oQ + qb * L::kQBuf;
             for (int j = 0; j <= nb && ok; ++j) {
-                if (j < nb) {
-                    // S_j = Q K_j^T into S buffer gb % 2
-                    const uint32_t slot = gs % NKV;
-                    const uint32_t sb = gb & 1;
-                    if (lane == 0) {
-                        ok = wait_or_abort(&full[slot], (gs / NKV) & 1, abort_flag) &&
-                             wait_or_abort(&sfree[sb], ((gb >> 1) & 1) ^ 1, abort_flag);
-                        if (ok) {
-                            tc_fence_after();
-                            const uint32_t kaddr = sbase + L::oKV + slot * L::kSlot;
+                if (j < nb && lane == 0) {
+                    // S_j = Q K_j^T
+                    const uint32_t slot = gb % NK;
+                    ok = wait_or_abort(&kfull[slot], (gb / NK) & 1, abort_flag) &&
+                         wait_or_abort(sfree, (gb & 1) ^ 1, abort_flag);
+                    if (ok) {
+                        tc_fence_after();
+                        const uint32_t kaddr = sbase + L::oK + slot * L::kSlot;
 #pragma unroll
-                            for (int kk = 0; kk < D / 16; ++kk) {
-                                const uint32_t off = (kk >> 2) * L::kQHalf + (kk & 3) * 32;
-                                const uint32_t koff = (kk >> 2) * L::kKVHalf + (kk & 3) * 32;
-                                umma_ss(tmem + kTmemS + sb * kTcKeys, umma_desc_sw128(qaddr + off, 16, 1024),
-                                        umma_desc_sw128(kaddr + koff, 16, 1024), idesc_s, kk > 0);
-                            }
-                            umma_commit(&sfull[sb]);
-                            if (j == nb - 1) umma_commit(&qempty[qb]);  // Q no longer read
+                        for (int kk = 0; kk < D / 16; ++kk) {
+                            const uint32_t off = (kk >> 2) * L::kQHalf + (kk & 3) * 32;
+                            const uint32_t koff = (kk >> 2) * L::kKVHalf + (kk & 3) * 32;
+                            umma_ss(tmem + kTmemS, umma_desc_sw128(qaddr + off, 16, 1024),
+                                    umma_desc_sw128(kaddr + koff, 16, 1024), idesc_s, kk > 0);
                         }
+                        umma_commit(sfull);
+                        umma_commit(&kempty[slot]);
+                        if (j == nb - 1) umma_commit(&qempty[qb]);  // Q no longer read
                     }
-                    ok = __shfl_sync(0xffffffffu, ok, 0);
                 }
-                if (j > 0 && ok) {
+                ok = __shfl_sync(0xffffffffu, ok, 0);
+                if (j > 0 && ok && lane == 0) {
                     // O += P_{j-1} V_{j-1}
                     const uint32_t pg = gb - 1;
                     const uint32_t pb = pg & 1;
-                    const uint32_t pslot = (gs - 1) % NKV;
-                    if (lane == 0) {
-                        ok = wait_or_abort(&pfull[pb], (pg >> 1) & 1, abort_flag);
-                        if (ok) {
-                            tc_fence_after();
-                            const uint32_t vaddr = sbase + L::oKV + pslot * L::kSlot + L::kHalves * L::kKVHalf;
+                    const uint32_t slot = pg % NK;
+                    ok = wait_or_abort(&vfull[slot], (pg / NK) & 1, abort_flag) &&
+                         wait_or_abort(&pfull[pb], (pg >> 1) & 1, abort_flag);
+                    if (ok) {
+                        tc_fence_after();
+                        const uint32_t vaddr = sbase + L::oV + slot * L::kSlot;
 #pragma unroll
-                            for (int kk = 0; kk < kTcKeys / 16; ++kk)
-                                umma_ts(tmem + kTmemO, tmem + kTmemP + pb * (kTcKeys / 2) + kk * 8,
-                                        umma_desc_sw128(vaddr + kk * 16 * 128, L::kKVHalf, 1024), idesc_o,
-                                        (j > 1 || kk > 0) ? 1u : 0u);
-                            umma_commit(odone);
-                            umma_commit(&empty[pslot]);
-                        }
+                        for (int kk = 0; kk < kTcKeys / 16; ++kk)
+                            umma_ts(tmem + kTmemO, tmem + kTmemP + pb * (kTcKeys / 2) + kk * 8,
+                                    umma_desc_sw128(vaddr + kk * 16 * 128, L::kKVHalf, 1024), idesc_o,
+                                    (j > 1 || kk > 0) ? 1u : 0u);
+                        umma_commit(odone);
+                        umma_commit(&vempty[slot]);
                     }
-                    ok = __shfl_sync(0xffffffffu, ok, 0);
                 }
-                if (j < nb) { ++gs; ++gb; }
+                ok = __shfl_sync(0xffffffffu, ok, 0);
+                if (j < nb) ++gb;
             }
         }
         // every MMA this thread issued has completed before tensor memory is freed
@@ -368,12 +467,12 @@ __global__ void __launch_bounds__(kTcThreads, 1) paged_prefill_tc_kernel(const _
         const int quarter = warp & 3;          // TMEM lane quarter of this warp
         const int r = quarter * 32 + lane;     // row = TMEM lane
         const uint32_t lane_addr = tmem + ((uint32_t)(quarter * 32) << 16);
-        const float scale_log2 = p.scale_log2;
+        const float c = p.scale_log2;          // > 0 (checked on the host)
         uint32_t gb = 0;
         bool ok = true;
         for (int ord = 0; ok; ++ord) {
-            const int qb = ord & 1;
-            ok = __all_sync(0xffffffffu, wait_or_abort(&qfull[qb], (ord >> 1) & 1, abort_flag));
+            const int qb = ord % NQ;
+            ok = __all_sync(0xffffffffu, wait_or_abort(&qfull[qb], (ord / NQ) & 1, abort_flag));
             if (!ok) break;
             const TcItem t = items[qb];
             mbar_arrive(&qempty[qb]);
@@ -382,54 +481,69 @@ __global__ void __launch_bounds__(kTcThreads, 1) paged_prefill_tc_kernel(const _
             const int tok = t.tile * p.QT + tt;
             const bool real = tt < p.QT && tok < t.q_len;
             const int qpos = real ? t.prefix + tok : t.n_keys - 1;
-            float m = PKV_NEG_INF, l = 0.f;
+            float m = PKV_NEG_INF, l0 = 0.f, l1 = 0.f;  // running max (scaled log2 units), sum
             for (int j = 0; j < t.n_blocks && ok; ++j, ++gb) {
-                const uint32_t sb = gb & 1;
-                ok = __all_sync(0xffffffffu, wait_or_abort(&sfull[sb], (gb >> 1) & 1, abort_flag));
+                ok = __all_sync(0xffffffffu, wait_or_abort(sfull, gb & 1, abort_flag));
                 if (!ok) break;
                 tc_fence_after();
-                uint32_t sv[2][32];
-                tmem_ld32(lane_addr + kTmemS + sb * kTcKeys, sv[0]);
-                tmem_ld32(lane_addr + kTmemS + sb * kTcKeys + 32, sv[1]);
+                uint32_t sv[64];
+                tmem_ld32(lane_addr + kTmemS, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
+                tmem_ld32(lane_addr + kTmemS + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
                 tc_wait_ld();
                 tc_fence_before();
-                mbar_arrive(&sfree[sb]);
-                // causal mask and scale; lazy running max
+                mbar_arrive(sfree);
+                // causal mask on the block the diagonal crosses; max of raw scores
                 const int kbase = j * kTcKeys;
-                float mx = PKV_NEG_INF;
+                if (__any_sync(0xffffffffu, kbase + kTcKeys - 1 > qpos)) {
 #pragma unroll
-                for (int h2 = 0; h2 < 2; ++h2)
+                    for (int i = 0; i < 64; ++i)
+                        if (kbase + i > qpos) sv[i] = __float_as_uint(PKV_NEG_INF);
+                }
+                // four independent chains of 3-input max
+                float a0 = __uint_as_float(sv[0]), a1 = __uint_as_float(sv[1]);
+                float a2 = __uint_as_float(sv[2]), a3 = __uint_as_float(sv[3]);
 #pragma unroll
-                    for (int c = 0; c < 32; ++c) {
-                        const int kpos = kbase + h2 * 32 + c;
-                        const float z = kpos <= qpos ? __uint_as_float(sv[h2][c]) * scale_log2 : PKV_NEG_INF;
-                        sv[h2][c] = __float_as_uint(z);
-                        mx = fmaxf(mx, z);
+                for (int i = 4; i < 60; i += 8) {
+                    a0 = fmax3f(a0, __uint_as_float(sv[i]), __uint_as_float(sv[i + 1]));
+                    a1 = fmax3f(a1, __uint_as_float(sv[i + 2]), __uint_as_float(sv[i + 3]));
+                    a2 = fmax3f(a2, __uint_as_float(sv[i + 4]), __uint_as_float(sv[i + 5]));
+                    a3 = fmax3f(a3, __uint_as_float(sv[i + 6]), __uint_as_float(sv[i + 7]));
+                }
+                a0 = fmax3f(a0, __uint_as_float(sv[60]), __uint_as_float(sv[61]));
+                a1 = fmax3f(a1, __uint_as_float(sv[62]), __uint_as_float(sv[63]));
+                const float mxs = fmax3f(a0, a1, fmaxf(a2, a3)) * c;
+                const bool up = mxs > m + kRescaleSlack;
+                const float alpha = up ? ex2_ftz(m - mxs) : 1.f;
+                if (up) m = mxs;
+                const float nm = -m;
+                float s0 = 0.f, s1 = 0.f;
+                uint32_t pk[32];
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    float z0, z1;
+                    ffma2_bcast(z0, z1, __uint_as_float(sv[2 * i]), __uint_as_float(sv[2 * i + 1]), c, nm);
+                    float p0, p1;
+                    if (kExpEmuEvery > 0 && i % (kExpEmuEvery > 0 ? kExpEmuEvery : 1) == kExpEmuEvery - 1) {
+                        exp2_poly2(z0, z1, p0, p1);
+                    } else {
+                        p0 = ex2_ftz(z0);
+                        p1 = ex2_ftz(z1);
                     }
-                const bool up = mx > m + kRescaleSlack;
-                const float alpha = up ? exp2f(m - mx) : 1.f;
-                if (up) m = mx;
-                float sum = 0.f;
-                uint32_t pk[2][16];
-#pragma unroll
-                for (int h2 = 0; h2 < 2; ++h2)
-#pragma unroll
-                    for (int c = 0; c < 16; ++c) {
-                        const float p0 = exp2f(__uint_as_float(sv[h2][2 * c]) - m);
-                        const float p1 = exp2f(__uint_as_float(sv[h2][2 * c + 1]) - m);
-                        sum += p0 + p1;
-                        pk[h2][c] = pack_bf16x2(p0, p1);
-                    }
-                l = l * alpha + sum;
-                tmem_st16(lane_addr + kTmemP + sb * (kTcKeys / 2), pk[0]);
-                tmem_st16(lane_addr + kTmemP + sb * (kTcKeys / 2) + 16, pk[1]);
+                    fadd2(s0, s1, p0, p1);
+                    pk[i] = pack_bf16x2(p0, p1);
+                }
+                l0 = l0 * alpha + s0;
+                l1 = l1 * alpha + s1;
+                const uint32_t pcol = kTmemP + (gb & 1) * (kTcKeys / 2);
+                tmem_st16(lane_addr + pcol, *reinterpret_cast<uint32_t(*)[16]>(&pk[0]));
+                tmem_st16(lane_addr + pcol + 16, *reinterpret_cast<uint32_t(*)[16]>(&pk[16]));
                 // The previous block's PV product (global index gb - 1) must be
                 // complete before O is touched or P of this block is released;
                 // observing every phase of odone in order keeps its parity
                 // unambiguous (the next PV needs this block's P).
                 if (gb > 0) ok = __all_sync(0xffffffffu, wait_or_abort(odone, (gb - 1) & 1, abort_flag));
                 // rescale this row of O (the warp does it if any of its rows raised the max)
-                if (j > 0 && __any_sync(0xffffffffu, up)) {
+                if (ok && j > 0 && __any_sync(0xffffffffu, up)) {
                     tc_fence_after();
 #pragma unroll
                     for (int c0 = 0; c0 < D; c0 += 32) {
@@ -437,19 +551,20 @@ __global__ void __launch_bounds__(kTcThreads, 1) paged_prefill_tc_kernel(const _
                         tmem_ld32(lane_addr + kTmemO + c0, ov);
                         tc_wait_ld();
 #pragma unroll
-                        for (int c = 0; c < 32; ++c) ov[c] = __float_as_uint(__uint_as_float(ov[c]) * alpha);
+                        for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
                         tmem_st32(lane_addr + kTmemO + c0, ov);
                     }
                 }
-                // keys past the context in the last block: zero their V rows so
-                // stale (possibly NaN) data cannot reach the MMA (P is 0 there)
-                if (j == t.n_blocks - 1 && (t.n_keys % kStageTok) != 0) {
+                // keys past the context in the last block: zero their V rows
+                // (once the block has landed) so stale, possibly NaN, data
+                // cannot reach the MMA (P is 0 there)
+                if (ok && j == t.n_blocks - 1 && (t.n_keys % kStageTok) != 0) {
+                    const uint32_t slot = gb % NK;
+                    ok = __all_sync(0xffffffffu, wait_or_abort(&vfull[slot], (gb / NK) & 1, abort_flag));
                     const int first = t.n_keys - kbase;  // first invalid key of the block
                     const int last = (first / kStageTok + 1) * kStageTok;
-                    const uint32_t slot = (uint32_t)(gb % NKV);
-                    // gb counts blocks; KV slots advance one per block as well
-                    uint8_t *vrow0 = smem + L::oKV + slot * L::kSlot + L::kHalves * L::kKVHalf;
-                    for (int i = r; i < (last - first) * L::kHalves * 8; i += kTcRows) {
+                    uint8_t *vrow0 = smem + L::oV + slot * L::kSlot;
+                    for (int i = r; ok && i < (last - first) * L::kHalves * 8; i += kTcRows) {
                         const int key = first + i / (L::kHalves * 8);
                         const int rest = i % (L::kHalves * 8);
                         *reinterpret_cast<uint4 *>(vrow0 + (rest / 8) * L::kKVHalf + key * 128 + (rest % 8) * 16) =
@@ -459,13 +574,14 @@ __global__ void __launch_bounds__(kTcThreads, 1) paged_prefill_tc_kernel(const _
                 }
                 tc_wait_st();
                 tc_fence_before();
-                mbar_arrive(&pfull[sb]);
+                mbar_arrive(&pfull[gb & 1]);
             }
             if (!ok) break;
             // epilogue: O / l for this row
             ok = __all_sync(0xffffffffu, wait_or_abort(odone, (gb - 1) & 1, abort_flag));
             if (!ok) break;
             tc_fence_after();
+            const float l = l0 + l1;
             const float inv = l > 0.f ? 1.f / l : 0.f;
             __nv_bfloat16 *orow =
                 real ? p.out + ((size_t)(t.q0 + tok) * p.Hq + (size_t)t.h * p.g + jh) * D : nullptr;
@@ -476,13 +592,13 @@ __global__ void __launch_bounds__(kTcThreads, 1) paged_prefill_tc_kernel(const _
                 tc_wait_ld();
                 if (real) {
 #pragma unroll
-                    for (int c = 0; c < 32; c += 8) {
+                    for (int i = 0; i < 32; i += 8) {
                         uint4 v;
-                        v.x = pack_bf16x2(__uint_as_float(ov[c]) * inv, __uint_as_float(ov[c + 1]) * inv);
-                        v.y = pack_bf16x2(__uint_as_float(ov[c + 2]) * inv, __uint_as_float(ov[c + 3]) * inv);
-                        v.z = pack_bf16x2(__uint_as_float(ov[c + 4]) * inv, __uint_as_float(ov[c + 5]) * inv);
-                        v.w = pack_bf16x2(__uint_as_float(ov[c + 6]) * inv, __uint_as_float(ov[c + 7]) * inv);
-                        *reinterpret_cast<uint4 *>(orow + c0 + c) = v;
+                        v.x = pack_bf16x2(__uint_as_float(ov[i]) * inv, __uint_as_float(ov[i + 1]) * inv);
+                        v.y = pack_bf16x2(__uint_as_float(ov[i + 2]) * inv, __uint_as_float(ov[i + 3]) * inv);
+                        v.z = pack_bf16x2(__uint_as_float(ov[i + 4]) * inv, __uint_as_float(ov[i + 5]) * inv);
+                        v.w = pack_bf16x2(__uint_as_float(ov[i + 6]) * inv, __uint_as_float(ov[i + 7]) * inv);
+                        *reinterpret_cast<uint4 *>(orow + c0 + i) = v;
                     }
                 }
             }

@@ -102,6 +102,38 @@ def test_decode_validation():
     assert _decode(lib, pool=_pool(hkv=2, d=256)) == EUNSUP
 
 
+def _prefill(lib, **kw):
+    a = dict(q=FAKE, kc=FAKE, vc=FAKE, tables=FAKE, mbs=4, ctx=FAKE, qs=FAKE, B=2, T=32, Hq=4, scale=0.1, Hkv=2,
+             out=FAKE, pool=_pool(hkv=2), max_q=16, max_ctx=64, ws=FAKE, ws_bytes=1 << 30)
+    a.update(kw)
+    f = lib.paged_attn_prefill
+    P, I32 = ctypes.c_void_p, ctypes.c_int32
+    f.argtypes = [P, P, P, P, I32, P, P, I32, I32, I32, ctypes.c_float, I32, P, _Pool, I32, I32, P,
+                  ctypes.c_size_t, P]
+    f.restype = ctypes.c_int
+    return f(a["q"], a["kc"], a["vc"], a["tables"], a["mbs"], a["ctx"], a["qs"], a["B"], a["T"], a["Hq"],
+             a["scale"], a["Hkv"], a["out"], a["pool"], a["max_q"], a["max_ctx"], a["ws"], a["ws_bytes"], None)
+
+
+def test_prefill_validation():
+    lib = pkv.load_library()
+    assert _prefill(lib, B=0) == 0
+    assert _prefill(lib, T=0) == 0  # no query rows: nothing to launch
+    assert _prefill(lib, T=-1) == EINVAL
+    assert _prefill(lib, Hq=5) == EINVAL
+    assert _prefill(lib, Hq=2 * 17) == EUNSUP
+    assert _prefill(lib, scale=0.0) == EINVAL  # the kernel keeps its running max on raw scores
+    assert _prefill(lib, scale=-0.1) == EINVAL
+    assert _prefill(lib, scale=float("inf")) == EINVAL
+    assert _prefill(lib, scale=float("nan")) == EINVAL
+    assert _prefill(lib, q=FAKE_ODD) == EINVAL
+    assert _prefill(lib, qs=None) == EINVAL
+    assert _prefill(lib, ws=ctypes.c_void_p(0x10010)) == EINVAL
+    assert _prefill(lib, ws_bytes=16) == EINVAL
+    assert _prefill(lib, mbs=0) == EINVAL
+    assert _prefill(lib, pool=_pool(hkv=2, bs=8)) == EUNSUP
+
+
 def test_workspace_size():
     f = pkv.decode_workspace_bytes
     # one partition per sequence: count + entries only
