@@ -51,10 +51,13 @@ def _load() -> ctypes.CDLL:
         lib.oracle_attention_partial.argtypes = [P, P, P, P, I, I, I, I, I, I, I, I, D, P, P, P]
         lib.oracle_lse_merge.argtypes = [P, P, P, I, I, P]
         lib.oracle_paged_prefill.argtypes = [P, P, P, P, I, P, P, I, I, I, I, I, I, D, P]
+        lib.oracle_swap_out.argtypes = [P, P, P, I, I, I, I, I, P, P]
+        lib.oracle_swap_in.argtypes = [P, P, P, I, I, I, I, I, P, P]
+        lib.oracle_lru_victims.argtypes = [P, P, I, I, P, P]
         lib.oracle_num_threads.argtypes = []
         for f in (lib.oracle_kv_write, lib.oracle_copy_blocks, lib.oracle_paged_attention,
                   lib.oracle_attention_partial, lib.oracle_lse_merge, lib.oracle_num_threads,
-                  lib.oracle_paged_prefill):
+                  lib.oracle_paged_prefill, lib.oracle_swap_out, lib.oracle_swap_in, lib.oracle_lru_victims):
             f.restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -93,6 +96,8 @@ def _check(rc: int, what: str):
         raise ValueError(f"oracle {what}: bad argument")
     if rc == 2:
         raise IndexError(f"oracle {what}: index out of range")
+    if rc == 3:
+        raise ValueError(f"oracle {what}: repeated block id")
     if rc:
         raise RuntimeError(f"oracle {what}: status {rc}")
 
@@ -126,6 +131,45 @@ def copy_blocks(k_cache, v_cache, pairs):
     rc = _load().oracle_copy_blocks(_ptr(kc), _ptr(vc), _ptr(pr), pr.shape[0], NB, Hkv, bs, d)
     _check(rc, "copy_blocks")
     return kc, vc
+
+
+def swap_out(k_cache, v_cache, block_ids):
+    """Returns (host_k, host_v) uint16 arrays [n, Hkv, bs, d]: copies of the
+    listed blocks of the two caches, in list order."""
+    kc, vc = bits(k_cache), bits(v_cache)
+    ids = np.ascontiguousarray(block_ids, dtype=np.int32).reshape(-1)
+    NB, Hkv, bs, d = kc.shape
+    hk = np.zeros((ids.shape[0], Hkv, bs, d), dtype=np.uint16)
+    hv = np.zeros_like(hk)
+    rc = _load().oracle_swap_out(_ptr(kc), _ptr(vc), _ptr(ids), ids.shape[0], NB, Hkv, bs, d, _ptr(hk), _ptr(hv))
+    _check(rc, "swap_out")
+    return hk, hv
+
+
+def swap_in(k_cache, v_cache, host_k, host_v, block_ids):
+    """Returns new (k_cache, v_cache) with block ids[i] replaced by host_k[i] /
+    host_v[i]; ids must be distinct."""
+    kc, vc = bits(k_cache).copy(), bits(v_cache).copy()
+    hk, hv = bits(host_k), bits(host_v)
+    ids = np.ascontiguousarray(block_ids, dtype=np.int32).reshape(-1)
+    NB, Hkv, bs, d = kc.shape
+    assert hk.shape == (ids.shape[0], Hkv, bs, d) and hv.shape == hk.shape
+    rc = _load().oracle_swap_in(_ptr(hk), _ptr(hv), _ptr(ids), ids.shape[0], NB, Hkv, bs, d, _ptr(kc), _ptr(vc))
+    _check(rc, "swap_in")
+    return kc, vc
+
+
+def lru_victims(last_use, evictable, k: int) -> np.ndarray:
+    """The k evictable blocks least recently used (oldest last_use first, ties
+    by lower block id)."""
+    lu = np.ascontiguousarray(last_use, dtype=np.int64).reshape(-1)
+    ev = np.ascontiguousarray(evictable, dtype=np.uint8).reshape(-1)
+    assert ev.shape == lu.shape
+    out = np.zeros(max(k, 1), dtype=np.int32)
+    cnt = np.zeros(1, dtype=np.int32)
+    rc = _load().oracle_lru_victims(_ptr(lu), _ptr(ev), lu.shape[0], int(k), _ptr(out), _ptr(cnt))
+    _check(rc, "lru_victims")
+    return out[:int(cnt[0])].copy()
 
 
 def paged_attention(q, k_cache, v_cache, block_tables, context_lens, scale: float) -> np.ndarray:

@@ -16,6 +16,9 @@
  *     computes ordinary attention over it (wkbse.com section 3.1, third point
  *     of the list), i.e. softmax(q K^T * scale) V.
  *   - copy-on-write of a shared block (intelliparadigm.com section 2.1, item 2).
+ *   - swap of cold blocks to CPU memory and back, victims chosen least
+ *     recently used first (intelliparadigm.com section 2.1, item 3; ai-stack.site
+ *     "Nano-vLLM 原理", practice 5, preemption by swapping a request's KV cache).
  *
  * Pool layout (the library's ABI; the oracle reads it through pool_row()):
  *   cache[num_blocks][num_kv_heads][bs][d], bf16 bit patterns (uint16).
@@ -287,4 +290,74 @@ int oracle_paged_prefill(const uint16_t *q, const uint16_t *k_cache, const uint1
         }
     }
     return status;
+}
+
+/*
+ * Swap-out: host_k[i] and host_v[i] (each num_kv_heads * bs * d elements, all
+ * heads of one block) become copies of block ids[i] of the two caches, for
+ * i < n.  The caches are not changed; an id may repeat.
+ */
+int oracle_swap_out(const uint16_t *k_cache, const uint16_t *v_cache, const int32_t *ids, int n, int num_blocks,
+                    int num_kv_heads, int bs, int d, uint16_t *host_k, uint16_t *host_v) {
+    if (n < 0 || num_blocks <= 0) return 1;
+    size_t block_elems = (size_t)num_kv_heads * bs * d;
+    for (int i = 0; i < n; ++i)
+        if (ids[i] < 0 || ids[i] >= num_blocks) return 2;
+    for (int i = 0; i < n; ++i) {
+        for (size_t e = 0; e < block_elems; ++e) {
+            host_k[(size_t)i * block_elems + e] = k_cache[(size_t)ids[i] * block_elems + e];
+            host_v[(size_t)i * block_elems + e] = v_cache[(size_t)ids[i] * block_elems + e];
+        }
+    }
+    return 0;
+}
+
+/*
+ * Swap-in: block ids[i] of the two caches becomes host_k[i] / host_v[i], for
+ * i < n.  Ids must be distinct (two copies into one block would leave it
+ * undefined): 3 otherwise.
+ */
+int oracle_swap_in(const uint16_t *host_k, const uint16_t *host_v, const int32_t *ids, int n, int num_blocks,
+                   int num_kv_heads, int bs, int d, uint16_t *k_cache, uint16_t *v_cache) {
+    if (n < 0 || num_blocks <= 0) return 1;
+    size_t block_elems = (size_t)num_kv_heads * bs * d;
+    for (int i = 0; i < n; ++i)
+        if (ids[i] < 0 || ids[i] >= num_blocks) return 2;
+    for (int i = 0; i < n; ++i)
+        for (int j = i + 1; j < n; ++j)
+            if (ids[i] == ids[j]) return 3;
+    for (int i = 0; i < n; ++i) {
+        for (size_t e = 0; e < block_elems; ++e) {
+            k_cache[(size_t)ids[i] * block_elems + e] = host_k[(size_t)i * block_elems + e];
+            v_cache[(size_t)ids[i] * block_elems + e] = host_v[(size_t)i * block_elems + e];
+        }
+    }
+    return 0;
+}
+
+/*
+ * LRU victim choice: among the blocks with evictable[b] != 0, the k with the
+ * oldest last_use[b] (smallest value; equal values by lower block id), in that
+ * order, written to victims[0 .. min(k, #evictable)).  Returns the count
+ * through *count.  Plain repeated selection of the minimum.
+ */
+int oracle_lru_victims(const int64_t *last_use, const uint8_t *evictable, int num_blocks, int k, int32_t *victims,
+                       int *count) {
+    if (num_blocks < 0 || k < 0) return 1;
+    uint8_t *taken = (uint8_t *)calloc((size_t)num_blocks + 1, 1);
+    if (!taken) return 1;
+    int c = 0;
+    while (c < k) {
+        int best = -1;
+        for (int b = 0; b < num_blocks; ++b) {
+            if (!evictable[b] || taken[b]) continue;
+            if (best < 0 || last_use[b] < last_use[best]) best = b;
+        }
+        if (best < 0) break;
+        taken[best] = 1;
+        victims[c++] = best;
+    }
+    free(taken);
+    *count = c;
+    return 0;
 }

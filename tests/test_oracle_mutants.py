@@ -15,6 +15,7 @@ import pytest
 import oracle
 from tests import test_oracle_pins as pins
 from tests import test_oracle_prefill as prefill_pins
+from tests import test_oracle_swap as swap_pins
 
 PIN_TESTS = [
     pins.test_block_count_golden,
@@ -32,6 +33,11 @@ PIN_TESTS = [
     pins.test_lse_merge_closed_form,
     lambda: prefill_pins.test_prefill_equals_sdpa_with_bottom_right_causal_mask([31, 17, 0, 64], [1, 20, 48, 3],
                                                                                  6, 3, 64, 16),
+    swap_pins.test_swap_out_then_in_equals_copy_blocks,
+    swap_pins.test_swap_round_trip_restores_and_swap_out_reads_only,
+    swap_pins.test_swap_of_a_permutation_is_a_gather,
+    swap_pins.test_lru_worked_example_golden,
+    lambda: swap_pins.test_lru_characterisation(0),
 ]
 
 MUTANTS = {
@@ -53,6 +59,13 @@ MUTANTS = {
     "prefill causal bound -1": ("bs, hq, 0, pos + 1, scale", "bs, hq, 0, pos, scale"),
     "prefill query position": ("int pos = context_lens[s] - q_len + (t - query_start[s]);",
                                "int pos = (t - query_start[s]);"),
+    # swap: the key region copied into both host buffers; a block shifted by one;
+    # the most recently used block chosen first; ties to the higher id
+    "swap key into value": ("host_v[(size_t)i * block_elems + e] = v_cache[", "host_v[(size_t)i * block_elems + e] = k_cache["),
+    "swap-in wrong block": ("k_cache[(size_t)ids[i] * block_elems + e] = host_k[",
+                            "k_cache[(size_t)((ids[i] + 1) % num_blocks) * block_elems + e] = host_k["),
+    "lru newest first": ("last_use[b] < last_use[best]", "last_use[b] > last_use[best]"),
+    "lru ties to higher id": ("last_use[b] < last_use[best]", "last_use[b] <= last_use[best]"),
     # the new token left out of the attended range (context_len - 1 tokens)
     "context off by one": ("hq, 0, context_lens[s], scale", "hq, 0, context_lens[s] - 1, scale"),
 }
