@@ -476,6 +476,111 @@ def run_prefill_cuda(args, rank, world, dist):
     }
 
 
+SWAP_WORKLOADS = ("llama2-13b-swap",)
+
+
+def run_swap_cuda(args, rank, world, dist):
+    """One step = swap-out of the LRU victim blocks of the Llama-2-13B pool to
+    pinned host memory, then swap-in of the same blocks (a preemption cycle,
+    about 256 MB each way).  Metric: GB/s moved over the host link; the
+    roofline peak is a plain pinned DMA copy of the same bytes (both ways),
+    measured in the same run."""
+    import paged_kv_cache_420_b200 as pkv
+
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
+    torch.cuda.set_device(dev)
+    w = workloads.make("llama2-13b", seed=args.seed + rank, values_device=dev, block_size=args.block_size)
+    nb = w.k_cache.shape[0]
+    rng = np.random.default_rng(args.seed + rank)
+    # blocks of a sequence share its last scheduling time; unowned blocks are free
+    owner_time = rng.permutation(w.num_seqs)
+    last_use = np.zeros(nb, dtype=np.int64)
+    evictable = np.zeros(nb, dtype=np.uint8)
+    for s in range(w.num_seqs):
+        nblk = (int(w.context_lens[s]) + w.block_size - 1) // w.block_size
+        blk = w.block_tables[s, :nblk]
+        last_use[blk] = owner_time[s]
+        evictable[blk] = 1
+    block_bytes = w.k_cache[0].numel() * 2
+    k = int(min(evictable.sum(), max(1, round((256 << 20) / (2 * block_bytes)))))
+    victims = pkv.lru_victims(last_use, evictable, k)
+    n = len(victims)
+    hk = torch.empty((n,) + tuple(w.k_cache.shape[1:]), dtype=torch.bfloat16).pin_memory()
+    hv = torch.empty_like(hk).pin_memory()
+    stream = torch.cuda.current_stream()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+
+    def step(i=None):
+        if i is not None:
+            ev[i][0].record(stream)
+        pkv.pkv_swap_out(w.k_cache, w.v_cache, victims, hk, hv, stream=stream)
+        if i is not None:
+            ev[i][1].record(stream)
+        pkv.pkv_swap_in(hk, hv, victims, w.k_cache, w.v_cache, stream=stream)
+        if i is not None:
+            ev[i][2].record(stream)
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize()
+    # the link: DMA copies of the same bytes, device -> pinned host and back
+    dk = torch.empty((n,) + tuple(w.k_cache.shape[1:]), dtype=torch.bfloat16, device=dev)
+    dv = torch.empty_like(dk)
+    d2h_ms, h2d_ms = [], []
+    for _ in range(5):
+        a, b, c = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+        a.record(stream)
+        hk.copy_(dk, non_blocking=True)
+        hv.copy_(dv, non_blocking=True)
+        b.record(stream)
+        dk.copy_(hk, non_blocking=True)
+        dv.copy_(hv, non_blocking=True)
+        c.record(stream)
+        torch.cuda.synchronize()
+        d2h_ms.append(a.elapsed_time(b))
+        h2d_ms.append(b.elapsed_time(c))
+    del dk, dv
+    if dist is not None:
+        dist.barrier()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(dev.index) as clocks:
+        t0.record(stream)
+        for i in range(args.steps):
+            step(i)
+        t1.record(stream)
+        torch.cuda.synchronize()
+        if dist is not None:
+            dist.barrier()
+        if t0.elapsed_time(t1) < 450:
+            time.sleep(0.45)
+    bytes_step = 2 * n * block_bytes * 2  # K and V, out and in
+    ms_max, bytes_all, _ = combine_ranks(dist, t0.elapsed_time(t1), bytes_step, n, dev)
+    out_ms = float(np.median([e[0].elapsed_time(e[1]) for e in ev]))
+    in_ms = float(np.median([e[1].elapsed_time(e[2]) for e in ev]))
+    one_way = 2 * n * block_bytes
+    dma_ms = float(np.median(d2h_ms)) + float(np.median(h2d_ms))
+    achieved = bytes_step / ((out_ms + in_ms) / 1e3) / 1e9
+    peak = bytes_step / (dma_ms / 1e3) / 1e9
+    return {
+        "metric": "block swap GB/s (out to pinned host memory and back in)",
+        "value": round(bytes_all * args.steps / (ms_max / 1e3) / 1e9, 2), "unit": "GB/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_max / args.steps, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": f"llama2-13b pool, {n} LRU victim blocks of {block_bytes * 2} B (K+V), "
+                               f"{one_way / 1e6:.1f} MB each way", "block_size": w.block_size, "seed": args.seed},
+        "roofline": {"kernel": "swap_blocks_kernel (out, in)", "bound": "host link",
+                     "achieved": round(achieved, 2), "peak": round(peak, 2),
+                     "peak_kind": "measured: pinned cudaMemcpyAsync of the same bytes, D2H then H2D",
+                     "unit": "GB/s", "frac": round(achieved / peak, 4),
+                     "swap_out_gbs": round(one_way / (out_ms / 1e3) / 1e9, 2),
+                     "swap_in_gbs": round(one_way / (in_ms / 1e3) / 1e9, 2),
+                     "dma_d2h_gbs": round(one_way / (float(np.median(d2h_ms)) / 1e3) / 1e9, 2),
+                     "dma_h2d_gbs": round(one_way / (float(np.median(h2d_ms)) / 1e3) / 1e9, 2),
+                     "traffic": None},
+        "e2e": None, "gpu_launches": 2 * args.steps, "clocks": clocks.summary(),
+    }
+
+
 def cpu_baseline(w, budget_s: float, label="oracle", pools=None):
     """Times the fp64 CPU oracle's paged attention on the first sequences of
     the workload until about `budget_s` seconds of CPU work are spent.  The
@@ -573,6 +678,38 @@ def run_prefill_reference(args, world):
     }
 
 
+def run_swap_reference(args, world):
+    """The oracle's swap-out and swap-in (plain C loops over host arrays) on a
+    sample with the Llama-2-13B block shape: 128 of 512 blocks out and back in."""
+    import oracle
+
+    rng = np.random.default_rng(args.seed)
+    shape = (512, 40, args.block_size or 16, 128)
+    kc = rng.integers(0, 1 << 16, size=shape, dtype=np.uint16)
+    vc = rng.integers(0, 1 << 16, size=shape, dtype=np.uint16)
+    ids = rng.permutation(shape[0])[:128].astype(np.int32)
+    block_bytes = int(np.prod(shape[1:])) * 2
+    times = []
+    for i in range(args.warmup + args.steps):
+        t = time.perf_counter()
+        hk, hv = oracle.swap_out(kc, vc, ids)
+        kc, vc = oracle.swap_in(kc, vc, hk, hv, ids)
+        if i >= args.warmup:
+            times.append(time.perf_counter() - t)
+    bytes_step = 2 * len(ids) * block_bytes * 2
+    value = round(bytes_step / statistics.median(times) / 1e9, 3)
+    sample = f"{len(ids)} of {shape[0]} blocks of shape {shape[1:]}, out and back in, per step"
+    return {
+        "impl": "reference", "metric": "block swap GB/s (out to pinned host memory and back in)",
+        "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(1e3 * sum(times) / len(times), 3), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "u16", "data": "synthetic",
+        "config": {"workload": "llama2-13b block shape swap sample", "block_size": shape[2], "seed": args.seed},
+        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
 def run_reference(args, rank, world):
     """The CPU oracle as the reference arm: rank 0 times it on the host cores,
     one bounded sample of the workload per step."""
@@ -580,6 +717,8 @@ def run_reference(args, rank, world):
         return None
     if args.workload in workloads.PREFILL_WORKLOADS:
         return run_prefill_reference(args, world)
+    if args.workload in SWAP_WORKLOADS:
+        return run_swap_reference(args, world)
     w = workloads.make(args.workload, seed=args.seed, values_device="cpu", block_size=args.block_size)
     per_step_budget = max(0.05, min(2.0, 150.0 / max(1, args.steps + args.warmup)))
     pools = oracle_pools(w)
@@ -616,7 +755,7 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["pkv", "reference"], default="pkv")
     ap.add_argument("--workload", default="llama2-13b",
-                    choices=list(workloads.WORKLOADS) + list(workloads.PREFILL_WORKLOADS))
+                    choices=list(workloads.WORKLOADS) + list(workloads.PREFILL_WORKLOADS) + list(SWAP_WORKLOADS))
     ap.add_argument("--block-size", type=int, default=None)
     ap.add_argument("--partition-tokens", type=int, default=-1, help="-1: the workload's choice, 0: library's")
     ap.add_argument("--seed", type=int, default=0)
@@ -642,6 +781,8 @@ def main(argv=None):
             line = run_reference(args, rank, world)
         elif args.workload in workloads.PREFILL_WORKLOADS:
             line = run_prefill_cuda(args, rank, world, dist)
+        elif args.workload in SWAP_WORKLOADS:
+            line = run_swap_cuda(args, rank, world, dist)
         else:
             line = run_cuda(args, rank, world, dist)
         if rank == 0 and line is not None:

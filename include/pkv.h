@@ -113,6 +113,44 @@ pkv_status pkv_copy_blocks(const int32_t *src_dst_pairs, int32_t num_pairs, void
                            void *v_cache, pkv_pool pool, pkv_stream_t stream);
 
 /*
+ * pkv_swap_out / pkv_swap_in -- move whole blocks between the pool and host
+ * memory: cold blocks go to CPU memory when device memory runs short
+ * (intelliparadigm.com section 2.1, item 3), and a preempted request's KV
+ * cache is swapped out and later back in (ai-stack.site "Nano-vLLM 原理",
+ * practice 5).  The block manager picks the blocks on the host (see
+ * pkv_lru_victims); one launch per 2048 ids moves them.
+ *
+ *   block_ids        HOST int32 [n], ids in [0, num_blocks) (else PKV_ERANGE)
+ *   host_k, host_v   pinned host memory the device can address (cudaHostAlloc /
+ *                    cudaMallocHost / a pinned torch tensor), 16-B aligned, each
+ *                    n * num_kv_heads * block_size * head_dim bf16, packed in
+ *                    list order: entry i is [num_kv_heads][block_size][head_dim].
+ *                    Pageable or device memory gives PKV_EINVAL.
+ * swap_out: host_k[i] / host_v[i] become bit-exact copies of block ids[i] of
+ *           k_cache / v_cache (the pool is only read; ids may repeat).
+ * swap_in:  block ids[i] of both caches becomes host_k[i] / host_v[i]; ids must
+ *           be distinct (PKV_EALIAS).
+ * Asynchronous on `stream`: the host buffers must stay alive and untouched
+ * until the stream reaches the call.  n == 0 is a no-op; nothing is enqueued
+ * when validation fails.
+ */
+pkv_status pkv_swap_out(const void *k_cache, const void *v_cache, pkv_pool pool, const int32_t *block_ids,
+                        int32_t n, void *host_k, void *host_v, pkv_stream_t stream);
+pkv_status pkv_swap_in(const void *host_k, const void *host_v, const int32_t *block_ids, int32_t n,
+                       void *k_cache, void *v_cache, pkv_pool pool, pkv_stream_t stream);
+
+/*
+ * pkv_lru_victims -- host-side choice of blocks to swap out, least recently
+ * used first (intelliparadigm.com section 2.1, item 3: block heat managed by
+ * LRU).  Among blocks b with evictable[b] != 0 (host arrays of num_blocks),
+ * writes the min(k, #evictable) with the oldest last_use[b] (smaller is older;
+ * equal values by lower id) to victims, oldest first, and their number to
+ * *count.  Pure host code: no device memory, no stream.
+ */
+pkv_status pkv_lru_victims(const int64_t *last_use, const uint8_t *evictable, int32_t num_blocks, int32_t k,
+                           int32_t *victims, int32_t *count);
+
+/*
  * pkv_decode_workspace_bytes -- device scratch needed by paged_attn_decode for
  * these sizes (a work list and the split-K partial results).  Returns 0 for
  * invalid sizes.  partition_tokens as for paged_attn_decode (0 = library's

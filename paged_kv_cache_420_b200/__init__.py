@@ -25,7 +25,8 @@ DEVERR_SLOT, DEVERR_BLOCK, DEVERR_CONTEXT, DEVERR_TIMEOUT, DEVERR_LAYOUT = 0x1, 
 # Every symbol include/pkv.h declares.
 EXPORTED = ("pkv_write", "pkv_copy_blocks", "pkv_decode_workspace_bytes", "paged_attn_decode",
             "paged_attn_decode_static_ws", "pkv_prefill_workspace_bytes", "paged_attn_prefill",
-            "pkv_get_device_error", "pkv_selftest_bounded_wait", "pkv_status_string", "pkv_version")
+            "pkv_get_device_error", "pkv_selftest_bounded_wait", "pkv_status_string", "pkv_version",
+            "pkv_swap_out", "pkv_swap_in", "pkv_lru_victims")
 STATIC_WS_BYTES = 32 << 20  # PKV_STATIC_WS_BYTES
 
 
@@ -57,10 +58,14 @@ def load_library() -> ctypes.CDLL:
         lib.pkv_decode_workspace_bytes.restype = SZ
         lib.paged_attn_decode.argtypes = [P, P, P, P, I32, P, I32, I32, F, I32, P, _Pool, I32, I32, P, SZ, P]
         lib.pkv_get_device_error.argtypes = [ctypes.POINTER(I32), P]
+        lib.pkv_swap_out.argtypes = [P, P, _Pool, P, I32, P, P, P]
+        lib.pkv_swap_in.argtypes = [P, P, P, I32, P, P, _Pool, P]
+        lib.pkv_lru_victims.argtypes = [P, P, I32, I32, P, P]
         lib.pkv_status_string.argtypes = [ctypes.c_int]
         lib.pkv_status_string.restype = ctypes.c_char_p
         lib.pkv_version.restype = I32
-        for f in ("pkv_write", "pkv_copy_blocks", "paged_attn_decode", "pkv_get_device_error"):
+        for f in ("pkv_write", "pkv_copy_blocks", "paged_attn_decode", "pkv_get_device_error", "pkv_swap_out",
+                  "pkv_swap_in", "pkv_lru_victims"):
             getattr(lib, f).restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -129,6 +134,60 @@ def pkv_copy_blocks(src_dst_pairs, k_cache: torch.Tensor, v_cache: torch.Tensor,
     st = load_library().pkv_copy_blocks(pairs.ctypes.data_as(ctypes.c_void_p), pairs.shape[0], _ptr(k_cache),
                                         _ptr(v_cache), _pool(k_cache), _stream(stream))
     _check(st, "pkv_copy_blocks")
+
+
+def _host_blocks(t: torch.Tensor, name: str, k_cache: torch.Tensor, n: int):
+    if t.dtype != torch.bfloat16 or not t.is_contiguous() or t.is_cuda:
+        raise ValueError(f"{name} must be a contiguous bf16 host tensor")
+    if not t.is_pinned():
+        raise ValueError(f"{name} must be pinned host memory")
+    if t.numel() < n * k_cache[0].numel():
+        raise ValueError(f"{name} holds fewer than {n} blocks")
+
+
+def _block_ids(block_ids) -> np.ndarray:
+    return np.ascontiguousarray(np.asarray(block_ids, dtype=np.int32).reshape(-1))
+
+
+def pkv_swap_out(k_cache: torch.Tensor, v_cache: torch.Tensor, block_ids, host_k: torch.Tensor,
+                 host_v: torch.Tensor, stream=None) -> None:
+    """host_k[i] / host_v[i] := block block_ids[i] of k_cache / v_cache (pinned
+    host tensors of at least len(block_ids) blocks); asynchronous on the stream."""
+    for t, n in ((k_cache, "k_cache"), (v_cache, "v_cache")):
+        _need(t, n, torch.bfloat16)
+    ids = _block_ids(block_ids)
+    _host_blocks(host_k, "host_k", k_cache, ids.shape[0])
+    _host_blocks(host_v, "host_v", k_cache, ids.shape[0])
+    st = load_library().pkv_swap_out(_ptr(k_cache), _ptr(v_cache), _pool(k_cache), ids.ctypes.data_as(ctypes.c_void_p),
+                                     ids.shape[0], _ptr(host_k), _ptr(host_v), _stream(stream))
+    _check(st, "pkv_swap_out")
+
+
+def pkv_swap_in(host_k: torch.Tensor, host_v: torch.Tensor, block_ids, k_cache: torch.Tensor,
+                v_cache: torch.Tensor, stream=None) -> None:
+    """Block block_ids[i] of k_cache / v_cache := host_k[i] / host_v[i] (ids distinct)."""
+    for t, n in ((k_cache, "k_cache"), (v_cache, "v_cache")):
+        _need(t, n, torch.bfloat16)
+    ids = _block_ids(block_ids)
+    _host_blocks(host_k, "host_k", k_cache, ids.shape[0])
+    _host_blocks(host_v, "host_v", k_cache, ids.shape[0])
+    st = load_library().pkv_swap_in(_ptr(host_k), _ptr(host_v), ids.ctypes.data_as(ctypes.c_void_p), ids.shape[0],
+                                    _ptr(k_cache), _ptr(v_cache), _pool(k_cache), _stream(stream))
+    _check(st, "pkv_swap_in")
+
+
+def lru_victims(last_use, evictable, k: int) -> np.ndarray:
+    """The k evictable blocks with the oldest last use (ties: lower id), oldest first."""
+    lu = np.ascontiguousarray(np.asarray(last_use, dtype=np.int64).reshape(-1))
+    ev = np.ascontiguousarray(np.asarray(evictable, dtype=np.uint8).reshape(-1))
+    if ev.shape != lu.shape:
+        raise ValueError("last_use and evictable must have one entry per block")
+    out = np.zeros(max(int(k), 1), dtype=np.int32)
+    cnt = ctypes.c_int32(0)
+    st = load_library().pkv_lru_victims(lu.ctypes.data_as(ctypes.c_void_p), ev.ctypes.data_as(ctypes.c_void_p),
+                                        lu.shape[0], int(k), out.ctypes.data_as(ctypes.c_void_p), ctypes.byref(cnt))
+    _check(st, "pkv_lru_victims")
+    return out[:cnt.value].copy()
 
 
 def decode_workspace_bytes(num_seqs: int, num_q_heads: int, num_kv_heads: int, head_dim: int,

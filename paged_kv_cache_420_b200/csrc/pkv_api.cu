@@ -281,6 +281,59 @@ pkv_status launch_prefill(const pkv::PrefillParams &prm, const CUtensorMap &mk, 
     return launch_status();
 }
 
+// Device address of host memory the GPU can reach (pinned; unified addressing
+// makes it the host address), or nullptr for pageable or device memory.
+void *mapped_host_pointer(const void *p) {
+    cudaPointerAttributes a;
+    if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+        cudaGetLastError();  // clear the sticky-free error of an unknown pointer
+        return nullptr;
+    }
+    if (a.type != cudaMemoryTypeHost || a.devicePointer == nullptr) return nullptr;
+    return a.devicePointer;
+}
+
+template <bool OUT>
+pkv_status swap_blocks(const int32_t *block_ids, int32_t n, void *k_cache, void *v_cache, const pkv_pool &pool,
+                       const void *host_k, const void *host_v, pkv_stream_t stream) {
+    const pkv_status ps = check_pool(pool);
+    if (ps != PKV_OK) return ps;
+    if (n < 0) return PKV_EINVAL;
+    if (n == 0) return PKV_OK;
+    if (!block_ids || !k_cache || !v_cache || !host_k || !host_v) return PKV_EINVAL;
+    if (!aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(host_k, 16) || !aligned(host_v, 16))
+        return PKV_EINVAL;
+    for (int i = 0; i < n; ++i)
+        if (block_ids[i] < 0 || block_ids[i] >= pool.num_blocks) return PKV_ERANGE;
+    if (!OUT) {  // two copies into one block would leave it undefined
+        std::vector<int32_t> ids(block_ids, block_ids + n);
+        std::sort(ids.begin(), ids.end());
+        for (int i = 1; i < n; ++i)
+            if (ids[i] == ids[i - 1]) return PKV_EALIAS;
+    }
+    uint8_t *hk = static_cast<uint8_t *>(mapped_host_pointer(host_k));
+    uint8_t *hv = static_cast<uint8_t *>(mapped_host_pointer(host_v));
+    if (!hk || !hv) return PKV_EINVAL;
+    const size_t block_bytes = (size_t)pool.num_kv_heads * pool.block_size * pool.head_dim * 2;
+    pkv::SwapParams p;
+    p.pool_k = static_cast<uint4 *>(k_cache);
+    p.pool_v = static_cast<uint4 *>(v_cache);
+    p.vec_per_block = (int64_t)(block_bytes / 16);
+    const long long per_cta = pkv::kSwapThreads * pkv::kSwapVecPerThread;
+    const unsigned gx = (unsigned)((p.vec_per_block + per_cta - 1) / per_cta);
+    for (int base = 0; base < n; base += pkv::kMaxSwapPerLaunch) {
+        const int m = std::min(pkv::kMaxSwapPerLaunch, n - base);
+        p.n = m;
+        p.host_k = reinterpret_cast<uint4 *>(hk + (size_t)base * block_bytes);
+        p.host_v = reinterpret_cast<uint4 *>(hv + (size_t)base * block_bytes);
+        std::memcpy(p.ids, block_ids + base, sizeof(int32_t) * m);
+        pkv::swap_blocks_kernel<OUT><<<dim3(gx, m), pkv::kSwapThreads, 0, (cudaStream_t)stream>>>(p);
+        const pkv_status st = launch_status();
+        if (st != PKV_OK) return st;
+    }
+    return PKV_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -364,6 +417,36 @@ pkv_status pkv_copy_blocks(const int32_t *src_dst_pairs, int32_t num_pairs, void
         const pkv_status st = launch_status();
         if (st != PKV_OK) return st;
     }
+    return PKV_OK;
+}
+
+pkv_status pkv_swap_out(const void *k_cache, const void *v_cache, pkv_pool pool, const int32_t *block_ids,
+                        int32_t n, void *host_k, void *host_v, pkv_stream_t stream) {
+    return swap_blocks<true>(block_ids, n, const_cast<void *>(k_cache), const_cast<void *>(v_cache), pool, host_k,
+                             host_v, stream);
+}
+
+pkv_status pkv_swap_in(const void *host_k, const void *host_v, const int32_t *block_ids, int32_t n, void *k_cache,
+                       void *v_cache, pkv_pool pool, pkv_stream_t stream) {
+    return swap_blocks<false>(block_ids, n, k_cache, v_cache, pool, host_k, host_v, stream);
+}
+
+pkv_status pkv_lru_victims(const int64_t *last_use, const uint8_t *evictable, int32_t num_blocks, int32_t k,
+                           int32_t *victims, int32_t *count) {
+    if (num_blocks < 0 || k < 0 || !count) return PKV_EINVAL;
+    if (num_blocks > 0 && (!last_use || !evictable)) return PKV_EINVAL;
+    if (k > 0 && !victims) return PKV_EINVAL;
+    std::vector<int32_t> cand;
+    cand.reserve(num_blocks);
+    for (int32_t b = 0; b < num_blocks; ++b)
+        if (evictable[b]) cand.push_back(b);
+    const size_t m = std::min<size_t>((size_t)k, cand.size());
+    auto older = [&](int32_t a, int32_t b) {
+        return last_use[a] < last_use[b] || (last_use[a] == last_use[b] && a < b);
+    };
+    std::partial_sort(cand.begin(), cand.begin() + m, cand.end(), older);
+    for (size_t i = 0; i < m; ++i) victims[i] = cand[i];
+    *count = (int32_t)m;
     return PKV_OK;
 }
 

@@ -90,4 +90,54 @@ __global__ void __launch_bounds__(kCopyThreads) copy_blocks_kernel(const __grid_
     }
 }
 
+// ----------------------------------------------------------------- swap ----
+// Whole blocks (all heads, K and V) between the pool and host memory that the
+// device can address (pinned, mapped through unified addressing).  Block ids
+// travel by value; grid.y = list position, grid.x = chunk of the block.
+// OUT gathers pool blocks into the packed host arrays [n][Hkv][bs][D]; IN
+// scatters them back.  Each thread keeps kSwapVecPerThread 16-byte vectors of
+// K and of V in flight (host memory is far: loads first, then stores).
+constexpr int kMaxSwapPerLaunch = 2048;  // 8 KB of parameters
+constexpr int kSwapThreads = 256;
+constexpr int kSwapVecPerThread = 4;
+
+struct SwapParams {
+    uint4 *pool_k;
+    uint4 *pool_v;
+    uint4 *host_k;  // first block of this launch
+    uint4 *host_v;
+    int64_t vec_per_block;  // Hkv * bs * D / 8
+    int n;
+    int32_t ids[kMaxSwapPerLaunch];
+};
+
+template <bool OUT>
+__global__ void __launch_bounds__(kSwapThreads) swap_blocks_kernel(const __grid_constant__ SwapParams p) {
+    const int i = blockIdx.y;
+    const int64_t pool_off = (int64_t)p.ids[i] * p.vec_per_block;
+    const int64_t host_off = (int64_t)i * p.vec_per_block;
+    const uint4 *sk = OUT ? p.pool_k + pool_off : p.host_k + host_off;
+    const uint4 *sv = OUT ? p.pool_v + pool_off : p.host_v + host_off;
+    uint4 *dk = OUT ? p.host_k + host_off : p.pool_k + pool_off;
+    uint4 *dv = OUT ? p.host_v + host_off : p.pool_v + pool_off;
+    const int64_t base = (int64_t)blockIdx.x * (kSwapThreads * kSwapVecPerThread) + threadIdx.x;
+    uint4 kv[kSwapVecPerThread], vv[kSwapVecPerThread];
+#pragma unroll
+    for (int u = 0; u < kSwapVecPerThread; ++u) {
+        const int64_t e = base + u * kSwapThreads;
+        if (e < p.vec_per_block) {
+            kv[u] = sk[e];
+            vv[u] = sv[e];
+        }
+    }
+#pragma unroll
+    for (int u = 0; u < kSwapVecPerThread; ++u) {
+        const int64_t e = base + u * kSwapThreads;
+        if (e < p.vec_per_block) {
+            dk[e] = kv[u];
+            dv[e] = vv[u];
+        }
+    }
+}
+
 }  // namespace pkv
