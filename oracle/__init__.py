@@ -54,10 +54,17 @@ def _load() -> ctypes.CDLL:
         lib.oracle_swap_out.argtypes = [P, P, P, I, I, I, I, I, P, P]
         lib.oracle_swap_in.argtypes = [P, P, P, I, I, I, I, I, P, P]
         lib.oracle_lru_victims.argtypes = [P, P, I, I, P, P]
+        lib.oracle_bm_init.argtypes = [P, P, P, I]
+        lib.oracle_bm_alloc.argtypes = [P, P, P, I, P, I, P, P, I, P]
+        lib.oracle_bm_free.argtypes = [P, P, P, I, P, I, P]
+        lib.oracle_bm_share.argtypes = [P, I, P, I, P]
+        lib.oracle_bm_append_slots.argtypes = [P, P, P, I, P, I, P, P, I, I, P, P, P, P]
         lib.oracle_num_threads.argtypes = []
         for f in (lib.oracle_kv_write, lib.oracle_copy_blocks, lib.oracle_paged_attention,
                   lib.oracle_attention_partial, lib.oracle_lse_merge, lib.oracle_num_threads,
-                  lib.oracle_paged_prefill, lib.oracle_swap_out, lib.oracle_swap_in, lib.oracle_lru_victims):
+                  lib.oracle_paged_prefill, lib.oracle_swap_out, lib.oracle_swap_in, lib.oracle_lru_victims,
+                  lib.oracle_bm_init, lib.oracle_bm_alloc, lib.oracle_bm_free, lib.oracle_bm_share,
+                  lib.oracle_bm_append_slots):
             f.restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -170,6 +177,91 @@ def lru_victims(last_use, evictable, k: int) -> np.ndarray:
     rc = _load().oracle_lru_victims(_ptr(lu), _ptr(ev), lu.shape[0], int(k), _ptr(out), _ptr(cnt))
     _check(rc, "lru_victims")
     return out[:int(cnt[0])].copy()
+
+
+# ---------------------------------------------------------------------------
+# block manager (state: free stack, its top, reference counts)
+# ---------------------------------------------------------------------------
+
+BM_ERR_NOSPACE, BM_ERR_RANGE, BM_ERR_DOUBLEFREE, BM_ERR_TABLE = 1, 2, 4, 8
+
+
+class BlockState:
+    """free_stack[:top] are the free ids (the next allocation pops
+    free_stack[top - 1]); refcount[b] counts the sequences mapping block b."""
+
+    def __init__(self, free_stack, top, refcount):
+        self.free_stack = np.ascontiguousarray(free_stack, dtype=np.int32)
+        self.top = int(top)
+        self.refcount = np.ascontiguousarray(refcount, dtype=np.int32)
+
+    def copy(self):
+        return BlockState(self.free_stack.copy(), self.top, self.refcount.copy())
+
+    @property
+    def num_blocks(self):
+        return self.refcount.shape[0]
+
+    def free_set(self):
+        return set(self.free_stack[:self.top].tolist())
+
+
+def _bm_call(fn, st: BlockState, *args):
+    top = np.array([st.top], dtype=np.int32)
+    rc = fn(_ptr(st.free_stack), _ptr(top), _ptr(st.refcount), st.num_blocks, *args)
+    st.top = int(top[0])
+    return rc
+
+
+def bm_init(num_blocks: int) -> BlockState:
+    st = BlockState(np.zeros(num_blocks, np.int32), 0, np.zeros(num_blocks, np.int32))
+    _check(_bm_call(_load().oracle_bm_init, st), "bm_init")
+    return st
+
+
+def bm_alloc(st: BlockState, counts, capacity: int):
+    """Returns (new state, offsets [n+1], ids [capacity], err)."""
+    st = st.copy()
+    c = np.ascontiguousarray(counts, dtype=np.int32).reshape(-1)
+    offsets = np.zeros(c.shape[0] + 1, dtype=np.int32)
+    ids = np.full(max(capacity, 1), -1, dtype=np.int32)
+    err = np.zeros(1, dtype=np.uint32)
+    _check(_bm_call(_load().oracle_bm_alloc, st, _ptr(c), c.shape[0], _ptr(offsets), _ptr(ids), int(capacity),
+                    _ptr(err)), "bm_alloc")
+    return st, offsets, ids[:capacity], int(err[0])
+
+
+def bm_free(st: BlockState, ids):
+    st = st.copy()
+    a = np.ascontiguousarray(ids, dtype=np.int32).reshape(-1)
+    err = np.zeros(1, dtype=np.uint32)
+    _check(_bm_call(_load().oracle_bm_free, st, _ptr(a), a.shape[0], _ptr(err)), "bm_free")
+    return st, int(err[0])
+
+
+def bm_share(st: BlockState, ids):
+    st = st.copy()
+    a = np.ascontiguousarray(ids, dtype=np.int32).reshape(-1)
+    err = np.zeros(1, dtype=np.uint32)
+    _check(_load().oracle_bm_share(_ptr(st.refcount), st.num_blocks, _ptr(a), a.shape[0], _ptr(err)), "bm_share")
+    return st, int(err[0])
+
+
+def bm_append_slots(st: BlockState, block_tables, context_lens, num_new, block_size: int):
+    """Returns (new state, tables, context_lens, slot_mapping int64, pairs [P, 2], err)."""
+    st = st.copy()
+    tables = np.ascontiguousarray(block_tables, dtype=np.int32).copy()
+    ctx = np.ascontiguousarray(context_lens, dtype=np.int32).copy()
+    nn = np.ascontiguousarray(num_new, dtype=np.int32).reshape(-1)
+    B, mbs = tables.shape
+    assert ctx.shape == (B,) and nn.shape == (B,)
+    slots = np.full(max(int(np.clip(nn, 0, None).sum()), 1), -7, dtype=np.int64)
+    pairs = np.zeros((max(B, 1), 2), dtype=np.int32)
+    npairs = np.zeros(1, dtype=np.int32)
+    err = np.zeros(1, dtype=np.uint32)
+    _check(_bm_call(_load().oracle_bm_append_slots, st, _ptr(tables), mbs, _ptr(ctx), _ptr(nn), B, int(block_size),
+                    _ptr(slots), _ptr(pairs), _ptr(npairs), _ptr(err)), "bm_append_slots")
+    return st, tables, ctx, slots[:int(np.clip(nn, 0, None).sum())], pairs[:int(npairs[0])].copy(), int(err[0])
 
 
 def paged_attention(q, k_cache, v_cache, block_tables, context_lens, scale: float) -> np.ndarray:

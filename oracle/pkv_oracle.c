@@ -16,6 +16,12 @@
  *     computes ordinary attention over it (wkbse.com section 3.1, third point
  *     of the list), i.e. softmax(q K^T * scale) V.
  *   - copy-on-write of a shared block (intelliparadigm.com section 2.1, item 2).
+ *   - the block manager: a free list popped on allocation, blocks allocated as
+ *     new tokens need them and the block table updated, blocks returned when
+ *     a sequence ends, shared blocks counted by reference and copied before a
+ *     sharer writes into them (wkbse.com section 3.1, "flexible memory
+ *     management" and "KV cache sharing"; intelliparadigm.com section 2.1,
+ *     items 1-2 and the block-allocation sketch).
  *   - swap of cold blocks to CPU memory and back, victims chosen least
  *     recently used first (intelliparadigm.com section 2.1, item 3; ai-stack.site
  *     "Nano-vLLM 原理", practice 5, preemption by swapping a request's KV cache).
@@ -359,5 +365,136 @@ int oracle_lru_victims(const int64_t *last_use, const uint8_t *evictable, int nu
     }
     free(taken);
     *count = c;
+    return 0;
+}
+
+/* ------------------------------------------------------------------------
+ * Block manager.  State: free_stack[0 .. *top) holds the free block ids; an
+ * allocation pops free_stack[*top - 1]; refcount[b] counts the sequences that
+ * map block b.  err collects the bits BM_ERR_* below.  Everything is a plain
+ * sequential loop in request order.
+ * ------------------------------------------------------------------------ */
+#define BM_ERR_NOSPACE 1u    /* a request found too few free blocks (or output room) */
+#define BM_ERR_RANGE 2u      /* a block id outside the pool */
+#define BM_ERR_DOUBLEFREE 4u /* a block freed more often than it was referenced */
+#define BM_ERR_TABLE 8u      /* a sequence outgrew its block-table row */
+
+int oracle_bm_init(int32_t *free_stack, int32_t *top, int32_t *refcount, int num_blocks) {
+    if (num_blocks <= 0) return 1;
+    for (int i = 0; i < num_blocks; ++i) {
+        free_stack[i] = num_blocks - 1 - i; /* block 0 is popped first */
+        refcount[i] = 0;
+    }
+    *top = num_blocks;
+    return 0;
+}
+
+static int32_t bm_pop(int32_t *free_stack, int32_t *top, int32_t *refcount) {
+    int32_t b = free_stack[--*top];
+    refcount[b] = 1;
+    return b;
+}
+
+/* Request r receives counts[r] blocks, written to ids[offsets[r] .. offsets[r+1]).
+ * Requests are served in order while the free list and the output room last;
+ * the first one that does not fit, and every later one, receives none. */
+int oracle_bm_alloc(int32_t *free_stack, int32_t *top, int32_t *refcount, int num_blocks, const int32_t *counts,
+                    int n, int32_t *offsets, int32_t *ids, int capacity, uint32_t *err) {
+    if (num_blocks <= 0 || n < 0 || capacity < 0) return 1;
+    int failed = 0;
+    offsets[0] = 0;
+    for (int r = 0; r < n; ++r) {
+        int c = counts[r] < 0 ? 0 : counts[r];
+        if (!failed && c <= *top && offsets[r] + c <= capacity) {
+            for (int k = 0; k < c; ++k) ids[offsets[r] + k] = bm_pop(free_stack, top, refcount);
+            offsets[r + 1] = offsets[r] + c;
+        } else {
+            if (c > 0 || failed) { failed = 1; *err |= BM_ERR_NOSPACE; }
+            offsets[r + 1] = offsets[r];
+        }
+    }
+    return 0;
+}
+
+/* Each listed id drops one reference, in list order; a block whose count
+ * reaches zero is pushed back onto the free list at that moment. */
+int oracle_bm_free(int32_t *free_stack, int32_t *top, int32_t *refcount, int num_blocks, const int32_t *ids, int n,
+                   uint32_t *err) {
+    if (num_blocks <= 0 || n < 0) return 1;
+    for (int i = 0; i < n; ++i) {
+        int32_t b = ids[i];
+        if (b < 0 || b >= num_blocks) { *err |= BM_ERR_RANGE; continue; }
+        if (refcount[b] <= 0) { *err |= BM_ERR_DOUBLEFREE; continue; }
+        if (--refcount[b] == 0) free_stack[(*top)++] = b;
+    }
+    return 0;
+}
+
+/* Each listed id gains one reference (a new sequence maps the block). */
+int oracle_bm_share(int32_t *refcount, int num_blocks, const int32_t *ids, int n, uint32_t *err) {
+    if (num_blocks <= 0 || n < 0) return 1;
+    for (int i = 0; i < n; ++i) {
+        if (ids[i] < 0 || ids[i] >= num_blocks) { *err |= BM_ERR_RANGE; continue; }
+        refcount[ids[i]] += 1;
+    }
+    return 0;
+}
+
+/* One step's slots for num_new[b] new tokens of every sequence b, in order:
+ *   - if the tokens go into a partly filled last block that other sequences
+ *     still map (refcount > 1), that block is first replaced by a private
+ *     copy: a new block, the pair (old, new) appended to pairs, one reference
+ *     of the old block dropped (copy-on-write);
+ *   - blocks for the logical indices the new tokens reach beyond the table
+ *     are popped in logical order;
+ *   - slot_mapping[off_b + t] = table[b][p / bs] * bs + p % bs for position
+ *     p = context_lens[b] + t, off_b the sum of num_new over earlier b;
+ *   - context_lens[b] grows by num_new[b].
+ * A sequence that finds too few free blocks or outgrows its table row, and
+ * every later one, is left unchanged with slots -1 (padding). */
+int oracle_bm_append_slots(int32_t *free_stack, int32_t *top, int32_t *refcount, int num_blocks,
+                           int32_t *block_tables, int mbs, int32_t *context_lens, const int32_t *num_new, int B,
+                           int bs, int64_t *slot_mapping, int32_t *pairs, int32_t *num_pairs, uint32_t *err) {
+    if (num_blocks <= 0 || B < 0 || bs <= 0 || mbs <= 0) return 1;
+    int failed = 0;
+    int64_t off = 0;
+    *num_pairs = 0;
+    for (int b = 0; b < B; ++b) {
+        int n = num_new[b] < 0 ? 0 : num_new[b];
+        int32_t pos0 = context_lens[b];
+        int32_t *row = block_tables + (size_t)b * mbs;
+        int first_new = (pos0 + bs - 1) / bs;              /* first logical block not yet mapped */
+        int last = n > 0 ? (pos0 + n - 1) / bs : first_new - 1;
+        int need_new = last >= first_new ? last - first_new + 1 : 0;
+        int cow = 0;
+        if (n > 0 && pos0 % bs != 0) {
+            int32_t cur = row[pos0 / bs];
+            if (cur < 0 || cur >= num_blocks) { *err |= BM_ERR_RANGE; failed = 1; }
+            else if (refcount[cur] > 1) cow = 1;
+        }
+        if (!failed && n > 0 && last >= mbs) { *err |= BM_ERR_TABLE; failed = 1; }
+        if (!failed && need_new + cow > *top) { *err |= BM_ERR_NOSPACE; failed = 1; }
+        if (failed) {
+            for (int t = 0; t < n; ++t) slot_mapping[off + t] = -1;
+            off += n;
+            continue;
+        }
+        if (cow) {
+            int32_t old = row[pos0 / bs];
+            int32_t fresh = bm_pop(free_stack, top, refcount);
+            refcount[old] -= 1;
+            row[pos0 / bs] = fresh;
+            pairs[2 * *num_pairs] = old;
+            pairs[2 * *num_pairs + 1] = fresh;
+            *num_pairs += 1;
+        }
+        for (int L = first_new; L <= last; ++L) row[L] = bm_pop(free_stack, top, refcount);
+        for (int t = 0; t < n; ++t) {
+            int32_t p = pos0 + t;
+            slot_mapping[off + t] = (int64_t)row[p / bs] * bs + p % bs;
+        }
+        context_lens[b] = pos0 + n;
+        off += n;
+    }
     return 0;
 }

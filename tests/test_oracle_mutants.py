@@ -15,6 +15,7 @@ import pytest
 import oracle
 from tests import test_oracle_pins as pins
 from tests import test_oracle_prefill as prefill_pins
+from tests import test_oracle_block_manager as bm_pins
 from tests import test_oracle_swap as swap_pins
 
 PIN_TESTS = [
@@ -37,6 +38,11 @@ PIN_TESTS = [
     swap_pins.test_swap_round_trip_restores_and_swap_out_reads_only,
     swap_pins.test_swap_of_a_permutation_is_a_gather,
     swap_pins.test_lru_worked_example_golden,
+    bm_pins.test_block_manager_worked_example_golden,
+    lambda: bm_pins.test_conservation_invariants(0),
+    lambda: bm_pins.test_append_block_counts_closed_form(0),
+    bm_pins.test_slots_feed_the_table_walk,
+    lambda: bm_pins.test_free_matches_python_restatement(0),
     lambda: swap_pins.test_lru_characterisation(0),
 ]
 
@@ -66,6 +72,19 @@ MUTANTS = {
                             "k_cache[(size_t)((ids[i] + 1) % num_blocks) * block_elems + e] = host_k["),
     "lru newest first": ("last_use[b] < last_use[best]", "last_use[b] > last_use[best]"),
     "lru ties to higher id": ("last_use[b] < last_use[best]", "last_use[b] <= last_use[best]"),
+    # block manager: copy-on-write of unshared blocks; the old block keeps its
+    # reference; a partly filled block allocated again; the slot offset from the
+    # wrong position; freeing pushes before the count reaches zero; the free
+    # list used first-in first-out
+    "cow unshared": ("else if (refcount[cur] > 1) cow = 1;", "else if (refcount[cur] >= 1) cow = 1;"),
+    "cow keeps reference": ("refcount[old] -= 1;", "refcount[old] -= 0;"),
+    "partial block reallocated": ("int first_new = (pos0 + bs - 1) / bs;", "int first_new = pos0 / bs + (pos0 > 0);"),
+    "slot offset": ("slot_mapping[off + t] = (int64_t)row[p / bs] * bs + p % bs;",
+                    "slot_mapping[off + t] = (int64_t)row[p / bs] * bs + t % bs;"),
+    "free pushes early": ("if (--refcount[b] == 0) free_stack[(*top)++] = b;",
+                          "--refcount[b]; free_stack[(*top)++] = b;"),
+    "fifo free list": ("int32_t b = free_stack[--*top];",
+                       "int32_t b = free_stack[0]; memmove(free_stack, free_stack + 1, sizeof(int32_t) * (size_t)(--*top));"),
     # the new token left out of the attended range (context_len - 1 tokens)
     "context off by one": ("hq, 0, context_lens[s], scale", "hq, 0, context_lens[s] - 1, scale"),
 }
