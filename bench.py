@@ -477,6 +477,135 @@ def run_prefill_cuda(args, rank, world, dist):
 
 
 SWAP_WORKLOADS = ("llama2-13b-swap",)
+BM_WORKLOADS = ("llama2-13b-blockmgr",)
+
+
+def run_blockmgr_cuda(args, rank, world, dist):
+    """Device block manager on the Llama-2-13B batch (128 sequences, their
+    context lengths): one step = append_slots for one new token per sequence
+    (block allocation as sequences cross a block boundary, slot mapping, copy-
+    on-write checks), timed per call; a 512-token chunk per sequence for 8
+    sequences is timed as the prefill case.  Metric: microseconds per decode
+    step; the floor is an empty kernel's launch-to-completion on the same
+    stream.  The CPU baseline is the oracle's sequential append on the host."""
+    import oracle
+    import paged_kv_cache_420_b200 as pkv
+
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
+    torch.cuda.set_device(dev)
+    w = workloads.make("llama2-13b", seed=args.seed + rank, values_device="cpu", block_size=args.block_size)
+    B, bs = w.num_seqs, w.block_size
+    steps = args.steps
+    mbs = (int(w.context_lens.max()) + steps + 2 * bs) // bs + 1
+    nb = B * mbs + 64
+    stream = torch.cuda.current_stream()
+
+    def fresh():
+        bm = pkv.BlockManager(nb, device=dev)
+        t = torch.full((B, mbs), -1, dtype=torch.int32, device=dev)
+        c = torch.zeros(B, dtype=torch.int32, device=dev)
+        fill = torch.from_numpy(w.context_lens.astype(np.int32)).to(dev)
+        bm.append_slots(t, c, fill, bs, int(w.context_lens.sum()))
+        return bm, t, c
+
+    bm, tables, ctx = fresh()
+    one = torch.ones(B, dtype=torch.int32, device=dev)
+    out = (torch.empty(B, dtype=torch.int64, device=dev), torch.empty((B, 2), dtype=torch.int32, device=dev),
+           torch.empty(1, dtype=torch.int32, device=dev))
+    for _ in range(max(args.warmup, 3)):
+        bm.append_slots(tables, ctx, one, bs, B, out=out)
+    torch.cuda.synchronize()
+    # the steps go into CUDA graphs of 64 calls: the device time, not the
+    # Python enqueue rate, is what is measured
+    per_graph = 64
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        for _ in range(per_graph):
+            bm.append_slots(tables, ctx, one, bs, B, out=out)
+    torch.cuda.synchronize()
+    reps = max(1, steps // per_graph)
+    steps = reps * per_graph
+    mbs_needed = (int(ctx.max().item()) + steps + bs) // bs
+    if mbs_needed > mbs:
+        raise RuntimeError("block-table rows too short for the timed steps")
+    if dist is not None:
+        dist.barrier()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(dev.index) as clocks:
+        t0.record(stream)
+        for _ in range(reps):
+            graph.replay()
+        t1.record(stream)
+        torch.cuda.synchronize()
+        if dist is not None:
+            dist.barrier()
+        if t0.elapsed_time(t1) < 450:
+            time.sleep(0.45)
+    if bm.error():
+        raise RuntimeError(f"block manager error word {bm.error():#x}")
+    ms_max, _, _ = combine_ranks(dist, t0.elapsed_time(t1), B, B, dev)
+    per_call_us = 1e3 * t0.elapsed_time(t1) / steps
+    del graph
+    # prefill-sized step: 8 sequences, 512 new tokens each
+    bm2, t2, c2 = fresh()
+    chunk = torch.zeros(B, dtype=torch.int32, device=dev)
+    chunk[:8] = 512
+    pre = []
+    pout = (torch.empty(8 * 512, dtype=torch.int64, device=dev), torch.empty((B, 2), dtype=torch.int32, device=dev),
+            torch.empty(1, dtype=torch.int32, device=dev))
+    for _ in range(5):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        bm2, t2, c2 = fresh()
+        torch.cuda.synchronize()
+        a.record(stream)
+        bm2.append_slots(t2, c2, chunk, bs, 8 * 512, out=pout)
+        b.record(stream)
+        torch.cuda.synchronize()
+        pre.append(a.elapsed_time(b) * 1e3)
+    # floor: an empty kernel, launch to completion
+    nop = torch.empty(1, device=dev)
+    g2 = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g2):
+        for _ in range(per_graph):
+            nop.zero_()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(10):
+        g2.replay()
+    b.record(stream)
+    torch.cuda.synchronize()
+    floor_us = 1e3 * a.elapsed_time(b) / (10 * per_graph)
+    del g2
+    # CPU baseline: the oracle's sequential append for the same decode step
+    st = oracle.bm_init(nb)
+    ot = np.full((B, mbs), -1, np.int32)
+    st, ot, oc, _, _, _ = oracle.bm_append_slots(st, ot, np.zeros(B, np.int32), w.context_lens.astype(np.int32), bs)
+    ones = np.ones(B, np.int32)
+    t = time.perf_counter()
+    n_cpu = 0
+    while time.perf_counter() - t < 2.0:
+        st, ot, oc, _, _, _ = oracle.bm_append_slots(st, ot, oc, ones, bs)
+        n_cpu += 1
+        if int(oc.max()) + 1 >= mbs * bs:
+            break
+    cpu_us = (time.perf_counter() - t) / max(n_cpu, 1) * 1e6
+    return {
+        "metric": "device block-manager append_slots microseconds per decode step",
+        "value": round(1e3 * ms_max / steps, 3), "unit": "us", "n_gpus": world, "steps": steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_max / steps, 5), "higher_is_better": False,
+        "scaling": "weak", "vs_baseline": None, "dtype": "int32", "data": "synthetic",
+        "config": {"workload": f"llama2-13b batch: {B} sequences, bs {bs}, one new token each per step; "
+                               f"prefill case 8 x 512 tokens", "block_size": bs, "seed": args.seed},
+        "roofline": {"kernel": "bm_append_slots_kernel", "bound": "latency", "achieved": round(per_call_us, 2),
+                     "peak": round(floor_us, 2),
+                     "peak_kind": "measured: one-thread kernel per graph node, back to back (launch floor)",
+                     "unit": "us", "frac": round(floor_us / per_call_us, 4),
+                     "prefill_8x512_us": round(float(np.median(pre)), 2), "traffic": None},
+        "cpu_baseline": {"value": round(cpu_us, 2), "unit": "us", "cores": 1, "kind": "oracle",
+                         "sample": f"{n_cpu} sequential append steps of the same batch"},
+        "e2e": None, "gpu_launches": steps, "clocks": clocks.summary(),
+    }
 
 
 def run_swap_cuda(args, rank, world, dist):
@@ -710,6 +839,36 @@ def run_swap_reference(args, world):
     }
 
 
+def run_blockmgr_reference(args, world):
+    """The oracle's sequential append_slots on the host for the same decode step."""
+    import oracle
+
+    w = workloads.make("llama2-13b", seed=args.seed, values_device="cpu", block_size=args.block_size)
+    B, bs = w.num_seqs, w.block_size
+    mbs = (int(w.context_lens.max()) + args.steps + args.warmup + 2 * bs) // bs + 1
+    st = oracle.bm_init(B * mbs + 64)
+    ot = np.full((B, mbs), -1, np.int32)
+    st, ot, oc, _, _, _ = oracle.bm_append_slots(st, ot, np.zeros(B, np.int32), w.context_lens.astype(np.int32), bs)
+    ones = np.ones(B, np.int32)
+    times = []
+    for i in range(args.warmup + args.steps):
+        t = time.perf_counter()
+        st, ot, oc, _, _, _ = oracle.bm_append_slots(st, ot, oc, ones, bs)
+        if i >= args.warmup:
+            times.append(time.perf_counter() - t)
+    value = round(statistics.median(times) * 1e6, 3)
+    return {
+        "impl": "reference", "metric": "device block-manager append_slots microseconds per decode step",
+        "value": value, "unit": "us", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(1e3 * sum(times) / len(times), 4), "higher_is_better": False, "scaling": "weak",
+        "vs_baseline": None, "dtype": "int32", "data": "synthetic",
+        "config": {"workload": f"llama2-13b batch: {B} sequences, one new token each", "block_size": bs},
+        "cpu_baseline": {"value": value, "unit": "us", "cores": 1, "kind": "oracle",
+                         "sample": "the whole decode step per step"},
+        "e2e": {"value": value, "unit": "us", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
 def run_reference(args, rank, world):
     """The CPU oracle as the reference arm: rank 0 times it on the host cores,
     one bounded sample of the workload per step."""
@@ -719,6 +878,8 @@ def run_reference(args, rank, world):
         return run_prefill_reference(args, world)
     if args.workload in SWAP_WORKLOADS:
         return run_swap_reference(args, world)
+    if args.workload in BM_WORKLOADS:
+        return run_blockmgr_reference(args, world)
     w = workloads.make(args.workload, seed=args.seed, values_device="cpu", block_size=args.block_size)
     per_step_budget = max(0.05, min(2.0, 150.0 / max(1, args.steps + args.warmup)))
     pools = oracle_pools(w)
@@ -755,7 +916,8 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["pkv", "reference"], default="pkv")
     ap.add_argument("--workload", default="llama2-13b",
-                    choices=list(workloads.WORKLOADS) + list(workloads.PREFILL_WORKLOADS) + list(SWAP_WORKLOADS))
+                    choices=list(workloads.WORKLOADS) + list(workloads.PREFILL_WORKLOADS) + list(SWAP_WORKLOADS)
+                    + list(BM_WORKLOADS))
     ap.add_argument("--block-size", type=int, default=None)
     ap.add_argument("--partition-tokens", type=int, default=-1, help="-1: the workload's choice, 0: library's")
     ap.add_argument("--seed", type=int, default=0)
@@ -783,6 +945,8 @@ def main(argv=None):
             line = run_prefill_cuda(args, rank, world, dist)
         elif args.workload in SWAP_WORKLOADS:
             line = run_swap_cuda(args, rank, world, dist)
+        elif args.workload in BM_WORKLOADS:
+            line = run_blockmgr_cuda(args, rank, world, dist)
         else:
             line = run_cuda(args, rank, world, dist)
         if rank == 0 and line is not None:

@@ -271,6 +271,78 @@ pkv_status paged_attn_prefill(const void *q, const void *k_cache, const void *v_
                               void *workspace, size_t workspace_bytes, pkv_stream_t stream);
 
 /*
+ * Block manager on the device -- the bookkeeping of the pages' block manager
+ * (wkbse.com section 3.1, "flexible memory management": blocks allocated only
+ * as new tokens need them, the block table updated, blocks returned when a
+ * sequence ends; "KV cache sharing": parallel samples map the same physical
+ * blocks; intelliparadigm.com section 2.1, items 1-2 and the allocation
+ * sketch: a free list popped on allocation, copy-on-write for shared
+ * prefixes), so a serving step needs no host round trip.
+ *
+ * State: one device buffer of pkv_bm_state_bytes(num_blocks), 256-B aligned,
+ * owned by the caller, laid out as
+ *   int32 [0] top, [1] error word (PKV_BM_ERR_* bits; the caller clears it)
+ *   at 256:            int32 free_stack[num_blocks]  (free_stack[0 .. top) are free,
+ *                      the next allocation pops free_stack[top - 1])
+ *   at 256 + A:        int32 refcount[num_blocks]     (sequences mapping each block)
+ *   at 256 + 2A..4A:   three int32 scratch arrays kept at their rest values
+ * with A = num_blocks * 4 rounded up to 256.  Every call is one kernel on
+ * `stream` (one CTA walking its list in order with block-wide scans), so its
+ * results are exactly the sequential, request-order ones; device-side
+ * failures set bits in the error word and leave the failing request (and,
+ * for alloc and append, every later one) unserved.  All arrays are device
+ * memory.  Calls on one state must be ordered (one stream).
+ */
+#define PKV_BM_ERR_NOSPACE 1u    /* too few free blocks, or no room in ids, for a request */
+#define PKV_BM_ERR_RANGE 2u      /* a block id outside [0, num_blocks) */
+#define PKV_BM_ERR_DOUBLEFREE 4u /* a block freed more often than referenced */
+#define PKV_BM_ERR_TABLE 8u      /* a sequence outgrew its block-table row, or its context was outside it */
+
+size_t pkv_bm_state_bytes(int32_t num_blocks);
+/* All blocks free, popped 0, 1, 2, ... first; reference counts 0; error word 0. */
+pkv_status pkv_bm_init(void *state, int32_t num_blocks, pkv_stream_t stream);
+/* Request r (of n) receives counts[r] blocks (reference count 1) at
+ * ids[offsets[r] .. offsets[r+1]) (offsets: int32 [n+1]); requests are served
+ * in order while free blocks and the capacity of ids last. */
+pkv_status pkv_bm_alloc(void *state, int32_t num_blocks, const int32_t *counts, int32_t n, int32_t *offsets,
+                        int32_t *ids, int32_t capacity, pkv_stream_t stream);
+/* Every listed block drops one reference, in list order; a block whose count
+ * reaches zero is pushed back on the free list at that point. */
+pkv_status pkv_bm_free(void *state, int32_t num_blocks, const int32_t *block_ids, int32_t n, pkv_stream_t stream);
+/* Every listed block gains one reference (a new sequence maps it, e.g. a fork). */
+pkv_status pkv_bm_share(void *state, int32_t num_blocks, const int32_t *block_ids, int32_t n, pkv_stream_t stream);
+/*
+ * One step's slots for num_new[b] new tokens of each sequence b < num_seqs, in
+ * sequence order: (1) if the tokens go into a partly filled last block that
+ * other sequences still map (reference count > 1), it is replaced by a fresh
+ * private block and the pair (old, fresh) is appended to cow_pairs (int32
+ * [num_seqs][2]; count in *num_cow_pairs) -- copy-on-write; of k sharers of one
+ * such block appending in the same step, the first min(k, refs - 1) copy and
+ * the last writes in place; (2) fresh blocks fill the table entries the new
+ * tokens reach; (3) slot_mapping[off_b + t] = table[b][p / bs] * bs + p % bs
+ * for p = context_lens[b] + t (off_b = the sum of num_new over earlier
+ * sequences; int64 [slot_capacity]; entries past the capacity are not written
+ * and set PKV_BM_ERR_NOSPACE), ready for pkv_write; (4) context_lens[b]
+ * grows by num_new[b].  block_tables is int32 [num_seqs][max_blocks_per_seq],
+ * updated in place.  The first sequence that finds too few free blocks or
+ * outgrows its row, and every later one, is left unchanged with slots -1.
+ * Run pkv_copy_blocks_dev on the pairs before writing the new tokens.
+ */
+pkv_status pkv_bm_append_slots(void *state, int32_t num_blocks, int32_t *block_tables, int32_t max_blocks_per_seq,
+                               int32_t *context_lens, const int32_t *num_new, int32_t num_seqs, int32_t block_size,
+                               int64_t *slot_mapping, int64_t slot_capacity, int32_t *cow_pairs,
+                               int32_t *num_cow_pairs, pkv_stream_t stream);
+/*
+ * pkv_copy_blocks sourced from the device: copies the first *num_pairs of
+ * cow_pairs (device int32 [max_pairs][2], as pkv_bm_append_slots leaves them)
+ * without a host round trip.  The destinations must be fresh blocks that are
+ * no pair's source (true of append's pairs); ids outside the pool set
+ * PKV_DEVERR_BLOCK and are skipped.
+ */
+pkv_status pkv_copy_blocks_dev(const int32_t *cow_pairs, const int32_t *num_pairs, int32_t max_pairs, void *k_cache,
+                               void *v_cache, pkv_pool pool, pkv_stream_t stream);
+
+/*
  * pkv_get_device_error -- copies the current device's error word to
  * *code_out and clears it, ordered after the work already on `stream`, and
  * waits for it.  Returns PKV_EDEVICE when the word was non-zero.

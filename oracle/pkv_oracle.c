@@ -463,6 +463,13 @@ int oracle_bm_append_slots(int32_t *free_stack, int32_t *top, int32_t *refcount,
         int n = num_new[b] < 0 ? 0 : num_new[b];
         int32_t pos0 = context_lens[b];
         int32_t *row = block_tables + (size_t)b * mbs;
+        if (pos0 < 0 || pos0 > mbs * bs) { /* the context is not inside its own table row */
+            if (!failed) *err |= BM_ERR_TABLE;
+            failed = 1;
+            for (int t = 0; t < n; ++t) slot_mapping[off + t] = -1;
+            off += n;
+            continue;
+        }
         int first_new = (pos0 + bs - 1) / bs;              /* first logical block not yet mapped */
         int last = n > 0 ? (pos0 + n - 1) / bs : first_new - 1;
         int need_new = last >= first_new ? last - first_new + 1 : 0;

@@ -26,7 +26,8 @@ DEVERR_SLOT, DEVERR_BLOCK, DEVERR_CONTEXT, DEVERR_TIMEOUT, DEVERR_LAYOUT = 0x1, 
 EXPORTED = ("pkv_write", "pkv_copy_blocks", "pkv_decode_workspace_bytes", "paged_attn_decode",
             "paged_attn_decode_static_ws", "pkv_prefill_workspace_bytes", "paged_attn_prefill",
             "pkv_get_device_error", "pkv_selftest_bounded_wait", "pkv_status_string", "pkv_version",
-            "pkv_swap_out", "pkv_swap_in", "pkv_lru_victims")
+            "pkv_swap_out", "pkv_swap_in", "pkv_lru_victims", "pkv_bm_state_bytes", "pkv_bm_init", "pkv_bm_alloc",
+            "pkv_bm_free", "pkv_bm_share", "pkv_bm_append_slots", "pkv_copy_blocks_dev")
 STATIC_WS_BYTES = 32 << 20  # PKV_STATIC_WS_BYTES
 
 
@@ -61,11 +62,20 @@ def load_library() -> ctypes.CDLL:
         lib.pkv_swap_out.argtypes = [P, P, _Pool, P, I32, P, P, P]
         lib.pkv_swap_in.argtypes = [P, P, P, I32, P, P, _Pool, P]
         lib.pkv_lru_victims.argtypes = [P, P, I32, I32, P, P]
+        lib.pkv_bm_state_bytes.argtypes = [I32]
+        lib.pkv_bm_state_bytes.restype = SZ
+        lib.pkv_bm_init.argtypes = [P, I32, P]
+        lib.pkv_bm_alloc.argtypes = [P, I32, P, I32, P, P, I32, P]
+        lib.pkv_bm_free.argtypes = [P, I32, P, I32, P]
+        lib.pkv_bm_share.argtypes = [P, I32, P, I32, P]
+        lib.pkv_bm_append_slots.argtypes = [P, I32, P, I32, P, P, I32, I32, P, I64, P, P, P]
+        lib.pkv_copy_blocks_dev.argtypes = [P, P, I32, P, P, _Pool, P]
         lib.pkv_status_string.argtypes = [ctypes.c_int]
         lib.pkv_status_string.restype = ctypes.c_char_p
         lib.pkv_version.restype = I32
         for f in ("pkv_write", "pkv_copy_blocks", "paged_attn_decode", "pkv_get_device_error", "pkv_swap_out",
-                  "pkv_swap_in", "pkv_lru_victims"):
+                  "pkv_swap_in", "pkv_lru_victims", "pkv_bm_init", "pkv_bm_alloc", "pkv_bm_free", "pkv_bm_share",
+                  "pkv_bm_append_slots", "pkv_copy_blocks_dev"):
             getattr(lib, f).restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -188,6 +198,98 @@ def lru_victims(last_use, evictable, k: int) -> np.ndarray:
                                         lu.shape[0], int(k), out.ctypes.data_as(ctypes.c_void_p), ctypes.byref(cnt))
     _check(st, "pkv_lru_victims")
     return out[:cnt.value].copy()
+
+
+BM_ERR_NOSPACE, BM_ERR_RANGE, BM_ERR_DOUBLEFREE, BM_ERR_TABLE = 1, 2, 4, 8
+
+
+def bm_state_bytes(num_blocks: int) -> int:
+    n = load_library().pkv_bm_state_bytes(int(num_blocks))
+    if n == 0:
+        raise ValueError("num_blocks must be positive")
+    return int(n)
+
+
+class BlockManager:
+    """The block manager's state on the device (free list, reference counts)
+    and its per-step calls; every array argument is a CUDA int32 tensor."""
+
+    def __init__(self, num_blocks: int, device="cuda", stream=None):
+        self.num_blocks = int(num_blocks)
+        self.state = torch.empty(bm_state_bytes(num_blocks), dtype=torch.uint8, device=device)
+        a = (self.num_blocks * 4 + 255) // 256 * 256
+        self.header = self.state[:8].view(torch.int32)  # top, error word
+        self.free_stack = self.state[256:256 + 4 * self.num_blocks].view(torch.int32)
+        self.refcount = self.state[256 + a:256 + a + 4 * self.num_blocks].view(torch.int32)
+        _check(load_library().pkv_bm_init(_ptr(self.state), self.num_blocks, _stream(stream)), "pkv_bm_init")
+
+    def top(self) -> int:
+        return int(self.header[0].item())
+
+    def error(self) -> int:
+        return int(self.header[1].item()) & 0xFFFFFFFF
+
+    def clear_error(self):
+        self.header[1:2].zero_()
+
+    def alloc(self, counts: torch.Tensor, capacity: int, stream=None):
+        """Returns (offsets [n+1], ids [capacity]) device tensors."""
+        _need(counts, "counts", torch.int32)
+        offsets = torch.empty(counts.numel() + 1, dtype=torch.int32, device=self.state.device)
+        ids = torch.full((max(int(capacity), 1),), -1, dtype=torch.int32, device=self.state.device)
+        _check(load_library().pkv_bm_alloc(_ptr(self.state), self.num_blocks, _ptr(counts), counts.numel(),
+                                           _ptr(offsets), _ptr(ids), int(capacity), _stream(stream)), "pkv_bm_alloc")
+        return offsets, ids[:int(capacity)]
+
+    def free(self, block_ids: torch.Tensor, stream=None):
+        _need(block_ids, "block_ids", torch.int32)
+        _check(load_library().pkv_bm_free(_ptr(self.state), self.num_blocks, _ptr(block_ids), block_ids.numel(),
+                                          _stream(stream)), "pkv_bm_free")
+
+    def share(self, block_ids: torch.Tensor, stream=None):
+        _need(block_ids, "block_ids", torch.int32)
+        _check(load_library().pkv_bm_share(_ptr(self.state), self.num_blocks, _ptr(block_ids), block_ids.numel(),
+                                           _stream(stream)), "pkv_bm_share")
+
+    def append_slots(self, block_tables: torch.Tensor, context_lens: torch.Tensor, num_new: torch.Tensor,
+                     block_size: int, num_tokens: int, stream=None, out=None):
+        """Updates block_tables and context_lens in place; returns
+        (slot_mapping int64 [num_tokens], cow_pairs [B, 2], num_cow_pairs [1]),
+        written into `out` when given (the same three tensors, preallocated)."""
+        for t, n in ((block_tables, "block_tables"), (context_lens, "context_lens"), (num_new, "num_new")):
+            _need(t, n, torch.int32)
+        B, mbs = block_tables.shape
+        if context_lens.shape != (B,) or num_new.shape != (B,):
+            raise ValueError("context_lens and num_new must be [num_seqs]")
+        dev = self.state.device
+        if out is None:
+            slots = torch.empty(max(int(num_tokens), 1), dtype=torch.int64, device=dev)
+            pairs = torch.empty((max(B, 1), 2), dtype=torch.int32, device=dev)
+            npairs = torch.empty(1, dtype=torch.int32, device=dev)
+        else:
+            slots, pairs, npairs = out
+            _need(slots, "slot_mapping", torch.int64)
+            _need(pairs, "cow_pairs", torch.int32)
+            _need(npairs, "num_cow_pairs", torch.int32)
+            if slots.numel() < num_tokens or pairs.shape[0] < B:
+                raise ValueError("out tensors too small")
+        _check(load_library().pkv_bm_append_slots(_ptr(self.state), self.num_blocks, _ptr(block_tables), mbs,
+                                                  _ptr(context_lens), _ptr(num_new), B, int(block_size), _ptr(slots),
+                                                  int(num_tokens), _ptr(pairs), _ptr(npairs), _stream(stream)),
+               "pkv_bm_append_slots")
+        return slots[:int(num_tokens)], pairs, npairs
+
+
+def copy_blocks_dev(cow_pairs: torch.Tensor, num_pairs: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+                    stream=None) -> None:
+    """Copies block src -> dst for the first num_pairs[0] rows of the device
+    pair list (as BlockManager.append_slots returns it)."""
+    _need(cow_pairs, "cow_pairs", torch.int32)
+    _need(num_pairs, "num_pairs", torch.int32)
+    for t, n in ((k_cache, "k_cache"), (v_cache, "v_cache")):
+        _need(t, n, torch.bfloat16)
+    _check(load_library().pkv_copy_blocks_dev(_ptr(cow_pairs), _ptr(num_pairs), cow_pairs.shape[0], _ptr(k_cache),
+                                              _ptr(v_cache), _pool(k_cache), _stream(stream)), "pkv_copy_blocks_dev")
 
 
 def decode_workspace_bytes(num_seqs: int, num_q_heads: int, num_kv_heads: int, head_dim: int,

@@ -1,0 +1,394 @@
+// block_manager.cuh -- the block manager's per-step bookkeeping on the device.
+//
+// The pages' block manager (wkbse.com "加速 LLM 推理：深入了解 vllm 引擎",
+// section 3.1, "flexible memory management" and "KV cache sharing";
+// intelliparadigm.com article 2012396, section 2.1, items 1-2 and the block
+// allocation sketch): a free list popped on allocation, blocks allocated only
+// as new tokens need them with the block table updated, blocks returned when a
+// sequence ends, shared blocks counted by reference and copied before a sharer
+// writes into them.
+//
+// State (one caller-owned device buffer, layout in pkv.h): the free stack
+// (free_stack[0 .. top) free, the next allocation pops free_stack[top - 1]),
+// reference counts, an error word, and per-block scratch kept at its rest
+// value between calls.  Every kernel is one CTA of 1024 threads walking its
+// items in chunks of 1024, in order, with block-wide scans: results are the
+// sequential (request-order) ones, bit for bit, without host round trips.
+#pragma once
+
+#include <cstdint>
+
+#include "ptx.cuh"
+
+namespace pkv {
+
+constexpr int kBmThreads = 1024;
+
+// error bits of the state's error word
+constexpr uint32_t kBmErrNoSpace = 1u;     // too few free blocks (or output room) for a request
+constexpr uint32_t kBmErrRange = 2u;       // a block id outside the pool
+constexpr uint32_t kBmErrDoubleFree = 4u;  // a block freed more often than referenced
+constexpr uint32_t kBmErrTable = 8u;       // a sequence outgrew its block-table row
+
+struct BmState {
+    int32_t *hdr;         // [0] top, [1] error word
+    int32_t *free_stack;  // [NB]
+    int32_t *refcount;    // [NB]
+    int32_t *last_idx;    // [NB] scratch: last list position of a block in a free batch (rest: -1)
+    int32_t *zeroed;      // [NB] scratch: its count reached zero in this batch (rest: 0)
+    int32_t *cow_rank;    // [NB] scratch: copy-on-write candidates seen so far in a chunk (rest: 0)
+};
+
+__device__ __forceinline__ void bm_error(const BmState &s, uint32_t bits) {
+    atomicOr(reinterpret_cast<unsigned int *>(s.hdr + 1), bits);
+}
+
+// The stack top as stored, clamped into [0, nb] (a corrupted state cannot
+// send a pop or push outside the stack).
+__device__ __forceinline__ int bm_top(const BmState &s, int nb) { return min(max(s.hdr[0], 0), nb); }
+
+// Block-wide exclusive scan of one int per thread (1024 threads); returns the
+// exclusive prefix and writes the block total to *total (all threads).
+__device__ __forceinline__ int block_scan_excl(int v, int *warp_sums, int *total) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    int x = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+    }
+    if (lane == 31) warp_sums[warp] = x;
+    __syncthreads();
+    if (warp == 0) {
+        int w = warp_sums[lane];
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, w, o);
+            if (lane >= o) w += y;
+        }
+        warp_sums[lane] = w;  // inclusive over warps
+    }
+    __syncthreads();
+    const int before = warp == 0 ? 0 : warp_sums[warp - 1];
+    *total = warp_sums[31];
+    __syncthreads();  // warp_sums reusable after return
+    return before + x - v;
+}
+
+__global__ void __launch_bounds__(256) bm_init_kernel(BmState s, int nb) {
+    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < nb; i += gridDim.x * blockDim.x) {
+        s.free_stack[i] = nb - 1 - i;  // block 0 is popped first
+        s.refcount[i] = 0;
+        s.last_idx[i] = -1;
+        s.zeroed[i] = 0;
+        s.cow_rank[i] = 0;
+    }
+    if (blockIdx.x == 0 && threadIdx.x == 0) {
+        s.hdr[0] = nb;
+        s.hdr[1] = 0;
+    }
+}
+
+// Block-wide maximum of one int per thread (1024 threads), on all threads.
+__device__ __forceinline__ int block_max(int v, int *warp_buf) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = max(v, __shfl_xor_sync(0xffffffffu, v, o));
+    if ((threadIdx.x & 31) == 0) warp_buf[threadIdx.x >> 5] = v;
+    __syncthreads();
+    int w = warp_buf[threadIdx.x & 31];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) w = max(w, __shfl_xor_sync(0xffffffffu, w, o));
+    __syncthreads();
+    return w;
+}
+
+// Request r receives counts[r] blocks at ids[offsets[r] .. offsets[r+1]),
+// requests served in order while the free list and the output room last.  The
+// inclusive sum of counts only grows, so the served requests are a prefix.
+__global__ void __launch_bounds__(kBmThreads) bm_alloc_kernel(BmState s, int nb, const int32_t *counts, int n,
+                                                               int32_t *offsets, int32_t *ids, int capacity) {
+    __shared__ int warp_buf[32];
+    const int top0 = bm_top(s, nb);
+    const int limit = min(top0, capacity);
+    int run = 0;     // counts of earlier chunks
+    int served = 0;  // blocks handed out (the largest fitting inclusive sum)
+    bool failed = false;
+    for (int base = 0; base < n; base += kBmThreads) {
+        const int r = base + threadIdx.x;
+        const int c = r < n ? max(__ldg(counts + r), 0) : 0;
+        int tot;
+        const int excl = run + block_scan_excl(c, warp_buf, &tot);
+        const int incl = excl + c;
+        const bool fits = r < n && incl <= limit;
+        if (fits) {
+            for (int k = 0; k < c; ++k) {
+                const int32_t blk = s.free_stack[top0 - 1 - (excl + k)];
+                ids[excl + k] = blk;
+                s.refcount[blk] = 1;
+            }
+        }
+        served = max(served, block_max(fits ? incl : 0, warp_buf));
+        failed = __syncthreads_or(r < n && !fits) || failed;
+        run += tot;
+    }
+    // second walk: offsets (needs the final served total for the unserved tail)
+    run = 0;
+    if (threadIdx.x == 0) offsets[0] = 0;
+    for (int base = 0; base < n; base += kBmThreads) {
+        const int r = base + threadIdx.x;
+        const int c = r < n ? max(__ldg(counts + r), 0) : 0;
+        int tot;
+        const int incl = run + block_scan_excl(c, warp_buf, &tot) + c;
+        if (r < n) offsets[r + 1] = incl <= limit ? incl : served;
+        run += tot;
+    }
+    if (threadIdx.x == 0) {
+        s.hdr[0] = top0 - served;
+        if (failed) bm_error(s, kBmErrNoSpace);
+    }
+}
+
+// Each listed id drops a reference; a block whose count reaches zero goes back
+// on the free list, pushed in list order at its last occurrence in the batch
+// (the sequential order when no block is freed more often than referenced).
+__global__ void __launch_bounds__(kBmThreads) bm_free_kernel(BmState s, int nb, const int32_t *list, int n) {
+    __shared__ int warp_sums[32];
+    for (int i = threadIdx.x; i < n; i += kBmThreads) {
+        const int32_t b = __ldg(list + i);
+        if (b < 0 || b >= nb) {
+            bm_error(s, kBmErrRange);
+            continue;
+        }
+        const int old = atomicSub(&s.refcount[b], 1);
+        if (old <= 0) {
+            atomicAdd(&s.refcount[b], 1);
+            bm_error(s, kBmErrDoubleFree);
+        } else if (old == 1) {
+            s.zeroed[b] = 1;
+        }
+        atomicMax(&s.last_idx[b], i);
+    }
+    __syncthreads();
+    const int top0 = bm_top(s, nb);
+    int run = 0;
+    for (int base = 0; base < n; base += kBmThreads) {
+        const int i = base + threadIdx.x;
+        int push = 0;
+        int32_t b = -1;
+        if (i < n) {
+            b = __ldg(list + i);
+            if (b >= 0 && b < nb && s.last_idx[b] == i) push = s.zeroed[b];
+        }
+        int tot;
+        const int excl = run + block_scan_excl(push, warp_sums, &tot);
+        if (push) {
+            if (top0 + excl < nb) s.free_stack[top0 + excl] = b;
+            else bm_error(s, kBmErrDoubleFree);  // more free blocks than the pool: the state was inconsistent
+        }
+        run += tot;
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < n; i += kBmThreads) {  // scratch back to rest
+        const int32_t b = __ldg(list + i);
+        if (b >= 0 && b < nb) {
+            s.last_idx[b] = -1;
+            s.zeroed[b] = 0;
+        }
+    }
+    if (threadIdx.x == 0) s.hdr[0] = min(top0 + run, nb);
+}
+
+__global__ void __launch_bounds__(256) bm_share_kernel(BmState s, int nb, const int32_t *list, int n) {
+    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) {
+        const int32_t b = __ldg(list + i);
+        if (b < 0 || b >= nb) bm_error(s, kBmErrRange);
+        else atomicAdd(&s.refcount[b], 1);
+    }
+}
+
+struct AppendParams {
+    BmState s;
+    int32_t *tables;  // [B][mbs]
+    int32_t *ctx;     // [B], grown in place
+    const int32_t *num_new;
+    int64_t *slots;   // [slot_cap]: sum num_new entries written, the rest untouched
+    int64_t slot_cap;
+    int32_t *pairs;   // [B][2]
+    int32_t *num_pairs;
+    int nb, mbs, B, bs;
+};
+
+// One step's slots, by the sequential rule: in sequence order, a sequence
+// whose new tokens go into a partly filled last block that others still map
+// first gets a private copy of it (copy-on-write), then blocks for the logical
+// indices its tokens reach, then its slots; the first sequence that finds too
+// few free blocks or outgrows its table row, and every later one, is left as
+// it was with slots -1.  A shared block with R references and k appending
+// sharers is copied for the first min(k, R - 1) of them in sequence order and
+// the last sharer writes in place; a candidate's rank among earlier
+// candidates on the same block comes from __match_any_sync within its warp
+// and a per-block counter walked warp by warp.
+__global__ void __launch_bounds__(kBmThreads) bm_append_slots_kernel(const AppendParams p) {
+    __shared__ int warp_buf[32];
+    // per sequence of the chunk, for the cooperative slot pass: its first
+    // slot index, and its first position (-1 unless it fits)
+    __shared__ int sh_slot0[kBmThreads], sh_pos0[kBmThreads];
+    const BmState &s = p.s;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int top0 = bm_top(s, p.nb);
+    int run_need = 0;   // blocks wanted by earlier sequences
+    int run_flags = 0;  // range / table failures at earlier sequences
+    int run_slots = 0;  // slot-mapping offset
+    int run_pairs = 0;
+    int handed = 0;     // blocks handed out
+    for (int base = 0; base < p.B; base += kBmThreads) {
+        const int b = base + threadIdx.x;
+        const bool live = b < p.B;
+        int n = 0, pos0 = 0, first_new = 0, last = -1, need_new = 0;
+        int32_t cur = -1;
+        bool cand = false, bad_range = false, overflow = false;
+        int32_t *row = p.tables + (size_t)(live ? b : 0) * p.mbs;
+        if (live) {
+            n = max(__ldg(p.num_new + b), 0);
+            pos0 = p.ctx[b];
+            if (pos0 < 0 || pos0 > p.mbs * p.bs) {
+                overflow = true;  // a context length outside its own table row (its slots stay -1)
+            } else {
+                first_new = (pos0 + p.bs - 1) / p.bs;
+                last = n > 0 ? (pos0 + n - 1) / p.bs : first_new - 1;
+                need_new = last >= first_new ? last - first_new + 1 : 0;
+                if (n > 0 && pos0 % p.bs != 0) {
+                    cur = row[pos0 / p.bs];
+                    if (cur < 0 || cur >= p.nb) bad_range = true;
+                    else cand = true;
+                }
+                overflow = n > 0 && last >= p.mbs;
+            }
+        }
+        // references of a candidate's block, after earlier chunks' copies
+        const int R = cand ? s.refcount[cur] : 0;
+        const unsigned same = __match_any_sync(0xffffffffu, cand ? cur : -2 - (int)threadIdx.x);
+        const int rank_in_warp = __popc(same & ((1u << lane) - 1u));
+        int rank = 0;
+        if (__syncthreads_or(cand)) {  // only when some sequence writes into a block it may share
+            const int live_warps = (min(kBmThreads, p.B - base) + 31) / 32;
+            for (int w = 0; w < live_warps; ++w) {
+                if (warp == w && cand) {
+                    rank = s.cow_rank[cur] + rank_in_warp;
+                    __syncwarp(same);
+                    if (rank_in_warp == 0) s.cow_rank[cur] += __popc(same);
+                }
+                __syncthreads();
+            }
+        }
+        const int cow = (cand && rank < R - 1) ? 1 : 0;
+        const int need = live ? need_new + cow : 0;
+        const int flag = (bad_range || overflow) ? 1 : 0;
+        int tot_flags, tot_need, tot_n;
+        const int flags_before = run_flags + block_scan_excl(flag, warp_buf, &tot_flags);
+        const int excl_need = run_need + block_scan_excl(need, warp_buf, &tot_need);
+        const int excl_slots = run_slots + block_scan_excl(n, warp_buf, &tot_n);
+        const bool earlier_ok = flags_before == 0 && excl_need <= top0;
+        const bool fits = live && earlier_ok && !flag && excl_need + need <= top0;
+        int tot_pairs, tot_handed;
+        const int excl_pairs = run_pairs + block_scan_excl(fits ? cow : 0, warp_buf, &tot_pairs);
+        (void)block_scan_excl(fits ? need : 0, warp_buf, &tot_handed);
+        if (live && bad_range) bm_error(s, kBmErrRange);
+        if (live && earlier_ok && !fits && !bad_range) bm_error(s, overflow ? kBmErrTable : kBmErrNoSpace);
+        if (fits) {
+            int k = 0;
+            if (cow) {
+                const int32_t fresh = s.free_stack[top0 - 1 - excl_need];
+                s.refcount[fresh] = 1;
+                atomicSub(&s.refcount[cur], 1);
+                row[pos0 / p.bs] = fresh;
+                p.pairs[2 * excl_pairs] = cur;
+                p.pairs[2 * excl_pairs + 1] = fresh;
+                k = 1;
+            }
+            for (int L = first_new; L <= last; ++L, ++k) {
+                const int32_t fresh = s.free_stack[top0 - 1 - (excl_need + k)];
+                s.refcount[fresh] = 1;
+                row[L] = fresh;
+            }
+            p.ctx[b] = pos0 + n;
+        }
+        sh_slot0[threadIdx.x] = live ? excl_slots : 0;
+        sh_pos0[threadIdx.x] = fits ? pos0 : -1;
+        __syncthreads();
+        // slots of the whole chunk, all threads: entry j belongs to the last
+        // sequence whose first slot is <= j (binary search over the chunk; a
+        // sequence without new tokens shares its first slot with the next one,
+        // so the last such sequence is always one that owns entry j)
+        const int chunk_first = sh_slot0[0];
+        const int nlive = min(kBmThreads, p.B - base);
+        for (int j = chunk_first + threadIdx.x; j < run_slots + tot_n; j += kBmThreads) {
+            int lo = 0, hi = nlive - 1;
+            while (lo < hi) {
+                const int mid = (lo + hi + 1) >> 1;
+                if (sh_slot0[mid] <= j) lo = mid;
+                else hi = mid - 1;
+            }
+            if (j >= p.slot_cap) continue;
+            const int q0 = sh_pos0[lo];
+            if (q0 < 0) {
+                p.slots[j] = -1;
+            } else {
+                const int pos = q0 + (j - sh_slot0[lo]);
+                const int32_t *qrow = p.tables + (size_t)(base + lo) * p.mbs;
+                p.slots[j] = (int64_t)qrow[pos / p.bs] * p.bs + pos % p.bs;
+            }
+        }
+        if (live && (int64_t)excl_slots + n > p.slot_cap) bm_error(s, kBmErrNoSpace);  // output too short
+        if (cand) s.cow_rank[cur] = 0;  // scratch back to rest
+        __syncthreads();
+        run_need += tot_need;
+        run_flags += tot_flags;
+        run_slots += tot_n;
+        run_pairs += tot_pairs;
+        handed += tot_handed;
+    }
+    if (threadIdx.x == 0) {
+        *p.num_pairs = run_pairs;
+        s.hdr[0] = top0 - handed;
+    }
+}
+
+// Copy-on-write pairs kept on the device (as bm_append_slots leaves them):
+// grid.y = pair slot up to max_pairs; slots at or past *num_pairs do nothing.
+// The pairs' destinations are fresh blocks, never another pair's source.
+constexpr int kCopyDevThreads = 256;
+constexpr int kCopyDevVec = 4;
+
+__global__ void __launch_bounds__(kCopyDevThreads) copy_blocks_dev_kernel(uint4 *k_cache, uint4 *v_cache,
+                                                                          const int32_t *pairs,
+                                                                          const int32_t *num_pairs,
+                                                                          int64_t vec_per_block, int nb, int first) {
+    const int pr = blockIdx.y;  // pair first + pr of the list; pairs points at pair first
+    if (first + pr >= *num_pairs) return;
+    const int32_t src = __ldg(pairs + 2 * pr), dst = __ldg(pairs + 2 * pr + 1);
+    if (src < 0 || src >= nb || dst < 0 || dst >= nb) {
+        if (blockIdx.x == 0 && threadIdx.x == 0) raise_error(PKV_DEVERR_BLOCK);
+        return;
+    }
+    const int64_t base = (int64_t)blockIdx.x * (kCopyDevThreads * kCopyDevVec) + threadIdx.x;
+    uint4 kv[kCopyDevVec], vv[kCopyDevVec];
+#pragma unroll
+    for (int u = 0; u < kCopyDevVec; ++u) {
+        const int64_t e = base + u * kCopyDevThreads;
+        if (e < vec_per_block) {
+            kv[u] = k_cache[src * vec_per_block + e];
+            vv[u] = v_cache[src * vec_per_block + e];
+        }
+    }
+#pragma unroll
+    for (int u = 0; u < kCopyDevVec; ++u) {
+        const int64_t e = base + u * kCopyDevThreads;
+        if (e < vec_per_block) {
+            k_cache[dst * vec_per_block + e] = kv[u];
+            v_cache[dst * vec_per_block + e] = vv[u];
+        }
+    }
+}
+
+}  // namespace pkv

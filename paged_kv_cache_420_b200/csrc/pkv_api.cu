@@ -13,6 +13,7 @@
 #include <mutex>
 #include <vector>
 
+#include "block_manager.cuh"
 #include "decode.cuh"
 #include "pkv.h"
 #include "prefill.cuh"
@@ -334,6 +335,25 @@ pkv_status swap_blocks(const int32_t *block_ids, int32_t n, void *k_cache, void 
     return PKV_OK;
 }
 
+
+// Block-manager state: a 256-byte header (top, error word), then five
+// 256-byte-aligned int32 arrays of num_blocks: free stack, reference counts and
+// three scratch arrays.
+size_t bm_array_bytes(int32_t nb) { return round256((size_t)nb * 4); }
+
+bool bm_state(void *state, int32_t nb, pkv::BmState *s) {
+    if (!state || nb <= 0 || !aligned(state, 256)) return false;
+    uint8_t *p = static_cast<uint8_t *>(state);
+    const size_t a = bm_array_bytes(nb);
+    s->hdr = reinterpret_cast<int32_t *>(p);
+    s->free_stack = reinterpret_cast<int32_t *>(p + 256);
+    s->refcount = reinterpret_cast<int32_t *>(p + 256 + a);
+    s->last_idx = reinterpret_cast<int32_t *>(p + 256 + 2 * a);
+    s->zeroed = reinterpret_cast<int32_t *>(p + 256 + 3 * a);
+    s->cow_rank = reinterpret_cast<int32_t *>(p + 256 + 4 * a);
+    return true;
+}
+
 }  // namespace
 
 extern "C" {
@@ -595,6 +615,102 @@ pkv_status paged_attn_prefill(const void *q, const void *k_cache, const void *v_
     return pool.head_dim == 128 ? launch_prefill_tc<128>(prm, mk, mv, mq, st, dev)
                                 : launch_prefill_tc<64>(prm, mk, mv, mq, st, dev);
 #endif
+}
+
+size_t pkv_bm_state_bytes(int32_t num_blocks) {
+    if (num_blocks <= 0) return 0;
+    return 256 + 5 * bm_array_bytes(num_blocks);
+}
+
+pkv_status pkv_bm_init(void *state, int32_t num_blocks, pkv_stream_t stream) {
+    pkv::BmState s;
+    if (!bm_state(state, num_blocks, &s)) return PKV_EINVAL;
+    const int grid = std::max(1, std::min(1024, (num_blocks + 255) / 256));
+    pkv::bm_init_kernel<<<grid, 256, 0, (cudaStream_t)stream>>>(s, num_blocks);
+    return launch_status();
+}
+
+pkv_status pkv_bm_alloc(void *state, int32_t num_blocks, const int32_t *counts, int32_t n, int32_t *offsets,
+                        int32_t *ids, int32_t capacity, pkv_stream_t stream) {
+    pkv::BmState s;
+    if (!bm_state(state, num_blocks, &s) || n < 0 || capacity < 0) return PKV_EINVAL;
+    if (!offsets || (n > 0 && !counts) || (capacity > 0 && !ids)) return PKV_EINVAL;
+    if (!aligned(counts, 4) || !aligned(offsets, 4) || !aligned(ids, 4)) return PKV_EINVAL;
+    pkv::bm_alloc_kernel<<<1, pkv::kBmThreads, 0, (cudaStream_t)stream>>>(s, num_blocks, counts, n, offsets, ids,
+                                                                         capacity);
+    return launch_status();
+}
+
+pkv_status pkv_bm_free(void *state, int32_t num_blocks, const int32_t *block_ids, int32_t n, pkv_stream_t stream) {
+    pkv::BmState s;
+    if (!bm_state(state, num_blocks, &s) || n < 0) return PKV_EINVAL;
+    if (n == 0) return PKV_OK;
+    if (!block_ids || !aligned(block_ids, 4)) return PKV_EINVAL;
+    pkv::bm_free_kernel<<<1, pkv::kBmThreads, 0, (cudaStream_t)stream>>>(s, num_blocks, block_ids, n);
+    return launch_status();
+}
+
+pkv_status pkv_bm_share(void *state, int32_t num_blocks, const int32_t *block_ids, int32_t n, pkv_stream_t stream) {
+    pkv::BmState s;
+    if (!bm_state(state, num_blocks, &s) || n < 0) return PKV_EINVAL;
+    if (n == 0) return PKV_OK;
+    if (!block_ids || !aligned(block_ids, 4)) return PKV_EINVAL;
+    const int grid = std::max(1, std::min(1024, (n + 255) / 256));
+    pkv::bm_share_kernel<<<grid, 256, 0, (cudaStream_t)stream>>>(s, num_blocks, block_ids, n);
+    return launch_status();
+}
+
+pkv_status pkv_bm_append_slots(void *state, int32_t num_blocks, int32_t *block_tables, int32_t max_blocks_per_seq,
+                               int32_t *context_lens, const int32_t *num_new, int32_t num_seqs, int32_t block_size,
+                               int64_t *slot_mapping, int64_t slot_capacity, int32_t *cow_pairs,
+                               int32_t *num_cow_pairs, pkv_stream_t stream) {
+    pkv::AppendParams p;
+    if (slot_capacity < 0) return PKV_EINVAL;
+    if (!bm_state(state, num_blocks, &p.s) || num_seqs < 0 || max_blocks_per_seq <= 0 || block_size <= 0)
+        return PKV_EINVAL;
+    if ((long long)max_blocks_per_seq * block_size >= (1ll << 31)) return PKV_EUNSUPPORTED;
+    if (!num_cow_pairs ||
+        (num_seqs > 0 && (!block_tables || !context_lens || !num_new || !cow_pairs || !slot_mapping)))
+        return PKV_EINVAL;
+    if (!aligned(block_tables, 4) || !aligned(context_lens, 4) || !aligned(num_new, 4) || !aligned(slot_mapping, 8) ||
+        !aligned(cow_pairs, 4) || !aligned(num_cow_pairs, 4))
+        return PKV_EINVAL;
+    p.tables = block_tables;
+    p.ctx = context_lens;
+    p.num_new = num_new;
+    p.slots = slot_mapping;
+    p.slot_cap = slot_capacity;
+    p.pairs = cow_pairs;
+    p.num_pairs = num_cow_pairs;
+    p.nb = num_blocks;
+    p.mbs = max_blocks_per_seq;
+    p.B = num_seqs;
+    p.bs = block_size;
+    pkv::bm_append_slots_kernel<<<1, pkv::kBmThreads, 0, (cudaStream_t)stream>>>(p);
+    return launch_status();
+}
+
+pkv_status pkv_copy_blocks_dev(const int32_t *cow_pairs, const int32_t *num_pairs, int32_t max_pairs, void *k_cache,
+                               void *v_cache, pkv_pool pool, pkv_stream_t stream) {
+    const pkv_status ps = check_pool(pool);
+    if (ps != PKV_OK) return ps;
+    if (max_pairs < 0) return PKV_EINVAL;
+    if (max_pairs == 0) return PKV_OK;
+    if (!cow_pairs || !num_pairs || !k_cache || !v_cache) return PKV_EINVAL;
+    if (!aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(cow_pairs, 4) || !aligned(num_pairs, 4))
+        return PKV_EINVAL;
+    const int64_t vec = (int64_t)pool.num_kv_heads * pool.block_size * pool.head_dim / 8;
+    const long long per_cta = pkv::kCopyDevThreads * pkv::kCopyDevVec;
+    const unsigned gx = (unsigned)((vec + per_cta - 1) / per_cta);
+    for (int base = 0; base < max_pairs; base += 65535) {  // grid.y limit
+        const int m = std::min(65535, max_pairs - base);
+        pkv::copy_blocks_dev_kernel<<<dim3(gx, m), pkv::kCopyDevThreads, 0, (cudaStream_t)stream>>>(
+            static_cast<uint4 *>(k_cache), static_cast<uint4 *>(v_cache), cow_pairs + 2 * base, num_pairs, vec,
+            pool.num_blocks, base);
+        const pkv_status st = launch_status();
+        if (st != PKV_OK) return st;
+    }
+    return PKV_OK;
 }
 
 pkv_status pkv_get_device_error(int32_t *code_out, pkv_stream_t stream) {

@@ -1,0 +1,248 @@
+"""GPU parity of the device block manager against the oracle's sequential
+block manager: every call's outputs and the whole state (free list, top,
+reference counts, error word) are compared bit for bit after each step.
+Cases: random operation mixes, forks whose sharers append together (more
+sharers than a warp, across the 1024-sequence chunk boundary), the worked
+example, errors, and a whole decode step driven from the device state."""
+import json
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import paged_kv_cache_420_b200 as pkv
+import workloads
+from tests._gpu_util import assert_attention_close, bits_equal
+
+pytestmark = pytest.mark.gpu
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
+
+def _same_state(bm: pkv.BlockManager, st: oracle.BlockState, err_expected: int):
+    torch.cuda.synchronize()
+    assert bm.top() == st.top
+    assert np.array_equal(bm.free_stack.cpu().numpy()[:st.top], st.free_stack[:st.top])
+    assert np.array_equal(bm.refcount.cpu().numpy(), st.refcount)
+    assert bm.error() == err_expected
+
+
+def _dev(a, dtype=torch.int32):
+    return torch.as_tensor(np.ascontiguousarray(a)).to(dtype).cuda()
+
+
+class Mirror:
+    """Applies each operation to the device manager and to the oracle."""
+
+    def __init__(self, nb, B, mbs, bs):
+        self.bm = pkv.BlockManager(nb)
+        self.st = oracle.bm_init(nb)
+        self.err = 0
+        self.bs = bs
+        self.tables = np.full((B, mbs), -1, np.int32)
+        self.ctx = np.zeros(B, np.int32)
+        self.t_dev = _dev(self.tables)
+        self.c_dev = _dev(self.ctx)
+        _same_state(self.bm, self.st, 0)
+
+    def append(self, num_new):
+        nn = np.asarray(num_new, np.int32)
+        T = int(np.clip(nn, 0, None).sum())
+        slots, pairs, npairs = self.bm.append_slots(self.t_dev, self.c_dev, _dev(nn), self.bs, T)
+        self.st, tables, ctx, oslots, opairs, e = oracle.bm_append_slots(self.st, self.tables, self.ctx, nn, self.bs)
+        self.err |= e
+        torch.cuda.synchronize()
+        assert np.array_equal(self.t_dev.cpu().numpy(), tables)
+        assert np.array_equal(self.c_dev.cpu().numpy(), ctx)
+        assert np.array_equal(slots.cpu().numpy(), oslots)
+        k = int(npairs.item())
+        assert k == len(opairs) and np.array_equal(pairs.cpu().numpy()[:k], opairs)
+        self.tables, self.ctx = tables, ctx
+        _same_state(self.bm, self.st, self.err)
+        return slots, pairs, npairs, opairs
+
+    def fork(self, a, b):
+        """Sequence b (after releasing its blocks) becomes a parallel sample of a."""
+        self.release(b)
+        nblk = (int(self.ctx[a]) + self.bs - 1) // self.bs
+        self.tables[b, :nblk] = self.tables[a, :nblk]
+        self.ctx[b] = self.ctx[a]
+        self.t_dev.copy_(_dev(self.tables))
+        self.c_dev.copy_(_dev(self.ctx))
+        if nblk:
+            self.bm.share(_dev(self.tables[a, :nblk]))
+            self.st, e = oracle.bm_share(self.st, self.tables[a, :nblk])
+            self.err |= e
+        _same_state(self.bm, self.st, self.err)
+
+    def release(self, b):
+        nblk = (int(self.ctx[b]) + self.bs - 1) // self.bs
+        if nblk:
+            self.bm.free(_dev(self.tables[b, :nblk]))
+            self.st, e = oracle.bm_free(self.st, self.tables[b, :nblk])
+            self.err |= e
+        self.tables[b] = -1
+        self.ctx[b] = 0
+        self.t_dev.copy_(_dev(self.tables))
+        self.c_dev.copy_(_dev(self.ctx))
+        _same_state(self.bm, self.st, self.err)
+
+
+@pytest.mark.parametrize("seed", range(4))
+def test_random_operation_mix(seed):
+    rng = np.random.default_rng(seed)
+    m = Mirror(nb=300, B=40, mbs=24, bs=int(rng.choice([4, 16])))
+    for _ in range(30):
+        r = rng.random()
+        if r < 0.55:
+            m.append(rng.integers(0, 9, 40) * (rng.random(40) < 0.8))
+        elif r < 0.8:
+            a, b = rng.choice(40, 2, replace=False)
+            m.fork(int(a), int(b))
+        else:
+            m.release(int(rng.integers(40)))
+
+
+def test_fork_storm_across_warps_and_chunks():
+    """1500 sequences: 60 parents, each with 24 forks spread over the batch, all
+    appending one token into the shared partly filled block in one step."""
+    rng = np.random.default_rng(1)
+    B = 1500
+    m = Mirror(nb=6000, B=B, mbs=8, bs=16)
+    parents = np.arange(60)
+    m.append(np.where(np.isin(np.arange(B), parents), rng.integers(17, 31, B), 0))  # partly filled 2nd block
+    forks = rng.permutation(np.arange(60, B))[:60 * 24].reshape(60, 24)
+    for p_, kids in zip(parents, forks):
+        for kid in kids:
+            nblk = (int(m.ctx[p_]) + 15) // 16
+            m.tables[kid, :nblk] = m.tables[p_, :nblk]
+            m.ctx[kid] = m.ctx[p_]
+    shared = np.concatenate([np.repeat(m.tables[p_, :(m.ctx[p_] + 15) // 16][None], 24, 0).reshape(-1)
+                             for p_ in parents])
+    m.t_dev.copy_(_dev(m.tables))
+    m.c_dev.copy_(_dev(m.ctx))
+    m.bm.share(_dev(shared))
+    m.st, _ = oracle.bm_share(m.st, shared)
+    _same_state(m.bm, m.st, 0)
+    active = np.zeros(B, np.int32)
+    active[np.concatenate([parents, forks.reshape(-1)])] = 1
+    slots, pairs, npairs, opairs = m.append(active)
+    assert len(opairs) == 60 * 24  # every sharer but the last in order copies
+
+
+def test_worked_example_on_device():
+    g = json.load(open(os.path.join(GOLDEN, "block_manager_example.json")))
+    bm = pkv.BlockManager(g["num_blocks"])
+    for step in g["steps"]:
+        if step["op"] == "append":
+            t = _dev(step["tables"])
+            c = _dev(step["context_lens"])
+            slots, pairs, npairs = bm.append_slots(t, c, _dev(step["num_new"]), g["block_size"],
+                                                   int(sum(step["num_new"])))
+            torch.cuda.synchronize()
+            assert t.cpu().tolist() == step["expect_tables"]
+            assert c.cpu().tolist() == step["expect_context_lens"]
+            assert slots.cpu().tolist() == step["expect_slots"]
+            assert pairs.cpu().numpy()[:int(npairs.item())].tolist() == step["expect_pairs"]
+            assert bm.top() == step["expect_top"]
+        elif step["op"] == "fork":
+            bm.share(_dev(step["share"]))
+        elif step["op"] == "free":
+            bm.free(_dev(step["ids"]))
+            assert bm.top() == step["expect_top"]
+        elif step["op"] == "alloc":
+            off, ids = bm.alloc(_dev(step["counts"]), 16)
+            torch.cuda.synchronize()
+            assert ids.cpu().numpy()[:int(off[-1].item())].tolist() == step["expect_ids"]
+        if "expect_refcount" in step:
+            torch.cuda.synchronize()
+            assert bm.refcount.cpu().tolist() == step["expect_refcount"]
+        assert bm.error() == 0
+
+
+def test_alloc_free_parity_and_errors():
+    rng = np.random.default_rng(3)
+    bm = pkv.BlockManager(700)
+    st = oracle.bm_init(700)
+    err = 0
+    for _ in range(6):
+        counts = rng.integers(0, 40, 2100).astype(np.int32) * (rng.random(2100) < 0.02)
+        off, ids = bm.alloc(_dev(counts), 500)
+        st, ooff, oids, e = oracle.bm_alloc(st, counts, 500)
+        err |= e
+        torch.cuda.synchronize()
+        assert np.array_equal(off.cpu().numpy(), ooff)
+        assert np.array_equal(ids.cpu().numpy()[:ooff[-1]], oids[:ooff[-1]])
+        _same_state(bm, st, err)
+        held = np.flatnonzero(st.refcount > 0)
+        batch = rng.choice(held, min(len(held), 300)).astype(np.int32) if len(held) else np.zeros(0, np.int32)
+        # no double frees: at most refcount occurrences of each block
+        keep = []
+        seen = {}
+        for b_ in batch:
+            seen[b_] = seen.get(b_, 0) + 1
+            if seen[b_] <= st.refcount[b_]:
+                keep.append(b_)
+        batch = np.array(keep, np.int32)
+        if len(batch):
+            bm.free(_dev(batch))
+            st, e = oracle.bm_free(st, batch)
+            err |= e
+            _same_state(bm, st, err)
+    assert err & oracle.BM_ERR_NOSPACE
+    # error paths: out of range, double free (the set of free blocks still matches)
+    bm.clear_error()
+    bm.free(_dev([700, -1]))
+    torch.cuda.synchronize()
+    assert bm.error() == oracle.BM_ERR_RANGE
+    bm.clear_error()
+    held = int(np.flatnonzero(st.refcount == 1)[0])
+    bm.free(_dev([held, held]))
+    st, e = oracle.bm_free(st, [held, held])
+    torch.cuda.synchronize()
+    assert bm.error() & oracle.BM_ERR_DOUBLEFREE and e & oracle.BM_ERR_DOUBLEFREE
+    assert set(bm.free_stack.cpu().numpy()[:bm.top()].tolist()) == st.free_set()
+
+
+def test_append_errors_match():
+    m = Mirror(nb=10, B=4, mbs=4, bs=4)
+    m.append([5, 3, 0, 0])          # 3 blocks
+    m.append([12, 1, 1, 0])         # seq0 outgrows its row (TABLE): it and every later one unchanged
+    m.release(0)
+    m.append([0, 1, 30, 2])         # seq2 asks for more than its row
+    m.append([8, 8, 8, 8])          # 8 blocks: fits
+    m.append([4, 4, 4, 4])          # one block left: seq0 gets it, seq1 on find none (NOSPACE)
+    assert m.err & oracle.BM_ERR_TABLE and m.err & oracle.BM_ERR_NOSPACE
+
+
+def test_decode_step_driven_by_the_device_block_manager():
+    """Forks share a prefix; one decode step appends a token to every sequence
+    from the device state, copies the copy-on-write pairs on the device, writes
+    the new K/V at the produced slots and runs decode attention: the result
+    equals the oracle's step on the oracle's own tables."""
+    rng = np.random.default_rng(11)
+    B, Hq, Hkv, D, bs, nb, mbs = 24, 8, 2, 128, 16, 400, 40
+    m = Mirror(nb=nb, B=B, mbs=mbs, bs=bs)
+    m.append(np.where(np.arange(B) < 8, rng.integers(20, 300, B), 0))
+    for kid in range(8, B):
+        m.fork(kid % 8, kid)
+    g = torch.Generator().manual_seed(5)
+    kc = torch.randn((nb, Hkv, bs, D), generator=g).to(torch.bfloat16)
+    vc = torch.randn((nb, Hkv, bs, D), generator=g).to(torch.bfloat16)
+    k_new = torch.randn((B, Hkv, D), generator=g).to(torch.bfloat16)
+    v_new = torch.randn((B, Hkv, D), generator=g).to(torch.bfloat16)
+    q = torch.randn((B, Hq, D), generator=g).to(torch.bfloat16)
+    kd, vd = kc.cuda(), vc.cuda()
+    slots, pairs, npairs, opairs = m.append(np.ones(B, np.int32))
+    assert len(opairs) > 0
+    pkv.copy_blocks_dev(pairs, npairs, kd, vd)
+    pkv.pkv_write(k_new.cuda(), v_new.cuda(), slots, kd, vd)
+    out = torch.empty((B, Hq, D), dtype=torch.bfloat16, device="cuda")
+    pkv.paged_attn_decode(q.cuda(), kd, vd, m.t_dev, m.c_dev, 1 / np.sqrt(D), Hkv, out, int(m.ctx.max()))
+    torch.cuda.synchronize()
+    okc, ovc = oracle.copy_blocks(kc, vc, opairs)
+    okc, ovc = oracle.kv_write(okc, ovc, k_new, v_new, slots.cpu().numpy())
+    assert bits_equal(kd, okc) and bits_equal(vd, ovc)
+    ref = oracle.paged_attention(q, okc, ovc, m.tables, m.ctx, float(np.float32(1 / np.sqrt(D))))
+    assert_attention_close(out, ref, "device block manager step")

@@ -56,3 +56,29 @@ def test_swap_validation():
     host = np.zeros(3 * 2 * 16 * 128, dtype=np.uint16)
     hp = host.ctypes.data_as(ctypes.c_void_p)
     assert lib.pkv_swap_out(FAKE, FAKE, pool, ids, 3, hp, hp, None) == EINVAL
+
+
+def test_block_manager_host_validation():
+    """Host checks of the device block manager's entry points (no GPU work)."""
+    lib = pkv.load_library()
+    assert lib.pkv_bm_state_bytes(0) == 0
+    assert lib.pkv_bm_state_bytes(10) == 256 + 5 * 256
+    assert lib.pkv_bm_state_bytes(100) == 256 + 5 * 512
+    assert lib.pkv_bm_init(None, 8, None) == EINVAL
+    assert lib.pkv_bm_init(ctypes.c_void_p(0x10080), 8, None) == EINVAL  # state not 256-B aligned
+    assert lib.pkv_bm_init(FAKE, 0, None) == EINVAL
+    assert lib.pkv_bm_alloc(FAKE, 8, FAKE, -1, FAKE, FAKE, 4, None) == EINVAL
+    assert lib.pkv_bm_alloc(FAKE, 8, FAKE, 2, None, FAKE, 4, None) == EINVAL
+    assert lib.pkv_bm_free(FAKE, 8, None, 0, None) == 0
+    assert lib.pkv_bm_free(FAKE, 8, None, 3, None) == EINVAL
+    assert lib.pkv_bm_share(FAKE, 8, ctypes.c_void_p(0x10002), 3, None) == EINVAL  # ids not 4-B aligned
+    args = [FAKE, 8, FAKE, 4, FAKE, FAKE, 2, 16, FAKE, 32, FAKE, FAKE, None]
+    bad = list(args); bad[8] = None  # no slot mapping
+    assert lib.pkv_bm_append_slots(*bad) == EINVAL
+    bad = list(args); bad[9] = -1  # negative capacity
+    assert lib.pkv_bm_append_slots(*bad) == EINVAL
+    bad = list(args); bad[7] = 0  # block size
+    assert lib.pkv_bm_append_slots(*bad) == EINVAL
+    pool = _Pool(8, 2, 16, 128)
+    assert lib.pkv_copy_blocks_dev(FAKE, FAKE, 0, FAKE, FAKE, pool, None) == 0
+    assert lib.pkv_copy_blocks_dev(None, FAKE, 4, FAKE, FAKE, pool, None) == EINVAL
