@@ -59,12 +59,18 @@ def _load() -> ctypes.CDLL:
         lib.oracle_bm_free.argtypes = [P, P, P, I, P, I, P]
         lib.oracle_bm_share.argtypes = [P, I, P, I, P]
         lib.oracle_bm_append_slots.argtypes = [P, P, P, I, P, I, P, P, I, I, P, P, P, P]
+        lib.oracle_e4m3_decode.argtypes = [ctypes.c_uint8]
+        lib.oracle_e4m3_decode.restype = D
+        lib.oracle_e4m3_encode_array.argtypes = [P, I, P]
+        lib.oracle_kv_write_fp8.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I]
+        lib.oracle_paged_attention_fp8.argtypes = [P, P, P, P, P, P, I, P, I, I, I, I, I, I, D, P]
         lib.oracle_num_threads.argtypes = []
         for f in (lib.oracle_kv_write, lib.oracle_copy_blocks, lib.oracle_paged_attention,
                   lib.oracle_attention_partial, lib.oracle_lse_merge, lib.oracle_num_threads,
                   lib.oracle_paged_prefill, lib.oracle_swap_out, lib.oracle_swap_in, lib.oracle_lru_victims,
                   lib.oracle_bm_init, lib.oracle_bm_alloc, lib.oracle_bm_free, lib.oracle_bm_share,
-                  lib.oracle_bm_append_slots):
+                  lib.oracle_bm_append_slots, lib.oracle_e4m3_encode_array, lib.oracle_kv_write_fp8,
+                  lib.oracle_paged_attention_fp8):
             f.restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -262,6 +268,62 @@ def bm_append_slots(st: BlockState, block_tables, context_lens, num_new, block_s
     _check(_bm_call(_load().oracle_bm_append_slots, st, _ptr(tables), mbs, _ptr(ctx), _ptr(nn), B, int(block_size),
                     _ptr(slots), _ptr(pairs), _ptr(npairs), _ptr(err)), "bm_append_slots")
     return st, tables, ctx, slots[:int(np.clip(nn, 0, None).sum())], pairs[:int(npairs[0])].copy(), int(err[0])
+
+
+# ---------------------------------------------------------------------------
+# FP8 (e4m3) KV cache
+# ---------------------------------------------------------------------------
+
+def e4m3_decode(codes) -> np.ndarray:
+    c = np.asarray(codes, dtype=np.uint8)
+    f = _load().oracle_e4m3_decode
+    return np.array([f(int(v)) for v in c.reshape(-1)], dtype=np.float64).reshape(c.shape)
+
+
+def e4m3_encode(x) -> np.ndarray:
+    a = np.ascontiguousarray(x, dtype=np.float64)
+    out = np.zeros(a.shape, dtype=np.uint8)
+    _load().oracle_e4m3_encode_array(_ptr(a), a.size, _ptr(out))
+    return out
+
+
+def kv_write_fp8(k_cache8, v_cache8, k, v, slot_mapping, k_scale, v_scale):
+    """Returns new uint8 (k_cache, v_cache) [NB, Hkv, bs, d] after the
+    quantizing slot-mapped write of bf16 k, v [T, Hkv, d]."""
+    kc = np.ascontiguousarray(k_cache8, dtype=np.uint8).copy()
+    vc = np.ascontiguousarray(v_cache8, dtype=np.uint8).copy()
+    kb, vb = bits(k), bits(v)
+    slots = np.ascontiguousarray(slot_mapping, dtype=np.int64)
+    ks = np.ascontiguousarray(k_scale, dtype=np.float32)
+    vs = np.ascontiguousarray(v_scale, dtype=np.float32)
+    NB, Hkv, bs, d = kc.shape
+    T = slots.shape[0]
+    assert kb.shape == (T, Hkv, d) and ks.shape == (Hkv,) and vs.shape == (Hkv,)
+    rc = _load().oracle_kv_write_fp8(_ptr(kc), _ptr(vc), _ptr(kb), _ptr(vb), _ptr(slots), _ptr(ks), _ptr(vs), T, NB,
+                                     Hkv, bs, d)
+    _check(rc, "kv_write_fp8")
+    return kc, vc
+
+
+def paged_attention_fp8(q, k_cache8, v_cache8, k_scale, v_scale, block_tables, context_lens,
+                        scale: float) -> np.ndarray:
+    """fp64 decode attention over an e4m3 pool: K = e4m3(code) * k_scale[h], V likewise."""
+    qb = bits(q)
+    kc = np.ascontiguousarray(k_cache8, dtype=np.uint8)
+    vc = np.ascontiguousarray(v_cache8, dtype=np.uint8)
+    ks = np.ascontiguousarray(k_scale, dtype=np.float32)
+    vs = np.ascontiguousarray(v_scale, dtype=np.float32)
+    tables = np.ascontiguousarray(block_tables, dtype=np.int32)
+    ctx = np.ascontiguousarray(context_lens, dtype=np.int32)
+    B, Hq, d = qb.shape
+    NB, Hkv, bs, d2 = kc.shape
+    assert d == d2
+    out = np.zeros((B, Hq, d), dtype=np.float64)
+    rc = _load().oracle_paged_attention_fp8(_ptr(qb), _ptr(kc), _ptr(vc), _ptr(ks), _ptr(vs), _ptr(tables),
+                                            tables.shape[1], _ptr(ctx), B, Hq, Hkv, d, bs, NB,
+                                            float(np.float64(np.float32(scale))), _ptr(out))
+    _check(rc, "paged_attention_fp8")
+    return out
 
 
 def paged_attention(q, k_cache, v_cache, block_tables, context_lens, scale: float) -> np.ndarray:

@@ -22,6 +22,10 @@
  *     sharer writes into them (wkbse.com section 3.1, "flexible memory
  *     management" and "KV cache sharing"; intelliparadigm.com section 2.1,
  *     items 1-2 and the block-allocation sketch).
+ *   - an FP8 KV cache (ai-stack.site "Nano-vLLM 原理", case study: FP8 mixed
+ *     precision): the pool holds OCP E4M3 codes with a static scale per kv
+ *     head for K and for V; a value is stored as the code nearest to
+ *     fp32(x) * fp32(1 / scale) and read back as the code's value times scale.
  *   - swap of cold blocks to CPU memory and back, victims chosen least
  *     recently used first (intelliparadigm.com section 2.1, item 3; ai-stack.site
  *     "Nano-vLLM 原理", practice 5, preemption by swapping a request's KV cache).
@@ -504,4 +508,124 @@ int oracle_bm_append_slots(int32_t *free_stack, int32_t *top, int32_t *refcount,
         off += n;
     }
     return 0;
+}
+
+/* ------------------------------------------------------------------------
+ * FP8 E4M3 (the OCP "E4M3FN" encoding): 1 sign bit, 4 exponent bits with
+ * bias 7, 3 mantissa bits; exponent field 0 holds the subnormals m/8 * 2^-6;
+ * no infinities; S.1111.111 is NaN; the largest finite value is 448.
+ * ------------------------------------------------------------------------ */
+double oracle_e4m3_decode(uint8_t c) {
+    int sgn = c >> 7, e = (c >> 3) & 15, m = c & 7;
+    double v;
+    if (e == 15 && m == 7) return NAN;
+    if (e == 0) v = ldexp((double)m / 8.0, -6);
+    else v = ldexp(1.0 + (double)m / 8.0, e - 7);
+    return sgn ? -v : v;
+}
+
+/* The code nearest to x (ties to the even code, i.e. the even mantissa), with
+ * magnitudes beyond 448 saturating to +-448 and NaN to 0x7F. */
+uint8_t oracle_e4m3_encode(double x) {
+    if (x != x) return 0x7F;
+    uint8_t sgn = signbit(x) ? 0x80 : 0x00;
+    double a = fabs(x);
+    if (a >= 448.0) return (uint8_t)(sgn | 0x7E);
+    int best = 0;
+    double best_err = a;
+    for (int c = 1; c <= 0x7E; ++c) {
+        double err = fabs(oracle_e4m3_decode((uint8_t)c) - a);
+        if (err < best_err || (err == best_err && (c & 1) == 0)) { best = c; best_err = err; }
+    }
+    return (uint8_t)(sgn | best);
+}
+
+int oracle_e4m3_encode_array(const double *x, int n, uint8_t *codes) {
+    for (int i = 0; i < n; ++i) codes[i] = oracle_e4m3_encode(x[i]);
+    return 0;
+}
+
+/* FP8 write: like oracle_kv_write, but row elements become e4m3 codes of
+ * fp32(x) * fp32(1 / scale[h]) (both products single-precision, rounded to
+ * nearest), with per-kv-head scales for K and V. */
+int oracle_kv_write_fp8(uint8_t *k_cache, uint8_t *v_cache, const uint16_t *k, const uint16_t *v,
+                        const int64_t *slot_mapping, const float *k_scale, const float *v_scale, int num_tokens,
+                        int num_blocks, int num_kv_heads, int bs, int d) {
+    if (num_tokens < 0 || num_blocks <= 0 || num_kv_heads <= 0 || bs <= 0 || d <= 0) return 1;
+    for (int t = 0; t < num_tokens; ++t) {
+        int64_t slot = slot_mapping[t];
+        if (slot < 0) continue;
+        if (slot >= (int64_t)num_blocks * bs) return 2;
+        int64_t block = slot / bs;
+        int offset = (int)(slot % bs);
+        for (int h = 0; h < num_kv_heads; ++h) {
+            float inv_k = 1.0f / k_scale[h], inv_v = 1.0f / v_scale[h];
+            size_t dst = pool_row(block, h, offset, num_kv_heads, bs, d);
+            size_t src = ((size_t)t * num_kv_heads + h) * (size_t)d;
+            for (int c = 0; c < d; ++c) {
+                float xk = (float)bf16_to_f64(k[src + c]) * inv_k;
+                float xv = (float)bf16_to_f64(v[src + c]) * inv_v;
+                k_cache[dst + c] = oracle_e4m3_encode((double)xk);
+                v_cache[dst + c] = oracle_e4m3_encode((double)xv);
+            }
+        }
+    }
+    return 0;
+}
+
+/* FP8 decode attention: the paged attention of oracle_paged_attention with
+ * K = e4m3(code) * k_scale[hkv] and V = e4m3(code) * v_scale[hkv], in double. */
+int oracle_paged_attention_fp8(const uint16_t *q, const uint8_t *k_cache, const uint8_t *v_cache,
+                               const float *k_scale, const float *v_scale, const int32_t *block_tables,
+                               int max_blocks_per_seq, const int32_t *context_lens, int B, int Hq, int Hkv, int d,
+                               int bs, int num_blocks, double scale, double *out) {
+    if (B < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || d <= 0 || bs <= 0) return 1;
+    for (int s = 0; s < B; ++s) {
+        if (context_lens[s] < 0) return 1;
+        if ((int64_t)context_lens[s] > (int64_t)max_blocks_per_seq * bs) return 2;
+    }
+    int g = Hq / Hkv, status = 0;
+#pragma omp parallel for schedule(dynamic, 1) collapse(2)
+    for (int s = 0; s < B; ++s) {
+        for (int hq = 0; hq < Hq; ++hq) {
+            int hkv = hq / g, n = context_lens[s];
+            double *o = out + ((size_t)s * Hq + hq) * (size_t)d;
+            double *z = (double *)malloc(sizeof(double) * (size_t)(n > 0 ? n : 1));
+            if (!z) {
+#pragma omp atomic write
+                status = 1;
+                continue;
+            }
+            const uint16_t *qr = q + ((size_t)s * Hq + hq) * (size_t)d;
+            double m = -INFINITY;
+            int bad = 0;
+            for (int i = 0; i < n; ++i) {
+                int32_t block = block_tables[(size_t)s * max_blocks_per_seq + i / bs];
+                if (block < 0 || block >= num_blocks) { bad = 1; break; }
+                const uint8_t *kr = k_cache + pool_row(block, hkv, i % bs, Hkv, bs, d);
+                double dot = 0.0;
+                for (int c = 0; c < d; ++c) dot += bf16_to_f64(qr[c]) * (oracle_e4m3_decode(kr[c]) * k_scale[hkv]);
+                z[i] = scale * dot;
+                if (z[i] > m) m = z[i];
+            }
+            if (bad) {
+#pragma omp atomic write
+                status = 2;
+                free(z);
+                continue;
+            }
+            double l = 0.0;
+            for (int c = 0; c < d; ++c) o[c] = 0.0;
+            for (int i = 0; i < n; ++i) {
+                int32_t block = block_tables[(size_t)s * max_blocks_per_seq + i / bs];
+                const uint8_t *vr = v_cache + pool_row(block, hkv, i % bs, Hkv, bs, d);
+                double w = exp(z[i] - m);
+                l += w;
+                for (int c = 0; c < d; ++c) o[c] += w * (oracle_e4m3_decode(vr[c]) * v_scale[hkv]);
+            }
+            for (int c = 0; c < d; ++c) o[c] = (l > 0.0) ? o[c] / l : 0.0;
+            free(z);
+        }
+    }
+    return status;
 }

@@ -16,6 +16,7 @@ import oracle
 from tests import test_oracle_pins as pins
 from tests import test_oracle_prefill as prefill_pins
 from tests import test_oracle_block_manager as bm_pins
+from tests import test_oracle_fp8 as fp8_pins
 from tests import test_oracle_swap as swap_pins
 
 PIN_TESTS = [
@@ -39,6 +40,10 @@ PIN_TESTS = [
     swap_pins.test_swap_of_a_permutation_is_a_gather,
     swap_pins.test_lru_worked_example_golden,
     bm_pins.test_block_manager_worked_example_golden,
+    fp8_pins.test_decode_table_matches_library,
+    fp8_pins.test_encode_golden,
+    fp8_pins.test_write_quantizes_into_the_bf16_layout,
+    lambda: fp8_pins.test_attention_equals_bf16_attention_on_exact_values(8, 2),
     lambda: bm_pins.test_conservation_invariants(0),
     lambda: bm_pins.test_append_block_counts_closed_form(0),
     bm_pins.test_slots_feed_the_table_walk,
@@ -85,6 +90,13 @@ MUTANTS = {
                           "--refcount[b]; free_stack[(*top)++] = b;"),
     "fifo free list": ("int32_t b = free_stack[--*top];",
                        "int32_t b = free_stack[0]; memmove(free_stack, free_stack + 1, sizeof(int32_t) * (size_t)(--*top));"),
+    # fp8: subnormals one binade off; ties to the odd code; the scale multiplied
+    # instead of divided on the way in; the key scale applied to the values
+    "e4m3 subnormal exponent": ("if (e == 0) v = ldexp((double)m / 8.0, -6);", "if (e == 0) v = ldexp((double)m / 8.0, -7);"),
+    "e4m3 ties to odd": ("(err == best_err && (c & 1) == 0)", "(err == best_err && (c & 1) == 1)"),
+    "fp8 write scale inverted": ("float inv_k = 1.0f / k_scale[h], inv_v = 1.0f / v_scale[h];",
+                                 "float inv_k = k_scale[h], inv_v = 1.0f / v_scale[h];"),
+    "fp8 value scale": ("(oracle_e4m3_decode(vr[c]) * v_scale[hkv])", "(oracle_e4m3_decode(vr[c]) * k_scale[hkv])"),
     # the new token left out of the attended range (context_len - 1 tokens)
     "context off by one": ("hq, 0, context_lens[s], scale", "hq, 0, context_lens[s] - 1, scale"),
 }
@@ -107,10 +119,11 @@ def test_pins_catch_planted_mistake(name, tmp_path, monkeypatch):
     so = _build_mutant(tmp_path, old, new)
     good = oracle._load()
     lib = ctypes.CDLL(so)
-    for fn in ("oracle_kv_write", "oracle_copy_blocks", "oracle_paged_attention",
-               "oracle_attention_partial", "oracle_lse_merge", "oracle_num_threads", "oracle_paged_prefill"):
-        getattr(lib, fn).argtypes = getattr(good, fn).argtypes
-        getattr(lib, fn).restype = getattr(good, fn).restype
+    # every function the oracle declared argument types for
+    for fn, f in list(vars(good).items()):
+        if fn.startswith("oracle_") and hasattr(f, "argtypes"):
+            getattr(lib, fn).argtypes = f.argtypes
+            getattr(lib, fn).restype = f.restype
     monkeypatch.setattr(oracle, "_lib", lib)
     caught = []
     for t in PIN_TESTS:
