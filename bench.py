@@ -45,10 +45,11 @@ DECODE_SOURCES = ["paged_kv_cache_420_b200/csrc/decode.cuh", "paged_kv_cache_420
 # algorithmic bytes
 # --------------------------------------------------------------------------
 
-def decode_bytes(w) -> int:
+def decode_bytes(w, kv_elem: int = 2) -> int:
     """Bytes paged decode attention must move: every distinct (block, kv head,
-    offset) K and V row of valid tokens once, q and out, the table entries
-    read and the context lengths."""
+    offset) K and V row of valid tokens once (kv_elem bytes per element: 2 for
+    bf16, 1 for an FP8 pool), q and out, the table entries read and the
+    context lengths."""
     bs = w.block_size
     NB = w.num_blocks
     used = np.zeros((NB, bs), dtype=bool)
@@ -61,7 +62,7 @@ def decode_bytes(w) -> int:
         if nb > 0:
             used[w.block_tables[s, nb - 1], : n - full * bs] = True
     token_rows = int(used.sum())
-    kv = token_rows * w.num_kv_heads * w.head_dim * 2 * 2
+    kv = token_rows * w.num_kv_heads * w.head_dim * kv_elem * 2
     qo = 2 * w.num_seqs * w.num_q_heads * w.head_dim * 2
     tables = 4 * int(sum((int(n) + bs - 1) // bs for n in w.context_lens))
     return kv + qo + tables + 4 * w.num_seqs
@@ -477,6 +478,81 @@ def run_prefill_cuda(args, rank, world, dist):
 
 
 SWAP_WORKLOADS = ("llama2-13b-swap",)
+FP8_WORKLOADS = ("llama2-13b-fp8",)
+
+
+def run_fp8_cuda(args, rank, world, dist):
+    """The Llama-2-13B decode step on an FP8 (e4m3) pool: the quantizing write
+    of each sequence's new token, then decode attention over the e4m3 codes
+    with per-kv-head K/V scales.  Metric: algorithmic HBM GB/s of the step (one
+    byte per cached element) and tokens*layers/s, comparable with the bf16
+    step's."""
+    import paged_kv_cache_420_b200 as pkv
+
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
+    torch.cuda.set_device(dev)
+    w = workloads.make("llama2-13b", seed=args.seed + rank, values_device=dev, block_size=args.block_size)
+    k8, v8, ks, vs = workloads.fp8_pools(w)
+    del w.k_cache, w.v_cache
+    torch.cuda.empty_cache()
+    slots = torch.from_numpy(w.slot_mapping).to(dev)
+    tables = torch.from_numpy(w.block_tables).to(dev)
+    ctx = torch.from_numpy(w.context_lens).to(dev)
+    out = torch.empty_like(w.q)
+    mctx = int(w.context_lens.max())
+    ws = torch.empty(pkv.decode_workspace_bytes(w.num_seqs, w.num_q_heads, w.num_kv_heads, w.head_dim, mctx),
+                     dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+
+    def step(i=None):
+        pkv.pkv_write_fp8(w.k_new, w.v_new, slots, ks, vs, k8, v8, stream=stream)
+        if i is not None:
+            ev[i][0].record(stream)
+        pkv.paged_attn_decode_fp8(w.q, k8, v8, ks, vs, tables, ctx, w.scale, w.num_kv_heads, out, mctx,
+                                  workspace=ws, stream=stream)
+        if i is not None:
+            ev[i][1].record(stream)
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(dev.index) as clocks:
+        t0.record(stream)
+        for i in range(args.steps):
+            step(i)
+        t1.record(stream)
+        torch.cuda.synchronize()
+        if dist is not None:
+            dist.barrier()
+        if t0.elapsed_time(t1) < 450:
+            time.sleep(0.45)
+    if pkv.get_device_error():
+        raise RuntimeError("device error word set during the timed region")
+    dec = decode_bytes(w, kv_elem=1)
+    wr = w.num_seqs * w.num_kv_heads * w.head_dim * (2 * 2 + 2) + 8 * w.num_seqs  # bf16 in, e4m3 out
+    ms_max, bytes_all, seqs_all = combine_ranks(dist, t0.elapsed_time(t1), dec + wr, w.num_seqs, dev)
+    dec_ms = sum(a.elapsed_time(b) for a, b in ev) / args.steps
+    peak, kind = measured_hbm_peak()
+    achieved = dec / (dec_ms / 1e3) / 1e9
+    return {
+        "metric": "paged decode attn HBM GB/s on an FP8 (e4m3) pool & tokens*layers/s at 13B shape",
+        "value": whole_job_gbs(bytes_all, args.steps, ms_max), "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_max / args.steps, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "e4m3 KV, bf16 q/out",
+        "data": "synthetic",
+        "config": {"workload": f"{w.name} with an FP8 pool: {w.description}", "block_size": w.block_size,
+                   "num_seqs": w.num_seqs, "seed": args.seed},
+        "tokens_layers_per_s": round(seqs_all * args.steps / (ms_max / 1e3), 1),
+        "roofline": {"kernel": "paged_attn_decode_fp8 (plan + attention kernels)", "bound": "hbm",
+                     "achieved": round(achieved, 1), "peak": peak, "peak_kind": kind, "unit": "GB/s",
+                     "frac": round(achieved / peak, 4), "algorithmic_bytes": dec,
+                     "decode_us": round(dec_ms * 1e3, 2), "traffic": None},
+        "e2e": None, "gpu_launches": 3 * args.steps, "clocks": clocks.summary(),
+    }
 BM_WORKLOADS = ("llama2-13b-blockmgr",)
 
 
@@ -839,6 +915,36 @@ def run_swap_reference(args, world):
     }
 
 
+def run_fp8_reference(args, world):
+    """The oracle's FP8 attention (fp64) on the first sequences of the 13B
+    batch with an FP8 pool, in the GPU line's unit (algorithmic GB/s)."""
+    import oracle
+
+    w = workloads.make("llama2-13b", seed=args.seed, values_device="cpu", block_size=args.block_size)
+    k8, v8, ks, vs = workloads.fp8_pools(w)
+    k8, v8, ks, vs = k8.numpy(), v8.numpy(), ks.numpy(), vs.numpy()
+    n = 8
+    sub = workloads.subset(w, n)
+    times = []
+    for i in range(args.warmup + args.steps):
+        t = time.perf_counter()
+        oracle.paged_attention_fp8(w.q[:n], k8, v8, ks, vs, w.block_tables[:n], w.context_lens[:n], w.scale)
+        if i >= args.warmup:
+            times.append(time.perf_counter() - t)
+    value = round(decode_bytes(sub, kv_elem=1) / statistics.median(times) / 1e9, 4)
+    return {
+        "impl": "reference",
+        "metric": "paged decode attn HBM GB/s on an FP8 (e4m3) pool & tokens*layers/s at 13B shape",
+        "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(1e3 * sum(times) / len(times), 3), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": f"llama2-13b with an FP8 pool, first {n} sequences", "block_size": w.block_size},
+        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": oracle.num_threads(), "kind": "oracle",
+                         "sample": f"first {n} of {w.num_seqs} sequences per step"},
+        "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
 def run_blockmgr_reference(args, world):
     """The oracle's sequential append_slots on the host for the same decode step."""
     import oracle
@@ -880,6 +986,8 @@ def run_reference(args, rank, world):
         return run_swap_reference(args, world)
     if args.workload in BM_WORKLOADS:
         return run_blockmgr_reference(args, world)
+    if args.workload in FP8_WORKLOADS:
+        return run_fp8_reference(args, world)
     w = workloads.make(args.workload, seed=args.seed, values_device="cpu", block_size=args.block_size)
     per_step_budget = max(0.05, min(2.0, 150.0 / max(1, args.steps + args.warmup)))
     pools = oracle_pools(w)
@@ -917,7 +1025,7 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["pkv", "reference"], default="pkv")
     ap.add_argument("--workload", default="llama2-13b",
                     choices=list(workloads.WORKLOADS) + list(workloads.PREFILL_WORKLOADS) + list(SWAP_WORKLOADS)
-                    + list(BM_WORKLOADS))
+                    + list(BM_WORKLOADS) + list(FP8_WORKLOADS))
     ap.add_argument("--block-size", type=int, default=None)
     ap.add_argument("--partition-tokens", type=int, default=-1, help="-1: the workload's choice, 0: library's")
     ap.add_argument("--seed", type=int, default=0)
@@ -947,6 +1055,8 @@ def main(argv=None):
             line = run_swap_cuda(args, rank, world, dist)
         elif args.workload in BM_WORKLOADS:
             line = run_blockmgr_cuda(args, rank, world, dist)
+        elif args.workload in FP8_WORKLOADS:
+            line = run_fp8_cuda(args, rank, world, dist)
         else:
             line = run_cuda(args, rank, world, dist)
         if rank == 0 and line is not None:

@@ -271,6 +271,37 @@ pkv_status paged_attn_prefill(const void *q, const void *k_cache, const void *v_
                               void *workspace, size_t workspace_bytes, pkv_stream_t stream);
 
 /*
+ * FP8 KV cache -- the pool holds OCP FP8 E4M3 codes (1 sign, 4 exponent bits
+ * with bias 7, 3 mantissa bits, no infinities, S.1111.111 NaN, largest finite
+ * 448), one byte per element, same [num_blocks][num_kv_heads][block_size]
+ * [head_dim] layout; half the bytes of bf16 per token.  The pages name FP8
+ * mixed precision as a way to cut memory and raise throughput (ai-stack.site
+ * "Nano-vLLM 原理", case study).  Each kv head has a static dequantisation
+ * scale for K and one for V (fp32 device arrays [num_kv_heads], chosen by the
+ * caller, e.g. from calibration): the value of a code c is e4m3(c) * scale.
+ *
+ * pkv_write_fp8: as pkv_write, storing for every element
+ *   code = e4m3_rne_satfinite(fp32(x) * fp32(1 / scale[h]))
+ * (IEEE round-to-nearest reciprocal and product; ties to the even code;
+ * magnitudes beyond 448 saturate).  Codes are bit-exact with that rule.
+ *
+ * paged_attn_decode_fp8: as paged_attn_decode over an FP8 pool, reading
+ * K = e4m3(code) * k_scale[h] and V = e4m3(code) * v_scale[h].  Supported at
+ * head_dim 128 with num_q_heads / num_kv_heads <= 2 (else PKV_EUNSUPPORTED);
+ * the codes are multiplied exactly as f16 with fp32 accumulation.  The
+ * workspace is the same as paged_attn_decode's.
+ */
+pkv_status pkv_write_fp8(const void *k, const void *v, const int64_t *slot_mapping, int32_t num_tokens,
+                         const float *k_scale, const float *v_scale, void *k_cache, void *v_cache, pkv_pool pool,
+                         pkv_stream_t stream);
+pkv_status paged_attn_decode_fp8(const void *q, const void *k_cache, const void *v_cache, const float *k_scale,
+                                 const float *v_scale, const int32_t *block_tables, int32_t max_blocks_per_seq,
+                                 const int32_t *context_lens, int32_t num_seqs, int32_t num_q_heads, float scale,
+                                 int32_t num_kv_heads, void *out, pkv_pool pool, int32_t max_context_len,
+                                 int32_t partition_tokens, void *workspace, size_t workspace_bytes,
+                                 pkv_stream_t stream);
+
+/*
  * Block manager on the device -- the bookkeeping of the pages' block manager
  * (wkbse.com section 3.1, "flexible memory management": blocks allocated only
  * as new tokens need them, the block table updated, blocks returned when a

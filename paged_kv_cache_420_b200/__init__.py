@@ -27,7 +27,8 @@ EXPORTED = ("pkv_write", "pkv_copy_blocks", "pkv_decode_workspace_bytes", "paged
             "paged_attn_decode_static_ws", "pkv_prefill_workspace_bytes", "paged_attn_prefill",
             "pkv_get_device_error", "pkv_selftest_bounded_wait", "pkv_status_string", "pkv_version",
             "pkv_swap_out", "pkv_swap_in", "pkv_lru_victims", "pkv_bm_state_bytes", "pkv_bm_init", "pkv_bm_alloc",
-            "pkv_bm_free", "pkv_bm_share", "pkv_bm_append_slots", "pkv_copy_blocks_dev")
+            "pkv_bm_free", "pkv_bm_share", "pkv_bm_append_slots", "pkv_copy_blocks_dev", "pkv_write_fp8",
+            "paged_attn_decode_fp8")
 STATIC_WS_BYTES = 32 << 20  # PKV_STATIC_WS_BYTES
 
 
@@ -70,12 +71,15 @@ def load_library() -> ctypes.CDLL:
         lib.pkv_bm_share.argtypes = [P, I32, P, I32, P]
         lib.pkv_bm_append_slots.argtypes = [P, I32, P, I32, P, P, I32, I32, P, I64, P, P, P]
         lib.pkv_copy_blocks_dev.argtypes = [P, P, I32, P, P, _Pool, P]
+        lib.pkv_write_fp8.argtypes = [P, P, P, I32, P, P, P, P, _Pool, P]
+        lib.paged_attn_decode_fp8.argtypes = [P, P, P, P, P, P, I32, P, I32, I32, F, I32, P, _Pool, I32, I32, P, SZ,
+                                              P]
         lib.pkv_status_string.argtypes = [ctypes.c_int]
         lib.pkv_status_string.restype = ctypes.c_char_p
         lib.pkv_version.restype = I32
         for f in ("pkv_write", "pkv_copy_blocks", "paged_attn_decode", "pkv_get_device_error", "pkv_swap_out",
                   "pkv_swap_in", "pkv_lru_victims", "pkv_bm_init", "pkv_bm_alloc", "pkv_bm_free", "pkv_bm_share",
-                  "pkv_bm_append_slots", "pkv_copy_blocks_dev"):
+                  "pkv_bm_append_slots", "pkv_copy_blocks_dev", "pkv_write_fp8", "paged_attn_decode_fp8"):
             getattr(lib, f).restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -290,6 +294,57 @@ def copy_blocks_dev(cow_pairs: torch.Tensor, num_pairs: torch.Tensor, k_cache: t
         _need(t, n, torch.bfloat16)
     _check(load_library().pkv_copy_blocks_dev(_ptr(cow_pairs), _ptr(num_pairs), cow_pairs.shape[0], _ptr(k_cache),
                                               _ptr(v_cache), _pool(k_cache), _stream(stream)), "pkv_copy_blocks_dev")
+
+
+def _need_scales(k_scale, v_scale, hkv):
+    for t, n in ((k_scale, "k_scale"), (v_scale, "v_scale")):
+        _need(t, n, torch.float32)
+        if t.numel() != hkv:
+            raise ValueError(f"{n} must hold one scale per kv head ({hkv})")
+
+
+def pkv_write_fp8(k: torch.Tensor, v: torch.Tensor, slot_mapping: torch.Tensor, k_scale: torch.Tensor,
+                  v_scale: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, stream=None) -> None:
+    """cache[slot // bs][h][slot % bs] = e4m3(fp32(k[t][h]) / scale[h]) (and v) for every token with slot >= 0;
+    the caches are uint8 tensors [num_blocks, num_kv_heads, block_size, head_dim]."""
+    for t, n in ((k, "k"), (v, "v")):
+        _need(t, n, torch.bfloat16)
+    for t, n in ((k_cache, "k_cache"), (v_cache, "v_cache")):
+        _need(t, n, torch.uint8)
+    _need(slot_mapping, "slot_mapping", torch.int64)
+    _need_scales(k_scale, v_scale, k_cache.shape[1])
+    T = slot_mapping.shape[0]
+    if k.shape != (T, k_cache.shape[1], k_cache.shape[3]) or v.shape != k.shape or v_cache.shape != k_cache.shape:
+        raise ValueError("k/v must be [num_tokens, num_kv_heads, head_dim] and the caches alike")
+    st = load_library().pkv_write_fp8(_ptr(k), _ptr(v), _ptr(slot_mapping), T, _ptr(k_scale), _ptr(v_scale),
+                                      _ptr(k_cache), _ptr(v_cache), _pool(k_cache), _stream(stream))
+    _check(st, "pkv_write_fp8")
+
+
+def paged_attn_decode_fp8(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, k_scale: torch.Tensor,
+                          v_scale: torch.Tensor, block_tables: torch.Tensor, context_lens: torch.Tensor, scale: float,
+                          num_kv_heads: int, out: torch.Tensor, max_context_len: int, partition_tokens: int = 0,
+                          workspace: Optional[torch.Tensor] = None, stream=None) -> None:
+    """paged_attn_decode over an FP8 (e4m3) pool with per-kv-head K and V scales."""
+    for t, n in ((q, "q"), (out, "out")):
+        _need(t, n, torch.bfloat16)
+    for t, n in ((k_cache, "k_cache"), (v_cache, "v_cache")):
+        _need(t, n, torch.uint8)
+    _need(block_tables, "block_tables", torch.int32)
+    _need(context_lens, "context_lens", torch.int32)
+    _need_scales(k_scale, v_scale, num_kv_heads)
+    B, Hq, D = q.shape
+    if out.shape != q.shape or v_cache.shape != k_cache.shape:
+        raise ValueError("out must match q and v_cache must match k_cache")
+    if workspace is None:
+        workspace = torch.empty(decode_workspace_bytes(B, Hq, num_kv_heads, D, max_context_len, partition_tokens),
+                                dtype=torch.uint8, device=q.device)
+    st = load_library().paged_attn_decode_fp8(
+        _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(k_scale), _ptr(v_scale), _ptr(block_tables),
+        block_tables.shape[1], _ptr(context_lens), B, Hq, float(scale), int(num_kv_heads), _ptr(out),
+        _pool(k_cache), int(max_context_len), int(partition_tokens), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(st, "paged_attn_decode_fp8")
 
 
 def decode_workspace_bytes(num_seqs: int, num_q_heads: int, num_kv_heads: int, head_dim: int,

@@ -63,6 +63,8 @@ struct DecodeParams {
     int B, Hq, Hkv, g, MBS, bs, NB, max_ctx, PT, maxP;
     int pool_rows;                // NB * Hkv * bs: first out-of-range TMA row
     float scale_log2;             // scale * log2(e)
+    const float *k_scale = nullptr;  // FP8 pool: dequantisation scale per kv head (nullptr: bf16 pool)
+    const float *v_scale = nullptr;
 };
 
 // Context length of sequence s, clamped to what the table and the workspace
@@ -163,11 +165,13 @@ struct StageInfo {
     int ord;                 // CTA-local item ordinal (selects the q buffer); -1 ends the stream
 };
 
-template <int D, int GP, int NS>
+template <int D, int GP, int NS, bool KV8 = false>
 struct DecodeSmem {
     static constexpr int kW = kConsumerWarps;
-    static constexpr int kHalfTile = kStageTok * 64 * 2;  // 16 rows x 64 elements = 2 KB
-    static constexpr int kTile = kStageTok * D * 2;       // one K (or V) stage tile
+    static constexpr int kElem = KV8 ? 1 : 2;             // bytes per K/V element (e4m3 or bf16)
+    static constexpr int kHalfTile = kStageTok * 128;     // one TMA box: 16 rows x 128 bytes = 2 KB
+    static constexpr int kBoxes = D * kElem / 128;        // boxes per row of a tile
+    static constexpr int kTile = kStageTok * D * kElem;   // one K (or V) stage tile
     static constexpr int kStage = 2 * kTile;
     static constexpr int kQBuf = GP * D * 2;              // the query heads of one kv head
     static constexpr int kMergeStride = D + 4;            // floats, padded against bank conflicts
@@ -211,11 +215,52 @@ __device__ __forceinline__ uint32_t tile_addr(uint32_t tile, int r, int c) {
     return tile + half * (kStageTok * 128) + r * 128 + ((chunk ^ (r & 7)) << 4) + ((c & 7) << 1);
 }
 
+// Byte address of e4m3 element (row r, column c) of an FP8 stage tile: one
+// 128-byte line per row, 16-byte chunks XOR-swizzled with (r & 7).
+__device__ __forceinline__ uint32_t tile_addr8(uint32_t tile, int r, int c) {
+    return tile + r * 128 + ((((c >> 4) ^ (r & 7))) << 4) + (c & 15);
+}
+
+__device__ __forceinline__ uint32_t f16x2_from_e4m3x2(uint32_t pair16) {
+    uint32_t r;
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(r) : "h"((unsigned short)pair16));
+    return r;
+}
+
+__device__ __forceinline__ uint32_t f16x2_from_f32(float lo, float hi) {
+    uint32_t r;
+    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+// acc + a * b with f16 a, b (the low or high halves of f16x2 words) and an
+// fp32 accumulator (mixed-precision FMA, sm_100).
+__device__ __forceinline__ float fma_f16lo(uint32_t a, uint32_t b, float acc) {
+    float r;
+    asm("{\n\t.reg .b16 al, ah, bl, bh;\n\tmov.b32 {al, ah}, %1;\n\tmov.b32 {bl, bh}, %2;\n\t"
+        "fma.rn.f32.f16 %0, al, bl, %3;\n\t}"
+        : "=f"(r) : "r"(a), "r"(b), "f"(acc));
+    return r;
+}
+__device__ __forceinline__ float fma_f16hi(uint32_t a, uint32_t b, float acc) {
+    float r;
+    asm("{\n\t.reg .b16 al, ah, bl, bh;\n\tmov.b32 {al, ah}, %1;\n\tmov.b32 {bl, bh}, %2;\n\t"
+        "fma.rn.f32.f16 %0, ah, bh, %3;\n\t}"
+        : "=f"(r) : "r"(a), "r"(b), "f"(acc));
+    return r;
+}
+
 // ----------------------------------------------- CUDA-core path (g <= 2) ----
-template <int D, int G>
+// KV8: the stage tiles hold e4m3 codes.  q is kept as exact f16 pairs, K and V
+// codes are converted to f16 (exactly) and multiplied in mixed precision with
+// fp32 accumulation; the K scale times scale * log2 e multiplies each summed
+// score, and the V scale is applied to the final output.
+template <int D, int G, bool KV8 = false>
 struct SimtState {
     static constexpr int EPL = D / 32;  // elements per lane
     float q[G][EPL];
+    uint32_t q16[G][EPL / 2];  // KV8: q as f16 pairs
+    float kscale;              // KV8: scale * log2(e) * k_scale of the kv head
     float acc[G][EPL];
     float m[G];
     float l_part;  // this lane's share of l for head (lane / 16) (G = 2) or head 0
@@ -231,14 +276,27 @@ struct SimtState {
     }
 
     __device__ __forceinline__ void load_q(const __nv_bfloat16 *qs, int lane, float scale_log2) {
+        kscale = scale_log2;
 #pragma unroll
         for (int j = 0; j < G; ++j)
 #pragma unroll
             for (int e = 0; e < EPL; e += 2) {
                 const uint32_t pr = *reinterpret_cast<const uint32_t *>(qs + j * D + lane * EPL + e);
-                q[j][e] = bf16lo_to_f32(pr) * scale_log2;
-                q[j][e + 1] = bf16hi_to_f32(pr) * scale_log2;
+                if constexpr (KV8) {
+                    q16[j][e / 2] = f16x2_from_f32(bf16lo_to_f32(pr), bf16hi_to_f32(pr));
+                } else {
+                    q[j][e] = bf16lo_to_f32(pr) * scale_log2;
+                    q[j][e + 1] = bf16hi_to_f32(pr) * scale_log2;
+                }
             }
+    }
+
+    // KV8: this lane's 4 codes of row r as two f16 pairs.
+    __device__ __forceinline__ void load_row8(uint32_t tile, int r, int lane, uint32_t (&h)[2]) {
+        uint32_t w;
+        asm volatile("ld.shared.u32 %0, [%1];" : "=r"(w) : "r"(tile_addr8(tile, r, lane * EPL)));
+        h[0] = f16x2_from_e4m3x2(w & 0xffffu);
+        h[1] = f16x2_from_e4m3x2(w >> 16);
     }
 
     // Loads this lane's EPL elements of row r of a tile as fp32.
@@ -261,18 +319,34 @@ struct SimtState {
         float v[NV];
         // q.k partial sums v[j*16 + r] for head j, token r; tokens r and r+1
         // share one packed fp32x2 FMA per element.
+        if constexpr (KV8) {
+            static_assert(EPL == 4, "FP8 stage tiles are 128-byte rows (head dim 128)");
 #pragma unroll
-        for (int r = 0; r < 16; r += 2) {
-            float x0[EPL], x1[EPL];
-            load_row(ktile, r, lane, x0);
-            load_row(ktile, r + 1, lane, x1);
+            for (int r = 0; r < 16; ++r) {
+                uint32_t k16[2];
+                load_row8(ktile, r, lane, k16);
 #pragma unroll
-            for (int j = 0; j < G; ++j) {
-                float d0 = 0.f, d1 = 0.f;
+                for (int j = 0; j < G; ++j) {
+                    float d = fma_f16lo(q16[j][0], k16[0], 0.f);
+                    d = fma_f16hi(q16[j][0], k16[0], d);
+                    d = fma_f16lo(q16[j][1], k16[1], d);
+                    v[j * 16 + r] = fma_f16hi(q16[j][1], k16[1], d);
+                }
+            }
+        } else {
 #pragma unroll
-                for (int e = 0; e < EPL; ++e) fma_f32x2(d0, d1, q[j][e], q[j][e], x0[e], x1[e]);
-                v[j * 16 + r] = d0;
-                v[j * 16 + r + 1] = d1;
+            for (int r = 0; r < 16; r += 2) {
+                float x0[EPL], x1[EPL];
+                load_row(ktile, r, lane, x0);
+                load_row(ktile, r + 1, lane, x1);
+#pragma unroll
+                for (int j = 0; j < G; ++j) {
+                    float d0 = 0.f, d1 = 0.f;
+#pragma unroll
+                    for (int e = 0; e < EPL; ++e) fma_f32x2(d0, d1, q[j][e], q[j][e], x0[e], x1[e]);
+                    v[j * 16 + r] = d0;
+                    v[j * 16 + r + 1] = d1;
+                }
             }
         }
         // Transposing butterfly: after it, lane holds the full 32-lane sum of
@@ -298,7 +372,7 @@ struct SimtState {
         }
         const int my_tok = (G == 1) ? (lane >> 1) : (lane & 15);
         const int my_head = (G == 1) ? 0 : (lane >> 4);
-        const float score = (my_tok < valid) ? v[0] : PKV_NEG_INF;
+        const float score = (my_tok < valid) ? (KV8 ? v[0] * kscale : v[0]) : PKV_NEG_INF;
         // stage max per head (one warp reduction each), lazy rescale
         float mx[G];
         if constexpr (G == 1) {
@@ -325,14 +399,30 @@ struct SimtState {
 #pragma unroll
         for (int r = 0; r < 16; ++r) {
             if (r < valid) {
-                float x[EPL];
-                load_row(vtile, r, lane, x);
+                if constexpr (KV8) {
+                    uint32_t v16[2];
+                    load_row8(vtile, r, lane, v16);
 #pragma unroll
-                for (int j = 0; j < G; ++j) {
-                    const int src = (G == 1) ? (2 * r) : (j * 16 + r);
-                    const float pj = __shfl_sync(0xffffffffu, pr, src);
+                    for (int j = 0; j < G; ++j) {
+                        const int src = (G == 1) ? (2 * r) : (j * 16 + r);
+                        const float pj = __shfl_sync(0xffffffffu, pr, src);
+                        const uint32_t p16 = f16x2_from_f32(pj, pj);
+                        acc[j][0] = fma_f16lo(p16, v16[0], acc[j][0]);
+                        acc[j][1] = fma_f16hi(p16, v16[0], acc[j][1]);
+                        acc[j][2] = fma_f16lo(p16, v16[1], acc[j][2]);
+                        acc[j][3] = fma_f16hi(p16, v16[1], acc[j][3]);
+                    }
+                } else {
+                    float x[EPL];
+                    load_row(vtile, r, lane, x);
 #pragma unroll
-                    for (int e = 0; e < EPL; e += 2) fma_f32x2(acc[j][e], acc[j][e + 1], pj, pj, x[e], x[e + 1]);
+                    for (int j = 0; j < G; ++j) {
+                        const int src = (G == 1) ? (2 * r) : (j * 16 + r);
+                        const float pj = __shfl_sync(0xffffffffu, pr, src);
+#pragma unroll
+                        for (int e = 0; e < EPL; e += 2)
+                            fma_f32x2(acc[j][e], acc[j][e + 1], pj, pj, x[e], x[e + 1]);
+                    }
                 }
             }
         }
@@ -520,14 +610,15 @@ struct MmaState {
 
 // PATH 0: CUDA cores with G = GSIMT heads per kv head; PATH 1: tensor cores
 // with query heads padded to GPAD in {4, 8, 16} (n-tiles of 8: GPAD/8 rounded up).
-template <int D, int PATH, int GSIMT, int GPAD, int NS>
+template <int D, int PATH, int GSIMT, int GPAD, int NS, bool KV8 = false>
 __global__ void __launch_bounds__(kDecodeThreads) paged_decode_kernel(const __grid_constant__ CUtensorMap tmap_k,
                                                                       const __grid_constant__ CUtensorMap tmap_v,
                                                                       const DecodeParams p) {
     constexpr int W = kConsumerWarps;
     constexpr int GP = PATH == 0 ? GSIMT : GPAD;
     constexpr int NT = (GPAD + 7) / 8;
-    using L = DecodeSmem<D, GP, NS>;
+    static_assert(!KV8 || (PATH == 0 && D == 128), "the FP8 pool runs on the CUDA-core path at head dim 128");
+    using L = DecodeSmem<D, GP, NS, KV8>;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     // 1024-B alignment: the 128-byte swizzle pattern repeats every 1 KB.
     // Everything below indexes the shared array itself, so accesses stay in
@@ -643,9 +734,10 @@ __global__ void __launch_bounds__(kDecodeThreads) paged_decode_kernel(const __gr
                             const uint32_t kt = tiles + slot * L::kStage;
                             mbar_arrive_expect_tx(&full[slot], (uint32_t)L::kStage);
 #pragma unroll
-                            for (int hf = 0; hf < D / 64; ++hf) {
-                                tma_load_2d_u32(kt + hf * L::kHalfTile, &tmap_k, &full[slot], hf * 64, row);
-                                tma_load_2d_u32(kt + L::kTile + hf * L::kHalfTile, &tmap_v, &full[slot], hf * 64, row);
+                            for (int hf = 0; hf < L::kBoxes; ++hf) {
+                                const int x = hf * (128 / L::kElem);  // box column in elements
+                                tma_load_2d_u32(kt + hf * L::kHalfTile, &tmap_k, &full[slot], x, row);
+                                tma_load_2d_u32(kt + L::kTile + hf * L::kHalfTile, &tmap_v, &full[slot], x, row);
                             }
                         } else {
                             mbar_arrive(&full[slot]);
@@ -683,7 +775,7 @@ __global__ void __launch_bounds__(kDecodeThreads) paged_decode_kernel(const __gr
         uint32_t gc = w;
         uint32_t mc = 0;  // merges done
         float scale_log2 = p.scale_log2;
-        SimtState<D, (PATH == 0 ? GSIMT : 1)> st0;
+        SimtState<D, (PATH == 0 ? GSIMT : 1), KV8> st0;
         MmaState<D, (PATH == 1 ? NT : 1)> st1;
         while (true) {
             const uint32_t slot = gc % NS;
@@ -695,7 +787,10 @@ __global__ void __launch_bounds__(kDecodeThreads) paged_decode_kernel(const __gr
                 const int qb = si.ord & 1;
                 if (!wait_or_abort(&qfull[qb], (si.ord >> 1) & 1, abort_flag)) break;
                 const __nv_bfloat16 *qs = qbuf + qb * (L::kQBuf / 2);
-                if constexpr (PATH == 0) { st0.reset(); st0.load_q(qs, lane, scale_log2); }
+                if constexpr (PATH == 0) {
+                    st0.reset();
+                    st0.load_q(qs, lane, KV8 ? scale_log2 * __ldg(p.k_scale + si.h) : scale_log2);
+                }
                 else { st1.reset(); st1.load_q(qs, lane, p.g); }
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&qempty[qb]);
@@ -733,7 +828,8 @@ __global__ void __launch_bounds__(kDecodeThreads) paged_decode_kernel(const __gr
                         f[u] = mu == PKV_NEG_INF ? 0.f : exp2f(mu - M);
                         Lsum = fmaf(mL[u * GP + j], f[u], Lsum);
                     }
-                    const float invL = Lsum > 0.f ? 1.f / Lsum : 0.f;
+                    float invL = Lsum > 0.f ? 1.f / Lsum : 0.f;
+                    if constexpr (KV8) invL *= __ldg(p.v_scale + si.h);
 #pragma unroll
                     for (int i = 0; i < D / 32; ++i) {
                         const int d = lane + 32 * i;
@@ -807,7 +903,8 @@ __global__ void __launch_bounds__(kReduceWarps * 32) splitk_reduce_kernel(const 
         float Lt = 0.f;
 #pragma unroll
         for (int u = 0; u < kReduceWarps; ++u) Lt += s_l[u];
-        const float inv = Lt > 0.f ? 1.f / Lt : 0.f;
+        float inv = Lt > 0.f ? 1.f / Lt : 0.f;
+        if (p.v_scale) inv *= __ldg(p.v_scale + (unit % p.Hq) / p.g);  // FP8 pool: the kv head's V scale
 #pragma unroll
         for (int e = 0; e < EPL; ++e) {
             float o = 0.f;

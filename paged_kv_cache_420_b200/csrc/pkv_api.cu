@@ -101,6 +101,22 @@ bool encode_pool_map(CUtensorMap *map, const void *base, const pkv_pool &pool) {
     return r == CUDA_SUCCESS;
 }
 
+// An FP8 pool (e4m3 codes) as 2-D [rows][D] bytes; a box is 16 rows x 128
+// bytes, the whole row at head dim 128.
+bool encode_pool_map_u8(CUtensorMap *map, const void *base, const pkv_pool &pool) {
+    auto fn = encode_fn();
+    if (!fn || pool.head_dim != 128) return false;
+    const cuuint64_t rows = (cuuint64_t)pool.num_blocks * pool.num_kv_heads * pool.block_size;
+    cuuint64_t dims[2] = {(cuuint64_t)pool.head_dim, rows};
+    cuuint64_t strides[1] = {(cuuint64_t)pool.head_dim};
+    cuuint32_t box[2] = {128, (cuuint32_t)pkv::kStageTok};
+    cuuint32_t estr[2] = {1, 1};
+    const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 // The query tensor [T][Hq][D] viewed as 3-D (columns, heads, tokens); a box is
 // 64 columns x g heads x QT tokens, so one tcgen05 prefill tile (rows = token x
 // head of the group) lands as [QT][g][64] with the 128-byte swizzle.
@@ -151,12 +167,12 @@ bool workspace_layout(int32_t B, int32_t Hq, int32_t D, int32_t max_ctx, int32_t
 
 // ---------------------------------------------------- decode dispatch ----
 
-template <int D, int PATH, int GS, int GPAD>
+template <int D, int PATH, int GS, int GPAD, bool KV8 = false>
 pkv_status launch_decode(const pkv::DecodeParams &prm, const CUtensorMap &mk, const CUtensorMap &mv,
                          cudaStream_t stream, int dev) {
     constexpr int NS = PATH == 0 ? kStagesSimt : kStagesMma;
-    using L = pkv::DecodeSmem<D, (PATH == 0 ? GS : GPAD), NS>;
-    auto kernel = pkv::paged_decode_kernel<D, PATH, GS, GPAD, NS>;
+    using L = pkv::DecodeSmem<D, (PATH == 0 ? GS : GPAD), NS, KV8>;
+    auto kernel = pkv::paged_decode_kernel<D, PATH, GS, GPAD, NS, KV8>;
     static int occ_cache[kMaxDevices] = {0};
     int occ = (dev >= 0 && dev < kMaxDevices) ? occ_cache[dev] : 0;
     if (occ == 0) {
@@ -354,6 +370,79 @@ bool bm_state(void *state, int32_t nb, pkv::BmState *s) {
     return true;
 }
 
+// Decode over a bf16 pool (scales null) or an FP8 (e4m3) pool with per-kv-head
+// dequantisation scales (head dim 128, GQA group <= 2: the CUDA-core path).
+pkv_status decode_impl(const void *q, const void *k_cache, const void *v_cache, const float *k_scale,
+                       const float *v_scale, const int32_t *block_tables, int32_t max_blocks_per_seq,
+                       const int32_t *context_lens, int32_t num_seqs, int32_t num_q_heads, float scale,
+                       int32_t num_kv_heads, void *out, pkv_pool pool, int32_t max_context_len,
+                       int32_t partition_tokens, void *workspace, size_t workspace_bytes, pkv_stream_t stream) {
+    const bool kv8 = k_scale != nullptr;
+    const pkv_status ps = check_pool(pool);
+    if (ps != PKV_OK) return ps;
+    if (num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || max_blocks_per_seq <= 0 || max_context_len < 0)
+        return PKV_EINVAL;
+    if (num_kv_heads != pool.num_kv_heads || num_q_heads % num_kv_heads != 0) return PKV_EINVAL;
+    const int g = num_q_heads / num_kv_heads;
+    if (g > 16) return PKV_EUNSUPPORTED;
+    if (kv8 && (pool.head_dim != 128 || g > 2)) return PKV_EUNSUPPORTED;
+    if (partition_tokens < 0 || partition_tokens % 16 != 0 || partition_tokens > 65536) return PKV_EINVAL;
+    if (num_seqs == 0) return PKV_OK;
+    if (!q || !k_cache || !v_cache || !block_tables || !context_lens || !out || !workspace) return PKV_EINVAL;
+    if (!aligned(q, 16) || !aligned(out, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) ||
+        !aligned(block_tables, 4) || !aligned(context_lens, 4) || !aligned(workspace, 256))
+        return PKV_EINVAL;
+    const int D = pool.head_dim;
+    const int PT = pick_partition_tokens(partition_tokens, max_context_len);
+    WorkspaceLayout wl;
+    if (!workspace_layout(num_seqs, num_q_heads, D, max_context_len, PT, &wl) || workspace_bytes < wl.total)
+        return PKV_EINVAL;
+
+    pkv::DecodeParams prm;
+    prm.q = static_cast<const __nv_bfloat16 *>(q);
+    prm.out = static_cast<__nv_bfloat16 *>(out);
+    prm.block_tables = block_tables;
+    prm.context_lens = context_lens;
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    prm.num_entries = reinterpret_cast<int32_t *>(ws + wl.off_count);
+    prm.work_counter = reinterpret_cast<int32_t *>(ws + wl.off_count) + 1;
+    prm.entries = reinterpret_cast<int2 *>(ws + wl.off_entries);
+    prm.part_ml = reinterpret_cast<float2 *>(ws + wl.off_ml);
+    prm.part_acc = reinterpret_cast<float *>(ws + wl.off_acc);
+    prm.B = num_seqs;
+    prm.Hq = num_q_heads;
+    prm.Hkv = num_kv_heads;
+    prm.g = g;
+    prm.MBS = max_blocks_per_seq;
+    prm.bs = pool.block_size;
+    prm.NB = pool.num_blocks;
+    prm.max_ctx = max_context_len;
+    prm.PT = PT;
+    prm.maxP = (int)std::max<long long>(1, ((long long)max_context_len + PT - 1) / PT);
+    prm.pool_rows = pool.num_blocks * pool.num_kv_heads * pool.block_size;
+    prm.scale_log2 = scale * 1.4426950408889634f;
+    prm.k_scale = k_scale;
+    prm.v_scale = v_scale;
+
+    CUtensorMap mk, mv;
+    if (kv8) {
+        if (!encode_pool_map_u8(&mk, k_cache, pool) || !encode_pool_map_u8(&mv, v_cache, pool)) return PKV_ECUDA;
+    } else if (!encode_pool_map(&mk, k_cache, pool) || !encode_pool_map(&mv, v_cache, pool)) {
+        return PKV_ECUDA;
+    }
+
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    pkv::plan_kernel<<<1, pkv::kPlanThreads, 0, st>>>(prm, D);
+    pkv_status r = launch_status();
+    if (r != PKV_OK) return r;
+    const int dev = current_device();
+    if (kv8) {
+        return g == 1 ? launch_decode<128, 0, 1, 1, true>(prm, mk, mv, st, dev)
+                      : launch_decode<128, 0, 2, 1, true>(prm, mk, mv, st, dev);
+    }
+    return D == 128 ? dispatch_group<128>(g, prm, mk, mv, st, dev) : dispatch_group<64>(g, prm, mk, mv, st, dev);
+}
+
 }  // namespace
 
 extern "C" {
@@ -486,58 +575,51 @@ pkv_status paged_attn_decode(const void *q, const void *k_cache, const void *v_c
                              int32_t num_q_heads, float scale, int32_t num_kv_heads, void *out, pkv_pool pool,
                              int32_t max_context_len, int32_t partition_tokens, void *workspace,
                              size_t workspace_bytes, pkv_stream_t stream) {
+    return decode_impl(q, k_cache, v_cache, nullptr, nullptr, block_tables, max_blocks_per_seq, context_lens,
+                       num_seqs, num_q_heads, scale, num_kv_heads, out, pool, max_context_len, partition_tokens,
+                       workspace, workspace_bytes, stream);
+}
+
+pkv_status paged_attn_decode_fp8(const void *q, const void *k_cache, const void *v_cache, const float *k_scale,
+                                 const float *v_scale, const int32_t *block_tables, int32_t max_blocks_per_seq,
+                                 const int32_t *context_lens, int32_t num_seqs, int32_t num_q_heads, float scale,
+                                 int32_t num_kv_heads, void *out, pkv_pool pool, int32_t max_context_len,
+                                 int32_t partition_tokens, void *workspace, size_t workspace_bytes,
+                                 pkv_stream_t stream) {
+    if (!k_scale || !v_scale || !aligned(k_scale, 4) || !aligned(v_scale, 4)) return PKV_EINVAL;
+    return decode_impl(q, k_cache, v_cache, k_scale, v_scale, block_tables, max_blocks_per_seq, context_lens,
+                       num_seqs, num_q_heads, scale, num_kv_heads, out, pool, max_context_len, partition_tokens,
+                       workspace, workspace_bytes, stream);
+}
+
+pkv_status pkv_write_fp8(const void *k, const void *v, const int64_t *slot_mapping, int32_t num_tokens,
+                         const float *k_scale, const float *v_scale, void *k_cache, void *v_cache, pkv_pool pool,
+                         pkv_stream_t stream) {
     const pkv_status ps = check_pool(pool);
     if (ps != PKV_OK) return ps;
-    if (num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || max_blocks_per_seq <= 0 || max_context_len < 0)
+    if (num_tokens < 0) return PKV_EINVAL;
+    if (num_tokens == 0) return PKV_OK;
+    if (!k || !v || !slot_mapping || !k_cache || !v_cache || !k_scale || !v_scale) return PKV_EINVAL;
+    if (!aligned(k, 16) || !aligned(v, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) ||
+        !aligned(slot_mapping, 8) || !aligned(k_scale, 4) || !aligned(v_scale, 4))
         return PKV_EINVAL;
-    if (num_kv_heads != pool.num_kv_heads || num_q_heads % num_kv_heads != 0) return PKV_EINVAL;
-    const int g = num_q_heads / num_kv_heads;
-    if (g > 16) return PKV_EUNSUPPORTED;
-    if (partition_tokens < 0 || partition_tokens % 16 != 0 || partition_tokens > 65536) return PKV_EINVAL;
-    if (num_seqs == 0) return PKV_OK;
-    if (!q || !k_cache || !v_cache || !block_tables || !context_lens || !out || !workspace) return PKV_EINVAL;
-    if (!aligned(q, 16) || !aligned(out, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) ||
-        !aligned(block_tables, 4) || !aligned(context_lens, 4) || !aligned(workspace, 256))
-        return PKV_EINVAL;
-    const int D = pool.head_dim;
-    const int PT = pick_partition_tokens(partition_tokens, max_context_len);
-    WorkspaceLayout wl;
-    if (!workspace_layout(num_seqs, num_q_heads, D, max_context_len, PT, &wl) || workspace_bytes < wl.total)
-        return PKV_EINVAL;
-
-    pkv::DecodeParams prm;
-    prm.q = static_cast<const __nv_bfloat16 *>(q);
-    prm.out = static_cast<__nv_bfloat16 *>(out);
-    prm.block_tables = block_tables;
-    prm.context_lens = context_lens;
-    uint8_t *ws = static_cast<uint8_t *>(workspace);
-    prm.num_entries = reinterpret_cast<int32_t *>(ws + wl.off_count);
-    prm.work_counter = reinterpret_cast<int32_t *>(ws + wl.off_count) + 1;
-    prm.entries = reinterpret_cast<int2 *>(ws + wl.off_entries);
-    prm.part_ml = reinterpret_cast<float2 *>(ws + wl.off_ml);
-    prm.part_acc = reinterpret_cast<float *>(ws + wl.off_acc);
-    prm.B = num_seqs;
-    prm.Hq = num_q_heads;
-    prm.Hkv = num_kv_heads;
-    prm.g = g;
-    prm.MBS = max_blocks_per_seq;
-    prm.bs = pool.block_size;
-    prm.NB = pool.num_blocks;
-    prm.max_ctx = max_context_len;
-    prm.PT = PT;
-    prm.maxP = (int)std::max<long long>(1, ((long long)max_context_len + PT - 1) / PT);
-    prm.pool_rows = pool.num_blocks * pool.num_kv_heads * pool.block_size;
-    prm.scale_log2 = scale * 1.4426950408889634f;
-
-    CUtensorMap mk, mv;
-    if (!encode_pool_map(&mk, k_cache, pool) || !encode_pool_map(&mv, v_cache, pool)) return PKV_ECUDA;
-
-    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    pkv::plan_kernel<<<1, pkv::kPlanThreads, 0, st>>>(prm, D);
-    pkv_status r = launch_status();
-    if (r != PKV_OK) return r;
+    pkv::WriteFp8Params p;
+    p.k = static_cast<const uint4 *>(k);
+    p.v = static_cast<const uint4 *>(v);
+    p.slots = slot_mapping;
+    p.k_scale = k_scale;
+    p.v_scale = v_scale;
+    p.k_cache = static_cast<uint2 *>(k_cache);
+    p.v_cache = static_cast<uint2 *>(v_cache);
+    p.vpr = pool.head_dim / 8;
+    p.num_kv_heads = pool.num_kv_heads;
+    p.block_size = pool.block_size;
+    p.pool_slots = (int64_t)pool.num_blocks * pool.block_size;
+    p.total = (int64_t)num_tokens * 2 * pool.num_kv_heads * p.vpr;
     const int dev = current_device();
-    return D == 128 ? dispatch_group<128>(g, prm, mk, mv, st, dev) : dispatch_group<64>(g, prm, mk, mv, st, dev);
+    const long long blocks = std::min<long long>((p.total + 255) / 256, (long long)sm_count(dev) * 16);
+    pkv::kv_write_fp8_kernel<<<(unsigned)std::max<long long>(blocks, 1), 256, 0, (cudaStream_t)stream>>>(p);
+    return launch_status();
 }
 
 size_t pkv_prefill_workspace_bytes(int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads,

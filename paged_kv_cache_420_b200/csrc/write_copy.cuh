@@ -50,6 +50,68 @@ __global__ void __launch_bounds__(256) kv_write_kernel(WriteParams p) {
     }
 }
 
+// ------------------------------------------------------------ fp8 write ----
+// The same slot-mapped write into an FP8 (e4m3) pool: each 16-byte vector of
+// 8 bf16 elements becomes 8 codes of fp32(x) * fp32(1 / scale[h]) (IEEE
+// round-to-nearest reciprocal and product), converted with round-to-nearest-
+// even and saturation to +-448.
+struct WriteFp8Params {
+    const uint4 *k;        // [T][Hkv][D] bf16 as 16-B vectors
+    const uint4 *v;
+    const int64_t *slots;  // [T]
+    const float *k_scale;  // [Hkv]
+    const float *v_scale;
+    uint2 *k_cache;        // [NB][Hkv][bs][D] e4m3 as 8-B vectors
+    uint2 *v_cache;
+    int64_t total;         // T * 2 * Hkv * vpr
+    int64_t pool_slots;
+    int num_kv_heads;
+    int block_size;
+    int vpr;               // vectors per row = D / 8
+};
+
+// Two fp32 values -> two e4m3 codes; lo lands in the low byte.
+__device__ __forceinline__ uint32_t e4m3x2_from_f32(float lo, float hi) {
+    uint16_t r;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+__global__ void __launch_bounds__(256) kv_write_fp8_kernel(WriteFp8Params p) {
+    const int per_token = 2 * p.num_kv_heads * p.vpr;
+    const int per_kv = p.num_kv_heads * p.vpr;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < p.total;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t t = i / per_token;
+        const int rem = (int)(i - t * per_token);
+        const int is_v = rem >= per_kv;
+        const int j = rem - is_v * per_kv;  // head * vpr + vector
+        const int64_t slot = __ldg(p.slots + t);
+        if (slot < 0) continue;  // padding token
+        if (slot >= p.pool_slots) {
+            if (j == 0 && !is_v) raise_error(PKV_DEVERR_SLOT);
+            continue;
+        }
+        const int64_t block = slot / p.block_size;
+        const int offset = (int)(slot - block * p.block_size);
+        const int h = j / p.vpr;
+        const int c = j - h * p.vpr;
+        const float inv = __frcp_rn(__ldg((is_v ? p.v_scale : p.k_scale) + h));
+        const uint4 val = __ldg((is_v ? p.v : p.k) + t * per_kv + j);
+        const uint32_t w[4] = {val.x, val.y, val.z, val.w};
+        uint32_t code[2];
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            const float x0 = __fmul_rn(bf16lo_to_f32(w[2 * u]), inv), x1 = __fmul_rn(bf16hi_to_f32(w[2 * u]), inv);
+            const float x2 = __fmul_rn(bf16lo_to_f32(w[2 * u + 1]), inv);
+            const float x3 = __fmul_rn(bf16hi_to_f32(w[2 * u + 1]), inv);
+            code[u] = e4m3x2_from_f32(x0, x1) | (e4m3x2_from_f32(x2, x3) << 16);
+        }
+        const int64_t dst = ((block * p.num_kv_heads + h) * p.block_size + offset) * p.vpr + c;
+        (is_v ? p.v_cache : p.k_cache)[dst] = make_uint2(code[0], code[1]);
+    }
+}
+
 // ----------------------------------------------------------------- copy ----
 // Pairs travel by value in the kernel parameters (validated on the host).
 // grid.y = pair, grid.x = chunk of the block; each thread moves kVecPerThread

@@ -167,6 +167,38 @@ def _finish(name, seed, ctx, per_seq_blocks, pre_cow_blocks, copy_pairs, NB,
                     description=description)
 
 
+E4M3_NAN_CODE = 0x7F  # an FP8 (e4m3) NaN code, used to poison unused FP8 pool rows
+
+
+def fp8_pools(w: Workload, seed: Optional[int] = None):
+    """An FP8 (e4m3) pool of the workload's shape: (k_cache8, v_cache8,
+    k_scale, v_scale).  Codes are drawn directly: a random sign, an exponent
+    field uniform in [1, 9] and a random mantissa (magnitudes 2^-6 .. 7.5), so
+    that code * scale spans a few binades; rows that are NaN in the workload's
+    bf16 pool (poison) get the NaN code.  Scales: one per kv head, uniform in
+    [0.05, 0.5], for K and for V.  Nothing here quantizes."""
+    seed = w.seed if seed is None else seed
+    dev = w.k_cache.device
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(int(seed) + 7919)
+    shape = tuple(w.k_cache.shape)
+
+    def codes():
+        sign = torch.randint(0, 2, shape, generator=gen, device=dev, dtype=torch.int32) << 7
+        expo = torch.randint(1, 10, shape, generator=gen, device=dev, dtype=torch.int32) << 3
+        mant = torch.randint(0, 8, shape, generator=gen, device=dev, dtype=torch.int32)
+        return (sign | expo | mant).to(torch.uint8)
+
+    k8, v8 = codes(), codes()
+    for src, dst in ((w.k_cache, k8), (w.v_cache, v8)):
+        dead = src.view(torch.int16) == torch.tensor(BF16_NAN_BITS, dtype=torch.int16, device=dev)
+        dst.masked_fill_(dead, E4M3_NAN_CODE)
+    rng = np.random.default_rng(int(seed) + 104729)
+    k_scale = torch.from_numpy(rng.uniform(0.05, 0.5, w.num_kv_heads).astype(np.float32)).to(dev)
+    v_scale = torch.from_numpy(rng.uniform(0.05, 0.5, w.num_kv_heads).astype(np.float32)).to(dev)
+    return k8, v8, k_scale, v_scale
+
+
 def _pop_tables(ctx, bs, free: list) -> list:
     """Pops each sequence's blocks (logical order) from the end of ``free``."""
     out = []
