@@ -7,7 +7,7 @@
 // 引擎", section 3.1).  An item is (sequence, kv head, tile of 128 query rows),
 // a row being (query token, head of the GQA group).
 //
-// Two CTAs per SM (each holds half of tensor memory and ~97 KB of shared
+// Two CTAs per SM (each holds half of tensor memory and ~113 KB of shared
 // memory), warp-specialised (192 threads):
 //   warp 0       producer: the item's Q tile (128 x D bf16) by a 3-D TMA load,
 //                and 64-key K and V blocks of the paged cache (4 stages of 16
@@ -49,12 +49,17 @@ struct TcItem {
     int s, h, tile, q_len, prefix, q0, n_keys, n_blocks;
 };
 
-// Shared memory of one CTA: NQ query buffers, NK-slot K and V rings.
+// Shared memory of one CTA: NQ query buffers, an NK-slot K ring and an
+// NV-slot V ring (two CTAs share an SM's 228 KB).
+#ifndef PKV_TC_NV128
+#define PKV_TC_NV128 3
+#endif
 template <int D>
 struct TcSmem {
     static constexpr int kHalves = D / 64;
     static constexpr int NQ = D == 128 ? 1 : 2;
     static constexpr int NK = D == 128 ? 2 : 4;
+    static constexpr int NV = D == 128 ? PKV_TC_NV128 : 4;
     static constexpr int kQHalf = kTcRows * 128;          // 16 KB: 128 rows x 64 columns
     static constexpr int kQBuf = kHalves * kQHalf;
     static constexpr int kKVHalf = kTcKeys * 128;         // 8 KB: 64 keys x 64 columns
@@ -62,10 +67,10 @@ struct TcSmem {
     static constexpr int oQ = 0;
     static constexpr int oK = NQ * kQBuf;
     static constexpr int oV = oK + NK * kSlot;
-    static constexpr int oBars = oV + NK * kSlot;
-    // kfull, kempty, vfull, vempty [NK]; qfull, qempty [NQ]; sfull, sfree,
-    // pfull[2], odone, drain
-    static constexpr int kNumBars = 4 * NK + 2 * NQ + 6;
+    static constexpr int oBars = oV + NV * kSlot;
+    // kfull, kempty [NK]; vfull, vempty [NV]; qfull, qempty [NQ]; sfull,
+    // sfree, pfull[2], odone, drain
+    static constexpr int kNumBars = 2 * NK + 2 * NV + 2 * NQ + 6;
     static constexpr int oItem = oBars + kNumBars * 8;
     static constexpr int oTmemSlot = oItem + NQ * (int)sizeof(TcItem);
     static constexpr int oAbort = oTmemSlot + 16;
@@ -263,7 +268,7 @@ __global__ void __launch_bounds__(kTcThreads, kTcCtasPerSm)
     paged_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v,
                             const __grid_constant__ CUtensorMap tmap_q, const PrefillParams p) {
     using L = TcSmem<D>;
-    constexpr int NQ = L::NQ, NK = L::NK;
+    constexpr int NQ = L::NQ, NK = L::NK, NV = L::NV;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     if ((smem_u32(smem_raw) & 1023u) != 0) {
         if (threadIdx.x == 0) raise_error(PKV_DEVERR_LAYOUT);
@@ -271,8 +276,8 @@ __global__ void __launch_bounds__(kTcThreads, kTcCtasPerSm)
     }
     uint8_t *smem = smem_raw;
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L::oBars);
-    uint64_t *kfull = bars, *kempty = bars + NK, *vfull = bars + 2 * NK, *vempty = bars + 3 * NK;
-    uint64_t *qfull = bars + 4 * NK, *qempty = qfull + NQ;
+    uint64_t *kfull = bars, *kempty = bars + NK, *vfull = bars + 2 * NK, *vempty = bars + 2 * NK + NV;
+    uint64_t *qfull = bars + 2 * NK + 2 * NV, *qempty = qfull + NQ;
     uint64_t *sfull = qempty + NQ, *sfree = sfull + 1, *pfull = sfree + 1, *odone = pfull + 2, *drain = odone + 1;
     TcItem *items = reinterpret_cast<TcItem *>(smem + L::oItem);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::oTmemSlot);
@@ -284,6 +289,8 @@ __global__ void __launch_bounds__(kTcThreads, kTcCtasPerSm)
         for (int i = 0; i < NK; ++i) {
             mbar_init(&kfull[i], 1);
             mbar_init(&kempty[i], 1);
+        }
+        for (int i = 0; i < NV; ++i) {
             mbar_init(&vfull[i], 1);
             mbar_init(&vempty[i], 1);
         }
@@ -368,10 +375,11 @@ __global__ void __launch_bounds__(kTcThreads, kTcCtasPerSm)
 #pragma unroll
                 for (int kv = 0; kv < 2 && ok; ++kv) {
                     const uint32_t g = kv ? gv : gk;
-                    const uint32_t slot = g % NK;
+                    const uint32_t depth = kv ? NV : NK;
+                    const uint32_t slot = g % depth;
                     uint64_t *fb = kv ? &vfull[slot] : &kfull[slot];
                     if (lane == 0) {
-                        ok = wait_or_abort(kv ? &vempty[slot] : &kempty[slot], ((g / NK) & 1) ^ 1, abort_flag);
+                        ok = wait_or_abort(kv ? &vempty[slot] : &kempty[slot], ((g / depth) & 1) ^ 1, abort_flag);
                         if (ok) mbar_arrive_expect_tx(fb, (uint32_t)L::kSlot);
                     }
                     ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -393,8 +401,8 @@ __global__ void __launch_bounds__(kTcThreads, kTcCtasPerSm)
         if (lane == 0 && *abort_flag) {
             for (uint32_t c = (gk > (uint32_t)NK ? gk - NK : 0); c < gk; ++c)
                 mbar_wait_bounded(&kfull[c % NK], (c / NK) & 1, kWaitLimitNs);
-            for (uint32_t c = (gv > (uint32_t)NK ? gv - NK : 0); c < gv; ++c)
-                mbar_wait_bounded(&vfull[c % NK], (c / NK) & 1, kWaitLimitNs);
+            for (uint32_t c = (gv > (uint32_t)NV ? gv - NV : 0); c < gv; ++c)
+                mbar_wait_bounded(&vfull[c % NV], (c / NV) & 1, kWaitLimitNs);
             if (q_issued >= 0) mbar_wait_bounded(&qfull[q_issued % NQ], ((q_issued / NQ) & 1), kWaitLimitNs);
         }
     } else if (warp == 1) {
@@ -437,8 +445,8 @@ __global__ void __launch_bounds__(kTcThreads, kTcCtasPerSm)
                     // O += P_{j-1} V_{j-1}
                     const uint32_t pg = gb - 1;
                     const uint32_t pb = pg & 1;
-                    const uint32_t slot = pg % NK;
-                    ok = wait_or_abort(&vfull[slot], (pg / NK) & 1, abort_flag) &&
+                    const uint32_t slot = pg % NV;
+                    ok = wait_or_abort(&vfull[slot], (pg / NV) & 1, abort_flag) &&
                          wait_or_abort(&pfull[pb], (pg >> 1) & 1, abort_flag);
                     if (ok) {
                         tc_fence_after();
@@ -559,8 +567,8 @@ __global__ void __launch_bounds__(kTcThreads, kTcCtasPerSm)
                 // (once the block has landed) so stale, possibly NaN, data
                 // cannot reach the MMA (P is 0 there)
                 if (ok && j == t.n_blocks - 1 && (t.n_keys % kStageTok) != 0) {
-                    const uint32_t slot = gb % NK;
-                    ok = __all_sync(0xffffffffu, wait_or_abort(&vfull[slot], (gb / NK) & 1, abort_flag));
+                    const uint32_t slot = gb % NV;
+                    ok = __all_sync(0xffffffffu, wait_or_abort(&vfull[slot], (gb / NV) & 1, abort_flag));
                     const int first = t.n_keys - kbase;  // first invalid key of the block
                     const int last = (first / kStageTok + 1) * kStageTok;
                     uint8_t *vrow0 = smem + L::oV + slot * L::kSlot;
