@@ -64,13 +64,20 @@ def _load() -> ctypes.CDLL:
         lib.oracle_e4m3_encode_array.argtypes = [P, I, P]
         lib.oracle_kv_write_fp8.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I]
         lib.oracle_paged_attention_fp8.argtypes = [P, P, P, P, P, P, I, P, I, I, I, I, I, I, D, P]
+        lib.oracle_bm_drop_hashes.argtypes = [P, P, I]
+        lib.oracle_fnv1a64.argtypes = [P, I]
+        lib.oracle_fnv1a64.restype = ctypes.c_uint64
+        lib.oracle_prefix_keys.argtypes = [P, I, I, P]
+        lib.oracle_prefix_lookup.argtypes = [P, P, I, P, P, I, P, P, I, I, P, I, P]
+        lib.oracle_prefix_insert.argtypes = [P, P, I, P, P, I, P, P, I, I, P, I, P]
         lib.oracle_num_threads.argtypes = []
         for f in (lib.oracle_kv_write, lib.oracle_copy_blocks, lib.oracle_paged_attention,
                   lib.oracle_attention_partial, lib.oracle_lse_merge, lib.oracle_num_threads,
                   lib.oracle_paged_prefill, lib.oracle_swap_out, lib.oracle_swap_in, lib.oracle_lru_victims,
                   lib.oracle_bm_init, lib.oracle_bm_alloc, lib.oracle_bm_free, lib.oracle_bm_share,
                   lib.oracle_bm_append_slots, lib.oracle_e4m3_encode_array, lib.oracle_kv_write_fp8,
-                  lib.oracle_paged_attention_fp8):
+                  lib.oracle_paged_attention_fp8, lib.oracle_bm_drop_hashes, lib.oracle_prefix_keys,
+                  lib.oracle_prefix_lookup, lib.oracle_prefix_insert):
             f.restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -196,13 +203,16 @@ class BlockState:
     """free_stack[:top] are the free ids (the next allocation pops
     free_stack[top - 1]); refcount[b] counts the sequences mapping block b."""
 
-    def __init__(self, free_stack, top, refcount):
+    def __init__(self, free_stack, top, refcount, block_hash=None):
         self.free_stack = np.ascontiguousarray(free_stack, dtype=np.int32)
         self.top = int(top)
         self.refcount = np.ascontiguousarray(refcount, dtype=np.int32)
+        n = self.refcount.shape[0]
+        self.block_hash = (np.zeros(n, np.uint64) if block_hash is None
+                           else np.ascontiguousarray(block_hash, dtype=np.uint64))
 
     def copy(self):
-        return BlockState(self.free_stack.copy(), self.top, self.refcount.copy())
+        return BlockState(self.free_stack.copy(), self.top, self.refcount.copy(), self.block_hash.copy())
 
     @property
     def num_blocks(self):
@@ -242,6 +252,7 @@ def bm_free(st: BlockState, ids):
     a = np.ascontiguousarray(ids, dtype=np.int32).reshape(-1)
     err = np.zeros(1, dtype=np.uint32)
     _check(_bm_call(_load().oracle_bm_free, st, _ptr(a), a.shape[0], _ptr(err)), "bm_free")
+    _load().oracle_bm_drop_hashes(_ptr(st.refcount), _ptr(st.block_hash), st.num_blocks)
     return st, int(err[0])
 
 
@@ -324,6 +335,65 @@ def paged_attention_fp8(q, k_cache8, v_cache8, k_scale, v_scale, block_tables, c
                                             float(np.float64(np.float32(scale))), _ptr(out))
     _check(rc, "paged_attention_fp8")
     return out
+
+
+# ---------------------------------------------------------------------------
+# prefix caching
+# ---------------------------------------------------------------------------
+
+def fnv1a64(data: bytes) -> int:
+    buf = np.frombuffer(bytes(data), dtype=np.uint8).copy() if len(data) else np.zeros(1, np.uint8)
+    return int(_load().oracle_fnv1a64(_ptr(buf), len(data)))
+
+
+def prefix_keys(tokens, block_size: int) -> np.ndarray:
+    """Chained keys of the full blocks of one prompt."""
+    t = np.ascontiguousarray(tokens, dtype=np.int32).reshape(-1)
+    keys = np.zeros(max(t.shape[0] // block_size, 1), dtype=np.uint64)
+    _load().oracle_prefix_keys(_ptr(t), t.shape[0], int(block_size), _ptr(keys))
+    return keys[:t.shape[0] // block_size]
+
+
+class PrefixCache:
+    """cap (key, block) pairs; key 0 = empty."""
+
+    def __init__(self, cap: int):
+        self.keys = np.zeros(cap, np.uint64)
+        self.vals = np.full(cap, -1, np.int32)
+
+    def copy(self):
+        c = PrefixCache(self.keys.shape[0])
+        c.keys, c.vals = self.keys.copy(), self.vals.copy()
+        return c
+
+
+def prefix_lookup(st: BlockState, cache: PrefixCache, tokens, query_start, block_size: int, block_tables):
+    """Returns (new state, tables, num_cached tokens per sequence)."""
+    st = st.copy()
+    t = np.ascontiguousarray(tokens, dtype=np.int32).reshape(-1)
+    qs = np.ascontiguousarray(query_start, dtype=np.int32)
+    tables = np.ascontiguousarray(block_tables, dtype=np.int32).copy()
+    B, mbs = tables.shape
+    nc = np.zeros(max(B, 1), np.int32)
+    _check(_load().oracle_prefix_lookup(_ptr(st.refcount), _ptr(st.block_hash), st.num_blocks, _ptr(cache.keys),
+                                        _ptr(cache.vals), cache.keys.shape[0], _ptr(t), _ptr(qs), B,
+                                        int(block_size), _ptr(tables), mbs, _ptr(nc)), "prefix_lookup")
+    return st, tables, nc[:B]
+
+
+def prefix_insert(st: BlockState, cache: PrefixCache, tokens, query_start, block_size: int, block_tables):
+    """Returns (new state, new cache, err)."""
+    st = st.copy()
+    cache = cache.copy()
+    t = np.ascontiguousarray(tokens, dtype=np.int32).reshape(-1)
+    qs = np.ascontiguousarray(query_start, dtype=np.int32)
+    tables = np.ascontiguousarray(block_tables, dtype=np.int32)
+    B, mbs = tables.shape
+    err = np.zeros(1, np.uint32)
+    _check(_load().oracle_prefix_insert(_ptr(st.refcount), _ptr(st.block_hash), st.num_blocks, _ptr(cache.keys),
+                                        _ptr(cache.vals), cache.keys.shape[0], _ptr(t), _ptr(qs), B,
+                                        int(block_size), _ptr(tables), mbs, _ptr(err)), "prefix_insert")
+    return st, cache, int(err[0])
 
 
 def paged_attention(q, k_cache, v_cache, block_tables, context_lens, scale: float) -> np.ndarray:

@@ -22,6 +22,11 @@
  *     sharer writes into them (wkbse.com section 3.1, "flexible memory
  *     management" and "KV cache sharing"; intelliparadigm.com section 2.1,
  *     items 1-2 and the block-allocation sketch).
+ *   - prefix caching (intelliparadigm.com section 3.1, --enable-prefix-caching:
+ *     prompt sharing; section 2.1's allocation sketch: a block whose prefix
+ *     matches is shared instead of allocated): full prompt blocks are keyed
+ *     by a chained FNV-1a 64-bit hash of their tokens and the key of the
+ *     block before, and looked up before allocation.
  *   - an FP8 KV cache (ai-stack.site "Nano-vLLM 原理", case study: FP8 mixed
  *     precision): the pool holds OCP E4M3 codes with a static scale per kv
  *     head for K and for V; a value is stored as the code nearest to
@@ -434,6 +439,14 @@ int oracle_bm_free(int32_t *free_stack, int32_t *top, int32_t *refcount, int num
     return 0;
 }
 
+/* A freed block's content no longer backs a prefix: its cached key is dropped
+ * when its count reaches zero (call after oracle_bm_free on the same list). */
+int oracle_bm_drop_hashes(const int32_t *refcount, uint64_t *block_hash, int num_blocks) {
+    for (int b = 0; b < num_blocks; ++b)
+        if (refcount[b] == 0) block_hash[b] = 0;
+    return 0;
+}
+
 /* Each listed id gains one reference (a new sequence maps the block). */
 int oracle_bm_share(int32_t *refcount, int num_blocks, const int32_t *ids, int n, uint32_t *err) {
     if (num_blocks <= 0 || n < 0) return 1;
@@ -628,4 +641,125 @@ int oracle_paged_attention_fp8(const uint16_t *q, const uint8_t *k_cache, const 
         }
     }
     return status;
+}
+
+/* ------------------------------------------------------------------------
+ * Prefix caching.  FNV-1a 64-bit (Fowler-Noll-Vo, "1a" order: xor the byte,
+ * then multiply): offset basis 14695981039346656037, prime 1099511628211.
+ * Block i of a prompt has digest d_i = FNV-1a over its bs tokens as
+ * little-endian int32 bytes and key k_i = FNV-1a over the 16 bytes
+ * le64(k_{i-1}) || le64(d_i) (k_{-1} = 0); a key of 0 is stored as 1 (0 marks
+ * an empty slot).  The cache maps keys to blocks; a mapping counts only while
+ * the block still holds that key (block_hash[b] == key) and is mapped by some
+ * sequence (refcount > 0).
+ * ------------------------------------------------------------------------ */
+static uint64_t fnv1a(uint64_t h, const uint8_t *p, size_t n) {
+    for (size_t i = 0; i < n; ++i) {
+        h ^= p[i];
+        h *= 1099511628211ull;
+    }
+    return h;
+}
+
+static uint64_t block_key(uint64_t prev, const int32_t *tokens, int bs) {
+    uint64_t d = 14695981039346656037ull;
+    for (int t = 0; t < bs; ++t) {
+        uint8_t b[4] = {(uint8_t)tokens[t], (uint8_t)(tokens[t] >> 8), (uint8_t)(tokens[t] >> 16),
+                        (uint8_t)(tokens[t] >> 24)};
+        d = fnv1a(d, b, 4);
+    }
+    uint8_t buf[16];
+    for (int i = 0; i < 8; ++i) {
+        buf[i] = (uint8_t)(prev >> (8 * i));
+        buf[8 + i] = (uint8_t)(d >> (8 * i));
+    }
+    uint64_t k = fnv1a(14695981039346656037ull, buf, 16);
+    return k ? k : 1;
+}
+
+uint64_t oracle_fnv1a64(const uint8_t *bytes, int n) { return fnv1a(14695981039346656037ull, bytes, (size_t)n); }
+
+int oracle_prefix_keys(const int32_t *tokens, int n_tokens, int bs, uint64_t *keys) {
+    uint64_t prev = 0;
+    for (int i = 0; i < n_tokens / bs; ++i) {
+        prev = block_key(prev, tokens + (size_t)i * bs, bs);
+        keys[i] = prev;
+    }
+    return 0;
+}
+
+/* The cache itself: parallel arrays of cap (key, block) pairs, cap a power of
+ * two; the oracle searches it linearly (a plain map, no probing). */
+static int cache_find(const uint64_t *keys, const int32_t *vals, int cap, uint64_t key) {
+    for (int i = 0; i < cap; ++i)
+        if (keys[i] == key) return vals[i];
+    return -1;
+}
+
+static int valid_holder(int32_t b, uint64_t key, const uint64_t *block_hash, const int32_t *refcount, int nb) {
+    return b >= 0 && b < nb && block_hash[b] == key && refcount[b] > 0;
+}
+
+/* Lookup, in sequence order: the longest run of leading full prompt blocks of
+ * sequence s whose keys have a valid holder -- leaving at least one prompt
+ * token uncached -- is mapped into its table row (one reference each);
+ * num_cached[s] = the tokens covered. */
+int oracle_prefix_lookup(int32_t *refcount, const uint64_t *block_hash, int num_blocks, const uint64_t *ckeys,
+                         const int32_t *cvals, int cap, const int32_t *tokens, const int32_t *query_start, int B,
+                         int bs, int32_t *block_tables, int mbs, int32_t *num_cached) {
+    if (num_blocks <= 0 || B < 0 || bs <= 0 || mbs <= 0) return 1;
+    for (int s = 0; s < B; ++s) {
+        int n = query_start[s + 1] - query_start[s];
+        int look = n > 0 ? (n - 1) / bs : 0;
+        if (look > mbs) look = mbs;
+        uint64_t prev = 0;
+        int hits = 0;
+        for (int i = 0; i < look; ++i) {
+            uint64_t key = block_key(prev, tokens + query_start[s] + (size_t)i * bs, bs);
+            prev = key;
+            int32_t b = cache_find(ckeys, cvals, cap, key);
+            if (!valid_holder(b, key, block_hash, refcount, num_blocks)) break;
+            block_tables[(size_t)s * mbs + i] = b;
+            refcount[b] += 1;
+            ++hits;
+        }
+        num_cached[s] = hits * bs;
+    }
+    return 0;
+}
+
+/* Insert, in sequence order, after the prompt's blocks hold its K/V: every full
+ * prompt block i of sequence s (block id table[s][i]) whose key has no valid
+ * holder becomes its holder (the first sequence in order wins); a block that
+ * already holds its key is left as it is. */
+int oracle_prefix_insert(const int32_t *refcount, uint64_t *block_hash, int num_blocks, uint64_t *ckeys,
+                         int32_t *cvals, int cap, const int32_t *tokens, const int32_t *query_start, int B, int bs,
+                         const int32_t *block_tables, int mbs, uint32_t *err) {
+    if (num_blocks <= 0 || B < 0 || bs <= 0 || mbs <= 0) return 1;
+    for (int s = 0; s < B; ++s) {
+        int n = query_start[s + 1] - query_start[s];
+        int full = n / bs;
+        if (full > mbs) full = mbs;
+        uint64_t prev = 0;
+        for (int i = 0; i < full; ++i) {
+            uint64_t key = block_key(prev, tokens + query_start[s] + (size_t)i * bs, bs);
+            prev = key;
+            int32_t b = block_tables[(size_t)s * mbs + i];
+            if (b < 0 || b >= num_blocks) { *err |= BM_ERR_RANGE; break; }
+            if (block_hash[b] == key) continue;
+            int slot = -1;
+            for (int j = 0; j < cap; ++j)
+                if (ckeys[j] == key) { slot = j; break; }
+            if (slot >= 0 && valid_holder(cvals[slot], key, block_hash, refcount, num_blocks)) continue;
+            if (slot < 0) {
+                for (int j = 0; j < cap; ++j)
+                    if (ckeys[j] == 0) { slot = j; break; }
+                if (slot < 0) { *err |= BM_ERR_NOSPACE; continue; }
+                ckeys[slot] = key;
+            }
+            cvals[slot] = b;
+            block_hash[b] = key;
+        }
+    }
+    return 0;
 }

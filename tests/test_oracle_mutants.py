@@ -17,6 +17,7 @@ from tests import test_oracle_pins as pins
 from tests import test_oracle_prefill as prefill_pins
 from tests import test_oracle_block_manager as bm_pins
 from tests import test_oracle_fp8 as fp8_pins
+from tests import test_oracle_prefix as prefix_pins
 from tests import test_oracle_swap as swap_pins
 
 PIN_TESTS = [
@@ -40,6 +41,11 @@ PIN_TESTS = [
     swap_pins.test_swap_of_a_permutation_is_a_gather,
     swap_pins.test_lru_worked_example_golden,
     bm_pins.test_block_manager_worked_example_golden,
+    prefix_pins.test_fnv1a64_published_vectors,
+    prefix_pins.test_keys_chain_over_the_prefix,
+    prefix_pins.test_worked_example,
+    prefix_pins.test_freed_holder_no_longer_matches,
+    prefix_pins.test_first_sequence_in_order_becomes_holder,
     fp8_pins.test_decode_table_matches_library,
     fp8_pins.test_encode_golden,
     fp8_pins.test_write_quantizes_into_the_bf16_layout,
@@ -90,6 +96,15 @@ MUTANTS = {
                           "--refcount[b]; free_stack[(*top)++] = b;"),
     "fifo free list": ("int32_t b = free_stack[--*top];",
                        "int32_t b = free_stack[0]; memmove(free_stack, free_stack + 1, sizeof(int32_t) * (size_t)(--*top));"),
+    # prefix cache: keys without the chain; a holder's validity ignored; the
+    # last inserter wins; the whole prompt looked up; FNV's multiply first
+    "prefix key unchained": ("buf[i] = (uint8_t)(prev >> (8 * i));", "buf[i] = 0;"),
+    "prefix holder unchecked": ("if (!valid_holder(b, key, block_hash, refcount, num_blocks)) break;",
+                                "if (b < 0) break;"),
+    "prefix last inserter wins": ("if (slot >= 0 && valid_holder(cvals[slot], key, block_hash, refcount, num_blocks)) continue;",
+                                  "if (0) continue;"),
+    "prefix whole prompt": ("int look = n > 0 ? (n - 1) / bs : 0;", "int look = n / bs;"),
+    "fnv multiply first": ("h ^= p[i];\n        h *= 1099511628211ull;", "h *= 1099511628211ull;\n        h ^= p[i];"),
     # fp8: subnormals one binade off; ties to the odd code; the scale multiplied
     # instead of divided on the way in; the key scale applied to the values
     "e4m3 subnormal exponent": ("if (e == 0) v = ldexp((double)m / 8.0, -6);", "if (e == 0) v = ldexp((double)m / 8.0, -7);"),
