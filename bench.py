@@ -638,6 +638,33 @@ def run_blockmgr_cuda(args, rank, world, dist):
         b.record(stream)
         torch.cuda.synchronize()
         pre.append(a.elapsed_time(b) * 1e3)
+    # prefix cache: 128 prompts of 512 tokens sharing a 256-token system prompt
+    rng = np.random.default_rng(args.seed)
+    system = rng.integers(0, 32000, 256)
+    prompts = [np.concatenate([system, rng.integers(0, 32000, 256)]).astype(np.int32) for _ in range(B)]
+    toks = torch.from_numpy(np.concatenate(prompts)).to(dev)
+    qs = torch.from_numpy(np.arange(B + 1, dtype=np.int32) * 512).to(dev)
+    pmbs = 512 // bs + 1
+    bm3 = pkv.BlockManager(B * pmbs + 64, device=dev)
+    pc = pkv.PrefixCache(1 << 16, device=dev)
+    t3 = torch.full((B, pmbs), -1, dtype=torch.int32, device=dev)
+    c3 = torch.zeros(B, dtype=torch.int32, device=dev)
+    bm3.append_slots(t3, c3, torch.full((B,), 512, dtype=torch.int32, device=dev), bs, B * 512)
+    pc.insert(bm3, toks, qs, bs, t3)  # the first batch fills the cache
+    lk, ins = [], []
+    for _ in range(5):
+        tl = torch.full((B, pmbs), -1, dtype=torch.int32, device=dev)
+        a, b, c = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+        a.record(stream)
+        cached = pc.lookup(bm3, toks, qs, bs, tl)
+        b.record(stream)
+        pc.insert(bm3, toks, qs, bs, t3)
+        c.record(stream)
+        torch.cuda.synchronize()
+        lk.append(a.elapsed_time(b) * 1e3)
+        ins.append(b.elapsed_time(c) * 1e3)
+        bm3.free(tl[tl >= 0].contiguous())  # drop the lookup's references again
+    prefix_hit_tokens = int(cached.sum().item())
     # floor: an empty kernel, launch to completion
     nop = torch.empty(1, device=dev)
     g2 = torch.cuda.CUDAGraph()
@@ -677,7 +704,10 @@ def run_blockmgr_cuda(args, rank, world, dist):
                      "peak": round(floor_us, 2),
                      "peak_kind": "measured: one-thread kernel per graph node, back to back (launch floor)",
                      "unit": "us", "frac": round(floor_us / per_call_us, 4),
-                     "prefill_8x512_us": round(float(np.median(pre)), 2), "traffic": None},
+                     "prefill_8x512_us": round(float(np.median(pre)), 2),
+                     "prefix_lookup_128x512_us": round(float(np.median(lk)), 2),
+                     "prefix_insert_128x512_us": round(float(np.median(ins)), 2),
+                     "prefix_hit_tokens": prefix_hit_tokens, "traffic": None},
         "cpu_baseline": {"value": round(cpu_us, 2), "unit": "us", "cores": 1, "kind": "oracle",
                          "sample": f"{n_cpu} sequential append steps of the same batch"},
         "e2e": None, "gpu_launches": steps, "clocks": clocks.summary(),

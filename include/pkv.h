@@ -317,6 +317,8 @@ pkv_status paged_attn_decode_fp8(const void *q, const void *k_cache, const void 
  *                      the next allocation pops free_stack[top - 1])
  *   at 256 + A:        int32 refcount[num_blocks]     (sequences mapping each block)
  *   at 256 + 2A..4A:   three int32 scratch arrays kept at their rest values
+ *   at 256 + 5A:       uint64 block_hash[num_blocks]  (the prefix-cache key a block
+ *                      holds, 0: none; cleared when its count reaches zero)
  * with A = num_blocks * 4 rounded up to 256.  Every call is one kernel on
  * `stream` (one CTA walking its list in order with block-wide scans), so its
  * results are exactly the sequential, request-order ones; device-side
@@ -363,6 +365,40 @@ pkv_status pkv_bm_append_slots(void *state, int32_t num_blocks, int32_t *block_t
                                int32_t *context_lens, const int32_t *num_new, int32_t num_seqs, int32_t block_size,
                                int64_t *slot_mapping, int64_t slot_capacity, int32_t *cow_pairs,
                                int32_t *num_cow_pairs, pkv_stream_t stream);
+/*
+ * Prefix caching (intelliparadigm.com section 3.1, --enable-prefix-caching:
+ * prompt sharing; section 2.1's allocation sketch shares an existing block
+ * whose prefix matches instead of allocating one).  Full prompt blocks are
+ * keyed by FNV-1a 64 (offset basis 14695981039346656037, prime
+ * 1099511628211, per byte xor then multiply) chained over the prefix:
+ * d_i = FNV-1a of the block's block_size tokens as little-endian int32 bytes,
+ * key_i = FNV-1a of le64(key_{i-1}) || le64(d_i), key_{-1} = 0, a key of 0
+ * stored as 1.  The cache is a caller-owned device buffer of
+ * pkv_prefix_cache_bytes(capacity) (capacity a power of two, 256-B aligned):
+ * an open-addressing table of (key, block) pairs.  An entry counts while its
+ * block still holds the key (block_hash) and is mapped (refcount > 0).
+ * tokens: int32 prompts concatenated, query_start: int32 [num_seqs + 1].
+ *
+ * pkv_prefix_lookup: for each sequence, the longest run of leading full
+ *   prompt blocks with a valid holder -- leaving at least one prompt token to
+ *   compute -- is written into its block-table row (int32 [num_seqs]
+ *   [max_blocks_per_seq]) with one reference each; num_cached[s] (int32
+ *   [num_seqs]) = the tokens covered.  Then pkv_bm_append_slots with
+ *   context_lens = num_cached and num_new = prompt length - num_cached.
+ * pkv_prefix_insert: after the prompt's K/V is written, in sequence order,
+ *   every full prompt block whose key has no valid holder becomes its holder
+ *   (the first sequence in order wins); a full table sets PKV_BM_ERR_NOSPACE.
+ */
+size_t pkv_prefix_cache_bytes(int32_t capacity);
+pkv_status pkv_prefix_cache_init(void *cache, int32_t capacity, pkv_stream_t stream);
+pkv_status pkv_prefix_lookup(void *state, int32_t num_blocks, void *cache, int32_t capacity, const int32_t *tokens,
+                             const int32_t *query_start, int32_t num_seqs, int32_t block_size,
+                             int32_t *block_tables, int32_t max_blocks_per_seq, int32_t *num_cached,
+                             pkv_stream_t stream);
+pkv_status pkv_prefix_insert(void *state, int32_t num_blocks, void *cache, int32_t capacity, const int32_t *tokens,
+                             const int32_t *query_start, int32_t num_seqs, int32_t block_size,
+                             const int32_t *block_tables, int32_t max_blocks_per_seq, pkv_stream_t stream);
+
 /*
  * pkv_copy_blocks sourced from the device: copies the first *num_pairs of
  * cow_pairs (device int32 [max_pairs][2], as pkv_bm_append_slots leaves them)

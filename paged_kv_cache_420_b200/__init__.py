@@ -28,7 +28,8 @@ EXPORTED = ("pkv_write", "pkv_copy_blocks", "pkv_decode_workspace_bytes", "paged
             "pkv_get_device_error", "pkv_selftest_bounded_wait", "pkv_status_string", "pkv_version",
             "pkv_swap_out", "pkv_swap_in", "pkv_lru_victims", "pkv_bm_state_bytes", "pkv_bm_init", "pkv_bm_alloc",
             "pkv_bm_free", "pkv_bm_share", "pkv_bm_append_slots", "pkv_copy_blocks_dev", "pkv_write_fp8",
-            "paged_attn_decode_fp8")
+            "paged_attn_decode_fp8", "pkv_prefix_cache_bytes", "pkv_prefix_cache_init", "pkv_prefix_lookup",
+            "pkv_prefix_insert")
 STATIC_WS_BYTES = 32 << 20  # PKV_STATIC_WS_BYTES
 
 
@@ -72,6 +73,11 @@ def load_library() -> ctypes.CDLL:
         lib.pkv_bm_append_slots.argtypes = [P, I32, P, I32, P, P, I32, I32, P, I64, P, P, P]
         lib.pkv_copy_blocks_dev.argtypes = [P, P, I32, P, P, _Pool, P]
         lib.pkv_write_fp8.argtypes = [P, P, P, I32, P, P, P, P, _Pool, P]
+        lib.pkv_prefix_cache_bytes.argtypes = [I32]
+        lib.pkv_prefix_cache_bytes.restype = SZ
+        lib.pkv_prefix_cache_init.argtypes = [P, I32, P]
+        lib.pkv_prefix_lookup.argtypes = [P, I32, P, I32, P, P, I32, I32, P, I32, P, P]
+        lib.pkv_prefix_insert.argtypes = [P, I32, P, I32, P, P, I32, I32, P, I32, P]
         lib.paged_attn_decode_fp8.argtypes = [P, P, P, P, P, P, I32, P, I32, I32, F, I32, P, _Pool, I32, I32, P, SZ,
                                               P]
         lib.pkv_status_string.argtypes = [ctypes.c_int]
@@ -79,7 +85,8 @@ def load_library() -> ctypes.CDLL:
         lib.pkv_version.restype = I32
         for f in ("pkv_write", "pkv_copy_blocks", "paged_attn_decode", "pkv_get_device_error", "pkv_swap_out",
                   "pkv_swap_in", "pkv_lru_victims", "pkv_bm_init", "pkv_bm_alloc", "pkv_bm_free", "pkv_bm_share",
-                  "pkv_bm_append_slots", "pkv_copy_blocks_dev", "pkv_write_fp8", "paged_attn_decode_fp8"):
+                  "pkv_bm_append_slots", "pkv_copy_blocks_dev", "pkv_write_fp8", "paged_attn_decode_fp8",
+                  "pkv_prefix_cache_init", "pkv_prefix_lookup", "pkv_prefix_insert"):
             getattr(lib, f).restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -225,6 +232,7 @@ class BlockManager:
         self.header = self.state[:8].view(torch.int32)  # top, error word
         self.free_stack = self.state[256:256 + 4 * self.num_blocks].view(torch.int32)
         self.refcount = self.state[256 + a:256 + a + 4 * self.num_blocks].view(torch.int32)
+        self.block_hash = self.state[256 + 5 * a:256 + 5 * a + 8 * self.num_blocks].view(torch.int64)
         _check(load_library().pkv_bm_init(_ptr(self.state), self.num_blocks, _stream(stream)), "pkv_bm_init")
 
     def top(self) -> int:
@@ -282,6 +290,41 @@ class BlockManager:
                                                   int(num_tokens), _ptr(pairs), _ptr(npairs), _stream(stream)),
                "pkv_bm_append_slots")
         return slots[:int(num_tokens)], pairs, npairs
+
+
+class PrefixCache:
+    """Device table of (prefix key, block) pairs for prefix caching."""
+
+    def __init__(self, capacity: int, device="cuda", stream=None):
+        n = load_library().pkv_prefix_cache_bytes(int(capacity))
+        if n == 0:
+            raise ValueError("capacity must be a power of two >= 2")
+        self.capacity = int(capacity)
+        self.buf = torch.empty(n, dtype=torch.uint8, device=device)
+        _check(load_library().pkv_prefix_cache_init(_ptr(self.buf), self.capacity, _stream(stream)),
+               "pkv_prefix_cache_init")
+
+    def lookup(self, bm: "BlockManager", tokens: torch.Tensor, query_start: torch.Tensor, block_size: int,
+               block_tables: torch.Tensor, stream=None) -> torch.Tensor:
+        """Maps cached leading blocks into block_tables; returns num_cached [B] (tokens)."""
+        for t, n in ((tokens, "tokens"), (query_start, "query_start"), (block_tables, "block_tables")):
+            _need(t, n, torch.int32)
+        B, mbs = block_tables.shape
+        num_cached = torch.empty(max(B, 1), dtype=torch.int32, device=self.buf.device)
+        _check(load_library().pkv_prefix_lookup(_ptr(bm.state), bm.num_blocks, _ptr(self.buf), self.capacity,
+                                                _ptr(tokens), _ptr(query_start), B, int(block_size),
+                                                _ptr(block_tables), mbs, _ptr(num_cached), _stream(stream)),
+               "pkv_prefix_lookup")
+        return num_cached[:B]
+
+    def insert(self, bm: "BlockManager", tokens: torch.Tensor, query_start: torch.Tensor, block_size: int,
+               block_tables: torch.Tensor, stream=None) -> None:
+        for t, n in ((tokens, "tokens"), (query_start, "query_start"), (block_tables, "block_tables")):
+            _need(t, n, torch.int32)
+        B, mbs = block_tables.shape
+        _check(load_library().pkv_prefix_insert(_ptr(bm.state), bm.num_blocks, _ptr(self.buf), self.capacity,
+                                                _ptr(tokens), _ptr(query_start), B, int(block_size),
+                                                _ptr(block_tables), mbs, _stream(stream)), "pkv_prefix_insert")
 
 
 def copy_blocks_dev(cow_pairs: torch.Tensor, num_pairs: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,

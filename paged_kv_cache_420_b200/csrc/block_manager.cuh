@@ -37,6 +37,7 @@ struct BmState {
     int32_t *last_idx;    // [NB] scratch: last list position of a block in a free batch (rest: -1)
     int32_t *zeroed;      // [NB] scratch: its count reached zero in this batch (rest: 0)
     int32_t *cow_rank;    // [NB] scratch: copy-on-write candidates seen so far in a chunk (rest: 0)
+    uint64_t *block_hash; // [NB] prefix-cache key the block holds (0: none)
 };
 
 __device__ __forceinline__ void bm_error(const BmState &s, uint32_t bits) {
@@ -82,6 +83,7 @@ __global__ void __launch_bounds__(256) bm_init_kernel(BmState s, int nb) {
         s.last_idx[i] = -1;
         s.zeroed[i] = 0;
         s.cow_rank[i] = 0;
+        s.block_hash[i] = 0;
     }
     if (blockIdx.x == 0 && threadIdx.x == 0) {
         s.hdr[0] = nb;
@@ -165,6 +167,7 @@ __global__ void __launch_bounds__(kBmThreads) bm_free_kernel(BmState s, int nb, 
             bm_error(s, kBmErrDoubleFree);
         } else if (old == 1) {
             s.zeroed[b] = 1;
+            s.block_hash[b] = 0;  // a freed block no longer backs a cached prefix
         }
         atomicMax(&s.last_idx[b], i);
     }
@@ -351,6 +354,155 @@ __global__ void __launch_bounds__(kBmThreads) bm_append_slots_kernel(const Appen
     if (threadIdx.x == 0) {
         *p.num_pairs = run_pairs;
         s.hdr[0] = top0 - handed;
+    }
+}
+
+// ------------------------------------------------------------ prefix cache --
+// Full prompt blocks are keyed by FNV-1a 64 (offset basis 14695981039346656037,
+// prime 1099511628211, xor then multiply per byte) chained over the prefix:
+// d_i = FNV-1a of the block's tokens as little-endian int32 bytes, key_i =
+// FNV-1a of le64(key_{i-1}) || le64(d_i) with key_{-1} = 0; key 0 is stored as
+// 1.  The cache is an open-addressing table of (key, block) pairs with linear
+// probing; an entry counts only while its block still holds the key
+// (block_hash) and some sequence maps it (refcount > 0).
+constexpr uint64_t kFnvBasis = 14695981039346656037ull;
+constexpr uint64_t kFnvPrime = 1099511628211ull;
+
+struct PrefixCache {
+    unsigned long long *keys;  // [cap], 0 = empty
+    int32_t *vals;             // [cap] block ids
+    int32_t *claim;            // [cap] scratch: earliest inserting sequence (rest: INT32_MAX)
+    int cap;                   // power of two
+};
+
+__device__ __forceinline__ uint64_t fnv_u32(uint64_t h, uint32_t w) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        h ^= (w >> (8 * i)) & 0xffu;
+        h *= kFnvPrime;
+    }
+    return h;
+}
+
+__device__ __forceinline__ uint64_t prefix_block_key(uint64_t prev, const int32_t *tok, int bs) {
+    uint64_t d = kFnvBasis;
+    for (int t = 0; t < bs; ++t) d = fnv_u32(d, (uint32_t)__ldg(tok + t));
+    uint64_t k = kFnvBasis;
+    k = fnv_u32(k, (uint32_t)prev);
+    k = fnv_u32(k, (uint32_t)(prev >> 32));
+    k = fnv_u32(k, (uint32_t)d);
+    k = fnv_u32(k, (uint32_t)(d >> 32));
+    return k ? k : 1;
+}
+
+// Slot holding key, or -1 (an empty slot ends the probe).
+__device__ __forceinline__ int cache_find(const PrefixCache &c, uint64_t key) {
+    int slot = (int)(key & (uint64_t)(c.cap - 1));
+    for (int n = 0; n < c.cap; ++n) {
+        const unsigned long long k = c.keys[slot];
+        if (k == key) return slot;
+        if (k == 0ull) return -1;
+        slot = (slot + 1) & (c.cap - 1);
+    }
+    return -1;
+}
+
+__device__ __forceinline__ bool holder_valid(const BmState &s, int nb, int32_t b, uint64_t key) {
+    return b >= 0 && b < nb && s.block_hash[b] == key && s.refcount[b] > 0;
+}
+
+__global__ void __launch_bounds__(256) prefix_cache_init_kernel(PrefixCache c) {
+    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < c.cap; i += gridDim.x * blockDim.x) {
+        c.keys[i] = 0ull;
+        c.vals[i] = -1;
+        c.claim[i] = 0x7fffffff;
+    }
+}
+
+struct PrefixParams {
+    BmState s;
+    PrefixCache c;
+    const int32_t *tokens;       // prompts, concatenated
+    const int32_t *query_start;  // [B+1]
+    int32_t *tables;             // [B][mbs]
+    int32_t *num_cached;         // [B] (lookup)
+    int nb, B, bs, mbs;
+};
+
+// Lookup, one thread per sequence: the leading prompt blocks whose keys have
+// a valid holder -- at least one prompt token is left to compute -- are
+// mapped into the sequence's table row with one reference each.
+__global__ void __launch_bounds__(256) prefix_lookup_kernel(const PrefixParams p) {
+    const int s = blockIdx.x * blockDim.x + threadIdx.x;
+    if (s >= p.B) return;
+    const int q0 = __ldg(p.query_start + s);
+    const int n = __ldg(p.query_start + s + 1) - q0;
+    const int look = min(n > 0 ? (n - 1) / p.bs : 0, p.mbs);
+    uint64_t prev = 0;
+    int hits = 0;
+    for (int i = 0; i < look; ++i) {
+        const uint64_t key = prefix_block_key(prev, p.tokens + q0 + i * p.bs, p.bs);
+        prev = key;
+        const int slot = cache_find(p.c, key);
+        const int32_t b = slot >= 0 ? p.c.vals[slot] : -1;
+        if (!holder_valid(p.s, p.nb, b, key)) break;
+        p.tables[(size_t)s * p.mbs + i] = b;
+        atomicAdd(&p.s.refcount[b], 1);
+        ++hits;
+    }
+    p.num_cached[s] = hits * p.bs;
+}
+
+// Insert, one CTA, sequences in order in chunks of 1024 (one thread each):
+// pass 1 puts each new key in the table (CAS into an empty slot) and, when the
+// key has no valid holder, claims the slot with the sequence index (atomicMin:
+// the earliest sequence wins, as in order); pass 2 lets the winners record
+// their blocks; pass 3 returns the claims to rest.
+__global__ void __launch_bounds__(kBmThreads) prefix_insert_kernel(const PrefixParams p) {
+    for (int base = 0; base < p.B; base += kBmThreads) {
+        const int s = base + threadIdx.x;
+        int q0 = 0, full = 0;
+        if (s < p.B) {
+            q0 = __ldg(p.query_start + s);
+            full = min((__ldg(p.query_start + s + 1) - q0) / p.bs, p.mbs);
+        }
+        for (int pass = 0; pass < 3; ++pass) {
+            uint64_t prev = 0;
+            for (int i = 0; i < full; ++i) {
+                const uint64_t key = prefix_block_key(prev, p.tokens + q0 + i * p.bs, p.bs);
+                prev = key;
+                const int32_t b = p.tables[(size_t)s * p.mbs + i];
+                if (b < 0 || b >= p.nb) {
+                    if (pass == 0) bm_error(p.s, kBmErrRange);
+                    break;
+                }
+                if (pass == 0) {
+                    if (p.s.block_hash[b] == key) continue;  // already the holder
+                    int slot = (int)(key & (uint64_t)(p.c.cap - 1));
+                    int found = -1;
+                    for (int t = 0; t < p.c.cap; ++t) {
+                        const unsigned long long k = atomicCAS(&p.c.keys[slot], 0ull, (unsigned long long)key);
+                        if (k == 0ull || k == key) { found = slot; break; }
+                        slot = (slot + 1) & (p.c.cap - 1);
+                    }
+                    if (found < 0) {
+                        bm_error(p.s, kBmErrNoSpace);
+                        continue;
+                    }
+                    if (!holder_valid(p.s, p.nb, p.c.vals[found], key)) atomicMin(&p.c.claim[found], s);
+                } else {
+                    const int slot = cache_find(p.c, key);
+                    if (slot < 0) continue;
+                    if (pass == 1 && p.c.claim[slot] == s) {
+                        p.c.vals[slot] = b;
+                        p.s.block_hash[b] = key;
+                    } else if (pass == 2) {
+                        p.c.claim[slot] = 0x7fffffff;
+                    }
+                }
+            }
+            __syncthreads();
+        }
     }
 }
 

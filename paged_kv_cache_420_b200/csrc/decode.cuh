@@ -394,6 +394,8 @@ struct SimtState {
         const float my_m = (G == 1 || my_head == 0) ? m[0] : m[G - 1];
         const float pr = exp2f(score - my_m);
         l_part += pr;
+        // KV8: p as an f16 pair, converted once here and shuffled as such
+        const uint32_t pr16 = KV8 ? f16x2_from_f32(pr, pr) : 0u;
         // PV: broadcast p of each valid token, accumulate its V row (packed
         // fp32x2 FMA over element pairs)
 #pragma unroll
@@ -405,8 +407,7 @@ struct SimtState {
 #pragma unroll
                     for (int j = 0; j < G; ++j) {
                         const int src = (G == 1) ? (2 * r) : (j * 16 + r);
-                        const float pj = __shfl_sync(0xffffffffu, pr, src);
-                        const uint32_t p16 = f16x2_from_f32(pj, pj);
+                        const uint32_t p16 = __shfl_sync(0xffffffffu, pr16, src);
                         acc[j][0] = fma_f16lo(p16, v16[0], acc[j][0]);
                         acc[j][1] = fma_f16hi(p16, v16[0], acc[j][1]);
                         acc[j][2] = fma_f16lo(p16, v16[1], acc[j][2]);

@@ -367,6 +367,18 @@ bool bm_state(void *state, int32_t nb, pkv::BmState *s) {
     s->last_idx = reinterpret_cast<int32_t *>(p + 256 + 2 * a);
     s->zeroed = reinterpret_cast<int32_t *>(p + 256 + 3 * a);
     s->cow_rank = reinterpret_cast<int32_t *>(p + 256 + 4 * a);
+    s->block_hash = reinterpret_cast<uint64_t *>(p + 256 + 5 * a);
+    return true;
+}
+
+// Prefix cache: keys (uint64), block ids and claims (int32), cap each.
+bool prefix_cache(void *cache, int32_t cap, pkv::PrefixCache *c) {
+    if (!cache || cap < 2 || (cap & (cap - 1)) != 0 || !aligned(cache, 256)) return false;
+    uint8_t *p = static_cast<uint8_t *>(cache);
+    c->keys = reinterpret_cast<unsigned long long *>(p);
+    c->vals = reinterpret_cast<int32_t *>(p + round256((size_t)cap * 8));
+    c->claim = reinterpret_cast<int32_t *>(p + round256((size_t)cap * 8) + round256((size_t)cap * 4));
+    c->cap = cap;
     return true;
 }
 
@@ -701,7 +713,66 @@ pkv_status paged_attn_prefill(const void *q, const void *k_cache, const void *v_
 
 size_t pkv_bm_state_bytes(int32_t num_blocks) {
     if (num_blocks <= 0) return 0;
-    return 256 + 5 * bm_array_bytes(num_blocks);
+    return 256 + 5 * bm_array_bytes(num_blocks) + round256((size_t)num_blocks * 8);
+}
+
+size_t pkv_prefix_cache_bytes(int32_t capacity) {
+    if (capacity < 2 || (capacity & (capacity - 1)) != 0) return 0;
+    return round256((size_t)capacity * 8) + 2 * round256((size_t)capacity * 4);
+}
+
+pkv_status pkv_prefix_cache_init(void *cache, int32_t capacity, pkv_stream_t stream) {
+    pkv::PrefixCache c;
+    if (!prefix_cache(cache, capacity, &c)) return PKV_EINVAL;
+    const int grid = std::max(1, std::min(1024, (capacity + 255) / 256));
+    pkv::prefix_cache_init_kernel<<<grid, 256, 0, (cudaStream_t)stream>>>(c);
+    return launch_status();
+}
+
+static pkv_status prefix_params(void *state, int32_t num_blocks, void *cache, int32_t capacity,
+                                const int32_t *tokens, const int32_t *query_start, int32_t num_seqs,
+                                int32_t block_size, int32_t *block_tables, int32_t max_blocks_per_seq,
+                                pkv::PrefixParams *p) {
+    if (!bm_state(state, num_blocks, &p->s) || !prefix_cache(cache, capacity, &p->c)) return PKV_EINVAL;
+    if (num_seqs < 0 || block_size <= 0 || max_blocks_per_seq <= 0) return PKV_EINVAL;
+    if (num_seqs > 0 && (!tokens || !query_start || !block_tables)) return PKV_EINVAL;
+    if (!aligned(tokens, 4) || !aligned(query_start, 4) || !aligned(block_tables, 4)) return PKV_EINVAL;
+    p->tokens = tokens;
+    p->query_start = query_start;
+    p->tables = block_tables;
+    p->nb = num_blocks;
+    p->B = num_seqs;
+    p->bs = block_size;
+    p->mbs = max_blocks_per_seq;
+    p->num_cached = nullptr;
+    return PKV_OK;
+}
+
+pkv_status pkv_prefix_lookup(void *state, int32_t num_blocks, void *cache, int32_t capacity, const int32_t *tokens,
+                             const int32_t *query_start, int32_t num_seqs, int32_t block_size,
+                             int32_t *block_tables, int32_t max_blocks_per_seq, int32_t *num_cached,
+                             pkv_stream_t stream) {
+    pkv::PrefixParams p;
+    const pkv_status st = prefix_params(state, num_blocks, cache, capacity, tokens, query_start, num_seqs,
+                                        block_size, block_tables, max_blocks_per_seq, &p);
+    if (st != PKV_OK) return st;
+    if (num_seqs == 0) return PKV_OK;
+    if (!num_cached || !aligned(num_cached, 4)) return PKV_EINVAL;
+    p.num_cached = num_cached;
+    pkv::prefix_lookup_kernel<<<(num_seqs + 255) / 256, 256, 0, (cudaStream_t)stream>>>(p);
+    return launch_status();
+}
+
+pkv_status pkv_prefix_insert(void *state, int32_t num_blocks, void *cache, int32_t capacity, const int32_t *tokens,
+                             const int32_t *query_start, int32_t num_seqs, int32_t block_size,
+                             const int32_t *block_tables, int32_t max_blocks_per_seq, pkv_stream_t stream) {
+    pkv::PrefixParams p;
+    const pkv_status st = prefix_params(state, num_blocks, cache, capacity, tokens, query_start, num_seqs,
+                                        block_size, const_cast<int32_t *>(block_tables), max_blocks_per_seq, &p);
+    if (st != PKV_OK) return st;
+    if (num_seqs == 0) return PKV_OK;
+    pkv::prefix_insert_kernel<<<1, pkv::kBmThreads, 0, (cudaStream_t)stream>>>(p);
+    return launch_status();
 }
 
 pkv_status pkv_bm_init(void *state, int32_t num_blocks, pkv_stream_t stream) {

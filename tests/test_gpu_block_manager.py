@@ -246,3 +246,77 @@ def test_decode_step_driven_by_the_device_block_manager():
     assert bits_equal(kd, okc) and bits_equal(vd, ovc)
     ref = oracle.paged_attention(q, okc, ovc, m.tables, m.ctx, float(np.float32(1 / np.sqrt(D))))
     assert_attention_close(out, ref, "device block manager step")
+
+
+def _systems(rng, bs, n_sys=4, vocab=100):
+    return [rng.integers(0, vocab, bs * int(rng.integers(1, 4))) for _ in range(n_sys)]
+
+
+def _prompts(rng, n, bs, systems, vocab=100):
+    """Prompts: one of the system prompts (1-3 blocks) plus a private tail."""
+    n_sys = len(systems)
+    out = []
+    for _ in range(n):
+        tail = rng.integers(0, vocab, int(rng.integers(0, 3 * bs)))
+        out.append(np.concatenate([systems[int(rng.integers(n_sys))], tail]).astype(np.int32))
+    return out
+
+
+def _serve_both(bm, pc, st, ocache, prompts, bs, mbs):
+    tokens = np.concatenate(prompts).astype(np.int32)
+    qs = np.concatenate([[0], np.cumsum([len(p) for p in prompts])]).astype(np.int32)
+    B = len(prompts)
+    tables = np.full((B, mbs), -1, np.int32)
+    t_dev = _dev(tables)
+    cached = pc.lookup(bm, _dev(tokens), _dev(qs), bs, t_dev)
+    st, otab, ocached = oracle.prefix_lookup(st, ocache, tokens, qs, bs, tables)
+    torch.cuda.synchronize()
+    assert np.array_equal(cached.cpu().numpy(), ocached)
+    assert np.array_equal(t_dev.cpu().numpy(), otab)
+    need = np.array([len(p) for p in prompts], np.int32) - ocached
+    c_dev = _dev(ocached)
+    slots, pairs, npairs = bm.append_slots(t_dev, c_dev, _dev(need), bs, int(need.sum()))
+    st, otab, octx, oslots, opairs, err = oracle.bm_append_slots(st, otab, ocached, need, bs)
+    torch.cuda.synchronize()
+    assert np.array_equal(t_dev.cpu().numpy(), otab) and np.array_equal(slots.cpu().numpy(), oslots)
+    pc.insert(bm, _dev(tokens), _dev(qs), bs, t_dev)
+    st, ocache, e2 = oracle.prefix_insert(st, ocache, tokens, qs, bs, otab)
+    torch.cuda.synchronize()
+    assert np.array_equal(bm.block_hash.cpu().numpy().view(np.uint64), st.block_hash)
+    _same_state(bm, st, err | e2)
+    return st, ocache, otab, octx, ocached
+
+
+@pytest.mark.parametrize("seed,B,bs", [(0, 40, 4), (1, 1300, 4), (2, 64, 16)])
+def test_prefix_cache_rounds_match_oracle(seed, B, bs):
+    """Rounds of requests sharing system prompts: lookup, the remaining blocks
+    through append_slots, insert; some sequences end between rounds."""
+    rng = np.random.default_rng(seed)
+    mbs = 8
+    nb = B * mbs * 2
+    bm = pkv.BlockManager(nb)
+    pc = pkv.PrefixCache(1 << int(np.ceil(np.log2(4 * B * mbs))))
+    st = oracle.bm_init(nb)
+    ocache = oracle.PrefixCache(4 * B * mbs)
+    live = []
+    total_hits = 0
+    systems = _systems(rng, bs)
+    for rnd in range(3):
+        prompts = _prompts(rng, B, bs, systems)
+        if rnd == 1:
+            prompts[B // 2] = prompts[B // 2 - 1].copy()  # the same prompt twice in one batch
+        st, ocache, tables, ctx, cached = _serve_both(bm, pc, st, ocache, prompts, bs, mbs)
+        total_hits += int((cached > 0).sum())
+        live.append((tables, ctx))
+        # half of the oldest round's sequences end
+        old_tables, old_ctx = live[0]
+        ends = np.flatnonzero(rng.random(len(old_ctx)) < 0.5)
+        ids = np.concatenate([old_tables[b, :(old_ctx[b] + bs - 1) // bs] for b in ends]) if len(ends) else []
+        ids = np.asarray(ids, np.int32)
+        if len(ids):
+            bm.free(_dev(ids))
+            st, _ = oracle.bm_free(st, ids)
+            _same_state(bm, st, 0)
+            assert np.array_equal(bm.block_hash.cpu().numpy().view(np.uint64), st.block_hash)
+        old_ctx[ends] = 0
+    assert total_hits > 0 and st.block_hash.any()
