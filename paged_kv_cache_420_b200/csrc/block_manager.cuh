@@ -429,80 +429,117 @@ struct PrefixParams {
     int nb, B, bs, mbs;
 };
 
-// Lookup, one thread per sequence: the leading prompt blocks whose keys have
-// a valid holder -- at least one prompt token is left to compute -- are
-// mapped into the sequence's table row with one reference each.
+// Keys of blocks base .. base+31 of one prompt, one warp: lane l hashes the
+// tokens of block base + l (its digest), then every lane walks the chain over
+// the shuffled digests in lockstep and keeps the key of its own block.  prev
+// enters as the key of block base - 1 (0 before block 0) and leaves as the key
+// of the group's last block; lanes past `count` get 0.
+__device__ __forceinline__ uint64_t warp_block_keys(const int32_t *tok0, int base, int count, int bs, uint64_t &prev) {
+    const int lane = threadIdx.x & 31;
+    const int i = base + lane;
+    uint64_t d = kFnvBasis;
+    if (i < count)
+        for (int t = 0; t < bs; ++t) d = fnv_u32(d, (uint32_t)__ldg(tok0 + (size_t)i * bs + t));
+    uint64_t mine = 0;
+    const int n = min(32, count - base);
+    for (int j = 0; j < n; ++j) {
+        const uint64_t dj = __shfl_sync(0xffffffffu, d, j);
+        uint64_t k = kFnvBasis;
+        k = fnv_u32(k, (uint32_t)prev);
+        k = fnv_u32(k, (uint32_t)(prev >> 32));
+        k = fnv_u32(k, (uint32_t)dj);
+        k = fnv_u32(k, (uint32_t)(dj >> 32));
+        prev = k ? k : 1;
+        if (lane == j) mine = prev;
+    }
+    return mine;
+}
+
+// Lookup, one warp per sequence: the leading prompt blocks whose keys have a
+// valid holder -- at least one prompt token is left to compute -- are mapped
+// into the sequence's table row with one reference each.
 __global__ void __launch_bounds__(256) prefix_lookup_kernel(const PrefixParams p) {
-    const int s = blockIdx.x * blockDim.x + threadIdx.x;
-    if (s >= p.B) return;
+    const int s = blockIdx.x * 8 + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (s >= p.B) return;  // whole warps
     const int q0 = __ldg(p.query_start + s);
     const int n = __ldg(p.query_start + s + 1) - q0;
     const int look = min(n > 0 ? (n - 1) / p.bs : 0, p.mbs);
     uint64_t prev = 0;
     int hits = 0;
-    for (int i = 0; i < look; ++i) {
-        const uint64_t key = prefix_block_key(prev, p.tokens + q0 + i * p.bs, p.bs);
-        prev = key;
-        const int slot = cache_find(p.c, key);
-        const int32_t b = slot >= 0 ? p.c.vals[slot] : -1;
-        if (!holder_valid(p.s, p.nb, b, key)) break;
-        p.tables[(size_t)s * p.mbs + i] = b;
-        atomicAdd(&p.s.refcount[b], 1);
-        ++hits;
+    for (int base = 0; base < look; base += 32) {
+        const uint64_t key = warp_block_keys(p.tokens + q0, base, look, p.bs, prev);
+        const int i = base + lane;
+        int32_t b = -1;
+        bool valid = false;
+        if (i < look) {
+            const int slot = cache_find(p.c, key);
+            b = slot >= 0 ? p.c.vals[slot] : -1;
+            valid = holder_valid(p.s, p.nb, b, key);
+        }
+        const unsigned hit = __ballot_sync(0xffffffffu, valid);
+        const int lead = hit == 0xffffffffu ? 32 : __ffs(~hit) - 1;  // leading run of hits
+        if (lane < lead) {
+            p.tables[(size_t)s * p.mbs + i] = b;
+            atomicAdd(&p.s.refcount[b], 1);
+        }
+        hits += lead;
+        if (lead < min(32, look - base)) break;
     }
-    p.num_cached[s] = hits * p.bs;
+    if (lane == 0) p.num_cached[s] = hits * p.bs;
 }
 
-// Insert, one CTA, sequences in order in chunks of 1024 (one thread each):
-// pass 1 puts each new key in the table (CAS into an empty slot) and, when the
-// key has no valid holder, claims the slot with the sequence index (atomicMin:
-// the earliest sequence wins, as in order); pass 2 lets the winners record
-// their blocks; pass 3 returns the claims to rest.
-__global__ void __launch_bounds__(kBmThreads) prefix_insert_kernel(const PrefixParams p) {
-    for (int base = 0; base < p.B; base += kBmThreads) {
-        const int s = base + threadIdx.x;
-        int q0 = 0, full = 0;
-        if (s < p.B) {
-            q0 = __ldg(p.query_start + s);
-            full = min((__ldg(p.query_start + s + 1) - q0) / p.bs, p.mbs);
-        }
-        for (int pass = 0; pass < 3; ++pass) {
-            uint64_t prev = 0;
-            for (int i = 0; i < full; ++i) {
-                const uint64_t key = prefix_block_key(prev, p.tokens + q0 + i * p.bs, p.bs);
-                prev = key;
-                const int32_t b = p.tables[(size_t)s * p.mbs + i];
-                if (b < 0 || b >= p.nb) {
-                    if (pass == 0) bm_error(p.s, kBmErrRange);
-                    break;
-                }
-                if (pass == 0) {
-                    if (p.s.block_hash[b] == key) continue;  // already the holder
+// Insert, one warp per sequence over all sequences at once, in three launches
+// (a kernel boundary orders the passes grid-wide): pass 0 puts each new key in
+// the table (CAS into an empty slot) and, when the key has no valid holder,
+// claims the slot with the sequence index (atomicMin: the earliest sequence
+// wins, as in sequence order); pass 1 lets the winners record their blocks;
+// pass 2 returns the claims to rest.  A block id outside the pool stops the
+// sequence there (and is reported).
+template <int PASS>
+__global__ void __launch_bounds__(256) prefix_insert_kernel(const PrefixParams p) {
+    const int s = blockIdx.x * 8 + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (s >= p.B) return;  // whole warps
+    const int q0 = __ldg(p.query_start + s);
+    const int full = min((__ldg(p.query_start + s + 1) - q0) / p.bs, p.mbs);
+    uint64_t prev = 0;
+    for (int gb = 0; gb < full; gb += 32) {
+        const uint64_t key = warp_block_keys(p.tokens + q0, gb, full, p.bs, prev);
+        const int i = gb + lane;
+        const int32_t b = i < full ? p.tables[(size_t)s * p.mbs + i] : 0;
+        const unsigned bad = __ballot_sync(0xffffffffu, i < full && (b < 0 || b >= p.nb));
+        const int stop = bad ? __ffs(bad) - 1 : 32;  // blocks from here on are not inserted
+        if (PASS == 0 && bad && lane == stop) bm_error(p.s, kBmErrRange);
+        if (i < full && lane < stop) {
+            if (PASS == 0) {
+                if (p.s.block_hash[b] != key) {
                     int slot = (int)(key & (uint64_t)(p.c.cap - 1));
                     int found = -1;
                     for (int t = 0; t < p.c.cap; ++t) {
                         const unsigned long long k = atomicCAS(&p.c.keys[slot], 0ull, (unsigned long long)key);
-                        if (k == 0ull || k == key) { found = slot; break; }
+                        if (k == 0ull || k == key) {
+                            found = slot;
+                            break;
+                        }
                         slot = (slot + 1) & (p.c.cap - 1);
                     }
-                    if (found < 0) {
-                        bm_error(p.s, kBmErrNoSpace);
-                        continue;
-                    }
-                    if (!holder_valid(p.s, p.nb, p.c.vals[found], key)) atomicMin(&p.c.claim[found], s);
-                } else {
-                    const int slot = cache_find(p.c, key);
-                    if (slot < 0) continue;
-                    if (pass == 1 && p.c.claim[slot] == s) {
+                    if (found < 0) bm_error(p.s, kBmErrNoSpace);
+                    else if (!holder_valid(p.s, p.nb, p.c.vals[found], key)) atomicMin(&p.c.claim[found], s);
+                }
+            } else {
+                const int slot = cache_find(p.c, key);
+                if (slot >= 0) {
+                    if (PASS == 1 && p.c.claim[slot] == s) {
                         p.c.vals[slot] = b;
                         p.s.block_hash[b] = key;
-                    } else if (pass == 2) {
+                    } else if (PASS == 2) {
                         p.c.claim[slot] = 0x7fffffff;
                     }
                 }
             }
-            __syncthreads();
         }
+        if (bad) break;
     }
 }
 

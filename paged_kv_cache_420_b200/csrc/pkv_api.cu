@@ -759,7 +759,7 @@ pkv_status pkv_prefix_lookup(void *state, int32_t num_blocks, void *cache, int32
     if (num_seqs == 0) return PKV_OK;
     if (!num_cached || !aligned(num_cached, 4)) return PKV_EINVAL;
     p.num_cached = num_cached;
-    pkv::prefix_lookup_kernel<<<(num_seqs + 255) / 256, 256, 0, (cudaStream_t)stream>>>(p);
+    pkv::prefix_lookup_kernel<<<(num_seqs + 7) / 8, 256, 0, (cudaStream_t)stream>>>(p);  // a warp per sequence
     return launch_status();
 }
 
@@ -771,7 +771,10 @@ pkv_status pkv_prefix_insert(void *state, int32_t num_blocks, void *cache, int32
                                         block_size, const_cast<int32_t *>(block_tables), max_blocks_per_seq, &p);
     if (st != PKV_OK) return st;
     if (num_seqs == 0) return PKV_OK;
-    pkv::prefix_insert_kernel<<<1, pkv::kBmThreads, 0, (cudaStream_t)stream>>>(p);
+    const unsigned grid = (unsigned)((num_seqs + 7) / 8);  // a warp per sequence
+    pkv::prefix_insert_kernel<0><<<grid, 256, 0, (cudaStream_t)stream>>>(p);
+    pkv::prefix_insert_kernel<1><<<grid, 256, 0, (cudaStream_t)stream>>>(p);
+    pkv::prefix_insert_kernel<2><<<grid, 256, 0, (cudaStream_t)stream>>>(p);
     return launch_status();
 }
 
