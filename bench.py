@@ -478,20 +478,22 @@ def run_prefill_cuda(args, rank, world, dist):
 
 
 SWAP_WORKLOADS = ("llama2-13b-swap",)
-FP8_WORKLOADS = ("llama2-13b-fp8",)
+FP8_WORKLOADS = ("llama2-13b-fp8", "llama3-8b-gqa-prefix-fp8")
 
 
 def run_fp8_cuda(args, rank, world, dist):
-    """The Llama-2-13B decode step on an FP8 (e4m3) pool: the quantizing write
-    of each sequence's new token, then decode attention over the e4m3 codes
-    with per-kv-head K/V scales.  Metric: algorithmic HBM GB/s of the step (one
-    byte per cached element) and tokens*layers/s, comparable with the bf16
-    step's."""
+    """A decode step on an FP8 (e4m3) pool (the Llama-2-13B batch, or the
+    Llama-3-8B shared-prefix batch): the quantizing write of each sequence's
+    new token, then decode attention over the e4m3 codes with per-kv-head K/V
+    scales (the shared-prefix batch's copy-on-write copies are not part of
+    this step).  Metric: algorithmic HBM GB/s of the step (one byte per cached
+    element) and tokens*layers/s, comparable with the bf16 step's."""
     import paged_kv_cache_420_b200 as pkv
 
     dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
     torch.cuda.set_device(dev)
-    w = workloads.make("llama2-13b", seed=args.seed + rank, values_device=dev, block_size=args.block_size)
+    base = args.workload[:-len("-fp8")]
+    w = workloads.make(base, seed=args.seed + rank, values_device=dev, block_size=args.block_size)
     k8, v8, ks, vs = workloads.fp8_pools(w)
     del w.k_cache, w.v_cache
     torch.cuda.empty_cache()
@@ -539,7 +541,7 @@ def run_fp8_cuda(args, rank, world, dist):
     peak, kind = measured_hbm_peak()
     achieved = dec / (dec_ms / 1e3) / 1e9
     return {
-        "metric": "paged decode attn HBM GB/s on an FP8 (e4m3) pool & tokens*layers/s at 13B shape",
+        "metric": f"paged decode attn HBM GB/s on an FP8 (e4m3) pool & tokens*layers/s ({base})",
         "value": whole_job_gbs(bytes_all, args.steps, ms_max), "unit": "GB/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_max / args.steps, 5),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "e4m3 KV, bf16 q/out",

@@ -173,10 +173,15 @@ struct DecodeSmem {
     static constexpr int kBoxes = D * kElem / 128;        // boxes per row of a tile
     static constexpr int kTile = kStageTok * D * kElem;   // one K (or V) stage tile
     static constexpr int kStage = 2 * kTile;
+    // FP8 pool on the tensor-core path (GP >= 4): each consumer warp converts
+    // its stage's V tile to f16 (bf16 tile layout) in a scratch of its own
+    static constexpr int kTileF16 = kStageTok * D * 2;
+    static constexpr int kScratch = (KV8 && GP >= 4) ? kW * kTileF16 : 0;
     static constexpr int kQBuf = GP * D * 2;              // the query heads of one kv head
     static constexpr int kMergeStride = D + 4;            // floats, padded against bank conflicts
     static constexpr int oTiles = 0;
-    static constexpr int oQ = oTiles + NS * kStage;
+    static constexpr int oScratch = oTiles + NS * kStage;
+    static constexpr int oQ = oScratch + kScratch;
     static constexpr int oMergeO = oQ + 2 * kQBuf;
     static constexpr int oMergeM = oMergeO + kW * GP * kMergeStride * 4;
     static constexpr int oMergeL = oMergeM + kW * GP * 4;
@@ -454,7 +459,40 @@ struct SimtState {
 };
 
 // ------------------------------------------- tensor-core path (3 <= g <= 16) --
-template <int D, int NT>
+// An FP8 stage tile (16 rows x 128 codes, tile_addr8 layout) -> the same tile
+// as f16 in the bf16 tile layout (tile_addr), by one warp: lane handles 16-code
+// chunks, one 16-byte load, eight pair conversions, two 16-byte stores.
+__device__ __forceinline__ void convert_tile_f16(uint32_t src8, uint32_t dst16, int lane) {
+#pragma unroll
+    for (int i = lane; i < kStageTok * 8; i += 32) {
+        const int r = i >> 3, ch = i & 7;
+        uint32_t w[4];
+        asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                     : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3])
+                     : "r"(tile_addr8(src8, r, ch * 16)));
+        uint32_t h[8];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            h[2 * k] = f16x2_from_e4m3x2(w[k] & 0xffffu);
+            h[2 * k + 1] = f16x2_from_e4m3x2(w[k] >> 16);
+        }
+        asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(tile_addr(dst16, r, ch * 16)), "r"(h[0]),
+                     "r"(h[1]), "r"(h[2]), "r"(h[3])
+                     : "memory");
+        asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(tile_addr(dst16, r, ch * 16 + 8)), "r"(h[4]),
+                     "r"(h[5]), "r"(h[6]), "r"(h[7])
+                     : "memory");
+    }
+}
+
+// H: an FP8 pool, f16 operands (the codes are exact in f16; q is converted to
+// f16 and P packed as f16), otherwise bf16.  With H the K operand comes
+// straight from the e4m3 stage tile: lane l (j = l % 4) loads the 4 codes of
+// columns k0 + 4j .. 4j + 3 of its rows as one word, and the pairs (4j, 4j+1)
+// and (4j+2, 4j+3) fill the k slots (2j, 2j+1) and (2j+8, 2j+9) of the
+// m16n8k16 A fragment.  The dot product does not depend on the order of k,
+// so q's B fragment takes its columns in the same order.
+template <int D, int NT, bool H = false>
 struct MmaState {
     static constexpr int KS = D / 16;  // k-steps of QK^T
     static constexpr int MT = D / 16;  // m-tiles of O^T
@@ -483,11 +521,18 @@ struct MmaState {
             const int head = nt * 8 + (lane >> 2);
 #pragma unroll
             for (int kk = 0; kk < KS; ++kk) {
-                const int col = kk * 16 + 2 * (lane & 3);
+                // k slots 2j, 2j+1 and 2j+8, 2j+9; with H they hold columns
+                // 4j, 4j+1 and 4j+2, 4j+3 (see above)
+                const int col0 = H ? kk * 16 + 4 * (lane & 3) : kk * 16 + 2 * (lane & 3);
+                const int col1 = H ? col0 + 2 : col0 + 8;
                 uint32_t b0 = 0, b1 = 0;
                 if (head < g) {
-                    b0 = *reinterpret_cast<const uint32_t *>(qs + head * D + col);
-                    b1 = *reinterpret_cast<const uint32_t *>(qs + head * D + col + 8);
+                    b0 = *reinterpret_cast<const uint32_t *>(qs + head * D + col0);
+                    b1 = *reinterpret_cast<const uint32_t *>(qs + head * D + col1);
+                    if constexpr (H) {
+                        b0 = f16x2_from_f32(bf16lo_to_f32(b0), bf16hi_to_f32(b0));
+                        b1 = f16x2_from_f32(bf16lo_to_f32(b1), bf16hi_to_f32(b1));
+                    }
                 }
                 qb[nt][kk][0] = b0;
                 qb[nt][kk][1] = b1;
@@ -507,14 +552,26 @@ struct MmaState {
 #pragma unroll
         for (int kk = 0; kk < KS; ++kk) {
             // matrices: (rows 0-7, cols k0..+7), (rows 8-15, k0..), (rows 0-7, k0+8..), (rows 8-15, k0+8..)
-            const int row = ri + 8 * (mi & 1);
-            const int col = kk * 16 + 8 * (mi >> 1);
             uint32_t a0, a1, a2, a3;
-            ldmatrix_x4(tile_addr(ktile, row, col), a0, a1, a2, a3);
+            if constexpr (H) {
+                uint32_t w0, w1;
+                const int c = kk * 16 + 4 * (lane & 3);
+                asm volatile("ld.shared.u32 %0, [%1];" : "=r"(w0) : "r"(tile_addr8(ktile, lane >> 2, c)));
+                asm volatile("ld.shared.u32 %0, [%1];" : "=r"(w1) : "r"(tile_addr8(ktile, (lane >> 2) + 8, c)));
+                a0 = f16x2_from_e4m3x2(w0 & 0xffffu);
+                a1 = f16x2_from_e4m3x2(w1 & 0xffffu);
+                a2 = f16x2_from_e4m3x2(w0 >> 16);
+                a3 = f16x2_from_e4m3x2(w1 >> 16);
+            } else {
+                const int row = ri + 8 * (mi & 1);
+                const int col = kk * 16 + 8 * (mi >> 1);
+                ldmatrix_x4(tile_addr(ktile, row, col), a0, a1, a2, a3);
+            }
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt) {
                 float *acc = (kk & 1) ? s2[nt] : s[nt];
-                mma_bf16_16816(acc[0], acc[1], acc[2], acc[3], a0, a1, a2, a3, qb[nt][kk][0], qb[nt][kk][1]);
+                if constexpr (H) mma_f16_16816(acc[0], acc[1], acc[2], acc[3], a0, a1, a2, a3, qb[nt][kk][0], qb[nt][kk][1]);
+                else mma_bf16_16816(acc[0], acc[1], acc[2], acc[3], a0, a1, a2, a3, qb[nt][kk][0], qb[nt][kk][1]);
             }
         }
 #pragma unroll
@@ -549,8 +606,8 @@ struct MmaState {
                 l[nt][c] = l[nt][c] * alpha[c] + p[c] + p[c + 2];
             }
             // accumulator layout (token row, head pair) -> operand layout of P^T
-            pb[nt][0] = movmatrix_trans(pack_bf16x2(p[0], p[1]));
-            pb[nt][1] = movmatrix_trans(pack_bf16x2(p[2], p[3]));
+            pb[nt][0] = movmatrix_trans(H ? f16x2_from_f32(p[0], p[1]) : pack_bf16x2(p[0], p[1]));
+            pb[nt][1] = movmatrix_trans(H ? f16x2_from_f32(p[2], p[3]) : pack_bf16x2(p[2], p[3]));
             if (__any_sync(0xffffffffu, raise)) {
 #pragma unroll
                 for (int mt = 0; mt < MT; ++mt) {
@@ -578,9 +635,14 @@ struct MmaState {
             ldmatrix_x4_trans(tile_addr(vtile, row, col), a0, a1, a2, a3);
             a0 &= mask01; a1 &= mask01; a2 &= mask23; a3 &= mask23;
 #pragma unroll
-            for (int nt = 0; nt < NT; ++nt)
-                mma_bf16_16816(o[nt][mt][0], o[nt][mt][1], o[nt][mt][2], o[nt][mt][3], a0, a1, a2, a3,
-                               pb[nt][0], pb[nt][1]);
+            for (int nt = 0; nt < NT; ++nt) {
+                if constexpr (H)
+                    mma_f16_16816(o[nt][mt][0], o[nt][mt][1], o[nt][mt][2], o[nt][mt][3], a0, a1, a2, a3,
+                                  pb[nt][0], pb[nt][1]);
+                else
+                    mma_bf16_16816(o[nt][mt][0], o[nt][mt][1], o[nt][mt][2], o[nt][mt][3], a0, a1, a2, a3,
+                                   pb[nt][0], pb[nt][1]);
+            }
         }
     }
 
@@ -618,7 +680,7 @@ __global__ void __launch_bounds__(kDecodeThreads) paged_decode_kernel(const __gr
     constexpr int W = kConsumerWarps;
     constexpr int GP = PATH == 0 ? GSIMT : GPAD;
     constexpr int NT = (GPAD + 7) / 8;
-    static_assert(!KV8 || (PATH == 0 && D == 128), "the FP8 pool runs on the CUDA-core path at head dim 128");
+    static_assert(!KV8 || D == 128, "FP8 stage tiles are 128-byte rows (head dim 128)");
     using L = DecodeSmem<D, GP, NS, KV8>;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     // 1024-B alignment: the 128-byte swizzle pattern repeats every 1 KB.
@@ -777,7 +839,7 @@ __global__ void __launch_bounds__(kDecodeThreads) paged_decode_kernel(const __gr
         uint32_t mc = 0;  // merges done
         float scale_log2 = p.scale_log2;
         SimtState<D, (PATH == 0 ? GSIMT : 1), KV8> st0;
-        MmaState<D, (PATH == 1 ? NT : 1)> st1;
+        MmaState<D, (PATH == 1 ? NT : 1), KV8> st1;
         while (true) {
             const uint32_t slot = gc % NS;
             if (!wait_or_abort(&full[slot], (gc / NS) & 1, abort_flag)) break;
@@ -798,8 +860,18 @@ __global__ void __launch_bounds__(kDecodeThreads) paged_decode_kernel(const __gr
             }
             if (si.valid > 0) {
                 const uint32_t kt = tiles + slot * L::kStage;
-                if constexpr (PATH == 0) st0.stage(kt, kt + L::kTile, si.valid, lane);
-                else st1.stage(kt, kt + L::kTile, si.valid, lane, scale_log2);
+                if constexpr (PATH == 0) {
+                    st0.stage(kt, kt + L::kTile, si.valid, lane);
+                } else if constexpr (KV8) {
+                    // K is read as codes; V goes through this warp's f16 copy
+                    const uint32_t sv = smem_u32(smem + L::oScratch) + w * L::kTileF16;
+                    convert_tile_f16(kt + L::kTile, sv, lane);
+                    __syncwarp();
+                    st1.stage(kt, sv, si.valid, lane, scale_log2 * __ldg(p.k_scale + si.h));
+                    __syncwarp();  // the next stage's conversion overwrites the scratch
+                } else {
+                    st1.stage(kt, kt + L::kTile, si.valid, lane, scale_log2);
+                }
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[slot]);

@@ -397,7 +397,7 @@ pkv_status decode_impl(const void *q, const void *k_cache, const void *v_cache, 
     if (num_kv_heads != pool.num_kv_heads || num_q_heads % num_kv_heads != 0) return PKV_EINVAL;
     const int g = num_q_heads / num_kv_heads;
     if (g > 16) return PKV_EUNSUPPORTED;
-    if (kv8 && (pool.head_dim != 128 || g > 2)) return PKV_EUNSUPPORTED;
+    if (kv8 && pool.head_dim != 128) return PKV_EUNSUPPORTED;
     if (partition_tokens < 0 || partition_tokens % 16 != 0 || partition_tokens > 65536) return PKV_EINVAL;
     if (num_seqs == 0) return PKV_OK;
     if (!q || !k_cache || !v_cache || !block_tables || !context_lens || !out || !workspace) return PKV_EINVAL;
@@ -449,8 +449,11 @@ pkv_status decode_impl(const void *q, const void *k_cache, const void *v_cache, 
     if (r != PKV_OK) return r;
     const int dev = current_device();
     if (kv8) {
-        return g == 1 ? launch_decode<128, 0, 1, 1, true>(prm, mk, mv, st, dev)
-                      : launch_decode<128, 0, 2, 1, true>(prm, mk, mv, st, dev);
+        if (g == 1) return launch_decode<128, 0, 1, 1, true>(prm, mk, mv, st, dev);
+        if (g == 2) return launch_decode<128, 0, 2, 1, true>(prm, mk, mv, st, dev);
+        if (g <= 4) return launch_decode<128, 1, 1, 4, true>(prm, mk, mv, st, dev);
+        if (g <= 8) return launch_decode<128, 1, 1, 8, true>(prm, mk, mv, st, dev);
+        return launch_decode<128, 1, 1, 16, true>(prm, mk, mv, st, dev);
     }
     return D == 128 ? dispatch_group<128>(g, prm, mk, mv, st, dev) : dispatch_group<64>(g, prm, mk, mv, st, dev);
 }

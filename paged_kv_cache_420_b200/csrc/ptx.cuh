@@ -145,6 +145,16 @@ __device__ __forceinline__ void mma_bf16_16816(float &d0, float &d1, float &d2, 
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
+// Same shape with f16 operands (fp32 accumulation).
+__device__ __forceinline__ void mma_f16_16816(float &d0, float &d1, float &d2, float &d3, uint32_t a0, uint32_t a1,
+                                              uint32_t a2, uint32_t a3, uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+        "{%0, %1, %2, %3};"
+        : "+f"(d0), "+f"(d1), "+f"(d2), "+f"(d3)
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
 // Orders this thread's generic-proxy shared-memory writes before later
 // async-proxy reads (TMA, tensor core) of the same CTA.
 __device__ __forceinline__ void fence_proxy_async_smem() {

@@ -1,7 +1,8 @@
 """GPU parity of the FP8 (e4m3) KV cache against the oracle: the quantizing
 write bit for bit (saturation, padding slots, several scales), and decode
-attention over e4m3 pools within the attention tolerance (GQA groups 1 and 2,
-ragged contexts, split-K partitions, poisoned unused rows)."""
+attention over e4m3 pools within the attention tolerance (GQA groups 1 to 16
+on both the CUDA-core and the tensor-core paths, ragged contexts, split-K
+partitions, poisoned unused rows)."""
 import numpy as np
 import pytest
 import torch
@@ -59,6 +60,10 @@ CASES = [
     ([5, 200, 511, 513], 16, 8, 0),          # g = 2
     ([1000, 3000, 77], 4, 4, 256),           # split-K partitions
     ([4096, 2049, 16], 8, 4, 512),           # g = 2, split-K
+    ([1, 15, 16, 17, 31, 100], 32, 8, 0),    # g = 4: tensor-core path
+    ([200, 511, 1000], 64, 8, 256),          # g = 8, split-K
+    ([50, 129], 12, 4, 0),                   # g = 3 (padded to 4)
+    ([33, 700], 16, 1, 0),                   # g = 16
 ]
 
 
@@ -116,11 +121,6 @@ def test_fp8_decode_matches_bf16_decode_on_exact_values():
 
 
 def test_fp8_refuses_unsupported_shapes():
-    w = workloads.make_custom([20], 8, 2, 128, 16, seed=1)  # g = 4
-    k8, v8, ks, vs = workloads.fp8_pools(w)
-    w.q = w.q.cuda()
-    with pytest.raises(pkv.PkvError):
-        _run_decode(w, k8.cuda(), v8.cuda(), ks.cuda(), vs.cuda())
     w = workloads.make_custom([20], 4, 4, 64, 16, seed=1)  # head dim 64
     k8, v8, ks, vs = workloads.fp8_pools(w)
     w.q = w.q.cuda()
