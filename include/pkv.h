@@ -287,9 +287,10 @@ pkv_status paged_attn_prefill(const void *q, const void *k_cache, const void *v_
  *
  * paged_attn_decode_fp8: as paged_attn_decode over an FP8 pool, reading
  * K = e4m3(code) * k_scale[h] and V = e4m3(code) * v_scale[h].  Supported at
- * head_dim 128 with num_q_heads / num_kv_heads <= 2 (else PKV_EUNSUPPORTED);
- * the codes are multiplied exactly as f16 with fp32 accumulation.  The
- * workspace is the same as paged_attn_decode's.
+ * head_dim 128 (else PKV_EUNSUPPORTED) for every GQA group <= 16: groups 1-2
+ * on CUDA cores, larger groups on the tensor cores; the codes are multiplied
+ * exactly as f16 with fp32 accumulation.  The workspace is the same as
+ * paged_attn_decode's.
  */
 pkv_status pkv_write_fp8(const void *k, const void *v, const int64_t *slot_mapping, int32_t num_tokens,
                          const float *k_scale, const float *v_scale, void *k_cache, void *v_cache, pkv_pool pool,
