@@ -485,9 +485,9 @@ def run_fp8_cuda(args, rank, world, dist):
     """A decode step on an FP8 (e4m3) pool (the Llama-2-13B batch, or the
     Llama-3-8B shared-prefix batch): the quantizing write of each sequence's
     new token, then decode attention over the e4m3 codes with per-kv-head K/V
-    scales (the shared-prefix batch's copy-on-write copies are not part of
-    this step).  Metric: algorithmic HBM GB/s of the step (one byte per cached
-    element) and tokens*layers/s, comparable with the bf16 step's."""
+    scales, after the batch's copy-on-write copies (if any).  Metric:
+    algorithmic HBM GB/s of the step (one byte per cached element) and
+    tokens*layers/s, comparable with the bf16 step's."""
     import paged_kv_cache_420_b200 as pkv
 
     dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
@@ -508,6 +508,8 @@ def run_fp8_cuda(args, rank, world, dist):
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
 
     def step(i=None):
+        if len(w.copy_pairs):
+            pkv.pkv_copy_blocks(w.copy_pairs, k8, v8, stream=stream)
         pkv.pkv_write_fp8(w.k_new, w.v_new, slots, ks, vs, k8, v8, stream=stream)
         if i is not None:
             ev[i][0].record(stream)
@@ -536,10 +538,14 @@ def run_fp8_cuda(args, rank, world, dist):
         raise RuntimeError("device error word set during the timed region")
     dec = decode_bytes(w, kv_elem=1)
     wr = w.num_seqs * w.num_kv_heads * w.head_dim * (2 * 2 + 2) + 8 * w.num_seqs  # bf16 in, e4m3 out
+    wr += copy_bytes(w) // 2  # e4m3 blocks
     ms_max, bytes_all, seqs_all = combine_ranks(dist, t0.elapsed_time(t1), dec + wr, w.num_seqs, dev)
     dec_ms = sum(a.elapsed_time(b) for a, b in ev) / args.steps
     peak, kind = measured_hbm_peak()
     achieved = dec / (dec_ms / 1e3) / 1e9
+    # copies (when the batch has pairs), write, plan, attention, and the
+    # split-K reduce when some context spans more than one partition
+    launches = (1 if len(w.copy_pairs) else 0) + 3 + (1 if mctx > library_partition_tokens(0, mctx) else 0)
     return {
         "metric": f"paged decode attn HBM GB/s on an FP8 (e4m3) pool & tokens*layers/s ({base})",
         "value": whole_job_gbs(bytes_all, args.steps, ms_max), "unit": "GB/s", "n_gpus": world,
@@ -553,7 +559,7 @@ def run_fp8_cuda(args, rank, world, dist):
                      "achieved": round(achieved, 1), "peak": peak, "peak_kind": kind, "unit": "GB/s",
                      "frac": round(achieved / peak, 4), "algorithmic_bytes": dec,
                      "decode_us": round(dec_ms * 1e3, 2), "traffic": None},
-        "e2e": None, "gpu_launches": 3 * args.steps, "clocks": clocks.summary(),
+        "e2e": None, "gpu_launches": args.steps * launches, "clocks": clocks.summary(),
     }
 BM_WORKLOADS = ("llama2-13b-blockmgr",)
 

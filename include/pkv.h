@@ -67,13 +67,19 @@ typedef enum pkv_status {
 #define PKV_DEVERR_TIMEOUT 0x8u  /* a bounded on-chip wait gave up (the call's results are invalid) */
 #define PKV_DEVERR_LAYOUT 0x10u  /* decode: shared memory window not 1 KB-aligned (results invalid) */
 
-/* Describes one physical pool (k_cache and v_cache share it). */
+/* Describes one physical pool (k_cache and v_cache share it).  Calls that
+ * move whole blocks (copy, device copy, swap) size them by kv_dtype; write,
+ * decode and prefill accept only their own element type (else PKV_EINVAL). */
 typedef struct pkv_pool {
     int32_t num_blocks;
     int32_t num_kv_heads;
     int32_t block_size;
     int32_t head_dim;
+    int32_t kv_dtype; /* PKV_KV_BF16 (0) or PKV_KV_E4M3 (1): the element type of k_cache / v_cache */
 } pkv_pool;
+
+#define PKV_KV_BF16 0 /* bf16 elements, 2 bytes */
+#define PKV_KV_E4M3 1 /* FP8 e4m3 codes, 1 byte (see pkv_write_fp8) */
 
 /*
  * pkv_write -- slot-mapped write of new tokens' K/V into their blocks.

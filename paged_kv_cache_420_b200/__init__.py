@@ -39,9 +39,12 @@ class PkvError(RuntimeError):
         super().__init__(f"{what}: {STATUS_NAMES.get(status, status)} ({status_string(status)})")
 
 
+KV_BF16, KV_E4M3 = 0, 1  # pkv_pool.kv_dtype
+
+
 class _Pool(ctypes.Structure):
     _fields_ = [("num_blocks", ctypes.c_int32), ("num_kv_heads", ctypes.c_int32),
-                ("block_size", ctypes.c_int32), ("head_dim", ctypes.c_int32)]
+                ("block_size", ctypes.c_int32), ("head_dim", ctypes.c_int32), ("kv_dtype", ctypes.c_int32)]
 
 
 _lib: Optional[ctypes.CDLL] = None
@@ -119,7 +122,12 @@ def _pool(k_cache: torch.Tensor) -> _Pool:
     if k_cache.dim() != 4:
         raise ValueError("cache must be [num_blocks, num_kv_heads, block_size, head_dim]")
     nb, hkv, bs, d = k_cache.shape
-    return _Pool(nb, hkv, bs, d)
+    return _Pool(nb, hkv, bs, d, KV_E4M3 if k_cache.dtype == torch.uint8 else KV_BF16)
+
+
+def _need_cache(t: torch.Tensor, name: str):
+    """A pool tensor: bf16, or uint8 e4m3 codes."""
+    _need(t, name, torch.uint8 if t.dtype == torch.uint8 else torch.bfloat16)
 
 
 def _need(t: torch.Tensor, name: str, dtype, cuda=True):
@@ -148,9 +156,11 @@ def pkv_write(k: torch.Tensor, v: torch.Tensor, slot_mapping: torch.Tensor, k_ca
 
 
 def pkv_copy_blocks(src_dst_pairs, k_cache: torch.Tensor, v_cache: torch.Tensor, stream=None) -> None:
-    """Copies block src -> dst of both caches for every (src, dst) host pair."""
+    """Copies block src -> dst of both caches for every (src, dst) host pair (bf16 or e4m3 pools)."""
     for t, n in ((k_cache, "k_cache"), (v_cache, "v_cache")):
-        _need(t, n, torch.bfloat16)
+        _need_cache(t, n)
+    if v_cache.dtype != k_cache.dtype:
+        raise TypeError("k_cache and v_cache must have the same element type")
     pairs = np.ascontiguousarray(np.asarray(src_dst_pairs, dtype=np.int32).reshape(-1, 2))
     st = load_library().pkv_copy_blocks(pairs.ctypes.data_as(ctypes.c_void_p), pairs.shape[0], _ptr(k_cache),
                                         _ptr(v_cache), _pool(k_cache), _stream(stream))
@@ -158,8 +168,8 @@ def pkv_copy_blocks(src_dst_pairs, k_cache: torch.Tensor, v_cache: torch.Tensor,
 
 
 def _host_blocks(t: torch.Tensor, name: str, k_cache: torch.Tensor, n: int):
-    if t.dtype != torch.bfloat16 or not t.is_contiguous() or t.is_cuda:
-        raise ValueError(f"{name} must be a contiguous bf16 host tensor")
+    if t.dtype != k_cache.dtype or not t.is_contiguous() or t.is_cuda:
+        raise ValueError(f"{name} must be a contiguous host tensor of the pool's element type")
     if not t.is_pinned():
         raise ValueError(f"{name} must be pinned host memory")
     if t.numel() < n * k_cache[0].numel():
@@ -175,7 +185,7 @@ def pkv_swap_out(k_cache: torch.Tensor, v_cache: torch.Tensor, block_ids, host_k
     """host_k[i] / host_v[i] := block block_ids[i] of k_cache / v_cache (pinned
     host tensors of at least len(block_ids) blocks); asynchronous on the stream."""
     for t, n in ((k_cache, "k_cache"), (v_cache, "v_cache")):
-        _need(t, n, torch.bfloat16)
+        _need_cache(t, n)
     ids = _block_ids(block_ids)
     _host_blocks(host_k, "host_k", k_cache, ids.shape[0])
     _host_blocks(host_v, "host_v", k_cache, ids.shape[0])
@@ -188,7 +198,7 @@ def pkv_swap_in(host_k: torch.Tensor, host_v: torch.Tensor, block_ids, k_cache: 
                 v_cache: torch.Tensor, stream=None) -> None:
     """Block block_ids[i] of k_cache / v_cache := host_k[i] / host_v[i] (ids distinct)."""
     for t, n in ((k_cache, "k_cache"), (v_cache, "v_cache")):
-        _need(t, n, torch.bfloat16)
+        _need_cache(t, n)
     ids = _block_ids(block_ids)
     _host_blocks(host_k, "host_k", k_cache, ids.shape[0])
     _host_blocks(host_v, "host_v", k_cache, ids.shape[0])
@@ -334,7 +344,7 @@ def copy_blocks_dev(cow_pairs: torch.Tensor, num_pairs: torch.Tensor, k_cache: t
     _need(cow_pairs, "cow_pairs", torch.int32)
     _need(num_pairs, "num_pairs", torch.int32)
     for t, n in ((k_cache, "k_cache"), (v_cache, "v_cache")):
-        _need(t, n, torch.bfloat16)
+        _need_cache(t, n)
     _check(load_library().pkv_copy_blocks_dev(_ptr(cow_pairs), _ptr(num_pairs), cow_pairs.shape[0], _ptr(k_cache),
                                               _ptr(v_cache), _pool(k_cache), _stream(stream)), "pkv_copy_blocks_dev")
 

@@ -57,12 +57,16 @@ int sm_count(int dev) {
 pkv_status check_pool(const pkv_pool &pool) {
     if (pool.num_blocks <= 0 || pool.num_kv_heads <= 0 || pool.block_size <= 0 || pool.head_dim <= 0)
         return PKV_EINVAL;
+    if (pool.kv_dtype != PKV_KV_BF16 && pool.kv_dtype != PKV_KV_E4M3) return PKV_EINVAL;
     if (pool.head_dim != 64 && pool.head_dim != 128) return PKV_EUNSUPPORTED;
     if (pool.block_size % 16 != 0 || pool.block_size > 1024) return PKV_EUNSUPPORTED;
     const long long rows = (long long)pool.num_blocks * pool.num_kv_heads * pool.block_size;
     if (rows >= (1ll << 31) - 1) return PKV_EUNSUPPORTED;  // TMA row coordinates are int32
     return PKV_OK;
 }
+
+// Bytes of one K/V element of the pool.
+int elem_bytes(const pkv_pool &pool) { return pool.kv_dtype == PKV_KV_E4M3 ? 1 : 2; }
 
 pkv_status launch_status() {
     const cudaError_t e = cudaGetLastError();
@@ -331,7 +335,7 @@ pkv_status swap_blocks(const int32_t *block_ids, int32_t n, void *k_cache, void 
     uint8_t *hk = static_cast<uint8_t *>(mapped_host_pointer(host_k));
     uint8_t *hv = static_cast<uint8_t *>(mapped_host_pointer(host_v));
     if (!hk || !hv) return PKV_EINVAL;
-    const size_t block_bytes = (size_t)pool.num_kv_heads * pool.block_size * pool.head_dim * 2;
+    const size_t block_bytes = (size_t)pool.num_kv_heads * pool.block_size * pool.head_dim * elem_bytes(pool);
     pkv::SwapParams p;
     p.pool_k = static_cast<uint4 *>(k_cache);
     p.pool_v = static_cast<uint4 *>(v_cache);
@@ -390,6 +394,7 @@ pkv_status decode_impl(const void *q, const void *k_cache, const void *v_cache, 
                        int32_t num_kv_heads, void *out, pkv_pool pool, int32_t max_context_len,
                        int32_t partition_tokens, void *workspace, size_t workspace_bytes, pkv_stream_t stream) {
     const bool kv8 = k_scale != nullptr;
+    if (pool.kv_dtype != (kv8 ? PKV_KV_E4M3 : PKV_KV_BF16)) return PKV_EINVAL;
     const pkv_status ps = check_pool(pool);
     if (ps != PKV_OK) return ps;
     if (num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || max_blocks_per_seq <= 0 || max_context_len < 0)
@@ -462,7 +467,7 @@ pkv_status decode_impl(const void *q, const void *k_cache, const void *v_cache, 
 
 extern "C" {
 
-int32_t pkv_version(void) { return 10000; }
+int32_t pkv_version(void) { return 10100; }
 
 const char *pkv_status_string(pkv_status s) {
     switch (s) {
@@ -481,6 +486,7 @@ pkv_status pkv_write(const void *k, const void *v, const int64_t *slot_mapping, 
                      void *v_cache, pkv_pool pool, pkv_stream_t stream) {
     const pkv_status ps = check_pool(pool);
     if (ps != PKV_OK) return ps;
+    if (pool.kv_dtype != PKV_KV_BF16) return PKV_EINVAL;
     if (num_tokens < 0) return PKV_EINVAL;
     if (num_tokens == 0) return PKV_OK;
     if (!k || !v || !slot_mapping || !k_cache || !v_cache) return PKV_EINVAL;
@@ -529,7 +535,7 @@ pkv_status pkv_copy_blocks(const int32_t *src_dst_pairs, int32_t num_pairs, void
     pkv::CopyParams p;
     p.k_cache = static_cast<uint4 *>(k_cache);
     p.v_cache = static_cast<uint4 *>(v_cache);
-    p.vec_per_block = (int64_t)pool.num_kv_heads * pool.block_size * pool.head_dim / 8;
+    p.vec_per_block = (int64_t)pool.num_kv_heads * pool.block_size * pool.head_dim * elem_bytes(pool) / 16;
     const long long per_cta = pkv::kCopyThreads * pkv::kCopyVecPerThread;
     const unsigned gx = (unsigned)((p.vec_per_block + per_cta - 1) / per_cta);
     for (int base = 0; base < num_pairs; base += pkv::kMaxPairsPerLaunch) {
@@ -612,6 +618,7 @@ pkv_status pkv_write_fp8(const void *k, const void *v, const int64_t *slot_mappi
                          pkv_stream_t stream) {
     const pkv_status ps = check_pool(pool);
     if (ps != PKV_OK) return ps;
+    if (pool.kv_dtype != PKV_KV_E4M3) return PKV_EINVAL;
     if (num_tokens < 0) return PKV_EINVAL;
     if (num_tokens == 0) return PKV_OK;
     if (!k || !v || !slot_mapping || !k_cache || !v_cache || !k_scale || !v_scale) return PKV_EINVAL;
@@ -652,6 +659,7 @@ pkv_status paged_attn_prefill(const void *q, const void *k_cache, const void *v_
                               int32_t max_context_len, void *workspace, size_t workspace_bytes, pkv_stream_t stream) {
     const pkv_status ps = check_pool(pool);
     if (ps != PKV_OK) return ps;
+    if (pool.kv_dtype != PKV_KV_BF16) return PKV_EINVAL;
     if (num_seqs < 0 || num_tokens < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || max_blocks_per_seq <= 0 ||
         max_context_len < 0 || max_query_len < 0)
         return PKV_EINVAL;
@@ -858,7 +866,7 @@ pkv_status pkv_copy_blocks_dev(const int32_t *cow_pairs, const int32_t *num_pair
     if (!cow_pairs || !num_pairs || !k_cache || !v_cache) return PKV_EINVAL;
     if (!aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(cow_pairs, 4) || !aligned(num_pairs, 4))
         return PKV_EINVAL;
-    const int64_t vec = (int64_t)pool.num_kv_heads * pool.block_size * pool.head_dim / 8;
+    const int64_t vec = (int64_t)pool.num_kv_heads * pool.block_size * pool.head_dim * elem_bytes(pool) / 16;
     const long long per_cta = pkv::kCopyDevThreads * pkv::kCopyDevVec;
     const unsigned gx = (unsigned)((vec + per_cta - 1) / per_cta);
     for (int base = 0; base < max_pairs; base += 65535) {  // grid.y limit

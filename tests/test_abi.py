@@ -36,7 +36,7 @@ def test_library_loads_and_exports_every_declared_symbol():
 
 
 def test_status_strings_and_version():
-    assert pkv.version() == 10000
+    assert pkv.version() == 10100
     for code in range(7):
         assert pkv.status_string(code)
     assert pkv.status_string(99) == "unknown status"
@@ -132,6 +132,21 @@ def test_prefill_validation():
     assert _prefill(lib, ws_bytes=16) == EINVAL
     assert _prefill(lib, mbs=0) == EINVAL
     assert _prefill(lib, pool=_pool(hkv=2, bs=8)) == EUNSUP
+
+
+def test_pool_element_type_validation():
+    lib = pkv.load_library()
+    ok = _pool()
+    fp8 = _Pool(8, 2, 16, 128, 1)
+    bad = _Pool(8, 2, 16, 128, 2)
+    assert _decode(lib, pool=bad) == EINVAL          # unknown element type
+    assert _decode(lib, pool=fp8) == EINVAL          # bf16 decode on an e4m3 pool
+    assert lib.pkv_write(FAKE, FAKE, FAKE, 4, FAKE, FAKE, fp8, None) == EINVAL
+    f = lib.pkv_write_fp8
+    f.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int32, ctypes.c_void_p,
+                  ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, _Pool, ctypes.c_void_p]
+    assert f(FAKE, FAKE, FAKE, 4, FAKE, FAKE, FAKE, FAKE, ok, None) == EINVAL   # e4m3 write on a bf16 pool
+    assert _prefill(lib, pool=_Pool(8, 2, 16, 128, 1)) == EINVAL
 
 
 def test_workspace_size():

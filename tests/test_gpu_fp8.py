@@ -140,3 +140,42 @@ def test_named_workload_fp8_full_size_sampled():
     ref = oracle.paged_attention_fp8(w.q[pick].cpu(), k8.cpu().numpy(), v8.cpu().numpy(), ks.cpu().numpy(),
                                      vs.cpu().numpy(), w.block_tables[pick], w.context_lens[pick], w.scale)
     assert_attention_close(out[pick], ref, "fp8 llama2-13b sampled")
+
+
+def _as_u16(a):
+    """An e4m3 pool [NB, Hkv, bs, D] viewed as 2-byte units [NB, Hkv, bs, D/2]:
+    whole-block copies move the same bytes either way."""
+    a = np.ascontiguousarray(a)
+    return a.view(np.uint16).reshape(a.shape[:-1] + (a.shape[-1] // 2,))
+
+
+def test_fp8_pool_copy_and_swap_match_oracle():
+    rng = np.random.default_rng(4)
+    NB, Hkv, bs, D = 64, 8, 16, 128
+    k8 = rng.integers(0, 256, (NB, Hkv, bs, D)).astype(np.uint8)
+    v8 = rng.integers(0, 256, (NB, Hkv, bs, D)).astype(np.uint8)
+    kd, vd = torch.from_numpy(k8).cuda(), torch.from_numpy(v8).cuda()
+    pairs = np.array([[3, 40], [7, 41], [63, 0], [12, 13]], np.int32)
+    pkv.pkv_copy_blocks(pairs, kd, vd)
+    torch.cuda.synchronize()
+    ok, ov = oracle.copy_blocks(_as_u16(k8), _as_u16(v8), pairs)
+    assert np.array_equal(_as_u16(kd.cpu().numpy()), ok) and np.array_equal(_as_u16(vd.cpu().numpy()), ov)
+    # the device-sourced copy, with a count on the device
+    pd = torch.from_numpy(np.array([[40, 50], [41, 51], [5, 52]], np.int32)).cuda()
+    pkv.copy_blocks_dev(pd, torch.tensor([2], dtype=torch.int32, device="cuda"), kd, vd)
+    torch.cuda.synchronize()
+    ok, ov = oracle.copy_blocks(ok, ov, np.array([[40, 50], [41, 51]], np.int32))
+    assert np.array_equal(_as_u16(kd.cpu().numpy()), ok) and np.array_equal(_as_u16(vd.cpu().numpy()), ov)
+    # swap out and back into other blocks
+    ids = np.array([50, 3, 63], np.int32)
+    hk = torch.empty((3, Hkv, bs, D), dtype=torch.uint8).pin_memory()
+    hv = torch.empty_like(hk).pin_memory()
+    pkv.pkv_swap_out(kd, vd, ids, hk, hv)
+    torch.cuda.synchronize()
+    ohk, ohv = oracle.swap_out(ok, ov, ids)
+    assert np.array_equal(_as_u16(hk.numpy()), ohk) and np.array_equal(_as_u16(hv.numpy()), ohv)
+    dst = np.array([20, 21, 22], np.int32)
+    pkv.pkv_swap_in(hk, hv, dst, kd, vd)
+    torch.cuda.synchronize()
+    ok, ov = oracle.swap_in(ok, ov, ohk, ohv, dst)
+    assert np.array_equal(_as_u16(kd.cpu().numpy()), ok) and np.array_equal(_as_u16(vd.cpu().numpy()), ov)
