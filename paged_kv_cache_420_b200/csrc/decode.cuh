@@ -173,15 +173,10 @@ struct DecodeSmem {
     static constexpr int kBoxes = D * kElem / 128;        // boxes per row of a tile
     static constexpr int kTile = kStageTok * D * kElem;   // one K (or V) stage tile
     static constexpr int kStage = 2 * kTile;
-    // FP8 pool on the tensor-core path (GP >= 4): each consumer warp converts
-    // its stage's V tile to f16 (bf16 tile layout) in a scratch of its own
-    static constexpr int kTileF16 = kStageTok * D * 2;
-    static constexpr int kScratch = (KV8 && GP >= 4) ? kW * kTileF16 : 0;
     static constexpr int kQBuf = GP * D * 2;              // the query heads of one kv head
     static constexpr int kMergeStride = D + 4;            // floats, padded against bank conflicts
     static constexpr int oTiles = 0;
-    static constexpr int oScratch = oTiles + NS * kStage;
-    static constexpr int oQ = oScratch + kScratch;
+    static constexpr int oQ = oTiles + NS * kStage;
     static constexpr int oMergeO = oQ + 2 * kQBuf;
     static constexpr int oMergeM = oMergeO + kW * GP * kMergeStride * 4;
     static constexpr int oMergeL = oMergeM + kW * GP * 4;
@@ -459,39 +454,34 @@ struct SimtState {
 };
 
 // ------------------------------------------- tensor-core path (3 <= g <= 16) --
-// An FP8 stage tile (16 rows x 128 codes, tile_addr8 layout) -> the same tile
-// as f16 in the bf16 tile layout (tile_addr), by one warp: lane handles 16-code
-// chunks, one 16-byte load, eight pair conversions, two 16-byte stores.
-__device__ __forceinline__ void convert_tile_f16(uint32_t src8, uint32_t dst16, int lane) {
-#pragma unroll
-    for (int i = lane; i < kStageTok * 8; i += 32) {
-        const int r = i >> 3, ch = i & 7;
-        uint32_t w[4];
-        asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
-                     : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3])
-                     : "r"(tile_addr8(src8, r, ch * 16)));
-        uint32_t h[8];
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            h[2 * k] = f16x2_from_e4m3x2(w[k] & 0xffffu);
-            h[2 * k + 1] = f16x2_from_e4m3x2(w[k] >> 16);
-        }
-        asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(tile_addr(dst16, r, ch * 16)), "r"(h[0]),
-                     "r"(h[1]), "r"(h[2]), "r"(h[3])
-                     : "memory");
-        asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(tile_addr(dst16, r, ch * 16 + 8)), "r"(h[4]),
-                     "r"(h[5]), "r"(h[6]), "r"(h[7])
-                     : "memory");
-    }
+// 8-bit transposing load of a 16 x 16 byte tile (rows from lanes 0-15): lane l
+// receives rows 4(l%4) .. 4(l%4)+3 of byte column l/4 in r0 and of column
+// l/4 + 8 in r1, row i of each group in byte i.
+__device__ __forceinline__ void ldmatrix_b8_trans(uint32_t addr, uint32_t &r0, uint32_t &r1) {
+    asm volatile("ldmatrix.sync.aligned.m16n16.x1.trans.shared.b8 {%0, %1}, [%2];" : "=r"(r0), "=r"(r1) : "r"(addr));
+}
+
+// Token order of the FP8 tensor-core stage: A row (and k slot) r of the 16
+// tokens holds token perm16(r) = 4j + {0, 1} for r = 2j + {0, 1} and
+// 4j + 2 + {0, 1} for r = 8 + 2j + {0, 1}.  It makes the S^T rows that
+// movmatrix turns into P^T's B fragment match the V^T A fragment that the
+// 8-bit transposing load delivers (tokens 4j .. 4j+3 per lane).
+__device__ __forceinline__ int perm16(int r) {
+    return r < 8 ? 4 * (r >> 1) + (r & 1) : 4 * ((r - 8) >> 1) + 2 + (r & 1);
 }
 
 // H: an FP8 pool, f16 operands (the codes are exact in f16; q is converted to
-// f16 and P packed as f16), otherwise bf16.  With H the K operand comes
-// straight from the e4m3 stage tile: lane l (j = l % 4) loads the 4 codes of
-// columns k0 + 4j .. 4j + 3 of its rows as one word, and the pairs (4j, 4j+1)
-// and (4j+2, 4j+3) fill the k slots (2j, 2j+1) and (2j+8, 2j+9) of the
-// m16n8k16 A fragment.  The dot product does not depend on the order of k,
-// so q's B fragment takes its columns in the same order.
+// f16 and P packed as f16), otherwise bf16.  With H both operands come
+// straight from the e4m3 stage tiles:
+//   K: lane l (j = l % 4) loads the 4 codes of columns k0 + 4j .. 4j + 3 of
+//      its two rows as one word each; the pairs (4j, 4j+1) and (4j+2, 4j+3)
+//      fill the k slots (2j, 2j+1) and (2j+8, 2j+9) of the m16n8k16 A
+//      fragment, and q's B fragment takes its columns in the same order (the
+//      dot product does not depend on the order of k).  The rows are the
+//      tokens in perm16 order.
+//   V: one 8-bit transposing load per 16 head-dim columns gives lane l the
+//      codes of tokens 4j .. 4j+3 at columns l/4 and l/4 + 8, which in perm16
+//      order are exactly its A fragment of V^T.
 template <int D, int NT, bool H = false>
 struct MmaState {
     static constexpr int KS = D / 16;  // k-steps of QK^T
@@ -556,8 +546,10 @@ struct MmaState {
             if constexpr (H) {
                 uint32_t w0, w1;
                 const int c = kk * 16 + 4 * (lane & 3);
-                asm volatile("ld.shared.u32 %0, [%1];" : "=r"(w0) : "r"(tile_addr8(ktile, lane >> 2, c)));
-                asm volatile("ld.shared.u32 %0, [%1];" : "=r"(w1) : "r"(tile_addr8(ktile, (lane >> 2) + 8, c)));
+                asm volatile("ld.shared.u32 %0, [%1];" : "=r"(w0) : "r"(tile_addr8(ktile, perm16(lane >> 2), c)));
+                asm volatile("ld.shared.u32 %0, [%1];"
+                             : "=r"(w1)
+                             : "r"(tile_addr8(ktile, perm16((lane >> 2) + 8), c)));
                 a0 = f16x2_from_e4m3x2(w0 & 0xffffu);
                 a1 = f16x2_from_e4m3x2(w1 & 0xffffu);
                 a2 = f16x2_from_e4m3x2(w0 >> 16);
@@ -578,8 +570,8 @@ struct MmaState {
         for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
             for (int c = 0; c < 4; ++c) s[nt][c] += s2[nt][c];
-        const int t0 = lane >> 2;  // tokens t0 and t0 + 8
-        const bool ok0 = t0 < valid, ok1 = t0 + 8 < valid;
+        const int t0 = lane >> 2;  // rows t0 and t0 + 8 (tokens, in perm16 order with H)
+        const bool ok0 = (H ? perm16(t0) : t0) < valid, ok1 = (H ? perm16(t0 + 8) : t0 + 8) < valid;
         uint32_t pb[NT][2];
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
@@ -618,21 +610,32 @@ struct MmaState {
                 }
             }
         }
-        // token masks of this thread's V^T operand halves: tokens 2(l%4)+{0,1} and +8
+        // token masks of this thread's V^T operand halves: k slots 2(l%4)+{0,1}
+        // and +8, i.e. tokens 2(l%4)+{0,1} and +8 (with H: 4(l%4)+{0,1} and +{2,3})
         uint32_t mask01 = 0xffffffffu, mask23 = 0xffffffffu;
         if (valid < 16) {
-            const int j0 = 2 * (lane & 3);
+            const int j0 = H ? 4 * (lane & 3) : 2 * (lane & 3);
+            const int j2 = H ? j0 + 2 : j0 + 8;
             mask01 = (j0 < valid ? 0x0000ffffu : 0u) | (j0 + 1 < valid ? 0xffff0000u : 0u);
-            mask23 = (j0 + 8 < valid ? 0x0000ffffu : 0u) | (j0 + 9 < valid ? 0xffff0000u : 0u);
+            mask23 = (j2 < valid ? 0x0000ffffu : 0u) | (j2 + 1 < valid ? 0xffff0000u : 0u);
         }
         // O^T[d][head] += V^T . P^T
 #pragma unroll
         for (int mt = 0; mt < MT; ++mt) {
-            // matrices (stored rows = tokens): (tok 0-7, d0..+7), (tok 0-7, d0+8..), (tok 8-15, d0..), (tok 8-15, d0+8..)
-            const int row = ri + 8 * (mi >> 1);
-            const int col = mt * 16 + 8 * (mi & 1);
             uint32_t a0, a1, a2, a3;
-            ldmatrix_x4_trans(tile_addr(vtile, row, col), a0, a1, a2, a3);
+            if constexpr (H) {
+                uint32_t r0, r1;
+                ldmatrix_b8_trans(tile_addr8(vtile, lane & 15, mt * 16), r0, r1);
+                a0 = f16x2_from_e4m3x2(r0 & 0xffffu);  // d = l/4: tokens 4j, 4j+1
+                a1 = f16x2_from_e4m3x2(r1 & 0xffffu);  // d = l/4 + 8
+                a2 = f16x2_from_e4m3x2(r0 >> 16);      // d = l/4: tokens 4j+2, 4j+3
+                a3 = f16x2_from_e4m3x2(r1 >> 16);
+            } else {
+                // matrices (stored rows = tokens): (tok 0-7, d0..+7), (tok 0-7, d0+8..), (tok 8-15, d0..), (tok 8-15, d0+8..)
+                const int row = ri + 8 * (mi >> 1);
+                const int col = mt * 16 + 8 * (mi & 1);
+                ldmatrix_x4_trans(tile_addr(vtile, row, col), a0, a1, a2, a3);
+            }
             a0 &= mask01; a1 &= mask01; a2 &= mask23; a3 &= mask23;
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt) {
@@ -863,12 +866,7 @@ __global__ void __launch_bounds__(kDecodeThreads) paged_decode_kernel(const __gr
                 if constexpr (PATH == 0) {
                     st0.stage(kt, kt + L::kTile, si.valid, lane);
                 } else if constexpr (KV8) {
-                    // K is read as codes; V goes through this warp's f16 copy
-                    const uint32_t sv = smem_u32(smem + L::oScratch) + w * L::kTileF16;
-                    convert_tile_f16(kt + L::kTile, sv, lane);
-                    __syncwarp();
-                    st1.stage(kt, sv, si.valid, lane, scale_log2 * __ldg(p.k_scale + si.h));
-                    __syncwarp();  // the next stage's conversion overwrites the scratch
+                    st1.stage(kt, kt + L::kTile, si.valid, lane, scale_log2 * __ldg(p.k_scale + si.h));
                 } else {
                     st1.stage(kt, kt + L::kTile, si.valid, lane, scale_log2);
                 }
