@@ -293,8 +293,8 @@ pkv_status paged_attn_prefill(const void *q, const void *k_cache, const void *v_
  *
  * paged_attn_decode_fp8: as paged_attn_decode over an FP8 pool, reading
  * K = e4m3(code) * k_scale[h] and V = e4m3(code) * v_scale[h].  Supported at
- * head_dim 128 (else PKV_EUNSUPPORTED) for every GQA group <= 16: groups 1-2
- * on CUDA cores, larger groups on the tensor cores; the codes are multiplied
+ * head_dim 128 (else PKV_EUNSUPPORTED) for every GQA group <= 16: group 1
+ * on CUDA cores, groups 2-16 on the tensor cores; the codes are multiplied
  * exactly as f16 with fp32 accumulation.  The workspace is the same as
  * paged_attn_decode's.
  */

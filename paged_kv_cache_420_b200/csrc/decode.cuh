@@ -19,11 +19,11 @@
 // goes to the workspace and a reduce kernel merges them by log-sum-exp.
 //
 // Two consumer arithmetic paths:
-//  * GQA group g <= 2 (MHA): CUDA cores.  A lane owns D/32 elements of every
-//    row; q.k partial sums of the 16 tokens are reduced by a transposing
-//    butterfly of warp shuffles; p is broadcast by shuffles for the PV sum.
-//  * 3 <= g <= 16: the g query heads of one kv head form a dense tile, so
-//    QK^T and PV run on tensor cores (mma.sync m16n8k16 bf16, fp32 accumulate):
+//  * MHA (g = 1): CUDA cores.  A lane owns D/32 elements of every row; q.k
+//    partial sums of the 16 tokens are reduced by a transposing butterfly of
+//    warp shuffles; p is broadcast by shuffles for the PV sum.
+//  * 2 <= g <= 16: the g query heads of one kv head form a tile, so QK^T and
+//    PV run on tensor cores (mma.sync m16n8k16 bf16, fp32 accumulate):
 //    S^T[16 tokens x 8 heads] = K_tile . Q^T, O^T[D x 8 heads] += V^T . P^T,
 //    with P^T moved from accumulator to operand layout by movmatrix.
 #pragma once
@@ -250,45 +250,42 @@ __device__ __forceinline__ float fma_f16hi(uint32_t a, uint32_t b, float acc) {
     return r;
 }
 
-// ----------------------------------------------- CUDA-core path (g <= 2) ----
+// ------------------------------------------------ CUDA-core path (g = 1) ----
+// One query head per kv head (MHA).  A lane owns EPL = D/32 contiguous
+// elements of every row.
 // KV8: the stage tiles hold e4m3 codes.  q is kept as exact f16 pairs, K and V
 // codes are converted to f16 (exactly) and multiplied in mixed precision with
 // fp32 accumulation; the K scale times scale * log2 e multiplies each summed
 // score, and the V scale is applied to the final output.
-template <int D, int G, bool KV8 = false>
+template <int D, bool KV8 = false>
 struct SimtState {
     static constexpr int EPL = D / 32;  // elements per lane
-    float q[G][EPL];
-    uint32_t q16[G][EPL / 2];  // KV8: q as f16 pairs
-    float kscale;              // KV8: scale * log2(e) * k_scale of the kv head
-    float acc[G][EPL];
-    float m[G];
-    float l_part;  // this lane's share of l for head (lane / 16) (G = 2) or head 0
+    float q[EPL];
+    uint32_t q16[EPL / 2];  // KV8: q as f16 pairs
+    float kscale;           // KV8: scale * log2(e) * k_scale of the kv head
+    float acc[EPL];
+    float m;
+    float l_part;  // this lane's share of l
 
     __device__ __forceinline__ void reset() {
+        m = PKV_NEG_INF;
 #pragma unroll
-        for (int j = 0; j < G; ++j) {
-            m[j] = PKV_NEG_INF;
-#pragma unroll
-            for (int e = 0; e < EPL; ++e) acc[j][e] = 0.f;
-        }
+        for (int e = 0; e < EPL; ++e) acc[e] = 0.f;
         l_part = 0.f;
     }
 
     __device__ __forceinline__ void load_q(const __nv_bfloat16 *qs, int lane, float scale_log2) {
         kscale = scale_log2;
 #pragma unroll
-        for (int j = 0; j < G; ++j)
-#pragma unroll
-            for (int e = 0; e < EPL; e += 2) {
-                const uint32_t pr = *reinterpret_cast<const uint32_t *>(qs + j * D + lane * EPL + e);
-                if constexpr (KV8) {
-                    q16[j][e / 2] = f16x2_from_f32(bf16lo_to_f32(pr), bf16hi_to_f32(pr));
-                } else {
-                    q[j][e] = bf16lo_to_f32(pr) * scale_log2;
-                    q[j][e + 1] = bf16hi_to_f32(pr) * scale_log2;
-                }
+        for (int e = 0; e < EPL; e += 2) {
+            const uint32_t pr = *reinterpret_cast<const uint32_t *>(qs + lane * EPL + e);
+            if constexpr (KV8) {
+                q16[e / 2] = f16x2_from_f32(bf16lo_to_f32(pr), bf16hi_to_f32(pr));
+            } else {
+                q[e] = bf16lo_to_f32(pr) * scale_log2;
+                q[e + 1] = bf16hi_to_f32(pr) * scale_log2;
             }
+        }
     }
 
     // KV8: this lane's 4 codes of row r as two f16 pairs.
@@ -315,23 +312,19 @@ struct SimtState {
     }
 
     __device__ __forceinline__ void stage(uint32_t ktile, uint32_t vtile, int valid, int lane) {
-        constexpr int NV = 16 * G;
-        float v[NV];
-        // q.k partial sums v[j*16 + r] for head j, token r; tokens r and r+1
-        // share one packed fp32x2 FMA per element.
+        float v[16];
+        // q.k partial sums v[r] of token r; tokens r and r+1 share one packed
+        // fp32x2 FMA per element.
         if constexpr (KV8) {
             static_assert(EPL == 4, "FP8 stage tiles are 128-byte rows (head dim 128)");
 #pragma unroll
             for (int r = 0; r < 16; ++r) {
                 uint32_t k16[2];
                 load_row8(ktile, r, lane, k16);
-#pragma unroll
-                for (int j = 0; j < G; ++j) {
-                    float d = fma_f16lo(q16[j][0], k16[0], 0.f);
-                    d = fma_f16hi(q16[j][0], k16[0], d);
-                    d = fma_f16lo(q16[j][1], k16[1], d);
-                    v[j * 16 + r] = fma_f16hi(q16[j][1], k16[1], d);
-                }
+                float d = fma_f16lo(q16[0], k16[0], 0.f);
+                d = fma_f16hi(q16[0], k16[0], d);
+                d = fma_f16lo(q16[1], k16[1], d);
+                v[r] = fma_f16hi(q16[1], k16[1], d);
             }
         } else {
 #pragma unroll
@@ -339,27 +332,24 @@ struct SimtState {
                 float x0[EPL], x1[EPL];
                 load_row(ktile, r, lane, x0);
                 load_row(ktile, r + 1, lane, x1);
+                float d0 = 0.f, d1 = 0.f;
 #pragma unroll
-                for (int j = 0; j < G; ++j) {
-                    float d0 = 0.f, d1 = 0.f;
-#pragma unroll
-                    for (int e = 0; e < EPL; ++e) fma_f32x2(d0, d1, q[j][e], q[j][e], x0[e], x1[e]);
-                    v[j * 16 + r] = d0;
-                    v[j * 16 + r + 1] = d1;
-                }
+                for (int e = 0; e < EPL; ++e) fma_f32x2(d0, d1, q[e], q[e], x0[e], x1[e]);
+                v[r] = d0;
+                v[r + 1] = d1;
             }
         }
-        // Transposing butterfly: after it, lane holds the full 32-lane sum of
-        // value index idx(lane): G = 1 -> token lane >> 1; G = 2 -> head
-        // lane >> 4, token lane & 15.
-        int n = NV;
+        // Transposing butterfly: each step halves the values a lane keeps and
+        // sums its half with the partner's; after it lanes 2t and 2t+1 both
+        // hold the full 32-lane sum of token t.
+        int n = 16;
 #pragma unroll
         for (int mask = 16; mask >= 1; mask >>= 1) {
             if (n > 1) {
                 const bool upper = (lane & mask) != 0;
                 n >>= 1;
 #pragma unroll
-                for (int i = 0; i < NV / 2; ++i) {
+                for (int i = 0; i < 8; ++i) {
                     if (i < n) {
                         const float send = upper ? v[i] : v[i + n];
                         const float keep = upper ? v[i + n] : v[i];
@@ -370,90 +360,58 @@ struct SimtState {
                 v[0] += __shfl_xor_sync(0xffffffffu, v[0], mask);
             }
         }
-        const int my_tok = (G == 1) ? (lane >> 1) : (lane & 15);
-        const int my_head = (G == 1) ? 0 : (lane >> 4);
+        const int my_tok = lane >> 1;
         const float score = (my_tok < valid) ? (KV8 ? v[0] * kscale : v[0]) : PKV_NEG_INF;
-        // stage max per head (one warp reduction each), lazy rescale
-        float mx[G];
-        if constexpr (G == 1) {
-            mx[0] = warp_max_f32(score);
-        } else {
-            mx[0] = warp_max_f32(my_head == 0 ? score : PKV_NEG_INF);
-            mx[1] = warp_max_f32(my_head == 1 ? score : PKV_NEG_INF);
-        }
+        // stage max (one warp reduction), lazy rescale
+        const float mx = warp_max_f32(score);
+        if (mx > m + kRescaleSlack) {  // warp-uniform, rare after the first stage
+            const float alpha = exp2f(m - mx);
+            m = mx;
 #pragma unroll
-        for (int j = 0; j < G; ++j) {
-            if (mx[j] > m[j] + kRescaleSlack) {  // warp-uniform, rare after the first stage
-                const float alpha = exp2f(m[j] - mx[j]);
-                m[j] = mx[j];
-#pragma unroll
-                for (int e = 0; e < EPL; ++e) acc[j][e] *= alpha;
-                if (G == 1 || my_head == j) l_part *= alpha;
-            }
+            for (int e = 0; e < EPL; ++e) acc[e] *= alpha;
+            l_part *= alpha;
         }
-        const float my_m = (G == 1 || my_head == 0) ? m[0] : m[G - 1];
-        const float pr = exp2f(score - my_m);
+        const float pr = exp2f(score - m);
         l_part += pr;
         // KV8: p as an f16 pair, converted once here and shuffled as such
         const uint32_t pr16 = KV8 ? f16x2_from_f32(pr, pr) : 0u;
-        // PV: broadcast p of each valid token, accumulate its V row (packed
-        // fp32x2 FMA over element pairs)
+        // PV: broadcast p of each valid token (from lane 2r), accumulate its V
+        // row (packed fp32x2 FMA over element pairs)
 #pragma unroll
         for (int r = 0; r < 16; ++r) {
             if (r < valid) {
                 if constexpr (KV8) {
                     uint32_t v16[2];
                     load_row8(vtile, r, lane, v16);
-#pragma unroll
-                    for (int j = 0; j < G; ++j) {
-                        const int src = (G == 1) ? (2 * r) : (j * 16 + r);
-                        const uint32_t p16 = __shfl_sync(0xffffffffu, pr16, src);
-                        acc[j][0] = fma_f16lo(p16, v16[0], acc[j][0]);
-                        acc[j][1] = fma_f16hi(p16, v16[0], acc[j][1]);
-                        acc[j][2] = fma_f16lo(p16, v16[1], acc[j][2]);
-                        acc[j][3] = fma_f16hi(p16, v16[1], acc[j][3]);
-                    }
+                    const uint32_t p16 = __shfl_sync(0xffffffffu, pr16, 2 * r);
+                    acc[0] = fma_f16lo(p16, v16[0], acc[0]);
+                    acc[1] = fma_f16hi(p16, v16[0], acc[1]);
+                    acc[2] = fma_f16lo(p16, v16[1], acc[2]);
+                    acc[3] = fma_f16hi(p16, v16[1], acc[3]);
                 } else {
                     float x[EPL];
                     load_row(vtile, r, lane, x);
+                    const float pj = __shfl_sync(0xffffffffu, pr, 2 * r);
 #pragma unroll
-                    for (int j = 0; j < G; ++j) {
-                        const int src = (G == 1) ? (2 * r) : (j * 16 + r);
-                        const float pj = __shfl_sync(0xffffffffu, pr, src);
-#pragma unroll
-                        for (int e = 0; e < EPL; e += 2)
-                            fma_f32x2(acc[j][e], acc[j][e + 1], pj, pj, x[e], x[e + 1]);
-                    }
+                    for (int e = 0; e < EPL; e += 2) fma_f32x2(acc[e], acc[e + 1], pj, pj, x[e], x[e + 1]);
                 }
             }
         }
     }
 
     // Writes this warp's partial (m, l, acc) into the merge buffers.
-    __device__ __forceinline__ void store_partial(float *mO, float *mM, float *mL, int w, int lane, int stride,
-                                                  int GPn) {
+    __device__ __forceinline__ void store_partial(float *mO, float *mM, float *mL, int w, int lane, int stride) {
+        // lanes 2t and 2t+1 hold the same p: sum over one lane of each pair
         float l = l_part;
-        if (G == 1) {
 #pragma unroll
-            for (int o = 2; o < 32; o <<= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
-        } else {
+        for (int o = 2; o < 32; o <<= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
 #pragma unroll
-            for (int o = 1; o < 16; o <<= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
-        }
-#pragma unroll
-        for (int j = 0; j < G; ++j)
-#pragma unroll
-            for (int e = 0; e < EPL; ++e) mO[(w * GPn + j) * stride + lane * EPL + e] = acc[j][e];
-        if constexpr (G == 1) {
-            if (lane == 0) { mM[w * GPn] = m[0]; mL[w * GPn] = l; }
-        } else {
-            if (lane == 0) { mM[w * GPn] = m[0]; mL[w * GPn] = l; }
-            if (lane == 16) { mM[w * GPn + 1] = m[1]; mL[w * GPn + 1] = l; }
-        }
+        for (int e = 0; e < EPL; ++e) mO[w * stride + lane * EPL + e] = acc[e];
+        if (lane == 0) { mM[w] = m; mL[w] = l; }
     }
 };
 
-// ------------------------------------------- tensor-core path (3 <= g <= 16) --
+// ------------------------------------------- tensor-core path (2 <= g <= 16) --
 // 8-bit transposing load of a 16 x 16 byte tile (rows from lanes 0-15): lane l
 // receives rows 4(l%4) .. 4(l%4)+3 of byte column l/4 in r0 and of column
 // l/4 + 8 in r1, row i of each group in byte i.
@@ -674,13 +632,15 @@ struct MmaState {
     }
 };
 
-// PATH 0: CUDA cores with G = GSIMT heads per kv head; PATH 1: tensor cores
-// with query heads padded to GPAD in {4, 8, 16} (n-tiles of 8: GPAD/8 rounded up).
+// PATH 0: CUDA cores, one query head per kv head (GSIMT = 1); PATH 1: tensor
+// cores with query heads padded to GPAD in {4, 8, 16} (n-tiles of 8: GPAD/8
+// rounded up).
 template <int D, int PATH, int GSIMT, int GPAD, int NS, bool KV8 = false>
 __global__ void __launch_bounds__(kDecodeThreads) paged_decode_kernel(const __grid_constant__ CUtensorMap tmap_k,
                                                                       const __grid_constant__ CUtensorMap tmap_v,
                                                                       const DecodeParams p) {
     constexpr int W = kConsumerWarps;
+    static_assert(PATH != 0 || GSIMT == 1, "the CUDA-core path serves one query head per kv head");
     constexpr int GP = PATH == 0 ? GSIMT : GPAD;
     constexpr int NT = (GPAD + 7) / 8;
     static_assert(!KV8 || D == 128, "FP8 stage tiles are 128-byte rows (head dim 128)");
@@ -841,7 +801,7 @@ __global__ void __launch_bounds__(kDecodeThreads) paged_decode_kernel(const __gr
         uint32_t gc = w;
         uint32_t mc = 0;  // merges done
         float scale_log2 = p.scale_log2;
-        SimtState<D, (PATH == 0 ? GSIMT : 1), KV8> st0;
+        SimtState<D, KV8> st0;
         MmaState<D, (PATH == 1 ? NT : 1), KV8> st1;
         while (true) {
             const uint32_t slot = gc % NS;
@@ -877,7 +837,7 @@ __global__ void __launch_bounds__(kDecodeThreads) paged_decode_kernel(const __gr
             if (si.k + W >= si.npad) {
                 // this warp's last stage of the item: merge the W partials
                 if (!wait_or_abort(mempty, (mc & 1) ^ 1, abort_flag)) break;
-                if constexpr (PATH == 0) st0.store_partial(mO, mM, mL, w, lane, L::kMergeStride, GP);
+                if constexpr (PATH == 0) st0.store_partial(mO, mM, mL, w, lane, L::kMergeStride);
                 else st1.store_partial(mO, mM, mL, w, lane, L::kMergeStride, GP, p.g);
                 __syncwarp();
                 if (lane == 0) mbar_arrive(mfull);

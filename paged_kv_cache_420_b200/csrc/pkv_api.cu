@@ -216,8 +216,9 @@ pkv_status launch_decode(const pkv::DecodeParams &prm, const CUtensorMap &mk, co
 template <int D>
 pkv_status dispatch_group(int g, const pkv::DecodeParams &prm, const CUtensorMap &mk, const CUtensorMap &mv,
                           cudaStream_t stream, int dev) {
+    // g = 1 on CUDA cores; from g = 2 up the heads of a kv head share the
+    // tensor-core tiles (measured faster than the two-head CUDA-core body)
     if (g == 1) return launch_decode<D, 0, 1, 1>(prm, mk, mv, stream, dev);
-    if (g == 2) return launch_decode<D, 0, 2, 1>(prm, mk, mv, stream, dev);
     if (g <= 4) return launch_decode<D, 1, 1, 4>(prm, mk, mv, stream, dev);
     if (g <= 8) return launch_decode<D, 1, 1, 8>(prm, mk, mv, stream, dev);
     return launch_decode<D, 1, 1, 16>(prm, mk, mv, stream, dev);
@@ -454,8 +455,9 @@ pkv_status decode_impl(const void *q, const void *k_cache, const void *v_cache, 
     if (r != PKV_OK) return r;
     const int dev = current_device();
     if (kv8) {
+        // g = 2 runs on the tensor cores too: over e4m3 codes the CUDA-core body
+        // is issue-bound (a conversion and four unpacked FMAs per code pair)
         if (g == 1) return launch_decode<128, 0, 1, 1, true>(prm, mk, mv, st, dev);
-        if (g == 2) return launch_decode<128, 0, 2, 1, true>(prm, mk, mv, st, dev);
         if (g <= 4) return launch_decode<128, 1, 1, 4, true>(prm, mk, mv, st, dev);
         if (g <= 8) return launch_decode<128, 1, 1, 8, true>(prm, mk, mv, st, dev);
         return launch_decode<128, 1, 1, 16, true>(prm, mk, mv, st, dev);

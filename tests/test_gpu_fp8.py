@@ -57,10 +57,10 @@ def _run_decode(w, k8, v8, ks, vs, pt=0):
 CASES = [
     # context lens, Hq, Hkv, partition tokens
     ([1, 15, 16, 17, 31, 100], 8, 8, 0),
-    ([5, 200, 511, 513], 16, 8, 0),          # g = 2
+    ([5, 200, 511, 513], 16, 8, 0),          # g = 2: tensor-core path (padded to 4 heads)
     ([1000, 3000, 77], 4, 4, 256),           # split-K partitions
     ([4096, 2049, 16], 8, 4, 512),           # g = 2, split-K
-    ([1, 15, 16, 17, 31, 100], 32, 8, 0),    # g = 4: tensor-core path
+    ([1, 15, 16, 17, 31, 100], 32, 8, 0),    # g = 4
     ([200, 511, 1000], 64, 8, 256),          # g = 8, split-K
     ([50, 129], 12, 4, 0),                   # g = 3 (padded to 4)
     ([33, 700], 16, 1, 0),                   # g = 16
