@@ -8,13 +8,15 @@
 // a row being (query token, head of the GQA group).
 //
 // Two CTAs per SM (each holds half of tensor memory and ~113 KB of shared
-// memory), warp-specialised (192 threads):
-//   warp 0       producer: the item's Q tile (128 x D bf16) by a 3-D TMA load,
-//                and 64-key K and V blocks of the paged cache (4 stages of 16
-//                keys each, addressed through the block table) into separate
-//                K and V rings; all 128-byte swizzled.  A K slot is released
-//                when its S product completes, a V slot when its PV product
-//                does, so the next K block streams in while P V still runs.
+// memory), warp-specialised (224 threads):
+//   warp 0       Q and K producer: the item's Q tile (128 x D bf16) by a 3-D
+//                TMA load, and 64-key K blocks of the paged cache (4 stages of
+//                16 keys each, addressed through the block table) into the K
+//                ring; all 128-byte swizzled.  A K slot is released when its S
+//                product completes.
+//   warp 6       V producer: the same blocks' V into the V ring, a slot being
+//                released when its PV product completes.  With its own warp
+//                the K stream never waits behind a V slot that PV still holds.
 //   warp 1       MMA issuer (one thread) and tensor-memory owner:
 //                S_j = Q K_j^T  (tcgen05.mma kind::f16, M 128, N 64, K-major
 //                smem operands, fp32 into the TMEM S buffer), then
@@ -37,7 +39,7 @@ namespace pkv {
 
 constexpr int kTcRows = 128;          // M: query rows per item
 constexpr int kTcKeys = 64;           // N: keys per block (4 stages of 16)
-constexpr int kTcThreads = 6 * 32;
+constexpr int kTcThreads = 7 * 32;
 constexpr int kTcCtasPerSm = 2;
 // Tensor memory of one CTA (256 of the SM's 512 columns):
 constexpr uint32_t kTmemCols = 256;
@@ -296,9 +298,9 @@ __global__ void __launch_bounds__(kTcThreads, kTcCtasPerSm)
         }
         for (int i = 0; i < NQ; ++i) {
             mbar_init(&qfull[i], 1);
-            // released by the MMA's commit (Q read) and by every softmax
-            // thread once it has taken the item description
-            mbar_init(&qempty[i], 1 + kTcRows);
+            // released by the MMA's commit (Q read), by every softmax thread
+            // and by the V producer once they have taken the item description
+            mbar_init(&qempty[i], 2 + kTcRows);
         }
         mbar_init(sfull, 1);
         mbar_init(sfree, kTcRows);
@@ -329,8 +331,8 @@ __global__ void __launch_bounds__(kTcThreads, kTcCtasPerSm)
     const int n_items = *reinterpret_cast<volatile int32_t *>(p.num_entries) * p.Hkv;
 
     if (warp == 0) {
-        // ------------------------------------------------------ producer --
-        uint32_t gk = 0, gv = 0;  // K and V blocks issued
+        // ------------------------------------------------ Q and K producer --
+        uint32_t gk = 0;          // K blocks issued
         int q_issued = -1;        // ord of the last Q tile load
         bool ok = true;
         int claimed = 0;
@@ -372,28 +374,19 @@ __global__ void __launch_bounds__(kTcThreads, kTcCtasPerSm)
                     if (blk >= 0 && blk < p.NB) row = (blk * p.Hkv + t.h) * p.bs + tok % p.bs;
                     else raise_error(PKV_DEVERR_BLOCK);
                 }
-#pragma unroll
-                for (int kv = 0; kv < 2 && ok; ++kv) {
-                    const uint32_t g = kv ? gv : gk;
-                    const uint32_t depth = kv ? NV : NK;
-                    const uint32_t slot = g % depth;
-                    uint64_t *fb = kv ? &vfull[slot] : &kfull[slot];
-                    if (lane == 0) {
-                        ok = wait_or_abort(kv ? &vempty[slot] : &kempty[slot], ((g / depth) & 1) ^ 1, abort_flag);
-                        if (ok) mbar_arrive_expect_tx(fb, (uint32_t)L::kSlot);
-                    }
-                    ok = __shfl_sync(0xffffffffu, ok, 0);
-                    if (ok && lane < 4) {
-                        const uint32_t dst = sbase + (kv ? L::oV : L::oK) + slot * L::kSlot + lane * (kStageTok * 128);
-#pragma unroll
-                        for (int hf = 0; hf < L::kHalves; ++hf)
-                            tma_load_2d_u32(dst + hf * L::kKVHalf, kv ? &tmap_v : &tmap_k, fb, hf * 64, row);
-                    }
-                    if (ok) {
-                        if (kv) ++gv;
-                        else ++gk;
-                    }
+                const uint32_t slot = gk % NK;
+                if (lane == 0) {
+                    ok = wait_or_abort(&kempty[slot], ((gk / NK) & 1) ^ 1, abort_flag);
+                    if (ok) mbar_arrive_expect_tx(&kfull[slot], (uint32_t)L::kSlot);
                 }
+                ok = __shfl_sync(0xffffffffu, ok, 0);
+                if (ok && lane < 4) {
+                    const uint32_t dst = sbase + L::oK + slot * L::kSlot + lane * (kStageTok * 128);
+#pragma unroll
+                    for (int hf = 0; hf < L::kHalves; ++hf)
+                        tma_load_2d_u32(dst + hf * L::kKVHalf, &tmap_k, &kfull[slot], hf * 64, row);
+                }
+                if (ok) ++gk;
             }
             it = __shfl_sync(0xffffffffu, claimed, 0);
         }
@@ -401,9 +394,47 @@ __global__ void __launch_bounds__(kTcThreads, kTcCtasPerSm)
         if (lane == 0 && *abort_flag) {
             for (uint32_t c = (gk > (uint32_t)NK ? gk - NK : 0); c < gk; ++c)
                 mbar_wait_bounded(&kfull[c % NK], (c / NK) & 1, kWaitLimitNs);
+            if (q_issued >= 0) mbar_wait_bounded(&qfull[q_issued % NQ], ((q_issued / NQ) & 1), kWaitLimitNs);
+        }
+    } else if (warp == 6) {
+        // ---------------------------------------------------- V producer --
+        uint32_t gv = 0;
+        bool ok = true;
+        for (int ord = 0; ok; ++ord) {
+            const int qb = ord % NQ;
+            ok = __all_sync(0xffffffffu, wait_or_abort(&qfull[qb], (ord / NQ) & 1, abort_flag));
+            if (!ok) break;
+            const TcItem t = items[qb];
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&qempty[qb]);
+            if (t.n_blocks < 0) break;
+            for (int j = 0; j < t.n_blocks && ok; ++j) {
+                // lane < 4: stage of 16 keys, as in the K producer
+                int row = p.pool_rows;
+                const int tok = j * kTcKeys + (lane & 3) * kStageTok;
+                if (lane < 4 && tok < t.n_keys) {
+                    const int blk = __ldg(p.block_tables + (size_t)t.s * p.MBS + tok / p.bs);
+                    if (blk >= 0 && blk < p.NB) row = (blk * p.Hkv + t.h) * p.bs + tok % p.bs;
+                    else raise_error(PKV_DEVERR_BLOCK);
+                }
+                const uint32_t slot = gv % NV;
+                if (lane == 0) {
+                    ok = wait_or_abort(&vempty[slot], ((gv / NV) & 1) ^ 1, abort_flag);
+                    if (ok) mbar_arrive_expect_tx(&vfull[slot], (uint32_t)L::kSlot);
+                }
+                ok = __shfl_sync(0xffffffffu, ok, 0);
+                if (ok && lane < 4) {
+                    const uint32_t dst = sbase + L::oV + slot * L::kSlot + lane * (kStageTok * 128);
+#pragma unroll
+                    for (int hf = 0; hf < L::kHalves; ++hf)
+                        tma_load_2d_u32(dst + hf * L::kKVHalf, &tmap_v, &vfull[slot], hf * 64, row);
+                }
+                if (ok) ++gv;
+            }
+        }
+        if (lane == 0 && *abort_flag) {
             for (uint32_t c = (gv > (uint32_t)NV ? gv - NV : 0); c < gv; ++c)
                 mbar_wait_bounded(&vfull[c % NV], (c / NV) & 1, kWaitLimitNs);
-            if (q_issued >= 0) mbar_wait_bounded(&qfull[q_issued % NQ], ((q_issued / NQ) & 1), kWaitLimitNs);
         }
     } else if (warp == 1) {
         // ---------------------------------------------------------- MMA --
