@@ -494,6 +494,8 @@ def run_fp8_cuda(args, rank, world, dist):
     torch.cuda.set_device(dev)
     base = args.workload[:-len("-fp8")]
     w = workloads.make(base, seed=args.seed + rank, values_device=dev, block_size=args.block_size)
+    if args.max_seqs and args.max_seqs < w.num_seqs:
+        w = workloads.subset(w, args.max_seqs)
     k8, v8, ks, vs = workloads.fp8_pools(w)
     del w.k_cache, w.v_cache
     torch.cuda.empty_cache()
