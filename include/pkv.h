@@ -176,7 +176,10 @@ size_t pkv_decode_workspace_bytes(int32_t num_seqs, int32_t num_q_heads, int32_t
  *   out[s][hq] = sum_i softmax(z)_i * V_i
  * where K_i, V_i are the rows of position i found through
  * block_tables[s][i / block_size] at offset i % block_size.  Accumulation is
- * fp32 with an online softmax; out is rounded to bf16 (nearest-even).
+ * fp32 with an online softmax; out is rounded to bf16 (nearest-even).  MHA
+ * (one query head per kv head) runs on CUDA cores with fp32 weights; GQA
+ * groups of 2 to 16 heads run on the tensor cores, where the softmax weights
+ * enter the weighted sum rounded to bf16.
  * Long contexts are split into partitions of partition_tokens tokens whose
  * (max, sum, acc) are merged by a log-sum-exp reduce.
  *
