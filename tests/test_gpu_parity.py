@@ -142,7 +142,7 @@ DECODE_CASES = [
     ([1, 17, 33, 64], 4, 4, 64, 16, 0),                 # the tiny shape
     ([1000, 5, 16, 31, 257, 640], 8, 8, 128, 16, 0),    # MHA, several stages, ragged tails
     ([1000, 5, 16, 31, 257, 640], 8, 8, 128, 16, 64),   # MHA, forced split-K
-    ([700, 3, 129, 1500], 8, 4, 128, 32, 0),            # g = 2 (CUDA-core path)
+    ([700, 3, 129, 1500], 8, 4, 128, 32, 0),            # g = 2 (tensor-core path, padded to 4 heads)
     ([700, 3, 129, 1500], 8, 4, 64, 32, 128),           # g = 2, d 64, split
     ([900, 2, 48, 333], 12, 4, 128, 16, 0),             # g = 3 (tensor-core path, padded tile)
     ([900, 2, 48, 333, 4097], 32, 8, 128, 16, 0),       # g = 4
