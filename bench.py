@@ -386,7 +386,8 @@ def run_cuda(args, rank, world, dist):
         "clocks": clocks.summary(),
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(w, budget_s=args.cpu_budget)
+        line["cpu_baseline"] = cpu_baseline(w, budget_s=args.cpu_budget,
+                                            single_thread_s=3.0 if w.name in SINGLE_THREAD_WORKLOADS else 0.0)
     return line
 
 
@@ -826,15 +827,36 @@ def run_swap_cuda(args, rank, world, dist):
     }
 
 
-def cpu_baseline(w, budget_s: float, label="oracle", pools=None):
+# workloads whose CPU baseline also reports a single-thread figure
+SINGLE_THREAD_WORKLOADS = ("tiny", "llama2-7b")
+
+
+def cpu_baseline(w, budget_s: float, label="oracle", pools=None, single_thread_s: float = 0.0):
     """Times the fp64 CPU oracle's paged attention on the first sequences of
     the workload until about `budget_s` seconds of CPU work are spent.  The
     step's copy-on-write copies and write are applied to the pools once,
-    untimed (they are under 1% of the step's bytes)."""
+    untimed (they are under 1% of the step's bytes).  With single_thread_s > 0
+    the same is timed on one thread for about that long and reported as
+    `single_thread`."""
     import oracle
 
     if pools is None:
         pools = oracle_pools(w)
+    line = _time_oracle(w, budget_s, label, pools)
+    if single_thread_s > 0:
+        prev = oracle.set_num_threads(1)
+        try:
+            one = _time_oracle(w, single_thread_s, label, pools)
+        finally:
+            oracle.set_num_threads(prev)
+        line["single_thread"] = {"value": one["value"], "unit": one["unit"], "cores": 1, "sample": one["sample"],
+                                 "tokens_layers_per_s": one["tokens_layers_per_s"]}
+    return line
+
+
+def _time_oracle(w, budget_s: float, label, pools):
+    import oracle
+
     kc, vc = pools
     done, elapsed, nbytes = 0, 0.0, 0
     chunk = 1
@@ -1042,6 +1064,9 @@ def run_reference(args, rank, world):
         tls.append(last["tokens_layers_per_s"])
     t_all = time.perf_counter() - t_all
     value = statistics.median(vals)
+    single = None
+    if w.name in SINGLE_THREAD_WORKLOADS:  # outside the timed steps
+        single = cpu_baseline(w, 0.05, pools=pools, single_thread_s=per_step_budget)["single_thread"]
     return {
         "impl": "reference",
         "metric": "paged decode attn HBM GB/s (% of B200 peak) & tokens·layers/s at 13B shape",
@@ -1051,8 +1076,8 @@ def run_reference(args, rank, world):
         "config": {"workload": f"{w.name}: {w.description}", "block_size": w.block_size,
                    "num_seqs": w.num_seqs, "seed": args.seed},
         "tokens_layers_per_s": statistics.median(tls),
-        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": last["cores"], "kind": "oracle",
-                         "sample": last["sample"]},
+        "cpu_baseline": dict({"value": value, "unit": "GB/s", "cores": last["cores"], "kind": "oracle",
+                              "sample": last["sample"]}, **({"single_thread": single} if single else {})),
         "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
 

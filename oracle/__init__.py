@@ -71,8 +71,10 @@ def _load() -> ctypes.CDLL:
         lib.oracle_prefix_lookup.argtypes = [P, P, I, P, P, I, P, P, I, I, P, I, P]
         lib.oracle_prefix_insert.argtypes = [P, P, I, P, P, I, P, P, I, I, P, I, P]
         lib.oracle_num_threads.argtypes = []
+        lib.oracle_set_num_threads.argtypes = [I]
         for f in (lib.oracle_kv_write, lib.oracle_copy_blocks, lib.oracle_paged_attention,
                   lib.oracle_attention_partial, lib.oracle_lse_merge, lib.oracle_num_threads,
+                  lib.oracle_set_num_threads,
                   lib.oracle_paged_prefill, lib.oracle_swap_out, lib.oracle_swap_in, lib.oracle_lru_victims,
                   lib.oracle_bm_init, lib.oracle_bm_alloc, lib.oracle_bm_free, lib.oracle_bm_share,
                   lib.oracle_bm_append_slots, lib.oracle_e4m3_encode_array, lib.oracle_kv_write_fp8,
@@ -85,6 +87,12 @@ def _load() -> ctypes.CDLL:
 
 def num_threads() -> int:
     return int(_load().oracle_num_threads())
+
+
+def set_num_threads(n: int) -> int:
+    """Threads of the oracle's later parallel loops (timing only); returns the
+    previous count."""
+    return int(_load().oracle_set_num_threads(int(n)))
 
 
 # ---------------------------------------------------------------------------

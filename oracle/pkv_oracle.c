@@ -73,6 +73,18 @@ int oracle_num_threads(void) {
 #endif
 }
 
+/* Threads used by later parallel regions (timing only; results do not depend
+ * on it).  Returns the previous count. */
+int oracle_set_num_threads(int n) {
+    int prev = oracle_num_threads();
+#ifdef _OPENMP
+    if (n > 0) omp_set_num_threads(n);
+#else
+    (void)n;
+#endif
+    return prev;
+}
+
 /*
  * Write: for every new token t with slot_mapping[t] >= 0, block = slot / bs,
  * offset = slot % bs, and for every kv head h the row

@@ -32,6 +32,8 @@ def test_reference_arm_prints_one_contract_line():
     assert line["config"]["workload"].startswith("tiny")
     cb = line["cpu_baseline"]
     assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == line["value"] and cb["sample"]
+    one = cb["single_thread"]  # reported for the tiny and 7B workloads
+    assert one["cores"] == 1 and one["value"] > 0 and one["unit"] == "GB/s"
     e2e = line["e2e"]
     assert e2e["value"] == line["value"] and e2e["unit"] == line["unit"]
     assert e2e["h2d_bytes_per_step"] == 0 and e2e["d2h_bytes_per_step"] == 0
