@@ -224,7 +224,10 @@ pkv_status paged_attn_decode(const void *q, const void *k_cache, const void *v_c
  *     invalid sizes return PKV_EINVAL as in paged_attn_decode.
  *   - The first call on each device looks up the array's device address
  *     (cudaGetSymbolAddress) with that device current; make that first call
- *     before any stream capture.
+ *     before any stream capture.  The address is kept for the life of the
+ *     process, which assumes one CUDA context per device for that long: after
+ *     a cudaDeviceReset, or with a driver-API context other than the primary
+ *     one current, the kept address no longer names this array.
  *   - All calls on a device share the one array, and it keeps the previous
  *     call's contents.  Nothing in it needs to start at zero (every call
  *     rewrites what it reads).  Calls whose kernels overlap on the GPU (for

@@ -32,12 +32,8 @@
 
 namespace pkv {
 
-#ifndef PKV_CONSUMER_WARPS
-#define PKV_CONSUMER_WARPS 4
-#endif
-
 constexpr int kStageTok = 16;                     // tokens per pipeline stage (one TMA box height)
-constexpr int kConsumerWarps = PKV_CONSUMER_WARPS;  // W
+constexpr int kConsumerWarps = 4;                 // W
 static_assert(32 % kConsumerWarps == 0, "stage groups must tile the 32-entry table prefetch");
 constexpr int kDecodeThreads = (kConsumerWarps + 1) * 32;
 constexpr int kPlanThreads = 1024;

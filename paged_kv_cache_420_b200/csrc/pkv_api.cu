@@ -7,6 +7,7 @@
 #include <cudaTypedefs.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cstdint>
 #include <cmath>
 #include <cstring>
@@ -23,15 +24,9 @@
 namespace {
 
 constexpr int kMaxDevices = 64;
-#ifndef PKV_STAGES_SIMT
-#define PKV_STAGES_SIMT 8
-#endif
-#ifndef PKV_STAGES_MMA
-#define PKV_STAGES_MMA 8
-#endif
 // NS: shared-memory ring slots per CTA (a multiple of the consumer warps)
-constexpr int kStagesSimt = PKV_STAGES_SIMT;
-constexpr int kStagesMma = PKV_STAGES_MMA;
+constexpr int kStagesSimt = 8;
+constexpr int kStagesMma = 8;
 static_assert(kStagesSimt % pkv::kConsumerWarps == 0 && kStagesMma % pkv::kConsumerWarps == 0,
               "ring slots must be a multiple of the consumer warps");
 
@@ -43,15 +38,20 @@ int current_device() {
     return dev;
 }
 
+// Per-device values computed on first use.  Several host threads may make
+// their first call on a device at once: each slot is an atomic, and a value
+// computed twice is the same value, so the last store is as good as the first.
+using DeviceCache = std::atomic<int>[kMaxDevices];
+
 int sm_count(int dev) {
-    static int cache[kMaxDevices] = {0};
+    static DeviceCache cache{};
     if (dev < 0 || dev >= kMaxDevices) return 148;
-    if (cache[dev] == 0) {
-        int n = 0;
+    int n = cache[dev].load(std::memory_order_acquire);
+    if (n == 0) {
         if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
-        cache[dev] = n;
+        cache[dev].store(n, std::memory_order_release);
     }
-    return cache[dev];
+    return n;
 }
 
 pkv_status check_pool(const pkv_pool &pool) {
@@ -177,8 +177,10 @@ pkv_status launch_decode(const pkv::DecodeParams &prm, const CUtensorMap &mk, co
     constexpr int NS = PATH == 0 ? kStagesSimt : kStagesMma;
     using L = pkv::DecodeSmem<D, (PATH == 0 ? GS : GPAD), NS, KV8>;
     auto kernel = pkv::paged_decode_kernel<D, PATH, GS, GPAD, NS, KV8>;
-    static int occ_cache[kMaxDevices] = {0};
-    int occ = (dev >= 0 && dev < kMaxDevices) ? occ_cache[dev] : 0;
+    // the shared-memory attribute is set before the occupancy query, so a
+    // cached occupancy also means the attribute is set on this device
+    static DeviceCache occ_cache{};
+    int occ = (dev >= 0 && dev < kMaxDevices) ? occ_cache[dev].load(std::memory_order_acquire) : 0;
     if (occ == 0) {
         if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc) != cudaSuccess)
             return PKV_ECUDA;
@@ -186,7 +188,7 @@ pkv_status launch_decode(const pkv::DecodeParams &prm, const CUtensorMap &mk, co
                 cudaSuccess ||
             occ <= 0)
             return PKV_ECUDA;
-        if (dev >= 0 && dev < kMaxDevices) occ_cache[dev] = occ;
+        if (dev >= 0 && dev < kMaxDevices) occ_cache[dev].store(occ, std::memory_order_release);
     }
     const long long items_upper = (long long)prm.B * prm.Hkv * prm.maxP;
     const long long grid = std::max<long long>(1, std::min<long long>(items_upper, (long long)sm_count(dev) * occ));
@@ -226,7 +228,7 @@ pkv_status dispatch_group(int g, const pkv::DecodeParams &prm, const CUtensorMap
 
 // -------------------------------------------------------- prefill ----
 
-int prefill_query_tile(int g) { return pkv::kPrefillRows / g; }
+int prefill_query_tile(int g) { return pkv::kTcRows / g; }
 
 bool prefill_layout(int32_t B, int32_t g, int32_t max_q, size_t *off_entries, size_t *total) {
     if (B < 0 || g <= 0 || max_q < 0) return false;
@@ -242,11 +244,11 @@ pkv_status launch_prefill_tc(const pkv::PrefillParams &prm, const CUtensorMap &m
                              const CUtensorMap &mq, cudaStream_t stream, int dev) {
     using L = pkv::TcSmem<D>;
     auto kernel = pkv::paged_prefill_tc_kernel<D>;
-    static bool attr_set[kMaxDevices] = {false};
-    if (dev >= 0 && dev < kMaxDevices && !attr_set[dev]) {
+    static DeviceCache attr_set{};
+    if (dev < 0 || dev >= kMaxDevices || attr_set[dev].load(std::memory_order_acquire) == 0) {
         if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kBytes) != cudaSuccess)
             return PKV_ECUDA;
-        attr_set[dev] = true;
+        if (dev >= 0 && dev < kMaxDevices) attr_set[dev].store(1, std::memory_order_release);
     }
     const long long tiles = std::max<long long>(1, ((long long)prm.max_q + prm.QT - 1) / prm.QT);
     const long long items_upper = (long long)prm.B * tiles * prm.Hkv;
@@ -265,41 +267,6 @@ pkv_status launch_prefill_tc(const pkv::PrefillParams &prm, const CUtensorMap &m
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     if (cudaLaunchKernelEx(&cfg, kernel, mk, mv, mq, prm) != cudaSuccess) return PKV_ECUDA;
-    return launch_status();
-}
-
-template <int D>
-pkv_status launch_prefill(const pkv::PrefillParams &prm, const CUtensorMap &mk, const CUtensorMap &mv,
-                          cudaStream_t stream, int dev) {
-    constexpr int NS = 8;
-    using L = pkv::PrefillSmem<D, NS>;
-    auto kernel = pkv::paged_prefill_kernel<D, NS>;
-    static int occ_cache[kMaxDevices] = {0};
-    int occ = (dev >= 0 && dev < kMaxDevices) ? occ_cache[dev] : 0;
-    if (occ == 0) {
-        if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kBytes) != cudaSuccess)
-            return PKV_ECUDA;
-        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kernel, pkv::kDecodeThreads, L::kBytes) !=
-                cudaSuccess ||
-            occ <= 0)
-            return PKV_ECUDA;
-        if (dev >= 0 && dev < kMaxDevices) occ_cache[dev] = occ;
-    }
-    const long long tiles = std::max<long long>(1, ((long long)prm.max_q + prm.QT - 1) / prm.QT);
-    const long long items_upper = (long long)prm.B * tiles * prm.Hkv;
-    const long long grid = std::max<long long>(1, std::min<long long>(items_upper, (long long)sm_count(dev) * occ));
-    cudaLaunchConfig_t cfg;
-    std::memset(&cfg, 0, sizeof cfg);
-    cfg.gridDim = dim3((unsigned)grid);
-    cfg.blockDim = dim3(pkv::kDecodeThreads);
-    cfg.dynamicSmemBytes = L::kBytes;
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, kernel, mk, mv, prm) != cudaSuccess) return PKV_ECUDA;
     return launch_status();
 }
 
@@ -697,31 +664,21 @@ pkv_status paged_attn_prefill(const void *q, const void *k_cache, const void *v_
     prm.NB = pool.num_blocks;
     prm.max_ctx = max_context_len;
     prm.max_q = max_query_len;
-#ifdef PKV_PREFILL_MMA_SYNC
     prm.QT = prefill_query_tile(g);
-#else
-    prm.QT = pkv::kTcRows / g;
-#endif
     prm.T = num_tokens;
     prm.pool_rows = pool.num_blocks * pool.num_kv_heads * pool.block_size;
     prm.scale_log2 = scale * 1.4426950408889634f;
     CUtensorMap mk, mv;
     if (!encode_pool_map(&mk, k_cache, pool) || !encode_pool_map(&mv, v_cache, pool)) return PKV_ECUDA;
-#ifndef PKV_PREFILL_MMA_SYNC
     CUtensorMap mq;
     if (!encode_query_map(&mq, q, num_tokens, num_q_heads, pool.head_dim, g, prm.QT)) return PKV_ECUDA;
-#endif
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     pkv::plan_prefill_kernel<<<1, pkv::kPlanThreads, 0, st>>>(prm);
     const pkv_status r = launch_status();
     if (r != PKV_OK) return r;
     const int dev = current_device();
-#ifdef PKV_PREFILL_MMA_SYNC
-    return pool.head_dim == 128 ? launch_prefill<128>(prm, mk, mv, st, dev) : launch_prefill<64>(prm, mk, mv, st, dev);
-#else
     return pool.head_dim == 128 ? launch_prefill_tc<128>(prm, mk, mv, mq, st, dev)
                                 : launch_prefill_tc<64>(prm, mk, mv, mq, st, dev);
-#endif
 }
 
 size_t pkv_bm_state_bytes(int32_t num_blocks) {

@@ -1,7 +1,7 @@
 // prefill_tc.cuh -- chunked-prefill paged attention on the 5th-generation
 // tensor cores (tcgen05, accumulators in tensor memory).
 //
-// Same operation as paged_prefill_kernel (prefill.cuh): query token i of a
+// Chunked prefill (parameters and planner in prefill.cuh): query token i of a
 // sequence's new chunk sits at position ctx - q_len + i and attends to positions
 // [0, pos] read through the block table (wkbse.com "加速 LLM 推理：深入了解 vllm
 // 引擎", section 3.1).  An item is (sequence, kv head, tile of 128 query rows),
@@ -53,15 +53,12 @@ struct TcItem {
 
 // Shared memory of one CTA: NQ query buffers, an NK-slot K ring and an
 // NV-slot V ring (two CTAs share an SM's 228 KB).
-#ifndef PKV_TC_NV128
-#define PKV_TC_NV128 3
-#endif
 template <int D>
 struct TcSmem {
     static constexpr int kHalves = D / 64;
     static constexpr int NQ = D == 128 ? 1 : 2;
     static constexpr int NK = D == 128 ? 2 : 4;
-    static constexpr int NV = D == 128 ? PKV_TC_NV128 : 4;
+    static constexpr int NV = D == 128 ? 3 : 4;
     static constexpr int kQHalf = kTcRows * 128;          // 16 KB: 128 rows x 64 columns
     static constexpr int kQBuf = kHalves * kQHalf;
     static constexpr int kKVHalf = kTcKeys * 128;         // 8 KB: 64 keys x 64 columns
@@ -183,60 +180,11 @@ __device__ __forceinline__ void ffma2_bcast(float &a0, float &a1, float b0, floa
         : "f"(b0), "f"(b1), "f"(c), "f"(d));
 }
 
-// Packed pair (d0, d1) = (a0 * b0 + c0, a1 * b1 + c1).
-__device__ __forceinline__ void ffma2(float &d0, float &d1, float a0, float a1, float b0, float b1, float c0,
-                                      float c1) {
-    asm("{\n\t.reg .b64 pa, pb, pc, pd;\n\t"
-        "mov.b64 pa, {%2, %3};\n\t"
-        "mov.b64 pb, {%4, %5};\n\t"
-        "mov.b64 pc, {%6, %7};\n\t"
-        "fma.rn.f32x2 pd, pa, pb, pc;\n\t"
-        "mov.b64 {%0, %1}, pd;\n\t}"
-        : "=f"(d0), "=f"(d1)
-        : "f"(a0), "f"(a1), "f"(b0), "f"(b1), "f"(c0), "f"(c1));
-}
-
 __device__ __forceinline__ float fmax3f(float a, float b, float c) {
     float r;
     asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
     return r;
 }
-
-// 2^x for a pair, x <= 64, on the FMA and integer pipes instead of the
-// special-function unit (which the softmax otherwise saturates):
-//   x = j + f, j = round(x) (by adding 1.5 * 2^23, which leaves j in the low
-//   mantissa bits), f = x - j in [-0.5, 0.5] exactly;
-//   2^f ~ c0 + f (c1 + f (c2 + f c3)), the relative-error minimax cubic on
-//   [-0.5, 0.5] (Remez exchange; fit_exp2_poly.py beside this file), max
-//   relative error 7.5e-5, far below bf16's 2^-9;
-//   2^j is added to the exponent field.
-// x is clamped to -126 first, so masked scores (-inf) give 2^-126 and the
-// exponent field cannot underflow.
-constexpr float kExp2C0 = 0.9999280571937561f;
-constexpr float kExp2C1 = 0.6932609677314758f;
-constexpr float kExp2C2 = 0.2426111251115799f;
-constexpr float kExp2C3 = 0.0551716685295105f;
-constexpr float kRoundMagic = 12582912.0f;  // 1.5 * 2^23
-
-__device__ __forceinline__ void exp2_poly2(float x0, float x1, float &y0, float &y1) {
-    x0 = fmaxf(x0, -126.f);
-    x1 = fmaxf(x1, -126.f);
-    float t0, t1, j0, j1, f0, f1, p0, p1;
-    ffma2(t0, t1, x0, x1, 1.f, 1.f, kRoundMagic, kRoundMagic);     // t = x + M (round to integer)
-    ffma2(j0, j1, t0, t1, 1.f, 1.f, -kRoundMagic, -kRoundMagic);   // j = t - M
-    ffma2(f0, f1, j0, j1, -1.f, -1.f, x0, x1);                     // f = x - j
-    ffma2(p0, p1, f0, f1, kExp2C3, kExp2C3, kExp2C2, kExp2C2);
-    ffma2(p0, p1, p0, p1, f0, f1, kExp2C1, kExp2C1);
-    ffma2(p0, p1, p0, p1, f0, f1, kExp2C0, kExp2C0);
-    y0 = __uint_as_float(__float_as_uint(p0) + (__float_as_uint(t0) << 23));
-    y1 = __uint_as_float(__float_as_uint(p1) + (__float_as_uint(t1) << 23));
-}
-
-// Every kExpEmuEvery-th pair of scores takes exp2_poly2 (0: none).
-#ifndef PKV_TC_EXP_EMU
-#define PKV_TC_EXP_EMU 0
-#endif
-constexpr int kExpEmuEvery = PKV_TC_EXP_EMU;
 
 // Packed pair (a0, a1) += (b0, b1).
 __device__ __forceinline__ void fadd2(float &a0, float &a1, float b0, float b1) {
@@ -561,13 +509,7 @@ __global__ void __launch_bounds__(kTcThreads, kTcCtasPerSm)
                 for (int i = 0; i < 32; ++i) {
                     float z0, z1;
                     ffma2_bcast(z0, z1, __uint_as_float(sv[2 * i]), __uint_as_float(sv[2 * i + 1]), c, nm);
-                    float p0, p1;
-                    if (kExpEmuEvery > 0 && i % (kExpEmuEvery > 0 ? kExpEmuEvery : 1) == kExpEmuEvery - 1) {
-                        exp2_poly2(z0, z1, p0, p1);
-                    } else {
-                        p0 = ex2_ftz(z0);
-                        p1 = ex2_ftz(z1);
-                    }
+                    const float p0 = ex2_ftz(z0), p1 = ex2_ftz(z1);
                     fadd2(s0, s1, p0, p1);
                     pk[i] = pack_bf16x2(p0, p1);
                 }

@@ -2,9 +2,11 @@
 configuration the benchmark times.
 
 Pools after the copy-on-write copies and the write are compared bit-exactly
-with the oracle's; attention is compared on a seeded sample of sequences that
-the fp64 oracle computes one by one (all of them when the batch is small), and
-every output row must be finite.
+with the oracle's.  Attention is compared with the fp64 oracle on every
+sequence of the 7B, 13B and long-context batches (the long-context batch
+includes both 131,072-token sequences, 256 partitions each), and on 64 of the
+256 shared-prefix sequences: a seeded sample, every copy-on-write fork, and one
+whole group of 8 sharers.  Every output row must be finite.
 """
 import numpy as np
 import pytest
@@ -16,15 +18,17 @@ from tests._gpu_util import assert_attention_close, bits_equal, no_device_error,
 
 pytestmark = pytest.mark.gpu
 
+# (workload, block size, sampled sequences; None = all)
 CASES = [
     ("tiny", 16, None),
-    ("llama2-7b", 16, 16),
+    ("llama2-7b", 16, None),
     ("llama2-13b", 16, None),
-    ("llama2-13b", 32, 32),
-    ("llama3-8b-gqa-prefix", 16, 24),
-    ("llama2-70b-long", 16, 2),
-    ("llama2-70b-long", 128, 2),
+    ("llama2-13b", 32, None),
+    ("llama3-8b-gqa-prefix", 16, 64),
+    ("llama2-70b-long", 16, None),
+    ("llama2-70b-long", 128, None),
 ]
+SHARERS_PER_GROUP = 8  # the shared-prefix batch: groups of 8 consecutive sequences
 
 
 @pytest.mark.parametrize("name,bs,sample", CASES)
@@ -43,11 +47,16 @@ def test_full_size_step(name, bs, sample):
     if sample is None or sample >= B:
         idx = np.arange(B)
     else:
-        rng = np.random.default_rng(123)
-        idx = np.sort(rng.choice(B, size=sample, replace=False))
-        if len(w.copy_pairs):  # always include the copy-on-write forks
+        must = set()
+        if len(w.copy_pairs):  # every copy-on-write fork, and the whole group of the first one
             forks = [int(np.nonzero((w.block_tables == d).any(axis=1))[0][0]) for d in w.copy_pairs[:, 1]]
-            idx = np.union1d(idx, forks)
+            g0 = forks[0] // SHARERS_PER_GROUP * SHARERS_PER_GROUP
+            must = set(forks) | set(range(g0, g0 + SHARERS_PER_GROUP))
+        rest = np.array(sorted(set(range(B)) - must))
+        rng = np.random.default_rng(123)
+        extra = rng.choice(rest, size=max(0, sample - len(must)), replace=False)
+        idx = np.array(sorted(must | set(int(x) for x in extra)))
+        assert len(idx) == sample
     q = w.q[torch.from_numpy(idx).cuda()]
     ref = oracle.paged_attention(q, okc, ovc, w.block_tables[idx], w.context_lens[idx], w.scale)
     assert_attention_close(out[torch.from_numpy(idx).cuda()], ref, f"{name} bs{bs}")

@@ -78,8 +78,10 @@ def test_named_prefill_workload_full_size(name):
     assert torch.isfinite(out.float()).all()
     okc, ovc = oracle.kv_write(kc0, vc0, w.k_new, w.v_new, w.slot_mapping)
     assert bits_equal(kc, okc) and bits_equal(vc, ovc)
-    # sampled rows: the first and last 32 query rows of two sequences
-    rows = np.concatenate([np.arange(s0, s0 + 32) for s0 in (int(w.query_start[1]), int(w.query_start[6]) - 32)])
+    # sampled rows: the first and last 128 query rows of every sequence's chunk
+    rows = np.unique(np.concatenate(
+        [np.r_[a:min(b, a + 128), max(a, b - 128):b]
+         for a, b in zip(w.query_start[:-1].astype(int), w.query_start[1:].astype(int))]))
     sub_q = w.q[torch.from_numpy(rows).cuda()]
     # oracle on single-row chunks with the rows' own context lengths
     seq_of = np.searchsorted(w.query_start, rows, side="right") - 1
