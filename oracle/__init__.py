@@ -54,22 +54,21 @@ def _load() -> ctypes.CDLL:
         lib.oracle_swap_out.argtypes = [P, P, P, I, I, I, I, I, P, P]
         lib.oracle_swap_in.argtypes = [P, P, P, I, I, I, I, I, P, P]
         lib.oracle_lru_victims.argtypes = [P, P, I, I, P, P]
-        lib.oracle_bm_init.argtypes = [P, P, P, I]
-        lib.oracle_bm_alloc.argtypes = [P, P, P, I, P, I, P, P, I, P]
-        lib.oracle_bm_free.argtypes = [P, P, P, I, P, I, P]
-        lib.oracle_bm_share.argtypes = [P, I, P, I, P]
-        lib.oracle_bm_append_slots.argtypes = [P, P, P, I, P, I, P, P, I, I, P, P, P, P]
+        lib.oracle_bm_init.argtypes = [P, P, P, P, P, P, I]
+        lib.oracle_bm_alloc.argtypes = [P, P, P, P, P, P, I, P, I, P, P, I, P]
+        lib.oracle_bm_free.argtypes = [P, P, P, P, P, P, I, P, I, P]
+        lib.oracle_bm_share.argtypes = [P, P, I, P, I, P]
+        lib.oracle_bm_append_slots.argtypes = [P, P, P, P, P, P, I, P, I, P, P, I, I, P, P, P, P]
         lib.oracle_e4m3_decode.argtypes = [ctypes.c_uint8]
         lib.oracle_e4m3_decode.restype = D
         lib.oracle_e4m3_encode_array.argtypes = [P, I, P]
         lib.oracle_kv_write_fp8.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I]
         lib.oracle_paged_attention_fp8.argtypes = [P, P, P, P, P, P, I, P, I, I, I, I, I, I, D, P]
-        lib.oracle_bm_drop_hashes.argtypes = [P, P, I]
         lib.oracle_fnv1a64.argtypes = [P, I]
         lib.oracle_fnv1a64.restype = ctypes.c_uint64
         lib.oracle_prefix_keys.argtypes = [P, I, I, P]
-        lib.oracle_prefix_lookup.argtypes = [P, P, I, P, P, I, P, P, I, I, P, I, P]
-        lib.oracle_prefix_insert.argtypes = [P, P, I, P, P, I, P, P, I, I, P, I, P]
+        lib.oracle_prefix_lookup.argtypes = [P, P, P, I, P, P, I, P, P, I, I, P, I, P]
+        lib.oracle_prefix_insert.argtypes = [P, I, P, P, I, P, P, I, I, P, I, P]
         lib.oracle_num_threads.argtypes = []
         lib.oracle_set_num_threads.argtypes = [I]
         for f in (lib.oracle_kv_write, lib.oracle_copy_blocks, lib.oracle_paged_attention,
@@ -78,7 +77,7 @@ def _load() -> ctypes.CDLL:
                   lib.oracle_paged_prefill, lib.oracle_swap_out, lib.oracle_swap_in, lib.oracle_lru_victims,
                   lib.oracle_bm_init, lib.oracle_bm_alloc, lib.oracle_bm_free, lib.oracle_bm_share,
                   lib.oracle_bm_append_slots, lib.oracle_e4m3_encode_array, lib.oracle_kv_write_fp8,
-                  lib.oracle_paged_attention_fp8, lib.oracle_bm_drop_hashes, lib.oracle_prefix_keys,
+                  lib.oracle_paged_attention_fp8, lib.oracle_prefix_keys,
                   lib.oracle_prefix_lookup, lib.oracle_prefix_insert):
             f.restype = ctypes.c_int
         _lib = lib
@@ -209,18 +208,25 @@ BM_ERR_NOSPACE, BM_ERR_RANGE, BM_ERR_DOUBLEFREE, BM_ERR_TABLE = 1, 2, 4, 8
 
 class BlockState:
     """free_stack[:top] are the free ids (the next allocation pops
-    free_stack[top - 1]); refcount[b] counts the sequences mapping block b."""
+    free_stack[top - 1]); refcount[b] counts the sequences mapping block b;
+    block_hash[b] is the prefix key block b holds (0: none); lru_stamp[b] is
+    the release clock of a cached block (refcount 0, key kept, evictable),
+    -1 for every other block; clock is the next release stamp."""
 
-    def __init__(self, free_stack, top, refcount, block_hash=None):
+    def __init__(self, free_stack, top, refcount, block_hash=None, lru_stamp=None, clock=0):
         self.free_stack = np.ascontiguousarray(free_stack, dtype=np.int32)
         self.top = int(top)
         self.refcount = np.ascontiguousarray(refcount, dtype=np.int32)
         n = self.refcount.shape[0]
         self.block_hash = (np.zeros(n, np.uint64) if block_hash is None
                            else np.ascontiguousarray(block_hash, dtype=np.uint64))
+        self.lru_stamp = (np.full(n, -1, np.int64) if lru_stamp is None
+                          else np.ascontiguousarray(lru_stamp, dtype=np.int64))
+        self.clock = int(clock)
 
     def copy(self):
-        return BlockState(self.free_stack.copy(), self.top, self.refcount.copy(), self.block_hash.copy())
+        return BlockState(self.free_stack.copy(), self.top, self.refcount.copy(), self.block_hash.copy(),
+                          self.lru_stamp.copy(), self.clock)
 
     @property
     def num_blocks(self):
@@ -229,11 +235,19 @@ class BlockState:
     def free_set(self):
         return set(self.free_stack[:self.top].tolist())
 
+    def lru_order(self):
+        """Cached blocks, least recently released first (the eviction order)."""
+        c = np.flatnonzero(self.lru_stamp >= 0)
+        return c[np.argsort(self.lru_stamp[c], kind="stable")].astype(np.int32)
+
 
 def _bm_call(fn, st: BlockState, *args):
     top = np.array([st.top], dtype=np.int32)
-    rc = fn(_ptr(st.free_stack), _ptr(top), _ptr(st.refcount), st.num_blocks, *args)
+    clock = np.array([st.clock], dtype=np.int64)
+    rc = fn(_ptr(st.free_stack), _ptr(top), _ptr(st.refcount), _ptr(st.block_hash), _ptr(st.lru_stamp),
+            _ptr(clock), st.num_blocks, *args)
     st.top = int(top[0])
+    st.clock = int(clock[0])
     return rc
 
 
@@ -260,7 +274,6 @@ def bm_free(st: BlockState, ids):
     a = np.ascontiguousarray(ids, dtype=np.int32).reshape(-1)
     err = np.zeros(1, dtype=np.uint32)
     _check(_bm_call(_load().oracle_bm_free, st, _ptr(a), a.shape[0], _ptr(err)), "bm_free")
-    _load().oracle_bm_drop_hashes(_ptr(st.refcount), _ptr(st.block_hash), st.num_blocks)
     return st, int(err[0])
 
 
@@ -268,7 +281,8 @@ def bm_share(st: BlockState, ids):
     st = st.copy()
     a = np.ascontiguousarray(ids, dtype=np.int32).reshape(-1)
     err = np.zeros(1, dtype=np.uint32)
-    _check(_load().oracle_bm_share(_ptr(st.refcount), st.num_blocks, _ptr(a), a.shape[0], _ptr(err)), "bm_share")
+    _check(_load().oracle_bm_share(_ptr(st.refcount), _ptr(st.lru_stamp), st.num_blocks, _ptr(a), a.shape[0],
+                                   _ptr(err)), "bm_share")
     return st, int(err[0])
 
 
@@ -383,7 +397,8 @@ def prefix_lookup(st: BlockState, cache: PrefixCache, tokens, query_start, block
     tables = np.ascontiguousarray(block_tables, dtype=np.int32).copy()
     B, mbs = tables.shape
     nc = np.zeros(max(B, 1), np.int32)
-    _check(_load().oracle_prefix_lookup(_ptr(st.refcount), _ptr(st.block_hash), st.num_blocks, _ptr(cache.keys),
+    _check(_load().oracle_prefix_lookup(_ptr(st.refcount), _ptr(st.lru_stamp), _ptr(st.block_hash), st.num_blocks,
+                                        _ptr(cache.keys),
                                         _ptr(cache.vals), cache.keys.shape[0], _ptr(t), _ptr(qs), B,
                                         int(block_size), _ptr(tables), mbs, _ptr(nc)), "prefix_lookup")
     return st, tables, nc[:B]
@@ -398,7 +413,7 @@ def prefix_insert(st: BlockState, cache: PrefixCache, tokens, query_start, block
     tables = np.ascontiguousarray(block_tables, dtype=np.int32)
     B, mbs = tables.shape
     err = np.zeros(1, np.uint32)
-    _check(_load().oracle_prefix_insert(_ptr(st.refcount), _ptr(st.block_hash), st.num_blocks, _ptr(cache.keys),
+    _check(_load().oracle_prefix_insert(_ptr(st.block_hash), st.num_blocks, _ptr(cache.keys),
                                         _ptr(cache.vals), cache.keys.shape[0], _ptr(t), _ptr(qs), B,
                                         int(block_size), _ptr(tables), mbs, _ptr(err)), "prefix_insert")
     return st, cache, int(err[0])

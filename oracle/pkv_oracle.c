@@ -26,7 +26,11 @@
  *     prompt sharing; section 2.1's allocation sketch: a block whose prefix
  *     matches is shared instead of allocated): full prompt blocks are keyed
  *     by a chained FNV-1a 64-bit hash of their tokens and the key of the
- *     block before, and looked up before allocation.
+ *     block before, and looked up before allocation.  A keyed block whose
+ *     last sequence ends stays cached (section 2.1 item 1: a block is free,
+ *     allocated or shareable) until allocation runs out of free blocks and
+ *     evicts it, least recently released first (item 3: LRU keeps the block
+ *     heat).
  *   - an FP8 KV cache (ai-stack.site "Nano-vLLM 原理", case study: FP8 mixed
  *     precision): the pool holds OCP E4M3 codes with a static scale per kv
  *     head for K and for V; a value is stored as the code nearest to
@@ -400,34 +404,69 @@ int oracle_lru_victims(const int64_t *last_use, const uint8_t *evictable, int nu
 #define BM_ERR_DOUBLEFREE 4u /* a block freed more often than it was referenced */
 #define BM_ERR_TABLE 8u      /* a sequence outgrew its block-table row */
 
-int oracle_bm_init(int32_t *free_stack, int32_t *top, int32_t *refcount, int num_blocks) {
+/* Block states (intelliparadigm.com section 2.1, item 1):
+ *   free       refcount 0, on the free stack, no key;
+ *   allocated  refcount > 0 (it may hold a prefix key);
+ *   cached     refcount 0 but still holding a prefix key: shareable again by
+ *              a prefix lookup, evictable by allocation.  lru_stamp[b] is the
+ *              value of the release clock when its count reached zero; every
+ *              other block has lru_stamp -1.
+ * Allocation takes the free stack first; when it is empty, the cached block
+ * with the smallest stamp (the least recently released, item 3) is evicted:
+ * its key is dropped and it is handed out. */
+int oracle_bm_init(int32_t *free_stack, int32_t *top, int32_t *refcount, uint64_t *block_hash, int64_t *lru_stamp,
+                   int64_t *clock, int num_blocks) {
     if (num_blocks <= 0) return 1;
     for (int i = 0; i < num_blocks; ++i) {
         free_stack[i] = num_blocks - 1 - i; /* block 0 is popped first */
         refcount[i] = 0;
+        block_hash[i] = 0;
+        lru_stamp[i] = -1;
     }
     *top = num_blocks;
+    *clock = 0;
     return 0;
 }
 
-static int32_t bm_pop(int32_t *free_stack, int32_t *top, int32_t *refcount) {
-    int32_t b = free_stack[--*top];
+/* Blocks allocation can hand out: the free stack and the cached blocks. */
+static int bm_available(const int32_t *top, const int64_t *lru_stamp, int num_blocks) {
+    int n = *top;
+    for (int b = 0; b < num_blocks; ++b)
+        if (lru_stamp[b] >= 0) ++n;
+    return n;
+}
+
+static int32_t bm_pop(int32_t *free_stack, int32_t *top, int32_t *refcount, uint64_t *block_hash, int64_t *lru_stamp,
+                      int num_blocks) {
+    int32_t b = -1;
+    if (*top > 0) {
+        b = free_stack[--*top];
+    } else {
+        for (int c = 0; c < num_blocks; ++c) /* the least recently released cached block */
+            if (lru_stamp[c] >= 0 && (b < 0 || lru_stamp[c] < lru_stamp[b])) b = c;
+        block_hash[b] = 0; /* evicted: its content no longer backs a prefix */
+        lru_stamp[b] = -1;
+    }
     refcount[b] = 1;
     return b;
 }
 
 /* Request r receives counts[r] blocks, written to ids[offsets[r] .. offsets[r+1]).
- * Requests are served in order while the free list and the output room last;
- * the first one that does not fit, and every later one, receives none. */
-int oracle_bm_alloc(int32_t *free_stack, int32_t *top, int32_t *refcount, int num_blocks, const int32_t *counts,
-                    int n, int32_t *offsets, int32_t *ids, int capacity, uint32_t *err) {
+ * Requests are served in order while the free and cached blocks and the
+ * output room last; the first one that does not fit, and every later one,
+ * receives none. */
+int oracle_bm_alloc(int32_t *free_stack, int32_t *top, int32_t *refcount, uint64_t *block_hash, int64_t *lru_stamp,
+                    int64_t *clock, int num_blocks, const int32_t *counts, int n, int32_t *offsets, int32_t *ids,
+                    int capacity, uint32_t *err) {
+    (void)clock;
     if (num_blocks <= 0 || n < 0 || capacity < 0) return 1;
     int failed = 0;
     offsets[0] = 0;
     for (int r = 0; r < n; ++r) {
         int c = counts[r] < 0 ? 0 : counts[r];
-        if (!failed && c <= *top && offsets[r] + c <= capacity) {
-            for (int k = 0; k < c; ++k) ids[offsets[r] + k] = bm_pop(free_stack, top, refcount);
+        if (!failed && c <= bm_available(top, lru_stamp, num_blocks) && offsets[r] + c <= capacity) {
+            for (int k = 0; k < c; ++k)
+                ids[offsets[r] + k] = bm_pop(free_stack, top, refcount, block_hash, lru_stamp, num_blocks);
             offsets[r + 1] = offsets[r] + c;
         } else {
             if (c > 0 || failed) { failed = 1; *err |= BM_ERR_NOSPACE; }
@@ -437,33 +476,32 @@ int oracle_bm_alloc(int32_t *free_stack, int32_t *top, int32_t *refcount, int nu
     return 0;
 }
 
-/* Each listed id drops one reference, in list order; a block whose count
- * reaches zero is pushed back onto the free list at that moment. */
-int oracle_bm_free(int32_t *free_stack, int32_t *top, int32_t *refcount, int num_blocks, const int32_t *ids, int n,
-                   uint32_t *err) {
+/* Each listed id drops one reference, in list order.  A block whose count
+ * reaches zero becomes cached (stamped with the release clock, which then
+ * advances) if it holds a prefix key, and is otherwise pushed back onto the
+ * free stack, at that moment. */
+int oracle_bm_free(int32_t *free_stack, int32_t *top, int32_t *refcount, uint64_t *block_hash, int64_t *lru_stamp,
+                   int64_t *clock, int num_blocks, const int32_t *ids, int n, uint32_t *err) {
     if (num_blocks <= 0 || n < 0) return 1;
     for (int i = 0; i < n; ++i) {
         int32_t b = ids[i];
         if (b < 0 || b >= num_blocks) { *err |= BM_ERR_RANGE; continue; }
         if (refcount[b] <= 0) { *err |= BM_ERR_DOUBLEFREE; continue; }
-        if (--refcount[b] == 0) free_stack[(*top)++] = b;
+        if (--refcount[b] == 0) {
+            if (block_hash[b] != 0) lru_stamp[b] = (*clock)++;
+            else free_stack[(*top)++] = b;
+        }
     }
     return 0;
 }
 
-/* A freed block's content no longer backs a prefix: its cached key is dropped
- * when its count reaches zero (call after oracle_bm_free on the same list). */
-int oracle_bm_drop_hashes(const int32_t *refcount, uint64_t *block_hash, int num_blocks) {
-    for (int b = 0; b < num_blocks; ++b)
-        if (refcount[b] == 0) block_hash[b] = 0;
-    return 0;
-}
-
-/* Each listed id gains one reference (a new sequence maps the block). */
-int oracle_bm_share(int32_t *refcount, int num_blocks, const int32_t *ids, int n, uint32_t *err) {
+/* Each listed id gains one reference (a new sequence maps the block); a cached
+ * block mapped again is no longer evictable. */
+int oracle_bm_share(int32_t *refcount, int64_t *lru_stamp, int num_blocks, const int32_t *ids, int n, uint32_t *err) {
     if (num_blocks <= 0 || n < 0) return 1;
     for (int i = 0; i < n; ++i) {
         if (ids[i] < 0 || ids[i] >= num_blocks) { *err |= BM_ERR_RANGE; continue; }
+        if (refcount[ids[i]] == 0) lru_stamp[ids[i]] = -1;
         refcount[ids[i]] += 1;
     }
     return 0;
@@ -475,15 +513,18 @@ int oracle_bm_share(int32_t *refcount, int num_blocks, const int32_t *ids, int n
  *     copy: a new block, the pair (old, new) appended to pairs, one reference
  *     of the old block dropped (copy-on-write);
  *   - blocks for the logical indices the new tokens reach beyond the table
- *     are popped in logical order;
+ *     are popped in logical order (free stack first, then cached blocks, the
+ *     least recently released first);
  *   - slot_mapping[off_b + t] = table[b][p / bs] * bs + p % bs for position
  *     p = context_lens[b] + t, off_b the sum of num_new over earlier b;
  *   - context_lens[b] grows by num_new[b].
- * A sequence that finds too few free blocks or outgrows its table row, and
- * every later one, is left unchanged with slots -1 (padding). */
-int oracle_bm_append_slots(int32_t *free_stack, int32_t *top, int32_t *refcount, int num_blocks,
-                           int32_t *block_tables, int mbs, int32_t *context_lens, const int32_t *num_new, int B,
-                           int bs, int64_t *slot_mapping, int32_t *pairs, int32_t *num_pairs, uint32_t *err) {
+ * A sequence that finds too few blocks or outgrows its table row, and every
+ * later one, is left unchanged with slots -1 (padding). */
+int oracle_bm_append_slots(int32_t *free_stack, int32_t *top, int32_t *refcount, uint64_t *block_hash,
+                           int64_t *lru_stamp, int64_t *clock, int num_blocks, int32_t *block_tables, int mbs,
+                           int32_t *context_lens, const int32_t *num_new, int B, int bs, int64_t *slot_mapping,
+                           int32_t *pairs, int32_t *num_pairs, uint32_t *err) {
+    (void)clock;
     if (num_blocks <= 0 || B < 0 || bs <= 0 || mbs <= 0) return 1;
     int failed = 0;
     int64_t off = 0;
@@ -509,7 +550,7 @@ int oracle_bm_append_slots(int32_t *free_stack, int32_t *top, int32_t *refcount,
             else if (refcount[cur] > 1) cow = 1;
         }
         if (!failed && n > 0 && last >= mbs) { *err |= BM_ERR_TABLE; failed = 1; }
-        if (!failed && need_new + cow > *top) { *err |= BM_ERR_NOSPACE; failed = 1; }
+        if (!failed && need_new + cow > bm_available(top, lru_stamp, num_blocks)) { *err |= BM_ERR_NOSPACE; failed = 1; }
         if (failed) {
             for (int t = 0; t < n; ++t) slot_mapping[off + t] = -1;
             off += n;
@@ -517,14 +558,15 @@ int oracle_bm_append_slots(int32_t *free_stack, int32_t *top, int32_t *refcount,
         }
         if (cow) {
             int32_t old = row[pos0 / bs];
-            int32_t fresh = bm_pop(free_stack, top, refcount);
+            int32_t fresh = bm_pop(free_stack, top, refcount, block_hash, lru_stamp, num_blocks);
             refcount[old] -= 1;
             row[pos0 / bs] = fresh;
             pairs[2 * *num_pairs] = old;
             pairs[2 * *num_pairs + 1] = fresh;
             *num_pairs += 1;
         }
-        for (int L = first_new; L <= last; ++L) row[L] = bm_pop(free_stack, top, refcount);
+        for (int L = first_new; L <= last; ++L)
+            row[L] = bm_pop(free_stack, top, refcount, block_hash, lru_stamp, num_blocks);
         for (int t = 0; t < n; ++t) {
             int32_t p = pos0 + t;
             slot_mapping[off + t] = (int64_t)row[p / bs] * bs + p % bs;
@@ -662,8 +704,8 @@ int oracle_paged_attention_fp8(const uint16_t *q, const uint8_t *k_cache, const 
  * little-endian int32 bytes and key k_i = FNV-1a over the 16 bytes
  * le64(k_{i-1}) || le64(d_i) (k_{-1} = 0); a key of 0 is stored as 1 (0 marks
  * an empty slot).  The cache maps keys to blocks; a mapping counts only while
- * the block still holds that key (block_hash[b] == key) and is mapped by some
- * sequence (refcount > 0).
+ * the block still holds that key (block_hash[b] == key): allocated, or cached
+ * and not yet evicted.
  * ------------------------------------------------------------------------ */
 static uint64_t fnv1a(uint64_t h, const uint8_t *p, size_t n) {
     for (size_t i = 0; i < n; ++i) {
@@ -708,17 +750,19 @@ static int cache_find(const uint64_t *keys, const int32_t *vals, int cap, uint64
     return -1;
 }
 
-static int valid_holder(int32_t b, uint64_t key, const uint64_t *block_hash, const int32_t *refcount, int nb) {
-    return b >= 0 && b < nb && block_hash[b] == key && refcount[b] > 0;
+static int valid_holder(int32_t b, uint64_t key, const uint64_t *block_hash, int nb) {
+    return b >= 0 && b < nb && block_hash[b] == key;
 }
 
 /* Lookup, in sequence order: the longest run of leading full prompt blocks of
  * sequence s whose keys have a valid holder -- leaving at least one prompt
- * token uncached -- is mapped into its table row (one reference each);
- * num_cached[s] = the tokens covered. */
-int oracle_prefix_lookup(int32_t *refcount, const uint64_t *block_hash, int num_blocks, const uint64_t *ckeys,
-                         const int32_t *cvals, int cap, const int32_t *tokens, const int32_t *query_start, int B,
-                         int bs, int32_t *block_tables, int mbs, int32_t *num_cached) {
+ * token uncached -- is mapped into its table row (one reference each; a
+ * cached holder is taken off the eviction order); num_cached[s] = the tokens
+ * covered. */
+int oracle_prefix_lookup(int32_t *refcount, int64_t *lru_stamp, const uint64_t *block_hash, int num_blocks,
+                         const uint64_t *ckeys, const int32_t *cvals, int cap, const int32_t *tokens,
+                         const int32_t *query_start, int B, int bs, int32_t *block_tables, int mbs,
+                         int32_t *num_cached) {
     if (num_blocks <= 0 || B < 0 || bs <= 0 || mbs <= 0) return 1;
     for (int s = 0; s < B; ++s) {
         int n = query_start[s + 1] - query_start[s];
@@ -730,8 +774,9 @@ int oracle_prefix_lookup(int32_t *refcount, const uint64_t *block_hash, int num_
             uint64_t key = block_key(prev, tokens + query_start[s] + (size_t)i * bs, bs);
             prev = key;
             int32_t b = cache_find(ckeys, cvals, cap, key);
-            if (!valid_holder(b, key, block_hash, refcount, num_blocks)) break;
+            if (!valid_holder(b, key, block_hash, num_blocks)) break;
             block_tables[(size_t)s * mbs + i] = b;
+            if (refcount[b] == 0) lru_stamp[b] = -1;
             refcount[b] += 1;
             ++hits;
         }
@@ -744,7 +789,7 @@ int oracle_prefix_lookup(int32_t *refcount, const uint64_t *block_hash, int num_
  * prompt block i of sequence s (block id table[s][i]) whose key has no valid
  * holder becomes its holder (the first sequence in order wins); a block that
  * already holds its key is left as it is. */
-int oracle_prefix_insert(const int32_t *refcount, uint64_t *block_hash, int num_blocks, uint64_t *ckeys,
+int oracle_prefix_insert(uint64_t *block_hash, int num_blocks, uint64_t *ckeys,
                          int32_t *cvals, int cap, const int32_t *tokens, const int32_t *query_start, int B, int bs,
                          const int32_t *block_tables, int mbs, uint32_t *err) {
     if (num_blocks <= 0 || B < 0 || bs <= 0 || mbs <= 0) return 1;
@@ -762,7 +807,7 @@ int oracle_prefix_insert(const int32_t *refcount, uint64_t *block_hash, int num_
             int slot = -1;
             for (int j = 0; j < cap; ++j)
                 if (ckeys[j] == key) { slot = j; break; }
-            if (slot >= 0 && valid_holder(cvals[slot], key, block_hash, refcount, num_blocks)) continue;
+            if (slot >= 0 && valid_holder(cvals[slot], key, block_hash, num_blocks)) continue;
             if (slot < 0) {
                 for (int j = 0; j < cap; ++j)
                     if (ckeys[j] == 0) { slot = j; break; }

@@ -44,7 +44,9 @@ PIN_TESTS = [
     prefix_pins.test_fnv1a64_published_vectors,
     prefix_pins.test_keys_chain_over_the_prefix,
     prefix_pins.test_worked_example,
-    prefix_pins.test_freed_holder_no_longer_matches,
+    prefix_pins.test_cached_blocks_worked_example,
+    prefix_pins.test_release_keeps_the_key_and_share_revives,
+    prefix_pins.test_allocation_evicts_least_recently_released_first,
     prefix_pins.test_first_sequence_in_order_becomes_holder,
     fp8_pins.test_decode_table_matches_library,
     fp8_pins.test_encode_golden,
@@ -92,17 +94,27 @@ MUTANTS = {
     "partial block reallocated": ("int first_new = (pos0 + bs - 1) / bs;", "int first_new = pos0 / bs + (pos0 > 0);"),
     "slot offset": ("slot_mapping[off + t] = (int64_t)row[p / bs] * bs + p % bs;",
                     "slot_mapping[off + t] = (int64_t)row[p / bs] * bs + t % bs;"),
-    "free pushes early": ("if (--refcount[b] == 0) free_stack[(*top)++] = b;",
-                          "--refcount[b]; free_stack[(*top)++] = b;"),
-    "fifo free list": ("int32_t b = free_stack[--*top];",
-                       "int32_t b = free_stack[0]; memmove(free_stack, free_stack + 1, sizeof(int32_t) * (size_t)(--*top));"),
+    "free pushes early": ("if (--refcount[b] == 0) {", "if (--refcount[b] >= 0) {"),
+    "fifo free list": ("        b = free_stack[--*top];",
+                       "        b = free_stack[0]; memmove(free_stack, free_stack + 1, sizeof(int32_t) * (size_t)(--*top));"),
     # prefix cache: keys without the chain; a holder's validity ignored; the
     # last inserter wins; the whole prompt looked up; FNV's multiply first
     "prefix key unchained": ("buf[i] = (uint8_t)(prev >> (8 * i));", "buf[i] = 0;"),
-    "prefix holder unchecked": ("if (!valid_holder(b, key, block_hash, refcount, num_blocks)) break;",
+    "prefix holder unchecked": ("if (!valid_holder(b, key, block_hash, num_blocks)) break;",
                                 "if (b < 0) break;"),
-    "prefix last inserter wins": ("if (slot >= 0 && valid_holder(cvals[slot], key, block_hash, refcount, num_blocks)) continue;",
+    "prefix last inserter wins": ("if (slot >= 0 && valid_holder(cvals[slot], key, block_hash, num_blocks)) continue;",
                                   "if (0) continue;"),
+    # cached blocks: the key dropped on release (no cached state); the most
+    # recently released block evicted first; eviction keeps the stale key; a
+    # prefix hit leaves the block evictable; cached blocks not counted as
+    # available
+    "release drops key": ("if (block_hash[b] != 0) lru_stamp[b] = (*clock)++;",
+                          "if (0) lru_stamp[b] = (*clock)++;"),
+    "evict most recent": ("lru_stamp[c] < lru_stamp[b]", "lru_stamp[c] > lru_stamp[b]"),
+    "eviction keeps key": ("block_hash[b] = 0; /* evicted", "/* evicted"),
+    "hit not revived": ("if (refcount[b] == 0) lru_stamp[b] = -1;\n            refcount[b] += 1;",
+                        "refcount[b] += 1;"),
+    "cached not available": ("if (lru_stamp[b] >= 0) ++n;", "if (0) ++n;"),
     "prefix whole prompt": ("int look = n > 0 ? (n - 1) / bs : 0;", "int look = n / bs;"),
     "fnv multiply first": ("h ^= p[i];\n        h *= 1099511628211ull;", "h *= 1099511628211ull;\n        h ^= p[i];"),
     # fp8: subnormals one binade off; ties to the odd code; the scale multiplied

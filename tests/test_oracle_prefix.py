@@ -2,7 +2,8 @@
 --enable-prefix-caching; section 2.1's allocation sketch shares a block whose
 prefix matches).  The hash is pinned by FNV-1a's published test vectors; the
 cache by a worked example, by the chaining (equal block contents under
-different prefixes do not match), by invalidation when the holder is freed,
+different prefixes do not match), by the cached state of released keyed
+blocks and their least-recently-released eviction (a second worked example),
 and by a composition pin: a prompt served partly from the cache attends to
 exactly its own tokens."""
 import json
@@ -72,15 +73,110 @@ def test_worked_example():
     assert c3.tolist() == [4]
 
 
-def test_freed_holder_no_longer_matches():
+def _key_names(prompts, bs):
+    """Key value -> name <prompt><block index> for every full block of the prompts."""
+    names = {}
+    for name, p in prompts.items():
+        for i, k in enumerate(oracle.prefix_keys(np.asarray(p, np.int32), bs)):
+            names.setdefault(int(k), f"{name}{i}")
+    return names
+
+
+def run_eviction_example(serve, finish, state):
+    """Replays the cached-block worked example through serve(prompt) ->
+    (num_cached, table row, err) and finish(table row, n_tokens); state() ->
+    (refcount, free stack [:top], lru order, block_hash)."""
+    g = json.load(open(os.path.join(GOLDEN, "prefix_eviction_example.json")))
+    names = _key_names(g["prompts"], g["block_size"])
+    rows = {}
+    for step in g["steps"]:
+        prompt = np.asarray(g["prompts"][step["prompt"]], np.int32)
+        if step["op"] == "serve":
+            cached, row, err = serve(prompt)
+            n_blk = -(-len(prompt) // g["block_size"])
+            assert cached == step["expect_cached"], step
+            assert list(row[:n_blk]) == step["expect_table"], step
+            assert err == step["expect_err"], step
+            rows[step["prompt"]] = row
+        else:
+            finish(rows[step["prompt"]], len(prompt))
+        refcount, free, lru, block_hash = state()
+        assert list(refcount) == step["expect_refcount"], step
+        assert list(free) == step["expect_free"], step
+        assert list(lru) == step["expect_lru"], step
+        keys = {str(b): names[int(h)] for b, h in enumerate(block_hash) if h}
+        assert keys == step["expect_keys"], step
+    return g
+
+
+def test_cached_blocks_worked_example():
+    g = json.load(open(os.path.join(GOLDEN, "prefix_eviction_example.json")))
+    bs = g["block_size"]
+    box = {"st": oracle.bm_init(g["num_blocks"]), "cache": oracle.PrefixCache(g["cache_capacity"])}
+
+    def serve(prompt):
+        tokens = prompt.astype(np.int32)
+        qs = np.array([0, len(prompt)], np.int32)
+        tables = np.full((1, 8), -1, np.int32)
+        st, tables, cached = oracle.prefix_lookup(box["st"], box["cache"], tokens, qs, bs, tables)
+        need = np.array([len(prompt)], np.int32) - cached
+        st, tables, ctx, slots, pairs, err = oracle.bm_append_slots(st, tables, cached, need, bs)
+        st, box["cache"], e2 = oracle.prefix_insert(st, box["cache"], tokens, qs, bs, tables)
+        box["st"] = st
+        return int(cached[0]), tables[0], err | e2
+
+    def finish(row, n):
+        box["st"], err = oracle.bm_free(box["st"], row[:-(-n // bs)])
+        assert err == 0
+
+    def state():
+        st = box["st"]
+        return st.refcount, st.free_stack[:st.top], st.lru_order(), st.block_hash
+
+    run_eviction_example(serve, finish, state)
+
+
+def test_release_keeps_the_key_and_share_revives():
+    """A keyed block whose count reaches zero keeps its key and joins the
+    eviction order; mapping it again (a fork) takes it off; an unkeyed block
+    returns to the free stack."""
     st = oracle.bm_init(16)
     cache = oracle.PrefixCache(32)
     p = np.arange(9, dtype=np.int32)
     st, cache, t, ctx, _, _ = _serve(st, cache, [p])
+    keys = oracle.prefix_keys(p, BS)
     st, _ = oracle.bm_free(st, t[0, :3])
-    assert st.block_hash.max() == 0
+    assert np.array_equal(st.block_hash[t[0, :2]], keys)
+    assert st.lru_order().tolist() == t[0, :2].tolist()
+    assert int(t[0, 2]) in st.free_set() and st.block_hash[t[0, 2]] == 0
+    st, err = oracle.bm_share(st, t[0, 1:2])
+    assert err == 0 and st.lru_order().tolist() == [int(t[0, 0])] and st.refcount[t[0, 1]] == 1
     st2, cache2, t2, _, cached, _ = _serve(st, cache, [p])
-    assert cached.tolist() == [0]
+    assert cached.tolist() == [8] and t2[0, :2].tolist() == t[0, :2].tolist()
+    assert st2.lru_order().tolist() == [] and st2.refcount[t[0, 0]] == 1 and st2.refcount[t[0, 1]] == 2
+
+
+def test_allocation_evicts_least_recently_released_first():
+    """With the free stack empty, bm_alloc hands out cached blocks in release
+    order and drops their keys; a lookup of an evicted prefix then misses."""
+    st = oracle.bm_init(4)
+    cache = oracle.PrefixCache(16)
+    prompts = [np.arange(5, dtype=np.int32) + 100 * i for i in range(2)]  # one full block each, 2 blocks
+    st, cache, t, ctx, _, _ = _serve(st, cache, prompts)
+    assert st.top == 0
+    st, _ = oracle.bm_free(st, [t[1, 0], t[1, 1], t[0, 0], t[0, 1]])  # prompt 1's keyed block is released first
+    assert st.lru_order().tolist() == [int(t[1, 0]), int(t[0, 0])]
+    assert sorted(st.free_set()) == sorted([int(t[1, 1]), int(t[0, 1])])
+    st, off, ids, err = oracle.bm_alloc(st, [3], 8)
+    assert err == 0 and ids[:3].tolist() == [int(t[0, 1]), int(t[1, 1]), int(t[1, 0])]
+    assert st.block_hash[t[1, 0]] == 0 and st.block_hash[t[0, 0]] != 0 and st.lru_order().tolist() == [int(t[0, 0])]
+    tables = np.full((2, 8), -1, np.int32)
+    tokens = np.concatenate(prompts)
+    qs = np.array([0, 5, 10], np.int32)
+    _, _, cached = oracle.prefix_lookup(st, cache, tokens, qs, BS, tables)
+    assert cached.tolist() == [4, 0]  # prompt 0's block is still cached, prompt 1's was evicted
+    st, off, ids, err = oracle.bm_alloc(st, [2], 8)  # one cached block left: the request does not fit
+    assert err == oracle.BM_ERR_NOSPACE and off.tolist() == [0, 0]
 
 
 def test_first_sequence_in_order_becomes_holder():
