@@ -388,7 +388,176 @@ def run_cuda(args, rank, world, dist):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w, budget_s=args.cpu_budget,
                                             single_thread_s=3.0 if w.name in SINGLE_THREAD_WORKLOADS else 0.0)
+    if world == 1 and not args.no_shapes and w.name == "llama2-13b" and not args.max_seqs:
+        del w, kc, vc, out, ws
+        torch.cuda.empty_cache()
+        line["shapes"] = other_shapes(dev, stream)
     return line
+
+
+# --------------------------------------------------------------------------
+# decode-alone timings of the other shapes, reported beside the headline step
+# --------------------------------------------------------------------------
+
+L2_FLUSH_BYTES = 256 << 20  # twice the 126 MB L2
+
+
+def time_calls(fn, stream, n: int, warm: int = 5, between=None):
+    """Median and mean CUDA-event time (us) of `fn` over n calls on `stream`,
+    after `warm` untimed calls.  `between` (untimed, outside the events) runs
+    before every call, e.g. an L2 flush."""
+    for _ in range(warm):
+        if between is not None:
+            between()
+        fn()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+    for a, b in ev:
+        if between is not None:
+            between()
+        a.record(stream)
+        fn()
+        b.record(stream)
+    torch.cuda.synchronize()
+    t = [1e3 * a.elapsed_time(b) for a, b in ev]
+    return statistics.median(t), statistics.fmean(t)
+
+
+def _timed_with_clocks(dev, fn, stream, n, warm=5, between=None):
+    with ClockSampler(dev.index) as clocks:
+        med, mean = time_calls(fn, stream, n, warm, between)
+        time.sleep(0.45)  # at least two clock samples
+    return med, mean, clocks.summary()
+
+
+def decode_shape(pkv, dev, stream, name, bs, pt, peak, n=50, fp8=False, flush=None):
+    """Decode attention alone (plan + attention + reduce) on one of the decode
+    workloads, after its copy-on-write copies and write."""
+    w = workloads.make(name, seed=0, values_device=dev, block_size=bs)
+    slots = torch.from_numpy(w.slot_mapping).to(dev)
+    tables = torch.from_numpy(w.block_tables).to(dev)
+    ctx = torch.from_numpy(w.context_lens).to(dev)
+    out = torch.empty_like(w.q)
+    ws = torch.empty(pkv.decode_workspace_bytes(w.num_seqs, w.num_q_heads, w.num_kv_heads, w.head_dim,
+                                                w.max_context_len, pt), dtype=torch.uint8, device=dev)
+    if fp8:
+        kc, vc, ks, vs = workloads.fp8_pools(w)
+        del w.k_cache, w.v_cache
+        if len(w.copy_pairs):
+            pkv.pkv_copy_blocks(w.copy_pairs, kc, vc, stream=stream)
+        pkv.pkv_write_fp8(w.k_new, w.v_new, slots, ks, vs, kc, vc, stream=stream)
+
+        def call():
+            pkv.paged_attn_decode_fp8(w.q, kc, vc, ks, vs, tables, ctx, w.scale, w.num_kv_heads, out,
+                                      w.max_context_len, pt, workspace=ws, stream=stream)
+    else:
+        kc, vc = w.k_cache, w.v_cache
+        if len(w.copy_pairs):
+            pkv.pkv_copy_blocks(w.copy_pairs, kc, vc, stream=stream)
+        pkv.pkv_write(w.k_new, w.v_new, slots, kc, vc, stream=stream)
+
+        def call():
+            pkv.paged_attn_decode(w.q, kc, vc, tables, ctx, w.scale, w.num_kv_heads, out, w.max_context_len, pt,
+                                  workspace=ws, stream=stream)
+    med, mean, clk = _timed_with_clocks(dev, call, stream, n, between=flush)
+    if pkv.get_device_error():
+        raise RuntimeError(f"device error word set on {name}")
+    nbytes = decode_bytes(w, kv_elem=1 if fp8 else 2)
+    gbs = nbytes / (med * 1e-6) / 1e9
+    rec = {"workload": f"{w.name}: {w.description}", "kv": "e4m3" if fp8 else "bf16", "block_size": w.block_size,
+           "partition_tokens": library_partition_tokens(pt, w.max_context_len), "decode_us": round(med, 2),
+           "decode_us_mean": round(mean, 2), "algorithmic_bytes": int(nbytes), "achieved_gbs": round(gbs, 1),
+           "frac": round(gbs / peak, 4), "calls": n, "clocks": clk}
+    if w.name == "llama3-8b-gqa-prefix":
+        rec["logical_bytes"] = int(logical_decode_bytes(w))
+    del w, kc, vc, out, ws
+    torch.cuda.empty_cache()
+    return rec
+
+
+def prefill_shape(pkv, dev, stream, name, tpeak, n=30):
+    w = workloads.make_prefill(name, seed=0, values_device=dev)
+    slots = torch.from_numpy(w.slot_mapping).to(dev)
+    tables = torch.from_numpy(w.block_tables).to(dev)
+    ctx = torch.from_numpy(w.context_lens).to(dev)
+    qs = torch.from_numpy(w.query_start).to(dev)
+    out = torch.empty_like(w.q)
+    ws = torch.empty(pkv.prefill_workspace_bytes(w.num_seqs, w.num_q_heads, w.num_kv_heads, w.max_query_len),
+                     dtype=torch.uint8, device=dev)
+    pkv.pkv_write(w.k_new, w.v_new, slots, w.k_cache, w.v_cache, stream=stream)
+
+    def call():
+        pkv.paged_attn_prefill(w.q, w.k_cache, w.v_cache, tables, ctx, qs, w.scale, w.num_kv_heads, out,
+                               w.max_query_len, w.max_context_len, workspace=ws, stream=stream)
+    med, mean, clk = _timed_with_clocks(dev, call, stream, n)
+    if pkv.get_device_error():
+        raise RuntimeError(f"device error word set on {name}")
+    flops = prefill_flops(w)
+    tf = flops / (med * 1e-6) / 1e12
+    rec = {"workload": f"{w.name}: {w.description}", "prefill_us": round(med, 2), "prefill_us_mean": round(mean, 2),
+           "algorithmic_flops": flops, "achieved_tflops": round(tf, 1), "frac": round(tf / tpeak, 4), "calls": n,
+           "clocks": clk}
+    del w, out, ws
+    torch.cuda.empty_cache()
+    return rec
+
+
+def copy_shape(pkv, dev, stream, peak, flush, pairs=256, n=50):
+    """pkv_copy_blocks on `pairs` copy-on-write pairs of the Llama-3-8B block
+    shape (8 kv heads x 16 tokens x 128, bf16: 32 KB of K and 32 KB of V per
+    block), sources and destinations distinct, L2 flushed before each call."""
+    rng = np.random.default_rng(7)
+    nb = 4 * pairs
+    kc = torch.randn(nb, 8, 16, 128, device=dev).to(torch.bfloat16)
+    vc = torch.randn(nb, 8, 16, 128, device=dev).to(torch.bfloat16)
+    ids = rng.permutation(nb)[:2 * pairs].astype(np.int32)
+    cp = np.stack([ids[:pairs], ids[pairs:]], axis=1)
+    med, mean, clk = _timed_with_clocks(dev, lambda: pkv.pkv_copy_blocks(cp, kc, vc, stream=stream), stream, n,
+                                        between=flush)
+    blk = kc[0].numel() * 2
+    nbytes = 2 * 2 * pairs * blk  # K and V, read and written
+    gbs = nbytes / (med * 1e-6) / 1e9
+    del kc, vc
+    torch.cuda.empty_cache()
+    return {"workload": f"{pairs} pairs of {2 * blk // 1024} KB blocks (K+V), 8 kv heads, bs16, d128",
+            "copy_us": round(med, 2), "copy_us_mean": round(mean, 2), "algorithmic_bytes": nbytes,
+            "achieved_gbs": round(gbs, 1), "frac": round(gbs / peak, 4), "calls": n, "l2": "256 MB read before each call",
+            "clocks": clk}
+
+
+def other_shapes(dev, stream):
+    """Decode alone at the GQA and long-context shapes (512-token partitions as
+    specified), the 13B decode with and without an L2 flush between calls, the
+    FP8 decode, the chunked prefill and a 256-pair block copy.  Each record
+    carries its own clocks; none of them enters the headline value."""
+    import paged_kv_cache_420_b200 as pkv
+
+    peak, _ = measured_hbm_peak()
+    tpeak, _ = measured_tensor_peak()
+    scratch = torch.ones(L2_FLUSH_BYTES // 8, dtype=torch.int64, device=dev)
+
+    def flush():
+        # a read of twice the L2 size: L2 then holds clean lines of the scratch
+        # (a write would leave dirty lines whose write-back the next call pays)
+        scratch.sum()
+
+    shapes = {}
+    for key, name, bs, pt in (("llama3-8b-gqa-prefix", "llama3-8b-gqa-prefix", 16, 0),
+                              ("llama2-70b-long bs16", "llama2-70b-long", 16, 512),
+                              ("llama2-70b-long bs128", "llama2-70b-long", 128, 512),
+                              ("llama2-7b", "llama2-7b", 16, 0)):
+        shapes[key] = decode_shape(pkv, dev, stream, name, bs, pt, peak)
+    shapes["llama2-13b l2-flushed"] = decode_shape(pkv, dev, stream, "llama2-13b", 16, 0, peak, flush=flush)
+    shapes["llama2-13b l2-flushed"]["l2"] = "256 MB read before each call"
+    shapes["llama2-13b unflushed"] = decode_shape(pkv, dev, stream, "llama2-13b", 16, 0, peak)
+    shapes["llama2-13b-fp8"] = decode_shape(pkv, dev, stream, "llama2-13b", 16, 0, peak, fp8=True)
+    shapes["llama3-8b-gqa-prefix-fp8"] = decode_shape(pkv, dev, stream, "llama3-8b-gqa-prefix", 16, 0, peak,
+                                                      fp8=True)
+    for name in workloads.PREFILL_WORKLOADS:
+        shapes[name] = prefill_shape(pkv, dev, stream, name, tpeak)
+    shapes["copy_blocks 256 pairs"] = copy_shape(pkv, dev, stream, peak, flush)
+    del scratch
+    torch.cuda.empty_cache()
+    return shapes
 
 
 def prefill_flops(w) -> float:
@@ -1097,6 +1266,8 @@ def main(argv=None):
     ap.add_argument("--max-seqs", type=int, default=0, help="time only the first N sequences (profiling)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-shapes", action="store_true",
+                    help="skip the decode-alone timings of the other shapes after the headline step")
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work for cpu_baseline")
     args = ap.parse_args(argv)
     args.warmup = max(args.warmup, 3)

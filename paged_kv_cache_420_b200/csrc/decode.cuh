@@ -63,10 +63,9 @@ struct DecodeParams {
     const float *v_scale = nullptr;
 };
 
-// Context length of sequence s, clamped to what the table and the workspace
-// can hold.  A value outside [0, cap] is reported (once, by the planner).
-__device__ __forceinline__ int clamped_context(const DecodeParams &p, int s, bool report) {
-    const int n = __ldg(p.context_lens + s);
+// A context length clamped to what the table and the workspace can hold.  A
+// value outside [0, cap] is reported (once, by the planner).
+__device__ __forceinline__ int clamp_context(const DecodeParams &p, int n, bool report) {
     const long long table_cap = (long long)p.MBS * p.bs;
     const int cap = (int)min(table_cap, (long long)p.max_ctx);
     if (n < 0 || n > cap) {
@@ -76,31 +75,43 @@ __device__ __forceinline__ int clamped_context(const DecodeParams &p, int s, boo
     return n;
 }
 
+__device__ __forceinline__ int clamped_context(const DecodeParams &p, int s, bool report) {
+    return clamp_context(p, __ldg(p.context_lens + s), report);
+}
+
 // ------------------------------------------------------------- planner ----
-// Writes entries[] = (s, partition) for every sequence and partition, in
-// sequence-major order, and the count, and zeroes the attention kernel's work
-// counter.  Zero-length sequences get a zero output row here (they have no
-// items).
+// Entry flag: the entry is a partition group, W consecutive partitions
+// (part .. part + W - 1) of one sequence.  Its W partitions stream
+// interleaved, one per consumer warp, and each warp writes its partition's
+// (m, l, acc) record itself, so the item needs no merge across warps.
+constexpr int kGroupFlag = 1 << 30;
+
+// Partition groups of a sequence with `parts` partitions: only split calls
+// (the records go to the workspace anyway) on the tensor-core path (a group
+// saves the merge of W multi-head partials; on the single-head CUDA-core path
+// the merge is cheap and groups measured slower), and only whole groups of W.
+__device__ __forceinline__ int group_count(const DecodeParams &p, int parts) {
+    return (p.maxP > 1 && p.g > 1) ? parts / kConsumerWarps : 0;
+}
+
+// Writes the entry list and its count, and zeroes the attention kernel's work
+// counter.  Every sequence's partition groups come first, then the remaining
+// single partitions (each sequence-major): the large items are claimed first
+// and the small ones fill the end of the kernel.  Zero-length sequences get a
+// zero output row here (they have no items).
 __global__ void __launch_bounds__(kPlanThreads) plan_kernel(DecodeParams p, int D) {
-    __shared__ int s_off[kPlanThreads + 1];
+    __shared__ int s_goff[kPlanThreads + 1], s_soff[kPlanThreads + 1];
+    __shared__ int s_n[kPlanThreads];
     __shared__ int s_warp[kPlanThreads / 32];
-    __shared__ int s_carry, s_any_zero;
+    __shared__ int s_any_zero;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     // The attention kernel may start its prologue now; it waits for this
     // grid's results with griddepcontrol.wait before reading them.
     grid_launch_dependents();
-    if (tid == 0) { s_carry = 0; s_any_zero = 0; }
+    if (tid == 0) s_any_zero = 0;
     __syncthreads();
-    for (int base = 0; base < p.B; base += kPlanThreads) {
-        const int s = base + tid;
-        int parts = 0;
-        if (s < p.B) {
-            const int n = clamped_context(p, s, true);
-            parts = (n + p.PT - 1) / p.PT;
-            if (n == 0) s_any_zero = 1;
-        }
-        // block-wide inclusive scan of parts
-        int x = parts;
+    // block-wide inclusive scan of one int per thread (all threads return)
+    auto scan = [&](int x) {
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
             const int y = __shfl_up_sync(0xffffffffu, x, o);
@@ -119,29 +130,73 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(DecodeParams p, int 
         }
         __syncthreads();
         const int incl = x + (warp > 0 ? s_warp[warp - 1] : 0);
-        s_off[tid + 1] = incl;
-        if (tid == 0) s_off[0] = 0;
+        __syncthreads();  // s_warp reusable
+        return incl;
+    };
+    // Single partitions go after all groups: with more sequences than one
+    // chunk the total of groups is counted first.
+    int groups_total = 0;
+    if (p.B > kPlanThreads) {
+        for (int base = 0; base < p.B; base += kPlanThreads) {
+            const int s = base + tid;
+            int c = 0;
+            if (s < p.B) c = group_count(p, (clamped_context(p, s, false) + p.PT - 1) / p.PT);
+            const int incl = scan(c);
+            if (tid == kPlanThreads - 1) s_goff[kPlanThreads] = incl;  // the chunk's total
+            __syncthreads();
+            groups_total += s_goff[kPlanThreads];
+            __syncthreads();
+        }
+    }
+    int carry_g = 0, carry_s = 0;
+    for (int base = 0; base < p.B; base += kPlanThreads) {
+        const int s = base + tid;
+        int groups = 0, singles = 0, n = 0;
+        if (s < p.B) {
+            n = clamped_context(p, s, true);
+            const int parts = (n + p.PT - 1) / p.PT;
+            groups = group_count(p, parts);
+            singles = parts - groups * kConsumerWarps;
+            if (n == 0) s_any_zero = 1;
+        }
+        s_n[tid] = n;
+        const int ig = scan(groups);
+        const int is = scan(singles);
+        s_goff[tid + 1] = ig;
+        s_soff[tid + 1] = is;
+        if (tid == 0) { s_goff[0] = 0; s_soff[0] = 0; }
         __syncthreads();
-        const int chunk_total = s_off[kPlanThreads];
-        const int carry = s_carry;
-        // cooperative fill: entry e of this chunk belongs to the last seq whose
-        // exclusive offset is <= e
-        for (int e = tid; e < chunk_total; e += kPlanThreads) {
+        const int chunk_g = s_goff[kPlanThreads], chunk_s = s_soff[kPlanThreads];
+        if (p.B <= kPlanThreads) groups_total = chunk_g;
+        // cooperative fill: entry e of this chunk belongs to the last seq
+        // whose exclusive offset is <= e
+        for (int e = tid; e < chunk_g + chunk_s; e += kPlanThreads) {
+            const bool is_group = e < chunk_g;
+            const int *off = is_group ? s_goff : s_soff;
+            const int ee = is_group ? e : e - chunk_g;
             int lo = 0, hi = kPlanThreads - 1;
             while (lo < hi) {
                 const int mid = (lo + hi + 1) >> 1;
-                if (s_off[mid] <= e) lo = mid; else hi = mid - 1;
+                if (off[mid] <= ee) lo = mid; else hi = mid - 1;
             }
-            p.entries[carry + e] = make_int2(base + lo, e - s_off[lo]);
+            const int i = ee - off[lo];
+            if (is_group) {
+                p.entries[carry_g + ee] = make_int2(base + lo, (i * kConsumerWarps) | kGroupFlag);
+            } else {
+                const int parts = (s_n[lo] + p.PT - 1) / p.PT;
+                p.entries[groups_total + carry_s + ee] =
+                    make_int2(base + lo, group_count(p, parts) * kConsumerWarps + i);
+            }
         }
-        __syncthreads();
-        if (tid == 0) s_carry = carry + chunk_total;
+        carry_g += chunk_g;
+        carry_s += chunk_s;
         __syncthreads();
     }
     if (tid == 0) {
-        *p.num_entries = s_carry;
+        *p.num_entries = carry_g + carry_s;
         *p.work_counter = 0;
     }
+    __syncthreads();
     if (s_any_zero) {
         const int vec_per_seq = p.Hq * D / 8;
         uint4 *out = reinterpret_cast<uint4 *>(p.out);
@@ -154,11 +209,37 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(DecodeParams p, int 
 
 // ------------------------------------------------------ attention kernel ----
 
-struct StageInfo {
-    int s, h, part, nparts;  // item
-    int k, npad;             // stage index within the item, stages padded to a multiple of W
-    int valid;               // valid tokens in this stage (0 = padding stage)
-    int ord;                 // CTA-local item ordinal (selects the q buffer); -1 ends the stream
+struct __align__(16) StageInfo {
+    int s, h;
+    int part;    // first partition, | kGroupFlag for a partition group (warp w owns partition part + w)
+    int nparts;  // partitions of the sequence
+    int k, npad; // stage index within the item, stages padded to a multiple of W
+    int valid;   // valid tokens in this stage (0 = padding stage)
+    int ord;     // CTA-local item ordinal (selects the q buffer); -1 ends the stream
+};
+
+// An item as the producer sees it.  A single partition streams its stages in
+// order; a partition group interleaves its W partitions (stage K is stage
+// K / W of partition part + K % W), so consumer warp w, which takes stages
+// w, w + W, ..., walks partition part + w alone.
+static_assert(kConsumerWarps == 4, "a partition group is 4 partitions: stage K -> (K & 3, K >> 2)");
+
+struct ItemMeta {
+    int s, h, part, grp, n, nparts;
+    int npad;  // stages, padded to a multiple of W
+
+    // partition (relative to part) and first token of stage K
+    __device__ __forceinline__ int stage_sub(int K) const { return grp ? (K & 3) : 0; }
+    __device__ __forceinline__ int stage_token(int K, int PT) const {
+        return (part + stage_sub(K)) * PT + (grp ? (K >> 2) : K) * kStageTok;
+    }
+    // valid tokens of stage K (0: a padding stage)
+    __device__ __forceinline__ int stage_valid(int K, int PT) const {
+        const int sub = stage_sub(K);
+        const int tok = stage_token(K, PT);
+        const int t1 = min(n, (part + sub + 1) * PT);
+        return tok < t1 ? min(kStageTok, t1 - tok) : 0;
+    }
 };
 
 template <int D, int GP, int NS, bool KV8 = false>
@@ -184,20 +265,43 @@ struct DecodeSmem {
     static constexpr int kAlloc = kBytes;  // the dynamic window is 1 KB-aligned (checked in the kernel)
 };
 
-// Bounded wait that also gives up when another warp has aborted.
+// Bounded wait that also gives up when another warp has aborted.  After the
+// first test the warp sleeps on the barrier (up to kWaitSleepNs per test, woken
+// by the phase's completion), so waiting warps do not take issue slots from
+// the warps that compute.
+constexpr uint32_t kWaitSleepNs = 20000;
 __device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
                                               uint64_t limit_ns = kWaitLimitNs) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_timer_ns();
-    for (uint32_t it = 1;; ++it) {
+    while (true) {
+        if (mbar_try_wait_sleep(bar, parity, kWaitSleepNs)) return true;
+        if (*abort_flag) return false;
+        if (global_timer_ns() - t0 > limit_ns) {
+            raise_error(PKV_DEVERR_TIMEOUT);
+            *abort_flag = 1;
+            return false;
+        }
+    }
+}
+
+// The producer's wait for a free ring slot.  The consumers free slots at the
+// rate they compute, so while the ring is full the producer backs off with a
+// short sleep between tests instead of spinning: on the CUDA-core path the
+// consumer warps are close to issue-bound and a spinning producer (one per
+// CTA, up to six CTAs per SM) would take their issue slots.
+constexpr uint32_t kProducerBackoffNs = 128;
+__device__ __forceinline__ bool wait_slot(uint64_t *bar, uint32_t parity, volatile int *abort_flag) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_timer_ns();
+    while (true) {
+        __nanosleep(kProducerBackoffNs);
         if (mbar_try_wait(bar, parity)) return true;
-        if ((it & 255u) == 0) {
-            if (*abort_flag) return false;
-            if (global_timer_ns() - t0 > limit_ns) {
-                raise_error(PKV_DEVERR_TIMEOUT);
-                *abort_flag = 1;
-                return false;
-            }
+        if (*abort_flag) return false;
+        if (global_timer_ns() - t0 > kWaitLimitNs) {
+            raise_error(PKV_DEVERR_TIMEOUT);
+            *abort_flag = 1;
+            return false;
         }
     }
 }
@@ -393,6 +497,23 @@ struct SimtState {
                 }
             }
         }
+    }
+
+    // Writes this warp's (m, l, acc) as the split-K record of partition part of
+    // query head `head` (a partition the warp walked alone).
+    template <class Params>
+    __device__ __forceinline__ void store_record(const Params &p, size_t head, int part, int lane) {
+        float l = l_part;
+#pragma unroll
+        for (int o = 2; o < 32; o <<= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
+        const size_t pi = head * p.maxP + part;
+        float *dst = p.part_acc + pi * D + lane * EPL;
+        if constexpr (EPL == 4) {
+            *reinterpret_cast<float4 *>(dst) = make_float4(acc[0], acc[1], acc[2], acc[3]);
+        } else {
+            *reinterpret_cast<float2 *>(dst) = make_float2(acc[0], acc[1]);
+        }
+        if (lane == 0) p.part_ml[pi] = make_float2(m, l);
     }
 
     // Writes this warp's partial (m, l, acc) into the merge buffers.
@@ -603,6 +724,34 @@ struct MmaState {
         }
     }
 
+    // Writes this warp's (m, l, O) of every head of the group as the split-K
+    // records of partition part (a partition the warp walked alone); head0 is
+    // the group's first query head.
+    template <class Params>
+    __device__ __forceinline__ void store_record(const Params &p, size_t head0, int part, int lane) {
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
+                float lsum = l[nt][c];
+                lsum += __shfl_xor_sync(0xffffffffu, lsum, 4);
+                lsum += __shfl_xor_sync(0xffffffffu, lsum, 8);
+                lsum += __shfl_xor_sync(0xffffffffu, lsum, 16);
+                const int head = nt * 8 + 2 * (lane & 3) + c;
+                if (head < p.g) {
+                    const size_t pi = (head0 + head) * p.maxP + part;
+                    if (lane < 4) p.part_ml[pi] = make_float2(m[nt][c], lsum);
+                    float *row = p.part_acc + pi * D;
+#pragma unroll
+                    for (int mt = 0; mt < MT; ++mt) {
+                        row[mt * 16 + (lane >> 2)] = o[nt][mt][c];
+                        row[mt * 16 + (lane >> 2) + 8] = o[nt][mt][c + 2];
+                    }
+                }
+            }
+        }
+    }
+
     __device__ __forceinline__ void store_partial(float *mO, float *mM, float *mL, int w, int lane, int stride,
                                                   int GPn, int g) {
 #pragma unroll
@@ -684,75 +833,122 @@ __global__ void __launch_bounds__(kDecodeThreads) paged_decode_kernel(const __gr
 
     if (warp == W) {
         // ------------------------------------------------------ producer --
-        // Items are claimed from a global counter (dynamic load balance); the
-        // claim of the next item is issued one item ahead so that its latency
-        // overlaps the current item's stage issue.
+        // Items are claimed from a global counter (dynamic load balance).  The
+        // next item's claim, entry, context length, first 32 table entries
+        // and query tile are fetched while the current item streams, so the
+        // ring does not drain at item boundaries.
         const int n_items = *reinterpret_cast<volatile int32_t *>(p.num_entries) * p.Hkv;
         uint32_t gc = 0;
-        int ord = 0;
         bool ok = true;
+        // entry -> item geometry; n_raw is the sequence's context length as loaded
+        auto describe = [&](int it, int2 sp, int n_raw) {
+            ItemMeta m;
+            const int e = it / p.Hkv;
+            m.h = it - e * p.Hkv;
+            m.s = sp.x;
+            m.grp = (sp.y & kGroupFlag) ? 1 : 0;
+            m.part = sp.y & ~kGroupFlag;
+            m.n = clamp_context(p, n_raw, false);
+            m.nparts = (m.n + p.PT - 1) / p.PT;
+            if (m.grp) {
+                m.npad = kConsumerWarps * (p.PT / kStageTok);
+            } else {
+                const int t0 = m.part * p.PT;
+                const int nst = (min(m.n, t0 + p.PT) - t0 + kStageTok - 1) / kStageTok;
+                m.npad = (nst + W - 1) / W * W;
+            }
+            return m;
+        };
+        // table entry of stage K of the item whose entry is sp (lane-parallel):
+        // loaded whenever the index lies inside the row, checked only when the
+        // stage holds tokens
+        auto table_entry = [&](int2 sp, int K) {
+            ItemMeta m;
+            m.grp = (sp.y & kGroupFlag) ? 1 : 0;
+            m.part = sp.y & ~kGroupFlag;
+            const int idx = m.stage_token(K, p.PT) / p.bs;
+            return idx < p.MBS ? __ldg(p.block_tables + (size_t)sp.x * p.MBS + idx) : -1;
+        };
+        int q_last = -1;  // ord of the last query tile load issued
+        auto load_q = [&](int it, int2 sp, int ord) -> bool {
+            bool r = true;
+            if (lane == 0) {
+                const int qb = ord & 1;
+                r = wait_or_abort(&qempty[qb], ((ord >> 1) & 1) ^ 1, abort_flag);
+                if (r) {
+                    const int h = it - (it / p.Hkv) * p.Hkv;
+                    const uint32_t bytes = (uint32_t)(p.g * D * 2);
+                    mbar_arrive_expect_tx(&qfull[qb], bytes);
+                    bulk_load(qbuf + qb * (L::kQBuf / 2), p.q + ((size_t)sp.x * p.Hq + (size_t)h * p.g) * D, bytes,
+                              &qfull[qb]);
+                    q_last = ord;
+                }
+            }
+            return __shfl_sync(0xffffffffu, r, 0);
+        };
+
         int claimed = 0;
         if (lane == 0) claimed = atomicAdd(p.work_counter, 1);
         int it = __shfl_sync(0xffffffffu, claimed, 0);
-        for (; it < n_items && ok; ++ord) {
-            if (lane == 0) claimed = atomicAdd(p.work_counter, 1);
-            const int e = it / p.Hkv;
-            const int h = it - e * p.Hkv;
-            const int2 sp = p.entries[e];
-            const int s = sp.x, part = sp.y;
-            const int n = clamped_context(p, s, false);
-            const int nparts = (n + p.PT - 1) / p.PT;
-            const int t0 = part * p.PT;
-            const int t1 = min(n, t0 + p.PT);
-            const int nst = (t1 - t0 + kStageTok - 1) / kStageTok;
-            const int npad = (nst + W - 1) / W * W;
-            if (lane == 0) {
-                const int qb = ord & 1;
-                ok = wait_or_abort(&qempty[qb], ((ord >> 1) & 1) ^ 1, abort_flag);
-                if (ok) {
-                    const uint32_t bytes = (uint32_t)(p.g * D * 2);
-                    mbar_arrive_expect_tx(&qfull[qb], bytes);
-                    bulk_load(qbuf + qb * (L::kQBuf / 2), p.q + ((size_t)s * p.Hq + (size_t)h * p.g) * D, bytes,
-                              &qfull[qb]);
+        int2 sp = make_int2(0, 0);
+        int n_raw = 0, blk_first = -1;
+        if (it < n_items) {
+            sp = p.entries[it / p.Hkv];
+            n_raw = __ldg(p.context_lens + sp.x);
+            blk_first = table_entry(sp, lane);
+            ok = load_q(it, sp, 0);
+        }
+        if (lane == 0) claimed = atomicAdd(p.work_counter, 1);  // the next item, one ahead
+        for (int ord = 0; it < n_items && ok; ++ord) {
+            const ItemMeta cur = describe(it, sp, n_raw);
+            // The next item's fetch chain, one step per pass (each step uses
+            // what the previous one loaded): claim -> entry -> context length,
+            // table entries and query tile.
+            int nxt = n_items, pf = 0, n_next = 0, blk_next = -1;
+            int2 sp_next = make_int2(0, 0);
+            auto prefetch_step = [&]() {
+                if (pf == 0) {
+                    nxt = __shfl_sync(0xffffffffu, claimed, 0);
+                    if (nxt < n_items) sp_next = p.entries[nxt / p.Hkv];
+                } else if (nxt < n_items) {
+                    n_next = __ldg(p.context_lens + sp_next.x);
+                    blk_next = table_entry(sp_next, lane);
+                    ok = load_q(nxt, sp_next, ord + 1) && ok;
                 }
-            }
-            ok = __shfl_sync(0xffffffffu, ok, 0);
+                ++pf;
+            };
             // Stages go out in groups of W, one per consumer warp: lane j < W
             // issues stage k0 + j into slot (gc + j) % NS, so one pass of the
             // warp issues W stages (waits, descriptors and TMA in lockstep).
-            int blk_reg = -1;
-            for (int k0 = 0; k0 < npad && ok; k0 += W) {
+            // Per 32 stages, lane l works out stage (k0 & ~31) + l once: its
+            // valid tokens and its TMA row, from the table entry loaded a
+            // chunk earlier; the issuing lanes take them by shuffle.
+            int blk_chunk = blk_first, row_reg = 0, valid_reg = 0;
+            for (int k0 = 0; k0 < cur.npad && ok; k0 += W) {
                 if ((k0 & 31) == 0) {
-                    // lane l fetches the block id of stage k0 + l
-                    const int kk = k0 + lane;
-                    int blk = -1;
-                    if (kk < nst) {
-                        const int tok = t0 + kk * kStageTok;
-                        blk = __ldg(p.block_tables + (size_t)s * p.MBS + tok / p.bs);
-                        if (blk < 0 || blk >= p.NB) {
-                            raise_error(PKV_DEVERR_BLOCK);
-                            blk = -1;
-                        }
+                    const int K = k0 + lane;
+                    valid_reg = K < cur.npad ? cur.stage_valid(K, p.PT) : 0;
+                    row_reg = p.pool_rows;  // an invalid id reads the zero fill
+                    if (valid_reg > 0) {
+                        if (blk_chunk < 0 || blk_chunk >= p.NB) raise_error(PKV_DEVERR_BLOCK);
+                        else row_reg = (blk_chunk * p.Hkv + cur.h) * p.bs + cur.stage_token(K, p.PT) % p.bs;
                     }
-                    blk_reg = blk;
+                    blk_chunk = k0 + 32 < cur.npad ? table_entry(sp, K + 32) : -1;  // the next chunk's
                 }
-                const int k = k0 + lane;
-                const int blk = __shfl_sync(0xffffffffu, blk_reg, k & 31);
+                const int src = (k0 + lane) & 31;
+                const int row = __shfl_sync(0xffffffffu, row_reg, src);
+                const int valid = __shfl_sync(0xffffffffu, valid_reg, src);
                 bool lane_ok = true;
                 if (lane < W) {
                     const uint32_t g = gc + lane;
                     const uint32_t slot = g % NS;
-                    lane_ok = wait_or_abort(&empty[slot], ((g / NS) & 1) ^ 1, abort_flag);
+                    lane_ok = wait_slot(&empty[slot], ((g / NS) & 1) ^ 1, abort_flag);
                     if (lane_ok) {
-                        const int tok = t0 + k * kStageTok;
-                        const int valid = k < nst ? min(kStageTok, t1 - tok) : 0;
                         StageInfo si;
-                        si.s = s; si.h = h; si.part = part; si.nparts = nparts;
-                        si.k = k; si.npad = npad; si.valid = valid; si.ord = ord;
+                        si.s = cur.s; si.h = cur.h; si.part = cur.part | (cur.grp ? kGroupFlag : 0);
+                        si.nparts = cur.nparts; si.k = k0 + lane; si.npad = cur.npad; si.valid = valid; si.ord = ord;
                         info[slot] = si;
                         if (valid > 0) {
-                            // rows of (block, head, offset): an invalid id reads the zero fill
-                            const int row = blk >= 0 ? (blk * p.Hkv + h) * p.bs + tok % p.bs : p.pool_rows;
                             const uint32_t kt = tiles + slot * L::kStage;
                             mbar_arrive_expect_tx(&full[slot], (uint32_t)L::kStage);
 #pragma unroll
@@ -766,10 +962,16 @@ __global__ void __launch_bounds__(kDecodeThreads) paged_decode_kernel(const __gr
                         }
                     }
                 }
-                ok = __all_sync(0xffffffffu, lane_ok);
+                ok = __all_sync(0xffffffffu, lane_ok) && ok;
                 gc += W;
+                if (pf < 2) prefetch_step();
             }
-            it = __shfl_sync(0xffffffffu, claimed, 0);
+            while (ok && pf < 2) prefetch_step();  // a short item: finish the chain here
+            if (lane == 0) claimed = atomicAdd(p.work_counter, 1);  // the item after next
+            it = nxt;
+            sp = sp_next;
+            n_raw = n_next;
+            blk_first = blk_next;
         }
         // end-of-stream marker for every consumer warp
         if (lane == 0) {
@@ -782,12 +984,15 @@ __global__ void __launch_bounds__(kDecodeThreads) paged_decode_kernel(const __gr
                 }
                 ++gc;
             }
-            // Drain: every TMA this CTA issued must have landed before exit.
-            // In a normal run the consumers already waited for all of them.
+            // Drain: every TMA and bulk copy this CTA issued must have landed
+            // before exit (the last two query tiles included).  In a normal run
+            // the consumers already waited for all of them.
             if (!ok) {
                 const uint32_t issued = gc;
                 for (uint32_t c = (issued > (uint32_t)NS ? issued - NS : 0); c < issued; ++c)
                     mbar_wait_bounded(&full[c % NS], (c / NS) & 1, kWaitLimitNs);
+                for (int o = max(0, q_last - 1); o <= q_last; ++o)
+                    mbar_wait_bounded(&qfull[o & 1], (o >> 1) & 1, kWaitLimitNs);
             }
         }
         grid_launch_dependents();
@@ -830,7 +1035,15 @@ __global__ void __launch_bounds__(kDecodeThreads) paged_decode_kernel(const __gr
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[slot]);
             gc += W;
-            if (si.k + W >= si.npad) {
+            const bool grp = (si.part & kGroupFlag) != 0;
+            if (grp && si.k + W >= si.npad) {
+                // partition group: this warp walked partition part + w alone
+                // and writes its record itself, no merge with the other warps
+                const size_t unit_head0 = (size_t)si.s * p.Hq + (size_t)si.h * p.g;
+                const int part = (si.part & ~kGroupFlag) + w;
+                if constexpr (PATH == 0) st0.store_record(p, unit_head0, part, lane);
+                else st1.store_record(p, unit_head0, part, lane);
+            } else if (si.k + W >= si.npad) {
                 // this warp's last stage of the item: merge the W partials
                 if (!wait_or_abort(mempty, (mc & 1) ^ 1, abort_flag)) break;
                 if constexpr (PATH == 0) st0.store_partial(mO, mM, mL, w, lane, L::kMergeStride);

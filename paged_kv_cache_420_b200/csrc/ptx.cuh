@@ -58,6 +58,22 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
     return done != 0;
 }
 
+// The same test, but a thread whose phase is not complete may be suspended for
+// up to `hint_ns` nanoseconds (it resumes as soon as the phase completes):
+// a waiting warp sleeps instead of spinning, leaving issue slots to the warps
+// that have work.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t *bar, uint32_t parity, uint32_t hint_ns) {
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+        : "memory");
+    return done != 0;
+}
+
 // Bounded wait for the phase with the given parity.  Gives up after about
 // `limit_ns` nanoseconds (checked every 256 polls), sets PKV_DEVERR_TIMEOUT
 // and returns false; the caller then stops issuing work and drains.

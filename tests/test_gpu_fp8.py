@@ -64,6 +64,8 @@ CASES = [
     ([200, 511, 1000], 64, 8, 256),          # g = 8, split-K
     ([50, 129], 12, 4, 0),                   # g = 3 (padded to 4)
     ([33, 700], 16, 1, 0),                   # g = 16
+    ([2048, 2047, 2049, 1537, 2576], 8, 8, 512),   # partition groups, MHA
+    ([2048, 2047, 2049, 1537, 2576], 32, 8, 256),  # partition groups, g = 4
 ]
 
 

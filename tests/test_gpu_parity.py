@@ -152,6 +152,11 @@ DECODE_CASES = [
     ([1111, 7, 300], 32, 2, 128, 16, 256),              # g = 16 (two n-tiles)
     ([1111, 7, 300], 16, 1, 64, 64, 0),                 # g = 16, d 64, bs 64
     ([15, 16, 17, 31, 32, 33, 47, 48, 49], 2, 1, 128, 16, 32),  # boundaries around stages/partitions
+    # partition groups (4 partitions, one per consumer warp): whole groups, a
+    # ragged last partition inside a group, groups followed by single partitions
+    ([2048, 2047, 2049, 1537, 1535, 2576], 8, 8, 128, 16, 512),    # MHA (CUDA-core path)
+    ([2048, 2047, 2049, 1537, 1535, 2576], 32, 8, 128, 16, 256),   # g = 4 (tensor-core path)
+    ([2048, 2047, 2049, 1537, 1535, 2576], 16, 1, 64, 32, 128),    # g = 16, d 64
 ]
 
 
@@ -257,6 +262,18 @@ def test_bad_block_id_and_context_are_reported():
     assert pkv.get_device_error() & pkv.DEVERR_CONTEXT
     ref = oracle.paged_attention(w.q, w.k_cache, w.v_cache, w.block_tables, np.array([64, 64], np.int32), w.scale)
     assert_attention_close(out, ref, "clamped ctx")
+    # the same bad id inside a partition group (16-token partitions: one group of 4)
+    ws = torch.empty(pkv.decode_workspace_bytes(2, 4, 4, 128, 64, 16), dtype=torch.uint8, device="cuda")
+    pkv.paged_attn_decode(w.q, w.k_cache, w.v_cache, t, d["ctx"], w.scale, 4, out, max_context_len=64,
+                          partition_tokens=16, workspace=ws)
+    assert pkv.get_device_error() & pkv.DEVERR_BLOCK
+    assert torch.isfinite(out.float()).all()
+    good = torch.empty_like(out)
+    pkv.paged_attn_decode(w.q, w.k_cache, w.v_cache, d["tables"], d["ctx"], w.scale, 4, good, max_context_len=64,
+                          partition_tokens=16, workspace=ws)
+    torch.cuda.synchronize()
+    assert pkv.get_device_error() == 0
+    assert torch.equal(out[1], good[1])  # the other sequence is untouched by the bad entry
 
 
 def test_many_sequences_over_planner_chunk():
@@ -267,4 +284,16 @@ def test_many_sequences_over_planner_chunk():
     okc, ovc, ref = oracle.decode_step(w)
     assert bits_equal(kc, okc)
     assert_attention_close(out, ref, "1300 seqs")
+    no_device_error()
+
+
+def test_many_sequences_with_partition_groups():
+    """More than 1024 sequences with partition groups: the planner lists the
+    groups of every chunk before all single partitions."""
+    lens = list(np.random.default_rng(12).integers(1, 200, size=1500))
+    w = to_cuda(workloads.make_custom(lens, 8, 2, 64, 16, seed=12, partition_tokens=32))
+    kc, vc, out = run_step(w)
+    okc, ovc, ref = oracle.decode_step(w)
+    assert bits_equal(kc, okc)
+    assert_attention_close(out, ref, "1500 seqs, groups")
     no_device_error()
