@@ -319,20 +319,37 @@ pkv_status paged_attn_decode_fp8(const void *q, const void *k_cache, const void 
  * (wkbse.com section 3.1, "flexible memory management": blocks allocated only
  * as new tokens need them, the block table updated, blocks returned when a
  * sequence ends; "KV cache sharing": parallel samples map the same physical
- * blocks; intelliparadigm.com section 2.1, items 1-2 and the allocation
+ * blocks; intelliparadigm.com section 2.1, items 1-3 and the allocation
  * sketch: a free list popped on allocation, copy-on-write for shared
- * prefixes), so a serving step needs no host round trip.
+ * prefixes, a block free, allocated or shareable, LRU for block heat), so a
+ * serving step needs no host round trip.
+ *
+ * Block states: free (on the free stack), allocated (refcount > 0), cached
+ * (refcount 0 but still holding a prefix key: a prefix lookup can map it
+ * again).  A block whose count reaches zero is cached if it holds a key and
+ * free otherwise.  Allocation pops the free stack first; when it is empty it
+ * evicts cached blocks, the least recently released first, dropping their
+ * keys.  A prefix hit or a share on a cached block takes it off the eviction
+ * order.
  *
  * State: one device buffer of pkv_bm_state_bytes(num_blocks), 256-B aligned,
- * owned by the caller, laid out as
- *   int32 [0] top, [1] error word (PKV_BM_ERR_* bits; the caller clears it)
+ * owned by the caller (num_blocks <= 2^29), laid out as
+ *   int32 [0] top, [1] error word (PKV_BM_ERR_* bits; the caller clears it),
+ *         [2] cached blocks, [3] and [4] head and tail of the eviction order
  *   at 256:            int32 free_stack[num_blocks]  (free_stack[0 .. top) are free,
  *                      the next allocation pops free_stack[top - 1])
  *   at 256 + A:        int32 refcount[num_blocks]     (sequences mapping each block)
  *   at 256 + 2A..4A:   three int32 scratch arrays kept at their rest values
  *   at 256 + 5A:       uint64 block_hash[num_blocks]  (the prefix-cache key a block
- *                      holds, 0: none; cleared when its count reaches zero)
- * with A = num_blocks * 4 rounded up to 256.  Every call is one kernel on
+ *                      holds, 0: none; dropped when the block is evicted)
+ *   at 256 + 5A + H:   uint32 lru_pos[num_blocks]     (a cached block's position in the
+ *                      eviction order; 0xffffffff for any other block)
+ *   at 256 + 6A + H:   int32 ring[2 num_blocks]       (the eviction order: entry at
+ *                      absolute position p is ring[p % (2 num_blocks)], live while
+ *                      lru_pos of its block equals p; head .. tail in release order)
+ *   at 256 + 6A + 2H:  int32 scratch[num_blocks]
+ * with A = num_blocks * 4 and H = num_blocks * 8, each rounded up to 256.
+ * Every call is one kernel on
  * `stream` (one CTA walking its list in order with block-wide scans), so its
  * results are exactly the sequential, request-order ones; device-side
  * failures set bits in the error word and leave the failing request (and,
@@ -345,17 +362,20 @@ pkv_status paged_attn_decode_fp8(const void *q, const void *k_cache, const void 
 #define PKV_BM_ERR_TABLE 8u      /* a sequence outgrew its block-table row, or its context was outside it */
 
 size_t pkv_bm_state_bytes(int32_t num_blocks);
-/* All blocks free, popped 0, 1, 2, ... first; reference counts 0; error word 0. */
+/* All blocks free, popped 0, 1, 2, ... first; reference counts 0; no keys, none
+ * cached; error word 0. */
 pkv_status pkv_bm_init(void *state, int32_t num_blocks, pkv_stream_t stream);
 /* Request r (of n) receives counts[r] blocks (reference count 1) at
  * ids[offsets[r] .. offsets[r+1]) (offsets: int32 [n+1]); requests are served
- * in order while free blocks and the capacity of ids last. */
+ * in order while free and cached blocks and the capacity of ids last. */
 pkv_status pkv_bm_alloc(void *state, int32_t num_blocks, const int32_t *counts, int32_t n, int32_t *offsets,
                         int32_t *ids, int32_t capacity, pkv_stream_t stream);
 /* Every listed block drops one reference, in list order; a block whose count
- * reaches zero is pushed back on the free list at that point. */
+ * reaches zero at that point is cached (appended to the eviction order) if it
+ * holds a prefix key, and otherwise pushed back on the free list. */
 pkv_status pkv_bm_free(void *state, int32_t num_blocks, const int32_t *block_ids, int32_t n, pkv_stream_t stream);
-/* Every listed block gains one reference (a new sequence maps it, e.g. a fork). */
+/* Every listed block gains one reference (a new sequence maps it, e.g. a fork);
+ * a cached block leaves the eviction order. */
 pkv_status pkv_bm_share(void *state, int32_t num_blocks, const int32_t *block_ids, int32_t n, pkv_stream_t stream);
 /*
  * One step's slots for num_new[b] new tokens of each sequence b < num_seqs, in
@@ -370,8 +390,10 @@ pkv_status pkv_bm_share(void *state, int32_t num_blocks, const int32_t *block_id
  * sequences; int64 [slot_capacity]; entries past the capacity are not written
  * and set PKV_BM_ERR_NOSPACE), ready for pkv_write; (4) context_lens[b]
  * grows by num_new[b].  block_tables is int32 [num_seqs][max_blocks_per_seq],
- * updated in place.  The first sequence that finds too few free blocks or
- * outgrows its row, and every later one, is left unchanged with slots -1.
+ * updated in place.  Fresh blocks come from the free stack, then from the
+ * cached blocks (least recently released first).  The first sequence that
+ * finds too few blocks or outgrows its row, and every later one, is left
+ * unchanged with slots -1.
  * Run pkv_copy_blocks_dev on the pairs before writing the new tokens.
  */
 pkv_status pkv_bm_append_slots(void *state, int32_t num_blocks, int32_t *block_tables, int32_t max_blocks_per_seq,
@@ -389,13 +411,15 @@ pkv_status pkv_bm_append_slots(void *state, int32_t num_blocks, int32_t *block_t
  * stored as 1.  The cache is a caller-owned device buffer of
  * pkv_prefix_cache_bytes(capacity) (capacity a power of two, 256-B aligned):
  * an open-addressing table of (key, block) pairs.  An entry counts while its
- * block still holds the key (block_hash) and is mapped (refcount > 0).
+ * block still holds the key (block_hash): allocated, or cached and not yet
+ * evicted.
  * tokens: int32 prompts concatenated, query_start: int32 [num_seqs + 1].
  *
  * pkv_prefix_lookup: for each sequence, the longest run of leading full
  *   prompt blocks with a valid holder -- leaving at least one prompt token to
  *   compute -- is written into its block-table row (int32 [num_seqs]
- *   [max_blocks_per_seq]) with one reference each; num_cached[s] (int32
+ *   [max_blocks_per_seq]) with one reference each (a cached holder leaves the
+ *   eviction order); num_cached[s] (int32
  *   [num_seqs]) = the tokens covered.  Then pkv_bm_append_slots with
  *   context_lens = num_cached and num_new = prompt length - num_cached.
  * pkv_prefix_insert: after the prompt's K/V is written, in sequence order,

@@ -232,21 +232,44 @@ def bm_state_bytes(num_blocks: int) -> int:
 
 
 class BlockManager:
-    """The block manager's state on the device (free list, reference counts)
-    and its per-step calls; every array argument is a CUDA int32 tensor."""
+    """The block manager's state on the device (free list, reference counts,
+    prefix keys, the eviction order of cached blocks) and its per-step calls;
+    every array argument is a CUDA int32 tensor."""
 
     def __init__(self, num_blocks: int, device="cuda", stream=None):
-        self.num_blocks = int(num_blocks)
+        self.num_blocks = nb = int(num_blocks)
         self.state = torch.empty(bm_state_bytes(num_blocks), dtype=torch.uint8, device=device)
-        a = (self.num_blocks * 4 + 255) // 256 * 256
-        self.header = self.state[:8].view(torch.int32)  # top, error word
-        self.free_stack = self.state[256:256 + 4 * self.num_blocks].view(torch.int32)
-        self.refcount = self.state[256 + a:256 + a + 4 * self.num_blocks].view(torch.int32)
-        self.block_hash = self.state[256 + 5 * a:256 + 5 * a + 8 * self.num_blocks].view(torch.int64)
-        _check(load_library().pkv_bm_init(_ptr(self.state), self.num_blocks, _stream(stream)), "pkv_bm_init")
+        a = (nb * 4 + 255) // 256 * 256
+        h = (nb * 8 + 255) // 256 * 256
+        self.header = self.state[:20].view(torch.int32)  # top, error word, cached, ring head, ring tail
+        self.free_stack = self.state[256:256 + 4 * nb].view(torch.int32)
+        self.refcount = self.state[256 + a:256 + a + 4 * nb].view(torch.int32)
+        self.block_hash = self.state[256 + 5 * a:256 + 5 * a + 8 * nb].view(torch.int64)
+        self.lru_pos = self.state[256 + 5 * a + h:256 + 5 * a + h + 4 * nb].view(torch.int32)
+        self.ring = self.state[256 + 6 * a + h:256 + 6 * a + h + 8 * nb].view(torch.int32)
+        _check(load_library().pkv_bm_init(_ptr(self.state), nb, _stream(stream)), "pkv_bm_init")
 
     def top(self) -> int:
         return int(self.header[0].item())
+
+    def cached(self) -> int:
+        """Blocks with no reference that still hold a prefix key."""
+        return int(self.header[2].item())
+
+    def lru_order(self):
+        """Cached blocks in eviction order (least recently released first), read
+        back from the device ring: the entries of head .. tail whose block still
+        records that position."""
+        import numpy as np
+        hdr = self.header.cpu().numpy().view(np.uint32)
+        head, tail = int(hdr[3]), int(hdr[4])
+        ring = self.ring.cpu().numpy()
+        pos_of = self.lru_pos.cpu().numpy().view(np.uint32)
+        pos = np.arange(head, tail, dtype=np.int64)
+        blocks = ring[pos % (2 * self.num_blocks)]
+        live = (blocks >= 0) & (blocks < self.num_blocks)
+        live[live] = pos_of[blocks[live]] == pos[live]
+        return blocks[live].astype(np.int32)
 
     def error(self) -> int:
         return int(self.header[1].item()) & 0xFFFFFFFF

@@ -14,6 +14,19 @@
 // value between calls.  Every kernel is one CTA of 1024 threads walking its
 // items in chunks of 1024, in order, with block-wide scans: results are the
 // sequential (request-order) ones, bit for bit, without host round trips.
+//
+// Cached blocks (intelliparadigm.com section 2.1, item 1: a block is free,
+// allocated or shareable; item 3: LRU keeps the block heat): a block that
+// holds a prefix key keeps it when its count reaches zero and waits in the
+// eviction order instead of on the free stack.  The order is a ring of
+// 2 * num_blocks entries addressed by absolute position (head .. tail): a
+// release appends the block at the tail and records the position in
+// lru_pos[b]; an entry is live while lru_pos[its block] equals its position,
+// so a prefix hit or a share takes a block out by clearing lru_pos alone.
+// Allocation pops the free stack first and then takes the live entries from
+// the head (least recently released first), dropping their keys.  When an
+// append would overflow the ring, the live entries are first compacted
+// toward the head, in order.
 #pragma once
 
 #include <cstdint>
@@ -31,17 +44,42 @@ constexpr uint32_t kBmErrDoubleFree = 4u;  // a block freed more often than refe
 constexpr uint32_t kBmErrTable = 8u;       // a sequence outgrew its block-table row
 
 struct BmState {
-    int32_t *hdr;         // [0] top, [1] error word
+    int32_t *hdr;         // [0] top, [1] error word, [2] cached blocks, [3] ring head, [4] ring tail
     int32_t *free_stack;  // [NB]
     int32_t *refcount;    // [NB]
     int32_t *last_idx;    // [NB] scratch: last list position of a block in a free batch (rest: -1)
     int32_t *zeroed;      // [NB] scratch: its count reached zero in this batch (rest: 0)
     int32_t *cow_rank;    // [NB] scratch: copy-on-write candidates seen so far in a chunk (rest: 0)
     uint64_t *block_hash; // [NB] prefix-cache key the block holds (0: none)
+    uint32_t *lru_pos;    // [NB] absolute ring position of a cached block's entry (kNotCached otherwise)
+    int32_t *ring;        // [2 NB] eviction order: ring[pos % (2 NB)] = block
+    int32_t *evicted;     // [NB] scratch: the blocks one allocation call takes from the ring, in order
 };
+
+constexpr uint32_t kNotCached = 0xffffffffu;
 
 __device__ __forceinline__ void bm_error(const BmState &s, uint32_t bits) {
     atomicOr(reinterpret_cast<unsigned int *>(s.hdr + 1), bits);
+}
+
+__device__ __forceinline__ int bm_cached(const BmState &s, int nb) { return min(max(s.hdr[2], 0), nb); }
+__device__ __forceinline__ uint32_t ring_head(const BmState &s) { return (uint32_t)s.hdr[3]; }
+__device__ __forceinline__ uint32_t ring_tail(const BmState &s) { return (uint32_t)s.hdr[4]; }
+
+// Whether the ring entry at absolute position pos is live (its block's
+// current entry); returns the block, or -1.
+__device__ __forceinline__ int32_t ring_live(const BmState &s, int nb, uint32_t pos) {
+    const int32_t b = s.ring[pos % (uint32_t)(2 * nb)];
+    return (b >= 0 && b < nb && s.lru_pos[b] == pos) ? b : -1;
+}
+
+// A block mapped again (a prefix hit or a share) whose count was zero leaves
+// the eviction order.
+__device__ __forceinline__ void bm_revive(const BmState &s, int32_t b) {
+    if (s.lru_pos[b] != kNotCached) {
+        s.lru_pos[b] = kNotCached;
+        atomicSub(&s.hdr[2], 1);
+    }
 }
 
 // The stack top as stored, clamped into [0, nb] (a corrupted state cannot
@@ -84,10 +122,14 @@ __global__ void __launch_bounds__(256) bm_init_kernel(BmState s, int nb) {
         s.zeroed[i] = 0;
         s.cow_rank[i] = 0;
         s.block_hash[i] = 0;
+        s.lru_pos[i] = kNotCached;
     }
     if (blockIdx.x == 0 && threadIdx.x == 0) {
         s.hdr[0] = nb;
         s.hdr[1] = 0;
+        s.hdr[2] = 0;  // cached blocks
+        s.hdr[3] = 0;  // ring head
+        s.hdr[4] = 0;  // ring tail
     }
 }
 
@@ -104,14 +146,84 @@ __device__ __forceinline__ int block_max(int v, int *warp_buf) {
     return w;
 }
 
+// Takes live ring entries from *cursor on until `target` blocks are in
+// s.evicted (the least recently released first): each taken block loses its
+// key and leaves the order.  Block-wide; `collected` (blocks already in
+// s.evicted) and *cursor are the same on every thread.  Returns the new
+// collected count (short of target only if the ring ran out, an inconsistent
+// state).
+__device__ int ring_collect(const BmState &s, int nb, int target, int collected, uint32_t *cursor,
+                            int *warp_buf) {
+    const uint32_t tail = ring_tail(s);
+    uint32_t cur = *cursor;
+    while (collected < target && cur != tail) {
+        const uint32_t span = min((uint32_t)kBmThreads, tail - cur);
+        const int32_t b = threadIdx.x < span ? ring_live(s, nb, cur + threadIdx.x) : -1;
+        int tot;
+        const int excl = block_scan_excl(b >= 0 ? 1 : 0, warp_buf, &tot);
+        const bool take = b >= 0 && collected + excl < target;
+        if (take) {
+            s.evicted[collected + excl] = b;
+            s.block_hash[b] = 0;  // evicted: its content no longer backs a prefix
+            s.lru_pos[b] = kNotCached;
+        }
+        const int took = min(tot, target - collected);
+        // past the whole span, or (stopped inside it) past the last entry taken
+        const uint32_t adv = took < tot ? (uint32_t)block_max(take ? (int)threadIdx.x + 1 : 0, warp_buf) : span;
+        collected += took;
+        cur += adv;
+    }
+    *cursor = cur;
+    __syncthreads();  // s.evicted visible to the whole block
+    return collected;
+}
+
+// Moves the live ring entries, in order, to positions 0 .. n-1 (through the
+// s.evicted scratch) and sets head = 0, tail = n.  Keeps the ring's span and
+// its absolute positions small.  Block-wide.
+__device__ void ring_compact(const BmState &s, int nb, int *warp_buf) {
+    const uint32_t head = ring_head(s), tail = ring_tail(s);
+    int n = 0;
+    for (uint32_t base = head; base != tail;) {
+        const uint32_t span = min((uint32_t)kBmThreads, tail - base);
+        const int32_t b = threadIdx.x < span ? ring_live(s, nb, base + threadIdx.x) : -1;
+        int tot;
+        const int excl = block_scan_excl(b >= 0 ? 1 : 0, warp_buf, &tot);
+        if (b >= 0 && n + excl < nb) s.evicted[n + excl] = b;
+        n += tot;
+        base += span;
+    }
+    n = min(n, nb);
+    __syncthreads();
+    for (int i = threadIdx.x; i < n; i += kBmThreads) {
+        const int32_t b = s.evicted[i];
+        s.ring[i] = b;
+        s.lru_pos[b] = (uint32_t)i;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        s.hdr[3] = 0;
+        s.hdr[4] = n;
+    }
+    __syncthreads();
+}
+
+// The j-th block one allocation call hands out: the free stack first, then
+// the blocks collected from the eviction order.
+__device__ __forceinline__ int32_t bm_pop_at(const BmState &s, int top0, int collected, int j) {
+    if (j < top0) return s.free_stack[top0 - 1 - j];
+    return j - top0 < collected ? s.evicted[j - top0] : -1;
+}
+
 // Request r receives counts[r] blocks at ids[offsets[r] .. offsets[r+1]),
-// requests served in order while the free list and the output room last.  The
-// inclusive sum of counts only grows, so the served requests are a prefix.
+// requests served in order while the free and cached blocks and the output
+// room last.  The inclusive sum of counts only grows, so the served requests
+// are a prefix.
 __global__ void __launch_bounds__(kBmThreads) bm_alloc_kernel(BmState s, int nb, const int32_t *counts, int n,
                                                                int32_t *offsets, int32_t *ids, int capacity) {
     __shared__ int warp_buf[32];
     const int top0 = bm_top(s, nb);
-    const int limit = min(top0, capacity);
+    const int limit = min(top0 + bm_cached(s, nb), capacity);
     int run = 0;     // counts of earlier chunks
     int served = 0;  // blocks handed out (the largest fitting inclusive sum)
     bool failed = false;
@@ -119,34 +231,41 @@ __global__ void __launch_bounds__(kBmThreads) bm_alloc_kernel(BmState s, int nb,
         const int r = base + threadIdx.x;
         const int c = r < n ? max(__ldg(counts + r), 0) : 0;
         int tot;
-        const int excl = run + block_scan_excl(c, warp_buf, &tot);
-        const int incl = excl + c;
+        const int incl = run + block_scan_excl(c, warp_buf, &tot) + c;
         const bool fits = r < n && incl <= limit;
-        if (fits) {
-            for (int k = 0; k < c; ++k) {
-                const int32_t blk = s.free_stack[top0 - 1 - (excl + k)];
-                ids[excl + k] = blk;
-                s.refcount[blk] = 1;
-            }
-        }
         served = max(served, block_max(fits ? incl : 0, warp_buf));
         failed = __syncthreads_or(r < n && !fits) || failed;
         run += tot;
     }
-    // second walk: offsets (needs the final served total for the unserved tail)
+    // blocks beyond the free stack come from the eviction order
+    uint32_t cursor = ring_head(s);
+    const int want = max(0, served - top0);
+    const int got = ring_collect(s, nb, want, 0, &cursor, warp_buf);
+    // second walk: ids and offsets (the unserved tail needs the final total)
     run = 0;
     if (threadIdx.x == 0) offsets[0] = 0;
     for (int base = 0; base < n; base += kBmThreads) {
         const int r = base + threadIdx.x;
         const int c = r < n ? max(__ldg(counts + r), 0) : 0;
         int tot;
-        const int incl = run + block_scan_excl(c, warp_buf, &tot) + c;
+        const int excl = run + block_scan_excl(c, warp_buf, &tot);
+        const int incl = excl + c;
         if (r < n) offsets[r + 1] = incl <= limit ? incl : served;
+        if (r < n && incl <= limit) {
+            for (int k = 0; k < c; ++k) {
+                const int32_t blk = bm_pop_at(s, top0, got, excl + k);
+                ids[excl + k] = blk;
+                if (blk >= 0) s.refcount[blk] = 1;
+            }
+        }
         run += tot;
     }
     if (threadIdx.x == 0) {
-        s.hdr[0] = top0 - served;
+        s.hdr[0] = top0 - min(served, top0);
+        s.hdr[2] -= got;
+        s.hdr[3] = (int32_t)cursor;
         if (failed) bm_error(s, kBmErrNoSpace);
+        if (got < want) bm_error(s, kBmErrDoubleFree);  // fewer cached blocks than counted: inconsistent state
     }
 }
 
@@ -167,28 +286,47 @@ __global__ void __launch_bounds__(kBmThreads) bm_free_kernel(BmState s, int nb, 
             bm_error(s, kBmErrDoubleFree);
         } else if (old == 1) {
             s.zeroed[b] = 1;
-            s.block_hash[b] = 0;  // a freed block no longer backs a cached prefix
         }
         atomicMax(&s.last_idx[b], i);
     }
     __syncthreads();
-    const int top0 = bm_top(s, nb);
-    int run = 0;
+    // a block whose count reached zero, at its last occurrence: cached if it
+    // holds a prefix key (appended to the eviction order), else free (pushed)
+    auto released = [&](int i, int32_t &b) -> int {  // 0: none, 1: free, 2: cached
+        if (i >= n) return 0;
+        b = __ldg(list + i);
+        if (b < 0 || b >= nb || s.last_idx[b] != i || !s.zeroed[b]) return 0;
+        return s.block_hash[b] != 0 ? 2 : 1;
+    };
+    int cached_total = 0;
     for (int base = 0; base < n; base += kBmThreads) {
-        const int i = base + threadIdx.x;
-        int push = 0;
+        int32_t b;
+        cached_total += __syncthreads_count(released(base + threadIdx.x, b) == 2);
+    }
+    // room in the ring (2 num_blocks entries) and small absolute positions
+    const uint32_t span = ring_tail(s) - ring_head(s);
+    if (cached_total > 0 && (span + (uint32_t)cached_total > (uint32_t)(2 * nb) ||
+                             ring_tail(s) + (uint32_t)cached_total >= 0x7fffffffu))
+        ring_compact(s, nb, warp_sums);
+    const int top0 = bm_top(s, nb);
+    const uint32_t tail0 = ring_tail(s);
+    int run = 0, run_c = 0;
+    for (int base = 0; base < n; base += kBmThreads) {
         int32_t b = -1;
-        if (i < n) {
-            b = __ldg(list + i);
-            if (b >= 0 && b < nb && s.last_idx[b] == i) push = s.zeroed[b];
-        }
-        int tot;
-        const int excl = run + block_scan_excl(push, warp_sums, &tot);
-        if (push) {
+        const int kind = released(base + threadIdx.x, b);
+        int tot, tot_c;
+        const int excl = run + block_scan_excl(kind == 1, warp_sums, &tot);
+        const int excl_c = run_c + block_scan_excl(kind == 2, warp_sums, &tot_c);
+        if (kind == 1) {
             if (top0 + excl < nb) s.free_stack[top0 + excl] = b;
             else bm_error(s, kBmErrDoubleFree);  // more free blocks than the pool: the state was inconsistent
+        } else if (kind == 2) {
+            const uint32_t pos = tail0 + (uint32_t)excl_c;
+            s.ring[pos % (uint32_t)(2 * nb)] = b;
+            s.lru_pos[b] = pos;
         }
         run += tot;
+        run_c += tot_c;
     }
     __syncthreads();
     for (int i = threadIdx.x; i < n; i += kBmThreads) {  // scratch back to rest
@@ -198,14 +336,18 @@ __global__ void __launch_bounds__(kBmThreads) bm_free_kernel(BmState s, int nb, 
             s.zeroed[b] = 0;
         }
     }
-    if (threadIdx.x == 0) s.hdr[0] = min(top0 + run, nb);
+    if (threadIdx.x == 0) {
+        s.hdr[0] = min(top0 + run, nb);
+        s.hdr[2] += run_c;
+        s.hdr[4] = (int32_t)(tail0 + (uint32_t)run_c);
+    }
 }
 
 __global__ void __launch_bounds__(256) bm_share_kernel(BmState s, int nb, const int32_t *list, int n) {
     for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) {
         const int32_t b = __ldg(list + i);
         if (b < 0 || b >= nb) bm_error(s, kBmErrRange);
-        else atomicAdd(&s.refcount[b], 1);
+        else if (atomicAdd(&s.refcount[b], 1) == 0) bm_revive(s, b);
     }
 }
 
@@ -239,6 +381,9 @@ __global__ void __launch_bounds__(kBmThreads) bm_append_slots_kernel(const Appen
     const BmState &s = p.s;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int top0 = bm_top(s, p.nb);
+    const int avail0 = top0 + bm_cached(s, p.nb);  // free, then cached blocks
+    uint32_t cursor = ring_head(s);               // eviction order: next entry to look at
+    int collected = 0;                            // blocks taken from it so far (in s.evicted)
     int run_need = 0;   // blocks wanted by earlier sequences
     int run_flags = 0;  // range / table failures at earlier sequences
     int run_slots = 0;  // slot-mapping offset
@@ -291,17 +436,19 @@ __global__ void __launch_bounds__(kBmThreads) bm_append_slots_kernel(const Appen
         const int flags_before = run_flags + block_scan_excl(flag, warp_buf, &tot_flags);
         const int excl_need = run_need + block_scan_excl(need, warp_buf, &tot_need);
         const int excl_slots = run_slots + block_scan_excl(n, warp_buf, &tot_n);
-        const bool earlier_ok = flags_before == 0 && excl_need <= top0;
-        const bool fits = live && earlier_ok && !flag && excl_need + need <= top0;
+        const bool earlier_ok = flags_before == 0 && excl_need <= avail0;
+        const bool fits = live && earlier_ok && !flag && excl_need + need <= avail0;
         int tot_pairs, tot_handed;
         const int excl_pairs = run_pairs + block_scan_excl(fits ? cow : 0, warp_buf, &tot_pairs);
         (void)block_scan_excl(fits ? need : 0, warp_buf, &tot_handed);
+        // this chunk's pops beyond the free stack come from the eviction order
+        collected = ring_collect(s, p.nb, max(0, handed + tot_handed - top0), collected, &cursor, warp_buf);
         if (live && bad_range) bm_error(s, kBmErrRange);
         if (live && earlier_ok && !fits && !bad_range) bm_error(s, overflow ? kBmErrTable : kBmErrNoSpace);
         if (fits) {
             int k = 0;
             if (cow) {
-                const int32_t fresh = s.free_stack[top0 - 1 - excl_need];
+                const int32_t fresh = bm_pop_at(s, top0, collected, excl_need);
                 s.refcount[fresh] = 1;
                 atomicSub(&s.refcount[cur], 1);
                 row[pos0 / p.bs] = fresh;
@@ -310,7 +457,7 @@ __global__ void __launch_bounds__(kBmThreads) bm_append_slots_kernel(const Appen
                 k = 1;
             }
             for (int L = first_new; L <= last; ++L, ++k) {
-                const int32_t fresh = s.free_stack[top0 - 1 - (excl_need + k)];
+                const int32_t fresh = bm_pop_at(s, top0, collected, excl_need + k);
                 s.refcount[fresh] = 1;
                 row[L] = fresh;
             }
@@ -353,7 +500,9 @@ __global__ void __launch_bounds__(kBmThreads) bm_append_slots_kernel(const Appen
     }
     if (threadIdx.x == 0) {
         *p.num_pairs = run_pairs;
-        s.hdr[0] = top0 - handed;
+        s.hdr[0] = top0 - min(handed, top0);
+        s.hdr[2] -= collected;
+        s.hdr[3] = (int32_t)cursor;
     }
 }
 
@@ -364,7 +513,7 @@ __global__ void __launch_bounds__(kBmThreads) bm_append_slots_kernel(const Appen
 // FNV-1a of le64(key_{i-1}) || le64(d_i) with key_{-1} = 0; key 0 is stored as
 // 1.  The cache is an open-addressing table of (key, block) pairs with linear
 // probing; an entry counts only while its block still holds the key
-// (block_hash) and some sequence maps it (refcount > 0).
+// (block_hash): allocated, or cached and not yet evicted.
 constexpr uint64_t kFnvBasis = 14695981039346656037ull;
 constexpr uint64_t kFnvPrime = 1099511628211ull;
 
@@ -408,7 +557,7 @@ __device__ __forceinline__ int cache_find(const PrefixCache &c, uint64_t key) {
 }
 
 __device__ __forceinline__ bool holder_valid(const BmState &s, int nb, int32_t b, uint64_t key) {
-    return b >= 0 && b < nb && s.block_hash[b] == key && s.refcount[b] > 0;
+    return b >= 0 && b < nb && s.block_hash[b] == key;
 }
 
 __global__ void __launch_bounds__(256) prefix_cache_init_kernel(PrefixCache c) {
@@ -457,7 +606,8 @@ __device__ __forceinline__ uint64_t warp_block_keys(const int32_t *tok0, int bas
 
 // Lookup, one warp per sequence: the leading prompt blocks whose keys have a
 // valid holder -- at least one prompt token is left to compute -- are mapped
-// into the sequence's table row with one reference each.
+// into the sequence's table row with one reference each (a cached holder
+// leaves the eviction order).
 __global__ void __launch_bounds__(256) prefix_lookup_kernel(const PrefixParams p) {
     const int s = blockIdx.x * 8 + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
@@ -481,7 +631,7 @@ __global__ void __launch_bounds__(256) prefix_lookup_kernel(const PrefixParams p
         const int lead = hit == 0xffffffffu ? 32 : __ffs(~hit) - 1;  // leading run of hits
         if (lane < lead) {
             p.tables[(size_t)s * p.mbs + i] = b;
-            atomicAdd(&p.s.refcount[b], 1);
+            if (atomicAdd(&p.s.refcount[b], 1) == 0) bm_revive(p.s, b);  // a cached holder is mapped again
         }
         hits += lead;
         if (lead < min(32, look - base)) break;

@@ -324,15 +324,19 @@ pkv_status swap_blocks(const int32_t *block_ids, int32_t n, void *k_cache, void 
 }
 
 
-// Block-manager state: a 256-byte header (top, error word), then five
-// 256-byte-aligned int32 arrays of num_blocks: free stack, reference counts and
-// three scratch arrays.
+// Block-manager state: a 256-byte header (top, error word, cached blocks,
+// ring head and tail), then 256-byte-aligned arrays: free stack, reference
+// counts and three scratch arrays (int32 [num_blocks] each), the prefix keys
+// (uint64 [num_blocks]), the ring positions of cached blocks (uint32
+// [num_blocks]), the eviction ring (int32 [2 num_blocks]) and the eviction
+// scratch (int32 [num_blocks]).
 size_t bm_array_bytes(int32_t nb) { return round256((size_t)nb * 4); }
 
 bool bm_state(void *state, int32_t nb, pkv::BmState *s) {
-    if (!state || nb <= 0 || !aligned(state, 256)) return false;
+    if (!state || nb <= 0 || nb > (1 << 29) || !aligned(state, 256)) return false;
     uint8_t *p = static_cast<uint8_t *>(state);
     const size_t a = bm_array_bytes(nb);
+    const size_t h = round256((size_t)nb * 8);
     s->hdr = reinterpret_cast<int32_t *>(p);
     s->free_stack = reinterpret_cast<int32_t *>(p + 256);
     s->refcount = reinterpret_cast<int32_t *>(p + 256 + a);
@@ -340,6 +344,9 @@ bool bm_state(void *state, int32_t nb, pkv::BmState *s) {
     s->zeroed = reinterpret_cast<int32_t *>(p + 256 + 3 * a);
     s->cow_rank = reinterpret_cast<int32_t *>(p + 256 + 4 * a);
     s->block_hash = reinterpret_cast<uint64_t *>(p + 256 + 5 * a);
+    s->lru_pos = reinterpret_cast<uint32_t *>(p + 256 + 5 * a + h);
+    s->ring = reinterpret_cast<int32_t *>(p + 256 + 6 * a + h);
+    s->evicted = reinterpret_cast<int32_t *>(p + 256 + 6 * a + h + round256((size_t)nb * 8));
     return true;
 }
 
@@ -682,8 +689,8 @@ pkv_status paged_attn_prefill(const void *q, const void *k_cache, const void *v_
 }
 
 size_t pkv_bm_state_bytes(int32_t num_blocks) {
-    if (num_blocks <= 0) return 0;
-    return 256 + 5 * bm_array_bytes(num_blocks) + round256((size_t)num_blocks * 8);
+    if (num_blocks <= 0 || num_blocks > (1 << 29)) return 0;
+    return 256 + 7 * bm_array_bytes(num_blocks) + 2 * round256((size_t)num_blocks * 8);
 }
 
 size_t pkv_prefix_cache_bytes(int32_t capacity) {

@@ -1,6 +1,7 @@
 """GPU parity of the device block manager against the oracle's sequential
 block manager: every call's outputs and the whole state (free list, top,
-reference counts, error word) are compared bit for bit after each step.
+reference counts, prefix keys, the eviction order of cached blocks, error
+word) are compared bit for bit after each step.
 Cases: random operation mixes, forks whose sharers append together (more
 sharers than a warp, across the 1024-sequence chunk boundary), the worked
 example, errors, and a whole decode step driven from the device state."""
@@ -25,6 +26,8 @@ def _same_state(bm: pkv.BlockManager, st: oracle.BlockState, err_expected: int):
     assert bm.top() == st.top
     assert np.array_equal(bm.free_stack.cpu().numpy()[:st.top], st.free_stack[:st.top])
     assert np.array_equal(bm.refcount.cpu().numpy(), st.refcount)
+    assert np.array_equal(bm.block_hash.cpu().numpy().view(np.uint64), st.block_hash)
+    assert np.array_equal(bm.lru_order(), st.lru_order()) and bm.cached() == len(st.lru_order())
     assert bm.error() == err_expected
 
 
@@ -320,3 +323,115 @@ def test_prefix_cache_rounds_match_oracle(seed, B, bs):
             assert np.array_equal(bm.block_hash.cpu().numpy().view(np.uint64), st.block_hash)
         old_ctx[ends] = 0
     assert total_hits > 0 and st.block_hash.any()
+
+
+def test_cached_blocks_worked_example_on_device():
+    """The cached-block worked example (a system prompt served again after its
+    first request finished; free blocks before cached ones; least recently
+    released evicted first, its key dropped) replayed on the device."""
+    from tests.test_oracle_prefix import run_eviction_example
+    g = json.load(open(os.path.join(GOLDEN, "prefix_eviction_example.json")))
+    bs = g["block_size"]
+    bm = pkv.BlockManager(g["num_blocks"])
+    pc = pkv.PrefixCache(g["cache_capacity"])
+
+    def serve(prompt):
+        tokens = _dev(prompt)
+        qs = _dev([0, len(prompt)])
+        t = _dev(np.full((1, 8), -1, np.int32))
+        cached = pc.lookup(bm, tokens, qs, bs, t)
+        need = _dev([len(prompt)]) - cached
+        bm.append_slots(t, cached.clone(), need.to(torch.int32), bs, len(prompt))
+        pc.insert(bm, tokens, qs, bs, t)
+        torch.cuda.synchronize()
+        err = bm.error()
+        bm.clear_error()
+        return int(cached[0].item()), t[0].cpu().numpy(), err
+
+    def finish(row, n):
+        bm.free(_dev(row[:-(-n // bs)]))
+
+    def state():
+        torch.cuda.synchronize()
+        return (bm.refcount.cpu().numpy(), bm.free_stack.cpu().numpy()[:bm.top()], bm.lru_order(),
+                bm.block_hash.cpu().numpy().view(np.uint64))
+
+    run_eviction_example(serve, finish, state)
+
+
+@pytest.mark.parametrize("seed,B,nb,rounds", [(0, 6, 40, 40), (1, 24, 90, 12), (2, 1100, 3000, 3)])
+def test_cached_blocks_under_pressure_match_oracle(seed, B, nb, rounds):
+    """Rounds of requests sharing system prompts on a pool too small to keep
+    every prefix: lookups revive cached blocks, allocation evicts the least
+    recently released, all requests finish between rounds.  The whole state,
+    the eviction order included, is compared after every call."""
+    rng = np.random.default_rng(seed)
+    bs, mbs = 4, 8
+    bm = pkv.BlockManager(nb)
+    pc = pkv.PrefixCache(1 << 12)
+    st = oracle.bm_init(nb)
+    ocache = oracle.PrefixCache(1 << 12)
+    systems = _systems(rng, bs, n_sys=6)
+    hits = evictions_seen = 0
+    for rnd in range(rounds):
+        prompts = _prompts(rng, B, bs, systems)
+        cached_before = len(st.lru_order())
+        st, ocache, tables, ctx, cached = _serve_both(bm, pc, st, ocache, prompts, bs, mbs)
+        bm.clear_error()
+        hits += int((cached > 0).sum())
+        evictions_seen += int(cached_before > len(st.lru_order()))
+        ids = np.concatenate([tables[b, :(ctx[b] + bs - 1) // bs] for b in range(B) if ctx[b] > 0]).astype(np.int32)
+        if len(ids):
+            bm.free(_dev(ids))
+            st, e = oracle.bm_free(st, ids)
+            _same_state(bm, st, e)
+            bm.clear_error()
+    assert hits > 0 and evictions_seen > 0 and len(st.lru_order()) > 0
+
+
+def test_alloc_takes_cached_blocks_after_the_free_stack():
+    rng = np.random.default_rng(5)
+    bs, B, mbs, nb = 4, 8, 6, 60
+    bm = pkv.BlockManager(nb)
+    pc = pkv.PrefixCache(256)
+    st = oracle.bm_init(nb)
+    ocache = oracle.PrefixCache(256)
+    systems = _systems(rng, bs, n_sys=3)
+    st, ocache, tables, ctx, _ = _serve_both(bm, pc, st, ocache, _prompts(rng, B, bs, systems), bs, mbs)
+    ids = np.concatenate([tables[b, :(ctx[b] + bs - 1) // bs] for b in range(B)]).astype(np.int32)
+    bm.free(_dev(ids))
+    st, _ = oracle.bm_free(st, ids)
+    _same_state(bm, st, 0)
+    assert len(st.lru_order()) > 0
+    counts = np.array([st.top, 2, 1, 3, 50], np.int32)  # the free stack, then cached blocks, then too many
+    off, out_ids = bm.alloc(_dev(counts), 100)
+    st, ooff, oids, e = oracle.bm_alloc(st, counts, 100)
+    torch.cuda.synchronize()
+    assert np.array_equal(off.cpu().numpy(), ooff)
+    assert np.array_equal(out_ids.cpu().numpy()[:ooff[-1]], oids[:ooff[-1]])
+    _same_state(bm, st, e)
+    assert e == oracle.BM_ERR_NOSPACE
+
+
+def test_eviction_ring_compacts_in_order():
+    """The same prompts served and finished round after round on a pool large
+    enough to evict nothing: every hit leaves a dead entry in the eviction
+    ring and every release appends one, so the ring fills up and is compacted
+    (its tail moves back); the order of the cached blocks stays the oracle's."""
+    rng = np.random.default_rng(9)
+    bs, mbs, nb = 4, 8, 40
+    bm = pkv.BlockManager(nb)
+    pc = pkv.PrefixCache(256)
+    st = oracle.bm_init(nb)
+    ocache = oracle.PrefixCache(256)
+    prompts = _prompts(rng, 3, bs, _systems(rng, bs, n_sys=2))
+    compactions = 0
+    for rnd in range(60):
+        st, ocache, tables, ctx, cached = _serve_both(bm, pc, st, ocache, prompts, bs, mbs)
+        ids = np.concatenate([tables[b, :(ctx[b] + bs - 1) // bs] for b in range(len(prompts))]).astype(np.int32)
+        tail_before = int(bm.header[4].item())
+        bm.free(_dev(ids))
+        st, e = oracle.bm_free(st, ids)
+        _same_state(bm, st, e)
+        compactions += int(int(bm.header[4].item()) < tail_before)
+    assert compactions > 0

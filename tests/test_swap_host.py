@@ -62,8 +62,9 @@ def test_block_manager_host_validation():
     """Host checks of the device block manager's entry points (no GPU work)."""
     lib = pkv.load_library()
     assert lib.pkv_bm_state_bytes(0) == 0
-    assert lib.pkv_bm_state_bytes(10) == 256 + 5 * 256 + 256
-    assert lib.pkv_bm_state_bytes(100) == 256 + 5 * 512 + 1024
+    assert lib.pkv_bm_state_bytes(10) == 256 + 7 * 256 + 2 * 256  # 7 int32 arrays, keys and ring
+    assert lib.pkv_bm_state_bytes(100) == 256 + 7 * 512 + 2 * 1024
+    assert lib.pkv_bm_state_bytes((1 << 29) + 1) == 0  # above the supported pool size
     assert lib.pkv_prefix_cache_bytes(0) == 0 and lib.pkv_prefix_cache_bytes(48) == 0  # power of two
     assert lib.pkv_prefix_cache_bytes(64) == 512 + 2 * 256
     assert lib.pkv_prefix_cache_init(FAKE, 48, None) == EINVAL
