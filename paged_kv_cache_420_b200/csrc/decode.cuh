@@ -94,6 +94,14 @@ __device__ __forceinline__ int group_count(const DecodeParams &p, int parts) {
     return (p.maxP > 1 && p.g > 1) ? parts / kConsumerWarps : 0;
 }
 
+// Split-K records of a sequence with `parts` partitions: one per partition
+// group (its W partitions merged inside the CTA), then one per single
+// partition.  Index of the record that holds partition `part`.
+__device__ __forceinline__ int record_index(const DecodeParams &p, int parts, int part) {
+    const int groups = group_count(p, parts);
+    return part < groups * kConsumerWarps ? part / kConsumerWarps : part - (kConsumerWarps - 1) * groups;
+}
+
 // Writes the entry list and its count, and zeroes the attention kernel's work
 // counter.  Every sequence's partition groups come first, then the remaining
 // single partitions (each sequence-major): the large items are claimed first
@@ -133,10 +141,13 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(DecodeParams p, int 
         __syncthreads();  // s_warp reusable
         return incl;
     };
+    // no sequence can hold a group: one scan per chunk (the planner runs
+    // before the attention kernel can read anything)
+    const bool can_group = group_count(p, p.maxP) > 0;
     // Single partitions go after all groups: with more sequences than one
     // chunk the total of groups is counted first.
     int groups_total = 0;
-    if (p.B > kPlanThreads) {
+    if (can_group && p.B > kPlanThreads) {
         for (int base = 0; base < p.B; base += kPlanThreads) {
             const int s = base + tid;
             int c = 0;
@@ -160,7 +171,7 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(DecodeParams p, int 
             if (n == 0) s_any_zero = 1;
         }
         s_n[tid] = n;
-        const int ig = scan(groups);
+        const int ig = can_group ? scan(groups) : 0;
         const int is = scan(singles);
         s_goff[tid + 1] = ig;
         s_soff[tid + 1] = is;
@@ -499,23 +510,6 @@ struct SimtState {
         }
     }
 
-    // Writes this warp's (m, l, acc) as the split-K record of partition part of
-    // query head `head` (a partition the warp walked alone).
-    template <class Params>
-    __device__ __forceinline__ void store_record(const Params &p, size_t head, int part, int lane) {
-        float l = l_part;
-#pragma unroll
-        for (int o = 2; o < 32; o <<= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
-        const size_t pi = head * p.maxP + part;
-        float *dst = p.part_acc + pi * D + lane * EPL;
-        if constexpr (EPL == 4) {
-            *reinterpret_cast<float4 *>(dst) = make_float4(acc[0], acc[1], acc[2], acc[3]);
-        } else {
-            *reinterpret_cast<float2 *>(dst) = make_float2(acc[0], acc[1]);
-        }
-        if (lane == 0) p.part_ml[pi] = make_float2(m, l);
-    }
-
     // Writes this warp's partial (m, l, acc) into the merge buffers.
     __device__ __forceinline__ void store_partial(float *mO, float *mM, float *mL, int w, int lane, int stride) {
         // lanes 2t and 2t+1 hold the same p: sum over one lane of each pair
@@ -724,34 +718,6 @@ struct MmaState {
         }
     }
 
-    // Writes this warp's (m, l, O) of every head of the group as the split-K
-    // records of partition part (a partition the warp walked alone); head0 is
-    // the group's first query head.
-    template <class Params>
-    __device__ __forceinline__ void store_record(const Params &p, size_t head0, int part, int lane) {
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-#pragma unroll
-            for (int c = 0; c < 2; ++c) {
-                float lsum = l[nt][c];
-                lsum += __shfl_xor_sync(0xffffffffu, lsum, 4);
-                lsum += __shfl_xor_sync(0xffffffffu, lsum, 8);
-                lsum += __shfl_xor_sync(0xffffffffu, lsum, 16);
-                const int head = nt * 8 + 2 * (lane & 3) + c;
-                if (head < p.g) {
-                    const size_t pi = (head0 + head) * p.maxP + part;
-                    if (lane < 4) p.part_ml[pi] = make_float2(m[nt][c], lsum);
-                    float *row = p.part_acc + pi * D;
-#pragma unroll
-                    for (int mt = 0; mt < MT; ++mt) {
-                        row[mt * 16 + (lane >> 2)] = o[nt][mt][c];
-                        row[mt * 16 + (lane >> 2) + 8] = o[nt][mt][c + 2];
-                    }
-                }
-            }
-        }
-    }
-
     __device__ __forceinline__ void store_partial(float *mO, float *mM, float *mL, int w, int lane, int stride,
                                                   int GPn, int g) {
 #pragma unroll
@@ -810,6 +776,7 @@ __global__ void __launch_bounds__(kDecodeThreads) paged_decode_kernel(const __gr
     uint64_t *mempty = mfull + 1;
     StageInfo *info = reinterpret_cast<StageInfo *>(smem + L::oInfo);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::oAbort);
+    int *grp_arrive = reinterpret_cast<int *>(smem + L::oAbort) + 1;  // warps done with a partition group
     const uint32_t tiles = smem_u32(smem + L::oTiles);
     __nv_bfloat16 *qbuf = reinterpret_cast<__nv_bfloat16 *>(smem + L::oQ);
     float *mO = reinterpret_cast<float *>(smem + L::oMergeO);
@@ -823,6 +790,7 @@ __global__ void __launch_bounds__(kDecodeThreads) paged_decode_kernel(const __gr
         mbar_init(mfull, W);
         mbar_init(mempty, W);
         *abort_flag = 0;
+        *grp_arrive = 0;
         fence_mbar_init();
         tma_prefetch_desc(&tmap_k);
         tma_prefetch_desc(&tmap_v);
@@ -1000,7 +968,8 @@ __global__ void __launch_bounds__(kDecodeThreads) paged_decode_kernel(const __gr
         // ------------------------------------------------------ consumer --
         const int w = warp;
         uint32_t gc = w;
-        uint32_t mc = 0;  // merges done
+        uint32_t mc = 0;   // merges done (each completes one phase of mempty)
+        uint32_t mfc = 0;  // merges of single partitions (each completes one phase of mfull)
         float scale_log2 = p.scale_log2;
         SimtState<D, KV8> st0;
         MmaState<D, (PATH == 1 ? NT : 1), KV8> st1;
@@ -1017,8 +986,10 @@ __global__ void __launch_bounds__(kDecodeThreads) paged_decode_kernel(const __gr
                 if constexpr (PATH == 0) {
                     st0.reset();
                     st0.load_q(qs, lane, KV8 ? scale_log2 * __ldg(p.k_scale + si.h) : scale_log2);
+                } else {
+                    st1.reset();
+                    st1.load_q(qs, lane, p.g);
                 }
-                else { st1.reset(); st1.load_q(qs, lane, p.g); }
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&qempty[qb]);
             }
@@ -1036,57 +1007,78 @@ __global__ void __launch_bounds__(kDecodeThreads) paged_decode_kernel(const __gr
             if (lane == 0) mbar_arrive(&empty[slot]);
             gc += W;
             const bool grp = (si.part & kGroupFlag) != 0;
-            if (grp && si.k + W >= si.npad) {
-                // partition group: this warp walked partition part + w alone
-                // and writes its record itself, no merge with the other warps
-                const size_t unit_head0 = (size_t)si.s * p.Hq + (size_t)si.h * p.g;
-                const int part = (si.part & ~kGroupFlag) + w;
-                if constexpr (PATH == 0) st0.store_record(p, unit_head0, part, lane);
-                else st1.store_record(p, unit_head0, part, lane);
-            } else if (si.k + W >= si.npad) {
-                // this warp's last stage of the item: merge the W partials
+            if (si.k + W >= si.npad) {
+                // this warp's last stage of the item: its partial (m, l, acc)
+                // goes to its merge buffer once the previous merge has read them
                 if (!wait_or_abort(mempty, (mc & 1) ^ 1, abort_flag)) break;
                 if constexpr (PATH == 0) st0.store_partial(mO, mM, mL, w, lane, L::kMergeStride);
                 else st1.store_partial(mO, mM, mL, w, lane, L::kMergeStride, GP, p.g);
                 __syncwarp();
-                if (lane == 0) mbar_arrive(mfull);
-                if (!wait_or_abort(mfull, mc & 1, abort_flag)) break;
-                // Combine: warp w takes heads w, w + W, ...; lane handles the
-                // elements lane, lane + 32, ... of the head (consecutive lanes on
-                // consecutive words: no bank conflicts), and the per-head factors
-                // 2^(m_u - M) are computed once per head.
                 const int g = p.g;
                 const size_t unit_head0 = (size_t)si.s * p.Hq + (size_t)si.h * g;
-                for (int j = w; j < g; j += W) {
-                    float M = PKV_NEG_INF;
+                const int part = si.part & ~kGroupFlag;
+                // merged result of heads j0, j0 + step, ...: out (a single
+                // partition sequence) or the split-K record `rec`
+                auto combine = [&](int j0, int step, int rec) {
+                    for (int j = j0; j < g; j += step) {
+                        float M = PKV_NEG_INF;
 #pragma unroll
-                    for (int u = 0; u < W; ++u) M = fmaxf(M, mM[u * GP + j]);
-                    float f[W], Lsum = 0.f;
+                        for (int u = 0; u < W; ++u) M = fmaxf(M, mM[u * GP + j]);
+                        float f[W], Lsum = 0.f;
 #pragma unroll
-                    for (int u = 0; u < W; ++u) {
-                        const float mu = mM[u * GP + j];
-                        f[u] = mu == PKV_NEG_INF ? 0.f : exp2f(mu - M);
-                        Lsum = fmaf(mL[u * GP + j], f[u], Lsum);
-                    }
-                    float invL = Lsum > 0.f ? 1.f / Lsum : 0.f;
-                    if constexpr (KV8) invL *= __ldg(p.v_scale + si.h);
+                        for (int u = 0; u < W; ++u) {
+                            const float mu = mM[u * GP + j];
+                            f[u] = mu == PKV_NEG_INF ? 0.f : exp2f(mu - M);
+                            Lsum = fmaf(mL[u * GP + j], f[u], Lsum);
+                        }
+                        float invL = Lsum > 0.f ? 1.f / Lsum : 0.f;
+                        if constexpr (KV8) invL *= __ldg(p.v_scale + si.h);
 #pragma unroll
-                    for (int i = 0; i < D / 32; ++i) {
-                        const int d = lane + 32 * i;
-                        float O = 0.f;
+                        for (int i = 0; i < D / 32; ++i) {
+                            const int d = lane + 32 * i;
+                            float O = 0.f;
 #pragma unroll
-                        for (int u = 0; u < W; ++u) O = fmaf(mO[(u * GP + j) * L::kMergeStride + d], f[u], O);
-                        if (si.nparts == 1) {
-                            p.out[(unit_head0 + j) * D + d] = __float2bfloat16_rn(O * invL);
-                        } else {
-                            const size_t pi = (unit_head0 + j) * p.maxP + si.part;
-                            p.part_acc[pi * D + d] = O;
-                            if (d == 0) p.part_ml[pi] = make_float2(M, Lsum);
+                            for (int u = 0; u < W; ++u) O = fmaf(mO[(u * GP + j) * L::kMergeStride + d], f[u], O);
+                            if (si.nparts == 1) {
+                                p.out[(unit_head0 + j) * D + d] = __float2bfloat16_rn(O * invL);
+                            } else {
+                                const size_t pi = (unit_head0 + j) * p.maxP + rec;
+                                p.part_acc[pi * D + d] = O;
+                                if (d == 0) p.part_ml[pi] = make_float2(M, Lsum);
+                            }
                         }
                     }
+                };
+                if (grp) {
+                    // partition group: warp u walked partition part + u alone.
+                    // The last warp to get here merges the W partitions into
+                    // the group's record (an fp32 log-sum-exp merge); the
+                    // others go on with the next item at once.
+                    int last = 0;
+                    if (lane == 0) {
+                        __threadfence_block();
+                        last = atomicAdd(grp_arrive, 1) == W - 1;
+                    }
+                    if (__shfl_sync(0xffffffffu, last, 0)) {
+                        __threadfence_block();
+                        combine(0, 1, part / W);
+                        __syncwarp();
+                        if (lane == 0) {
+                            *grp_arrive = 0;
+                            mbar_arrive_count(mempty, W);
+                        }
+                    }
+                } else {
+                    // the W warps shared the partition's stages: merge
+                    // together, warp w taking heads w, w + W, ...; lanes on
+                    // consecutive words (no bank conflicts)
+                    if (lane == 0) mbar_arrive(mfull);
+                    if (!wait_or_abort(mfull, mfc & 1, abort_flag)) break;
+                    ++mfc;
+                    combine(w, W, record_index(p, si.nparts, part));
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(mempty);
                 }
-                __syncwarp();
-                if (lane == 0) mbar_arrive(mempty);
                 ++mc;
             }
         }
@@ -1095,10 +1087,11 @@ __global__ void __launch_bounds__(kDecodeThreads) paged_decode_kernel(const __gr
 }
 
 // --------------------------------------------------------------- reduce ----
-// Log-sum-exp merge of the partitions of every (s, hq) with more than one
-// partition: M = max_p m_p, L = sum_p l_p 2^(m_p - M),
+// Log-sum-exp merge of the split-K records of every (s, hq) with more than
+// one partition (a record per partition group, then one per single
+// partition): M = max_p m_p, L = sum_p l_p 2^(m_p - M),
 // out = sum_p acc_p 2^(m_p - M) / L.  One CTA per (s, hq); warp w takes
-// partitions w, w + 4, ...; lanes own D/32 consecutive elements.
+// records w, w + 4, ...; lanes own D/32 consecutive elements.
 template <int D>
 __global__ void __launch_bounds__(kReduceWarps * 32) splitk_reduce_kernel(const DecodeParams p) {
     constexpr int EPL = D / 32;
@@ -1109,8 +1102,9 @@ __global__ void __launch_bounds__(kReduceWarps * 32) splitk_reduce_kernel(const 
     const int s = unit / p.Hq;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int n = clamped_context(p, s, false);
-    const int P = (n + p.PT - 1) / p.PT;
-    if (P <= 1) return;  // written directly by the attention kernel
+    const int parts = (n + p.PT - 1) / p.PT;
+    if (parts <= 1) return;  // written directly by the attention kernel
+    const int P = parts - (kConsumerWarps - 1) * group_count(p, parts);  // records
     const float2 *ml = p.part_ml + (size_t)unit * p.maxP;
     float M = PKV_NEG_INF;
     for (int i = lane; i < P; i += 32) M = fmaxf(M, ml[i].x);
