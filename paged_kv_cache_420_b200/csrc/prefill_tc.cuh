@@ -19,18 +19,21 @@
 //                the K stream never waits behind a V slot that PV still holds.
 //   warp 1       MMA issuer (one thread) and tensor-memory owner:
 //                S_j = Q K_j^T  (tcgen05.mma kind::f16, M 128, N 64, K-major
-//                smem operands, fp32 into the TMEM S buffer), then
-//                O += P_j V_j   (A = P_j in TMEM, B = V_j MN-major in smem,
+//                smem operands, fp32 into TMEM S buffer j % 2), then
+//                O += P_{j-1} V_{j-1}  (A = P in TMEM, B = V MN-major in smem,
 //                N = D), each followed by tcgen05.commit onto an mbarrier.
-//   warps 2-5    softmax: thread r owns row r (TMEM lane r).  It loads S_j
-//                (releasing the S buffer at once), masks the diagonal block,
-//                keeps the row's running max in scaled log2 units (raised
-//                lazily, as in decode) and sum, writes P_j as bf16 into one of
-//                two TMEM P buffers, rescales its O row when the max was raised
-//                (after the previous PV product has completed), and at the end
-//                of the item normalises O and stores the row.
-// S_{j+1} runs on the tensor cores while the softmax works on S_j, and the
-// other CTA on the SM fills the gaps of this one.
+//   warps 2-5    softmax: thread r owns row r (TMEM lane r).  It loads S_j,
+//                masks the diagonal block, keeps the row's running max in
+//                scaled log2 units (raised lazily, as in decode) and sum, writes
+//                P_j as bf16 over the first half of S_j's own buffer, rescales
+//                its O row when the max was raised (after the previous PV
+//                product has completed), and at the end of the item normalises
+//                O and stores the row.
+// Two S buffers: S_{j+1} is issued right behind S_j, so it is ready when the
+// softmax finishes S_j.  S_{j+2} reuses S_j's buffer; the MMA thread issues it
+// after P_j V_j, and the tensor core runs one thread's MMAs in order, so P_j
+// has been read before S_{j+2} overwrites it.  The other CTA on the SM fills
+// the gaps of this one.
 #pragma once
 
 #include "prefill.cuh"
@@ -43,8 +46,8 @@ constexpr int kTcThreads = 7 * 32;
 constexpr int kTcCtasPerSm = 2;
 // Tensor memory of one CTA (256 of the SM's 512 columns):
 constexpr uint32_t kTmemCols = 256;
-constexpr uint32_t kTmemS = 0;        // S: fp32, columns [0, 64)
-constexpr uint32_t kTmemP = 64;       // two P buffers (bf16 pairs): [64, 96) and [96, 128)
+constexpr uint32_t kTmemS = 0;        // S buffers: fp32, columns [0, 64) and [64, 128); P_j (bf16
+                                      // pairs) over the first 32 columns of S_j's buffer
 constexpr uint32_t kTmemO = 128;      // O: fp32, [128, 128 + D)
 
 struct TcItem {
@@ -67,8 +70,8 @@ struct TcSmem {
     static constexpr int oK = NQ * kQBuf;
     static constexpr int oV = oK + NK * kSlot;
     static constexpr int oBars = oV + NV * kSlot;
-    // kfull, kempty [NK]; vfull, vempty [NV]; qfull, qempty [NQ]; sfull,
-    // sfree, pfull[2], odone, drain
+    // kfull, kempty [NK]; vfull, vempty [NV]; qfull, qempty [NQ]; sfull[2],
+    // pfull[2], odone, drain
     static constexpr int kNumBars = 2 * NK + 2 * NV + 2 * NQ + 6;
     static constexpr int oItem = oBars + kNumBars * 8;
     static constexpr int oTmemSlot = oItem + NQ * (int)sizeof(TcItem);
@@ -228,7 +231,7 @@ __global__ void __launch_bounds__(kTcThreads, kTcCtasPerSm)
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L::oBars);
     uint64_t *kfull = bars, *kempty = bars + NK, *vfull = bars + 2 * NK, *vempty = bars + 2 * NK + NV;
     uint64_t *qfull = bars + 2 * NK + 2 * NV, *qempty = qfull + NQ;
-    uint64_t *sfull = qempty + NQ, *sfree = sfull + 1, *pfull = sfree + 1, *odone = pfull + 2, *drain = odone + 1;
+    uint64_t *sfull = qempty + NQ, *pfull = sfull + 2, *odone = pfull + 2, *drain = odone + 1;
     TcItem *items = reinterpret_cast<TcItem *>(smem + L::oItem);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::oTmemSlot);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::oAbort);
@@ -250,8 +253,8 @@ __global__ void __launch_bounds__(kTcThreads, kTcCtasPerSm)
             // and by the V producer once they have taken the item description
             mbar_init(&qempty[i], 2 + kTcRows);
         }
-        mbar_init(sfull, 1);
-        mbar_init(sfree, kTcRows);
+        mbar_init(&sfull[0], 1);
+        mbar_init(&sfull[1], 1);
         mbar_init(&pfull[0], kTcRows);
         mbar_init(&pfull[1], kTcRows);
         mbar_init(odone, 1);
@@ -400,21 +403,22 @@ __global__ void __launch_bounds__(kTcThreads, kTcCtasPerSm)
             const uint32_t qaddr = sbase + L::oQ + qb * L::kQBuf;
             for (int j = 0; j <= nb && ok; ++j) {
                 if (j < nb && lane == 0) {
-                    // S_j = Q K_j^T
+                    // S_j = Q K_j^T into buffer gb % 2.  That buffer last held
+                    // P_{gb-2}, read by a P·V this thread issued before: in order.
                     const uint32_t slot = gb % NK;
-                    ok = wait_or_abort(&kfull[slot], (gb / NK) & 1, abort_flag) &&
-                         wait_or_abort(sfree, (gb & 1) ^ 1, abort_flag);
+                    ok = wait_or_abort(&kfull[slot], (gb / NK) & 1, abort_flag);
                     if (ok) {
                         tc_fence_after();
                         const uint32_t kaddr = sbase + L::oK + slot * L::kSlot;
+                        const uint32_t sbuf = tmem + kTmemS + (gb & 1) * kTcKeys;
 #pragma unroll
                         for (int kk = 0; kk < D / 16; ++kk) {
                             const uint32_t off = (kk >> 2) * L::kQHalf + (kk & 3) * 32;
                             const uint32_t koff = (kk >> 2) * L::kKVHalf + (kk & 3) * 32;
-                            umma_ss(tmem + kTmemS, umma_desc_sw128(qaddr + off, 16, 1024),
+                            umma_ss(sbuf, umma_desc_sw128(qaddr + off, 16, 1024),
                                     umma_desc_sw128(kaddr + koff, 16, 1024), idesc_s, kk > 0);
                         }
-                        umma_commit(sfull);
+                        umma_commit(&sfull[gb & 1]);
                         umma_commit(&kempty[slot]);
                         if (j == nb - 1) umma_commit(&qempty[qb]);  // Q no longer read
                     }
@@ -432,7 +436,7 @@ __global__ void __launch_bounds__(kTcThreads, kTcCtasPerSm)
                         const uint32_t vaddr = sbase + L::oV + slot * L::kSlot;
 #pragma unroll
                         for (int kk = 0; kk < kTcKeys / 16; ++kk)
-                            umma_ts(tmem + kTmemO, tmem + kTmemP + pb * (kTcKeys / 2) + kk * 8,
+                            umma_ts(tmem + kTmemO, tmem + kTmemS + pb * kTcKeys + kk * 8,
                                     umma_desc_sw128(vaddr + kk * 16 * 128, L::kKVHalf, 1024), idesc_o,
                                     (j > 1 || kk > 0) ? 1u : 0u);
                         umma_commit(odone);
@@ -470,15 +474,14 @@ __global__ void __launch_bounds__(kTcThreads, kTcCtasPerSm)
             const int qpos = real ? t.prefix + tok : t.n_keys - 1;
             float m = PKV_NEG_INF, l0 = 0.f, l1 = 0.f;  // running max (scaled log2 units), sum
             for (int j = 0; j < t.n_blocks && ok; ++j, ++gb) {
-                ok = __all_sync(0xffffffffu, wait_or_abort(sfull, gb & 1, abort_flag));
+                const uint32_t sbuf = kTmemS + (gb & 1) * kTcKeys;  // S_j, then P_j over it
+                ok = __all_sync(0xffffffffu, wait_or_abort(&sfull[gb & 1], (gb >> 1) & 1, abort_flag));
                 if (!ok) break;
                 tc_fence_after();
                 uint32_t sv[64];
-                tmem_ld32(lane_addr + kTmemS, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
-                tmem_ld32(lane_addr + kTmemS + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
+                tmem_ld32(lane_addr + sbuf, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
+                tmem_ld32(lane_addr + sbuf + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
                 tc_wait_ld();
-                tc_fence_before();
-                mbar_arrive(sfree);
                 // causal mask on the block the diagonal crosses; max of raw scores
                 const int kbase = j * kTcKeys;
                 if (__any_sync(0xffffffffu, kbase + kTcKeys - 1 > qpos)) {
@@ -515,9 +518,8 @@ __global__ void __launch_bounds__(kTcThreads, kTcCtasPerSm)
                 }
                 l0 = l0 * alpha + s0;
                 l1 = l1 * alpha + s1;
-                const uint32_t pcol = kTmemP + (gb & 1) * (kTcKeys / 2);
-                tmem_st16(lane_addr + pcol, *reinterpret_cast<uint32_t(*)[16]>(&pk[0]));
-                tmem_st16(lane_addr + pcol + 16, *reinterpret_cast<uint32_t(*)[16]>(&pk[16]));
+                tmem_st16(lane_addr + sbuf, *reinterpret_cast<uint32_t(*)[16]>(&pk[0]));
+                tmem_st16(lane_addr + sbuf + 16, *reinterpret_cast<uint32_t(*)[16]>(&pk[16]));
                 // The previous block's PV product (global index gb - 1) must be
                 // complete before O is touched or P of this block is released;
                 // observing every phase of odone in order keeps its parity
