@@ -270,6 +270,22 @@ pkv_status launch_prefill_tc(const pkv::PrefillParams &prm, const CUtensorMap &m
     return launch_status();
 }
 
+// One copy launch of n <= CAP validated pairs (host int32 [n][2]), by value.
+template <int CAP>
+pkv_status copy_launch(const int32_t *pairs, int n, void *k_cache, void *v_cache, int64_t vec_per_block,
+                       pkv_stream_t stream) {
+    pkv::CopyParams<CAP> p;
+    p.k_cache = static_cast<uint4 *>(k_cache);
+    p.v_cache = static_cast<uint4 *>(v_cache);
+    p.vec_per_block = vec_per_block;
+    p.num_pairs = n;
+    for (int i = 0; i < n; ++i) p.pairs[i] = make_int2(pairs[2 * i], pairs[2 * i + 1]);
+    const long long per_cta = pkv::kCopyThreads * pkv::kCopyVecPerThread;
+    const unsigned gx = (unsigned)((vec_per_block + per_cta - 1) / per_cta);
+    pkv::copy_blocks_kernel<CAP><<<dim3(gx, n), pkv::kCopyThreads, 0, (cudaStream_t)stream>>>(p);
+    return launch_status();
+}
+
 // Device address of host memory the GPU can reach (pinned; unified addressing
 // makes it the host address), or nullptr for pageable or device memory.
 void *mapped_host_pointer(const void *p) {
@@ -508,19 +524,13 @@ pkv_status pkv_copy_blocks(const int32_t *src_dst_pairs, int32_t num_pairs, void
     for (int i = 0; i < num_pairs; ++i)
         if (std::binary_search(src.begin(), src.end(), dsorted[i])) return PKV_EALIAS;
 
-    pkv::CopyParams p;
-    p.k_cache = static_cast<uint4 *>(k_cache);
-    p.v_cache = static_cast<uint4 *>(v_cache);
-    p.vec_per_block = (int64_t)pool.num_kv_heads * pool.block_size * pool.head_dim * elem_bytes(pool) / 16;
-    const long long per_cta = pkv::kCopyThreads * pkv::kCopyVecPerThread;
-    const unsigned gx = (unsigned)((p.vec_per_block + per_cta - 1) / per_cta);
+    const int64_t vec = (int64_t)pool.num_kv_heads * pool.block_size * pool.head_dim * elem_bytes(pool) / 16;
     for (int base = 0; base < num_pairs; base += pkv::kMaxPairsPerLaunch) {
         const int n = std::min(pkv::kMaxPairsPerLaunch, num_pairs - base);
-        p.num_pairs = n;
-        for (int i = 0; i < n; ++i)
-            p.pairs[i] = make_int2(src_dst_pairs[2 * (base + i)], src_dst_pairs[2 * (base + i) + 1]);
-        pkv::copy_blocks_kernel<<<dim3(gx, n), pkv::kCopyThreads, 0, (cudaStream_t)stream>>>(p);
-        const pkv_status st = launch_status();
+        const int32_t *pr = src_dst_pairs + 2 * base;
+        const pkv_status st = n <= 32    ? copy_launch<32>(pr, n, k_cache, v_cache, vec, stream)
+                              : n <= 256 ? copy_launch<256>(pr, n, k_cache, v_cache, vec, stream)
+                                         : copy_launch<pkv::kMaxPairsPerLaunch>(pr, n, k_cache, v_cache, vec, stream);
         if (st != PKV_OK) return st;
     }
     return PKV_OK;

@@ -113,22 +113,27 @@ __global__ void __launch_bounds__(256) kv_write_fp8_kernel(WriteFp8Params p) {
 }
 
 // ----------------------------------------------------------------- copy ----
-// Pairs travel by value in the kernel parameters (validated on the host).
+// Pairs travel by value in the kernel parameters (validated on the host),
+// in a parameter block of CAP pairs: the host picks the smallest of 32, 256
+// and 1024 that holds a launch's pairs (the launch latency grows with the
+// parameter bytes: 8 KB cost about 1 us more than 2 KB for 256 pairs).
 // grid.y = pair, grid.x = chunk of the block; each thread moves kVecPerThread
 // vectors of K and of V, loads first, then stores.
 constexpr int kMaxPairsPerLaunch = 1024;  // 8 KB of parameters
 constexpr int kCopyThreads = 256;
 constexpr int kCopyVecPerThread = 4;
 
+template <int CAP>
 struct CopyParams {
     uint4 *k_cache;
     uint4 *v_cache;
     int64_t vec_per_block;  // Hkv * bs * D / 8
     int num_pairs;
-    int2 pairs[kMaxPairsPerLaunch];
+    int2 pairs[CAP];
 };
 
-__global__ void __launch_bounds__(kCopyThreads) copy_blocks_kernel(const __grid_constant__ CopyParams p) {
+template <int CAP>
+__global__ void __launch_bounds__(kCopyThreads) copy_blocks_kernel(const __grid_constant__ CopyParams<CAP> p) {
     const int pair = blockIdx.y;
     const int64_t src = (int64_t)p.pairs[pair].x * p.vec_per_block;
     const int64_t dst = (int64_t)p.pairs[pair].y * p.vec_per_block;
