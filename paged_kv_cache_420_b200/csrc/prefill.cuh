@@ -34,12 +34,12 @@ struct PrefillParams {
 
 // Query length and cached prefix of sequence s, clamped to what the table, the
 // workspace and the context allow (reported once, by the planner).
-__device__ __forceinline__ void prefill_lengths(const PrefillParams &p, int s, bool report, int &q_len,
-                                                int &prefix) {
-    int ctx = __ldg(p.context_lens + s);
+// From the loaded values: ctx = context_lens[s], q_begin = query_start[s],
+// q_end = query_start[s + 1].
+__device__ __forceinline__ void prefill_lengths_of(const PrefillParams &p, int ctx, int q_begin, int q_end,
+                                                   bool report, int &q_len, int &prefix) {
     const long long cap = min((long long)p.MBS * p.bs, (long long)p.max_ctx);
-    const int q_begin = __ldg(p.query_start + s);
-    int ql = __ldg(p.query_start + s + 1) - q_begin;
+    int ql = q_end - q_begin;
     bool bad = false;
     if (q_begin < 0 || q_begin > p.T) { bad = true; ql = 0; }
     else if (ql > p.T - q_begin) { bad = true; ql = p.T - q_begin; }
@@ -48,6 +48,12 @@ __device__ __forceinline__ void prefill_lengths(const PrefillParams &p, int s, b
     if (bad && report) raise_error(PKV_DEVERR_CONTEXT);
     q_len = ql;
     prefix = ctx - ql;
+}
+
+__device__ __forceinline__ void prefill_lengths(const PrefillParams &p, int s, bool report, int &q_len,
+                                                int &prefix) {
+    prefill_lengths_of(p, __ldg(p.context_lens + s), __ldg(p.query_start + s), __ldg(p.query_start + s + 1),
+                       report, q_len, prefix);
 }
 
 // Planner: entries (s, tile) sequence-major, each sequence's last (longest)

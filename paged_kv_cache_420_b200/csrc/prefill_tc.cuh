@@ -20,7 +20,7 @@
 //   warp 1       MMA issuer (one thread) and tensor-memory owner:
 //                S_j = Q K_j^T  (tcgen05.mma kind::f16, M 128, N 64, K-major
 //                smem operands, fp32 into TMEM S buffer j % 2), then
-//                O += P_{j-1} V_{j-1}  (A = P in TMEM, B = V MN-major in smem,
+//                O += P_j V_j  (A = P in TMEM, B = V MN-major in smem,
 //                N = D), each followed by tcgen05.commit onto an mbarrier.
 //   warps 2-5    softmax: thread r owns row r (TMEM lane r).  It loads S_j,
 //                masks the diagonal block, keeps the row's running max in
@@ -29,11 +29,11 @@
 //                its O row when the max was raised (after the previous PV
 //                product has completed), and at the end of the item normalises
 //                O and stores the row.
-// Two S buffers: S_{j+1} is issued right behind S_j, so it is ready when the
-// softmax finishes S_j.  S_{j+2} reuses S_j's buffer; the MMA thread issues it
-// after P_j V_j, and the tensor core runs one thread's MMAs in order, so P_j
-// has been read before S_{j+2} overwrites it.  The other CTA on the SM fills
-// the gaps of this one.
+// Two S buffers: the MMA thread issues P_j V_j as soon as P_j is ready and
+// then S_{j+2} into S_j's buffer (the tensor core runs one thread's MMAs in
+// order, so P_j has been read before S_{j+2} overwrites it).  S stays two
+// blocks ahead of the softmax and no P·V queues behind an S issue.  The other
+// CTA on the SM fills the gaps of this one.
 #pragma once
 
 #include "prefill.cuh"
@@ -52,6 +52,7 @@ constexpr uint32_t kTmemO = 128;      // O: fp32, [128, 128 + D)
 
 struct TcItem {
     int s, h, tile, q_len, prefix, q0, n_keys, n_blocks;
+    int row0[4];  // TMA rows of the first 64-key block's four 16-key stages
 };
 
 // Shared memory of one CTA: NQ query buffers, an NK-slot K ring and an
@@ -200,20 +201,46 @@ __device__ __forceinline__ void fadd2(float &a0, float &a1, float b0, float b1) 
         : "f"(b0), "f"(b1));
 }
 
-// Item geometry shared by the three roles.
-__device__ __forceinline__ TcItem tc_item(const PrefillParams &p, int it) {
+// Item geometry from the item's planner entry `st` and its sequence's loaded
+// lengths (ln = context_lens[s], query_start[s], query_start[s + 1]).
+__device__ __forceinline__ TcItem tc_item(const PrefillParams &p, int it, int2 st, int3 ln) {
     TcItem t;
     const int e = it / p.Hkv;
     t.h = it - e * p.Hkv;
-    const int2 st = p.entries[e];
     t.s = st.x;
     t.tile = st.y;
-    prefill_lengths(p, t.s, false, t.q_len, t.prefix);
-    t.q0 = __ldg(p.query_start + t.s);
+    prefill_lengths_of(p, ln.x, ln.y, ln.z, false, t.q_len, t.prefix);
+    t.q0 = ln.y;
     const int last_tok = min(t.q_len, (t.tile + 1) * p.QT) - 1;
     t.n_keys = t.prefix + last_tok + 1;
     t.n_blocks = (t.n_keys + kTcKeys - 1) / kTcKeys;
     return t;
+}
+
+__device__ __forceinline__ int3 tc_lengths(const PrefillParams &p, int s) {
+    return make_int3(__ldg(p.context_lens + s), __ldg(p.query_start + s), __ldg(p.query_start + s + 1));
+}
+
+// Table entry of stage `lane` (< 4) of 64-key block j of item t (-1 for a
+// stage past the keys, or a lane past 4).
+__device__ __forceinline__ int tc_stage_block(const PrefillParams &p, const TcItem &t, int j, int lane) {
+    const int tok = j * kTcKeys + (lane & 3) * kStageTok;
+    return (lane < 4 && tok < t.n_keys) ? __ldg(p.block_tables + (size_t)t.s * p.MBS + tok / p.bs) : -1;
+}
+
+// TMA row of that stage from its table entry: an entry outside the pool, or a
+// stage past the keys, reads rows beyond the pool (zero fill); the former is
+// reported.
+__device__ __forceinline__ int tc_stage_row_of(const PrefillParams &p, const TcItem &t, int j, int lane, int blk) {
+    const int tok = j * kTcKeys + (lane & 3) * kStageTok;
+    if (lane >= 4 || tok >= t.n_keys) return p.pool_rows;
+    if (blk >= 0 && blk < p.NB) return (blk * p.Hkv + t.h) * p.bs + tok % p.bs;
+    raise_error(PKV_DEVERR_BLOCK);
+    return p.pool_rows;
+}
+
+__device__ __forceinline__ int tc_stage_row(const PrefillParams &p, const TcItem &t, int j, int lane) {
+    return tc_stage_row_of(p, t, j, lane, tc_stage_block(p, t, j, lane));
 }
 
 template <int D>
@@ -283,20 +310,34 @@ __global__ void __launch_bounds__(kTcThreads, kTcCtasPerSm)
 
     if (warp == 0) {
         // ------------------------------------------------ Q and K producer --
+        // The next item's claim, entry, lengths and first-block table entries
+        // are fetched one step per K block while the current item streams, so
+        // an item boundary waits on no dependent global load.
         uint32_t gk = 0;          // K blocks issued
         int q_issued = -1;        // ord of the last Q tile load
         bool ok = true;
         int claimed = 0;
         if (lane == 0) claimed = atomicAdd(p.work_counter, 1);
         int it = __shfl_sync(0xffffffffu, claimed, 0);
+        TcItem cur;
+        cur.n_blocks = -1;
+        int row0 = p.pool_rows;
+        if (it < n_items) {
+            const int2 sp = p.entries[it / p.Hkv];
+            cur = tc_item(p, it, sp, tc_lengths(p, sp.x));
+            row0 = tc_stage_row(p, cur, 0, lane);
+        }
+        if (lane == 0) claimed = atomicAdd(p.work_counter, 1);  // the next item, one ahead
         for (int ord = 0; ok; ++ord) {
             const int qb = ord % NQ;
+            // the first block's rows travel with the item (the V producer uses them)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) cur.row0[i] = __shfl_sync(0xffffffffu, row0, i);
             if (lane == 0) {
                 ok = wait_or_abort(&qempty[qb], ((ord / NQ) & 1) ^ 1, abort_flag);
                 if (ok) {
-                    TcItem t;
-                    if (it < n_items) t = tc_item(p, it);
-                    else t.n_blocks = -1;  // end of stream
+                    TcItem t = cur;
+                    if (it >= n_items) t.n_blocks = -1;  // end of stream
                     items[qb] = t;
                     if (it < n_items) {
                         q_issued = ord;
@@ -313,18 +354,32 @@ __global__ void __launch_bounds__(kTcThreads, kTcCtasPerSm)
             }
             ok = __shfl_sync(0xffffffffu, ok, 0);
             if (it >= n_items || !ok) break;
-            if (lane == 0) claimed = atomicAdd(p.work_counter, 1);
-            const TcItem t = tc_item(p, it);
-            for (int j = 0; j < t.n_blocks && ok; ++j) {
-                // lane < 4: stage of 16 keys within the block; stages past the
-                // keys read rows beyond the pool (zero fill)
-                int row = p.pool_rows;
-                const int tok = j * kTcKeys + (lane & 3) * kStageTok;
-                if (lane < 4 && tok < t.n_keys) {
-                    const int blk = __ldg(p.block_tables + (size_t)t.s * p.MBS + tok / p.bs);
-                    if (blk >= 0 && blk < p.NB) row = (blk * p.Hkv + t.h) * p.bs + tok % p.bs;
-                    else raise_error(PKV_DEVERR_BLOCK);
+            // one step per K block, each using what the step before loaded:
+            // claim -> entry -> lengths -> item geometry and first-block rows
+            int nxt = n_items, pf = 0, nrow0 = p.pool_rows, nblk = -1;
+            int2 nsp = make_int2(0, 0);
+            int3 nln = make_int3(0, 0, 0);
+            TcItem nt;
+            nt.n_blocks = -1;
+            auto prefetch_step = [&]() {
+                if (pf == 0) {
+                    nxt = __shfl_sync(0xffffffffu, claimed, 0);
+                    if (nxt < n_items) nsp = p.entries[nxt / p.Hkv];
+                } else if (pf == 1) {
+                    if (nxt < n_items) nln = tc_lengths(p, nsp.x);
+                } else if (pf == 2) {
+                    if (nxt < n_items) {
+                        nt = tc_item(p, nxt, nsp, nln);
+                        nblk = tc_stage_block(p, nt, 0, lane);
+                    }
+                } else if (nxt < n_items) {
+                    nrow0 = tc_stage_row_of(p, nt, 0, lane, nblk);
                 }
+                ++pf;
+            };
+            for (int j = 0; j < cur.n_blocks && ok; ++j) {
+                // lane < 4: stage of 16 keys within the block
+                const int row = j == 0 ? row0 : tc_stage_row(p, cur, j, lane);
                 const uint32_t slot = gk % NK;
                 if (lane == 0) {
                     ok = wait_or_abort(&kempty[slot], ((gk / NK) & 1) ^ 1, abort_flag);
@@ -338,8 +393,13 @@ __global__ void __launch_bounds__(kTcThreads, kTcCtasPerSm)
                         tma_load_2d_u32(dst + hf * L::kKVHalf, &tmap_k, &kfull[slot], hf * 64, row);
                 }
                 if (ok) ++gk;
+                if (pf < 4) prefetch_step();
             }
-            it = __shfl_sync(0xffffffffu, claimed, 0);
+            while (ok && pf < 4) prefetch_step();  // a short item: finish the chain here
+            if (lane == 0) claimed = atomicAdd(p.work_counter, 1);  // the item after next
+            it = nxt;
+            cur = nt;
+            row0 = nrow0;
         }
         // After an abort, loads this CTA issued must land before it exits.
         if (lane == 0 && *abort_flag) {
@@ -360,13 +420,14 @@ __global__ void __launch_bounds__(kTcThreads, kTcCtasPerSm)
             if (lane == 0) mbar_arrive(&qempty[qb]);
             if (t.n_blocks < 0) break;
             for (int j = 0; j < t.n_blocks && ok; ++j) {
-                // lane < 4: stage of 16 keys, as in the K producer
+                // lane < 4: stage of 16 keys, as in the K producer (the first
+                // block's rows come with the item; the error, if any, was
+                // reported there)
                 int row = p.pool_rows;
-                const int tok = j * kTcKeys + (lane & 3) * kStageTok;
-                if (lane < 4 && tok < t.n_keys) {
-                    const int blk = __ldg(p.block_tables + (size_t)t.s * p.MBS + tok / p.bs);
-                    if (blk >= 0 && blk < p.NB) row = (blk * p.Hkv + t.h) * p.bs + tok % p.bs;
-                    else raise_error(PKV_DEVERR_BLOCK);
+                if (j == 0) {
+                    row = lane == 0 ? t.row0[0] : lane == 1 ? t.row0[1] : lane == 2 ? t.row0[2] : t.row0[3];
+                } else {
+                    row = tc_stage_row(p, t, j, lane);
                 }
                 const uint32_t slot = gv % NV;
                 if (lane == 0) {
@@ -401,51 +462,58 @@ __global__ void __launch_bounds__(kTcThreads, kTcCtasPerSm)
             if (nb < 0) break;
             tc_fence_after();
             const uint32_t qaddr = sbase + L::oQ + qb * L::kQBuf;
-            for (int j = 0; j <= nb && ok; ++j) {
-                if (j < nb && lane == 0) {
-                    // S_j = Q K_j^T into buffer gb % 2.  That buffer last held
-                    // P_{gb-2}, read by a P·V this thread issued before: in order.
-                    const uint32_t slot = gb % NK;
-                    ok = wait_or_abort(&kfull[slot], (gb / NK) & 1, abort_flag);
-                    if (ok) {
-                        tc_fence_after();
-                        const uint32_t kaddr = sbase + L::oK + slot * L::kSlot;
-                        const uint32_t sbuf = tmem + kTmemS + (gb & 1) * kTcKeys;
+            // Order: S_0, S_1, then for every block j: P_j V_j as soon as P_j is
+            // ready, then S_{j+2} into the buffer P_j just vacated (the tensor
+            // core runs this thread's MMAs in order, so P_j is read first).
+            // S stays two blocks ahead of the softmax, and no P·V waits
+            // behind an S issue.
+            const uint32_t gb0 = gb;  // global index of the item's first block
+            auto issue_s = [&](int jj) -> bool {
+                const uint32_t g = gb0 + jj;
+                const uint32_t slot = g % NK;
+                if (!wait_or_abort(&kfull[slot], (g / NK) & 1, abort_flag)) return false;
+                tc_fence_after();
+                const uint32_t kaddr = sbase + L::oK + slot * L::kSlot;
+                const uint32_t sbuf = tmem + kTmemS + (g & 1) * kTcKeys;
 #pragma unroll
-                        for (int kk = 0; kk < D / 16; ++kk) {
-                            const uint32_t off = (kk >> 2) * L::kQHalf + (kk & 3) * 32;
-                            const uint32_t koff = (kk >> 2) * L::kKVHalf + (kk & 3) * 32;
-                            umma_ss(sbuf, umma_desc_sw128(qaddr + off, 16, 1024),
-                                    umma_desc_sw128(kaddr + koff, 16, 1024), idesc_s, kk > 0);
-                        }
-                        umma_commit(&sfull[gb & 1]);
-                        umma_commit(&kempty[slot]);
-                        if (j == nb - 1) umma_commit(&qempty[qb]);  // Q no longer read
-                    }
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t off = (kk >> 2) * L::kQHalf + (kk & 3) * 32;
+                    const uint32_t koff = (kk >> 2) * L::kKVHalf + (kk & 3) * 32;
+                    umma_ss(sbuf, umma_desc_sw128(qaddr + off, 16, 1024), umma_desc_sw128(kaddr + koff, 16, 1024),
+                            idesc_s, kk > 0);
                 }
-                ok = __shfl_sync(0xffffffffu, ok, 0);
-                if (j > 0 && ok && lane == 0) {
-                    // O += P_{j-1} V_{j-1}
-                    const uint32_t pg = gb - 1;
-                    const uint32_t pb = pg & 1;
-                    const uint32_t slot = pg % NV;
-                    ok = wait_or_abort(&vfull[slot], (pg / NV) & 1, abort_flag) &&
-                         wait_or_abort(&pfull[pb], (pg >> 1) & 1, abort_flag);
-                    if (ok) {
-                        tc_fence_after();
-                        const uint32_t vaddr = sbase + L::oV + slot * L::kSlot;
+                umma_commit(&sfull[g & 1]);
+                umma_commit(&kempty[slot]);
+                if (jj == nb - 1) umma_commit(&qempty[qb]);  // Q no longer read
+                return true;
+            };
+            auto issue_pv = [&](int jj) -> bool {
+                const uint32_t g = gb0 + jj;
+                const uint32_t pb = g & 1;
+                const uint32_t slot = g % NV;
+                if (!wait_or_abort(&vfull[slot], (g / NV) & 1, abort_flag) ||
+                    !wait_or_abort(&pfull[pb], (g >> 1) & 1, abort_flag))
+                    return false;
+                tc_fence_after();
+                const uint32_t vaddr = sbase + L::oV + slot * L::kSlot;
 #pragma unroll
-                        for (int kk = 0; kk < kTcKeys / 16; ++kk)
-                            umma_ts(tmem + kTmemO, tmem + kTmemS + pb * kTcKeys + kk * 8,
-                                    umma_desc_sw128(vaddr + kk * 16 * 128, L::kKVHalf, 1024), idesc_o,
-                                    (j > 1 || kk > 0) ? 1u : 0u);
-                        umma_commit(odone);
-                        umma_commit(&vempty[slot]);
-                    }
+                for (int kk = 0; kk < kTcKeys / 16; ++kk)
+                    umma_ts(tmem + kTmemO, tmem + kTmemS + pb * kTcKeys + kk * 8,
+                            umma_desc_sw128(vaddr + kk * 16 * 128, L::kKVHalf, 1024), idesc_o,
+                            (jj > 0 || kk > 0) ? 1u : 0u);
+                umma_commit(odone);
+                umma_commit(&vempty[slot]);
+                return true;
+            };
+            if (lane == 0) {
+                ok = issue_s(0) && (nb < 2 || issue_s(1));
+                for (int jj = 0; jj < nb && ok; ++jj) {
+                    ok = issue_pv(jj);
+                    if (ok && jj + 2 < nb) ok = issue_s(jj + 2);
                 }
-                ok = __shfl_sync(0xffffffffu, ok, 0);
-                if (j < nb) ++gb;
             }
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+            gb += nb;
         }
         // every MMA this thread issued has completed before tensor memory is freed
         if (lane == 0) {
