@@ -157,6 +157,9 @@ DECODE_CASES = [
     ([2048, 2047, 2049, 1537, 1535, 2576], 8, 8, 128, 16, 512),    # MHA (CUDA-core path)
     ([2048, 2047, 2049, 1537, 1535, 2576], 32, 8, 128, 16, 256),   # g = 4 (tensor-core path)
     ([2048, 2047, 2049, 1537, 1535, 2576], 16, 1, 64, 32, 128),    # g = 16, d 64
+    ([3000, 1024, 1025, 9], 64, 8, 128, 1024, 256),               # bs 1024: partitions and groups inside one block
+    ([1000, 47, 48, 49, 2000], 8, 2, 128, 48, 0),                 # bs 48 (not a power of two), g = 4
+    ([1000, 47, 48, 49, 2000], 2, 2, 128, 48, 96),                # bs 48, MHA, split
 ]
 
 

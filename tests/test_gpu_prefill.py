@@ -44,6 +44,7 @@ CASES = [
     ([0, 513], [384, 300], 8, 8, 64, 16),                # MHA head dim 64, several 128-token tiles
     ([70], [200], 20, 4, 128, 32),                       # g = 5: 25-token tiles, 3 padding rows
     ([129, 1], [777, 64], 14, 2, 128, 16),               # g = 7: 18-token tiles, long chunk
+    ([100, 2000, 0], [300, 130, 513], 8, 2, 128, 48),    # bs 48 (not a power of two), g = 4, many items
 ]
 
 
