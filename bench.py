@@ -196,6 +196,36 @@ def whole_job_gbs(bytes_all_ranks: float, steps: int, ms_max: float) -> float:
     return bytes_all_ranks * steps / (ms_max / 1e3) / 1e9
 
 
+def timed_passes(dev, stream, step, steps: int, dist):
+    """Two timed passes of `steps` steps, clocks sampled over both.
+
+    The first records only its two end events and gives the step time; the
+    second calls step(i), which records an event pair around the kernel the
+    roofline is about.  An event between two launches costs about 2 us of
+    idle device time, so those events stay out of the first pass.
+    Returns (ms of the first pass, ClockSampler).
+    """
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(dev.index) as clocks:
+        t0.record(stream)
+        for _ in range(steps):
+            step()
+        t1.record(stream)
+        torch.cuda.synchronize()
+        if dist is not None:
+            dist.barrier()
+        for i in range(steps):
+            step(i)
+        torch.cuda.synchronize()
+        # keep sampling a little if the timed region was shorter than one sample
+        if t0.elapsed_time(t1) < 450:
+            time.sleep(0.45)
+    return t0.elapsed_time(t1), clocks
+
+
 def make_workload(args, rank: int, device):
     bs = args.block_size
     w = workloads.make(args.workload, seed=args.seed + rank, values_device=device, block_size=bs)
@@ -256,22 +286,7 @@ def run_cuda(args, rank, world, dist):
     if err:
         raise RuntimeError(f"device error word {err:#x} during warm-up")
 
-    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    if dist is not None:
-        dist.barrier()
-    torch.cuda.synchronize()
-    with ClockSampler(dev.index) as clocks:
-        t0.record(stream)
-        for i in range(args.steps):
-            step(i)
-        t1.record(stream)
-        torch.cuda.synchronize()
-        if dist is not None:
-            dist.barrier()
-        # keep sampling a little if the timed region was shorter than one sample
-        if t0.elapsed_time(t1) < 450:
-            time.sleep(0.45)
-    ms_total = t0.elapsed_time(t1)
+    ms_total, clocks = timed_passes(dev, stream, step, args.steps, dist)
     decode_ms = sum(a.elapsed_time(b) for a, b in ev_d) / args.steps
     if pkv.get_device_error():
         raise RuntimeError("device error word set during the timed region")
@@ -296,7 +311,7 @@ def run_cuda(args, rank, world, dist):
         out_h = [torch.empty(out.shape, dtype=out.dtype).pin_memory() for _ in range(2)]
         h2d = sum(v.numel() * v.element_size() for v in host.values())
         d2h = out_h[0].numel() * out_h[0].element_size()
-        k_e2e = max(3, min(args.steps, 1000))
+        k_e2e = max(3, args.steps)  # as long as the device-resident pass: same power state
         copy = torch.cuda.Stream(device=dev)
         ev_in = [torch.cuda.Event() for _ in range(2)]
         ev_done = [torch.cuda.Event() for _ in range(2)]
@@ -332,12 +347,13 @@ def run_cuda(args, rank, world, dist):
         if dist is not None:
             dist.barrier()
         a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record(copy)
-        stream.wait_stream(copy)
-        e2e_run(k_e2e)
-        copy.wait_stream(stream)
-        b_.record(copy)
-        torch.cuda.synchronize()
+        with ClockSampler(dev.index) as e2e_clocks:
+            a.record(copy)
+            stream.wait_stream(copy)
+            e2e_run(k_e2e)
+            copy.wait_stream(stream)
+            b_.record(copy)
+            torch.cuda.synchronize()
         if not torch.equal(out_h[(k_e2e - 1) % 2].to(dev), out):
             raise RuntimeError("end-to-end output differs from the device-resident run")
         e_ms = torch.tensor([a.elapsed_time(b_)], dtype=torch.float64, device=dev)
@@ -345,7 +361,7 @@ def run_cuda(args, rank, world, dist):
             dist.all_reduce(e_ms, op=dist.ReduceOp.MAX)
         e2e = {"value": round(bytes_all * k_e2e / (float(e_ms[0]) / 1e3) / 1e9, 2), "unit": "GB/s",
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "steps": k_e2e,
-               "overlap": "copies on a second stream, double-buffered"}
+               "overlap": "copies on a second stream, double-buffered", "clocks": e2e_clocks.summary()}
 
     peak, peak_kind = measured_hbm_peak()
     achieved = dec_bytes / (decode_ms / 1e3) / 1e9
@@ -610,23 +626,11 @@ def run_prefill_cuda(args, rank, world, dist):
     for _ in range(max(args.warmup, 3)):
         step()
     torch.cuda.synchronize()
-    if dist is not None:
-        dist.barrier()
-    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with ClockSampler(dev.index) as clocks:
-        t0.record(stream)
-        for i in range(args.steps):
-            step(i)
-        t1.record(stream)
-        torch.cuda.synchronize()
-        if dist is not None:
-            dist.barrier()
-        if t0.elapsed_time(t1) < 450:
-            time.sleep(0.45)
+    ms_run, clocks = timed_passes(dev, stream, step, args.steps, dist)
     if pkv.get_device_error():
         raise RuntimeError("device error word set during the timed region")
     flops = prefill_flops(w)
-    ms_max, flops_all, tok_all = combine_ranks(dist, t0.elapsed_time(t1), int(flops), w.num_tokens, dev)
+    ms_max, flops_all, tok_all = combine_ranks(dist, ms_run, int(flops), w.num_tokens, dev)
     attn_ms = sum(a.elapsed_time(b) for a, b in ev) / args.steps
     peak, kind = measured_tensor_peak()
     achieved = flops / (attn_ms / 1e3) / 1e12
@@ -693,25 +697,13 @@ def run_fp8_cuda(args, rank, world, dist):
     for _ in range(max(args.warmup, 3)):
         step()
     torch.cuda.synchronize()
-    if dist is not None:
-        dist.barrier()
-    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with ClockSampler(dev.index) as clocks:
-        t0.record(stream)
-        for i in range(args.steps):
-            step(i)
-        t1.record(stream)
-        torch.cuda.synchronize()
-        if dist is not None:
-            dist.barrier()
-        if t0.elapsed_time(t1) < 450:
-            time.sleep(0.45)
+    ms_run, clocks = timed_passes(dev, stream, step, args.steps, dist)
     if pkv.get_device_error():
         raise RuntimeError("device error word set during the timed region")
     dec = decode_bytes(w, kv_elem=1)
     wr = w.num_seqs * w.num_kv_heads * w.head_dim * (2 * 2 + 2) + 8 * w.num_seqs  # bf16 in, e4m3 out
     wr += copy_bytes(w) // 2  # e4m3 blocks
-    ms_max, bytes_all, seqs_all = combine_ranks(dist, t0.elapsed_time(t1), dec + wr, w.num_seqs, dev)
+    ms_max, bytes_all, seqs_all = combine_ranks(dist, ms_run, dec + wr, w.num_seqs, dev)
     dec_ms = sum(a.elapsed_time(b) for a, b in ev) / args.steps
     peak, kind = measured_hbm_peak()
     achieved = dec / (dec_ms / 1e3) / 1e9
@@ -955,21 +947,9 @@ def run_swap_cuda(args, rank, world, dist):
         d2h_ms.append(a.elapsed_time(b))
         h2d_ms.append(b.elapsed_time(c))
     del dk, dv
-    if dist is not None:
-        dist.barrier()
-    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with ClockSampler(dev.index) as clocks:
-        t0.record(stream)
-        for i in range(args.steps):
-            step(i)
-        t1.record(stream)
-        torch.cuda.synchronize()
-        if dist is not None:
-            dist.barrier()
-        if t0.elapsed_time(t1) < 450:
-            time.sleep(0.45)
+    ms_run, clocks = timed_passes(dev, stream, step, args.steps, dist)
     bytes_step = 2 * n * block_bytes * 2  # K and V, out and in
-    ms_max, bytes_all, _ = combine_ranks(dist, t0.elapsed_time(t1), bytes_step, n, dev)
+    ms_max, bytes_all, _ = combine_ranks(dist, ms_run, bytes_step, n, dev)
     out_ms = float(np.median([e[0].elapsed_time(e[1]) for e in ev]))
     in_ms = float(np.median([e[1].elapsed_time(e[2]) for e in ev]))
     one_way = 2 * n * block_bytes
