@@ -230,12 +230,16 @@ pkv_status dispatch_group(int g, const pkv::DecodeParams &prm, const CUtensorMap
 
 int prefill_query_tile(int g) { return pkv::kTcRows / g; }
 
-bool prefill_layout(int32_t B, int32_t g, int32_t max_q, size_t *off_entries, size_t *total) {
+// Workspace: entry count and work counter, the work list, and its staging
+// copy in sequence order.
+bool prefill_layout(int32_t B, int32_t g, int32_t max_q, size_t *off_entries, size_t *off_staged, size_t *total) {
     if (B < 0 || g <= 0 || max_q < 0) return false;
     const int QT = prefill_query_tile(g);
     const long long max_tiles = std::max<long long>(1, ((long long)max_q + QT - 1) / QT);
+    const size_t list = round256((size_t)B * max_tiles * sizeof(int2));
     *off_entries = 256;
-    *total = 256 + round256((size_t)B * max_tiles * sizeof(int2));
+    *off_staged = 256 + list;
+    *total = 256 + 2 * list;
     return true;
 }
 
@@ -633,8 +637,8 @@ pkv_status pkv_write_fp8(const void *k, const void *v, const int64_t *slot_mappi
 size_t pkv_prefill_workspace_bytes(int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads,
                                    int32_t max_query_len) {
     if (num_kv_heads <= 0 || num_q_heads <= 0 || num_q_heads % num_kv_heads) return 0;
-    size_t off, total;
-    if (!prefill_layout(num_seqs, num_q_heads / num_kv_heads, max_query_len, &off, &total)) return 0;
+    size_t off, off_staged, total;
+    if (!prefill_layout(num_seqs, num_q_heads / num_kv_heads, max_query_len, &off, &off_staged, &total)) return 0;
     return total;
 }
 
@@ -659,8 +663,8 @@ pkv_status paged_attn_prefill(const void *q, const void *k_cache, const void *v_
     if (!aligned(q, 16) || !aligned(out, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) ||
         !aligned(block_tables, 4) || !aligned(context_lens, 4) || !aligned(query_start, 4) || !aligned(workspace, 256))
         return PKV_EINVAL;
-    size_t off_entries, total;
-    if (!prefill_layout(num_seqs, g, max_query_len, &off_entries, &total) || workspace_bytes < total)
+    size_t off_entries, off_staged, total;
+    if (!prefill_layout(num_seqs, g, max_query_len, &off_entries, &off_staged, &total) || workspace_bytes < total)
         return PKV_EINVAL;
     pkv::PrefillParams prm;
     prm.q = static_cast<const __nv_bfloat16 *>(q);
@@ -672,6 +676,7 @@ pkv_status paged_attn_prefill(const void *q, const void *k_cache, const void *v_
     prm.num_entries = reinterpret_cast<int32_t *>(ws);
     prm.work_counter = reinterpret_cast<int32_t *>(ws) + 1;
     prm.entries = reinterpret_cast<int2 *>(ws + off_entries);
+    prm.staged = reinterpret_cast<int2 *>(ws + off_staged);
     prm.B = num_seqs;
     prm.Hq = num_q_heads;
     prm.Hkv = num_kv_heads;

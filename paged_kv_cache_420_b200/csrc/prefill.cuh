@@ -10,8 +10,8 @@
 //
 // This header holds what the attention kernel (prefill_tc.cuh) builds on: the
 // call's parameters, the clamped lengths of a sequence, and the planner that
-// lists the (sequence, query tile) items, each sequence's longest tile first.
-// No split-K: an item walks its whole causal key range.
+// lists the (sequence, query tile) items, longest first.  No split-K: an item
+// walks its whole causal key range.
 #pragma once
 
 #include "decode.cuh"
@@ -24,7 +24,8 @@ struct PrefillParams {
     const int32_t *block_tables;  // [B][MBS]
     const int32_t *context_lens;  // [B]
     const int32_t *query_start;   // [B+1]
-    int2 *entries;                // workspace: (seq, query tile)
+    int2 *entries;                // workspace: (seq, query tile), longest first
+    int2 *staged;                 // workspace: the same entries in sequence order
     int32_t *num_entries;
     int32_t *work_counter;
     int B, Hq, Hkv, g, MBS, bs, NB, max_ctx, max_q, QT, T;
@@ -56,24 +57,41 @@ __device__ __forceinline__ void prefill_lengths(const PrefillParams &p, int s, b
                        report, q_len, prefix);
 }
 
-// Planner: entries (s, tile) sequence-major, each sequence's last (longest)
-// tile first; zeroes the work counter.
+// Keys an item walks, in 64-key units, as the planner's sort key (an item's
+// cost grows with it); items longer than the histogram share its last bucket.
+constexpr int kPlanBuckets = 4096;
+__device__ __forceinline__ int prefill_sort_key(const PrefillParams &p, int q_len, int prefix, int tile) {
+    const int n_keys = prefix + min(q_len, (tile + 1) * p.QT);
+    return min(n_keys >> 6, kPlanBuckets - 1);
+}
+
+// Planner: lists the (s, tile) entries, longest first, and zeroes the work
+// counter.  The attention kernel's CTAs claim items in list order, so the
+// last items claimed are the shortest and the CTAs finish close together.
+// Entries go to `staged` in sequence order with a histogram of their sort
+// keys; a descending scan of the histogram gives each key's first slot and
+// the entries are scattered to `entries` (order within a key is arbitrary:
+// items are independent).
 __global__ void __launch_bounds__(kPlanThreads) plan_prefill_kernel(PrefillParams p) {
     __shared__ int s_off[kPlanThreads + 1];
     __shared__ int s_warp[kPlanThreads / 32];
     __shared__ int s_carry;
+    __shared__ int s_ql[kPlanThreads], s_pre[kPlanThreads];
+    __shared__ int s_hist[kPlanBuckets];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     grid_launch_dependents();
+    for (int i = tid; i < kPlanBuckets; i += kPlanThreads) s_hist[i] = 0;
     if (tid == 0) s_carry = 0;
     __syncthreads();
     for (int base = 0; base < p.B; base += kPlanThreads) {
         const int s = base + tid;
-        int tiles = 0;
+        int tiles = 0, ql = 0, prefix = 0;
         if (s < p.B) {
-            int ql, prefix;
             prefill_lengths(p, s, true, ql, prefix);
             tiles = (ql + p.QT - 1) / p.QT;
         }
+        s_ql[tid] = ql;
+        s_pre[tid] = prefix;
         int x = tiles;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
@@ -104,14 +122,60 @@ __global__ void __launch_bounds__(kPlanThreads) plan_prefill_kernel(PrefillParam
                 if (s_off[mid] <= e) lo = mid; else hi = mid - 1;
             }
             const int n_tiles = s_off[lo + 1] - s_off[lo];
-            p.entries[carry + e] = make_int2(base + lo, n_tiles - 1 - (e - s_off[lo]));
+            const int tile = n_tiles - 1 - (e - s_off[lo]);
+            p.staged[carry + e] = make_int2(base + lo, tile);
+            atomicAdd(&s_hist[prefill_sort_key(p, s_ql[lo], s_pre[lo], tile)], 1);
         }
         __syncthreads();
         if (tid == 0) s_carry = carry + chunk_total;
         __syncthreads();
     }
+    const int total = s_carry;
+    // first slot of each key, longest key first: exclusive scan of the
+    // histogram from the top bucket down (thread t owns 4 buckets)
+    static_assert(kPlanBuckets == 4 * kPlanThreads, "four buckets per thread");
+    {
+        const int b0 = kPlanBuckets - 1 - 4 * tid;  // this thread's buckets: b0, b0-1, b0-2, b0-3
+        int c[4], sum = 0;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            c[i] = s_hist[b0 - i];
+            sum += c[i];
+        }
+        int x = sum;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, x, o);
+            if (lane >= o) x += y;
+        }
+        if (lane == 31) s_warp[warp] = x;
+        __syncthreads();
+        if (warp == 0) {
+            int w = s_warp[lane];
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int y = __shfl_up_sync(0xffffffffu, w, o);
+                if (lane >= o) w += y;
+            }
+            s_warp[lane] = w;
+        }
+        __syncthreads();
+        int start = x - sum + (warp > 0 ? s_warp[warp - 1] : 0);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            s_hist[b0 - i] = start;
+            start += c[i];
+        }
+    }
+    __syncthreads();
+    for (int e = tid; e < total; e += kPlanThreads) {
+        const int2 st = p.staged[e];
+        int ql, prefix;
+        prefill_lengths(p, st.x, false, ql, prefix);
+        p.entries[atomicAdd(&s_hist[prefill_sort_key(p, ql, prefix, st.y)], 1)] = st;
+    }
     if (tid == 0) {
-        *p.num_entries = s_carry;
+        *p.num_entries = total;
         *p.work_counter = 0;
     }
 }

@@ -636,20 +636,31 @@ __global__ void __launch_bounds__(kTcThreads, kTcCtasPerSm)
             const float inv = l > 0.f ? 1.f / l : 0.f;
             __nv_bfloat16 *orow =
                 real ? p.out + ((size_t)(t.q0 + tok) * p.Hq + (size_t)t.h * p.g + jh) * D : nullptr;
+            // A row is 2*D bytes, so with `out` 32-byte aligned every 16-column
+            // piece of it is too, and it goes out in 32-byte stores (full
+            // sectors, half the store instructions); 16-byte stores otherwise.
+            const bool wide = (reinterpret_cast<uintptr_t>(p.out) & 31u) == 0;
 #pragma unroll
             for (int c0 = 0; c0 < D; c0 += 32) {
                 uint32_t ov[32];
                 tmem_ld32(lane_addr + kTmemO + c0, ov);
                 tc_wait_ld();
                 if (real) {
+                    uint32_t lo[8], hi[8];
 #pragma unroll
-                    for (int i = 0; i < 32; i += 8) {
-                        uint4 v;
-                        v.x = pack_bf16x2(__uint_as_float(ov[i]) * inv, __uint_as_float(ov[i + 1]) * inv);
-                        v.y = pack_bf16x2(__uint_as_float(ov[i + 2]) * inv, __uint_as_float(ov[i + 3]) * inv);
-                        v.z = pack_bf16x2(__uint_as_float(ov[i + 4]) * inv, __uint_as_float(ov[i + 5]) * inv);
-                        v.w = pack_bf16x2(__uint_as_float(ov[i + 6]) * inv, __uint_as_float(ov[i + 7]) * inv);
-                        *reinterpret_cast<uint4 *>(orow + c0 + i) = v;
+                    for (int i = 0; i < 8; ++i) {
+                        lo[i] = pack_bf16x2(__uint_as_float(ov[2 * i]) * inv, __uint_as_float(ov[2 * i + 1]) * inv);
+                        hi[i] = pack_bf16x2(__uint_as_float(ov[16 + 2 * i]) * inv,
+                                            __uint_as_float(ov[16 + 2 * i + 1]) * inv);
+                    }
+                    if (wide) {
+                        st_global_v8(orow + c0, lo);
+                        st_global_v8(orow + c0 + 16, hi);
+                    } else {
+                        *reinterpret_cast<uint4 *>(orow + c0) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+                        *reinterpret_cast<uint4 *>(orow + c0 + 8) = make_uint4(lo[4], lo[5], lo[6], lo[7]);
+                        *reinterpret_cast<uint4 *>(orow + c0 + 16) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+                        *reinterpret_cast<uint4 *>(orow + c0 + 24) = make_uint4(hi[4], hi[5], hi[6], hi[7]);
                     }
                 }
             }

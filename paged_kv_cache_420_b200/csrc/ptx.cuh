@@ -212,4 +212,14 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     return *reinterpret_cast<uint32_t *>(&v);
 }
 
+// ---------------------------------------------------------------- stores --
+
+// One 32-byte global store (a 256-bit vector store, sm_100 and later); `ptr`
+// must be 32-byte aligned.
+__device__ __forceinline__ void st_global_v8(void *ptr, const uint32_t (&v)[8]) {
+    asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(ptr), "r"(v[0]), "r"(v[1]),
+                 "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7])
+                 : "memory");
+}
+
 }  // namespace pkv

@@ -60,6 +60,23 @@ def test_prefill_parity(prefix, chunk, Hq, Hkv, D, bs, poison):
     no_device_error()
 
 
+@pytest.mark.parametrize("case", [1, 2, 4, 0])
+def test_prefill_out_only_16_byte_aligned(case):
+    """`out` 16 bytes past a 32-byte boundary takes the 16-byte store path of
+    the epilogue; it must write the same bits as the paired 32-byte stores."""
+    w = workloads.make_prefill_custom(*CASES[case], seed=5)
+    kc, vc, out = run_prefill(w)
+    base = torch.full((out.numel() + 8,), float("nan"), dtype=out.dtype, device="cuda")
+    out16 = base[8:].view(out.shape)
+    assert out16.data_ptr() % 32 == 16 and out.data_ptr() % 32 == 0
+    pkv.paged_attn_prefill(w.q, kc, vc, torch.from_numpy(w.block_tables).cuda(),
+                           torch.from_numpy(w.context_lens).cuda(), torch.from_numpy(w.query_start).cuda(),
+                           w.scale, w.num_kv_heads, out16, w.max_query_len, w.max_context_len)
+    torch.cuda.synchronize()
+    no_device_error()
+    assert torch.equal(out16, out)  # also false if any element stayed NaN
+
+
 def test_prefill_single_token_equals_decode_kernel():
     w = workloads.make_prefill_custom([300, 1000, 0], [1, 1, 1], 32, 8, 128, 16, seed=9)
     kc, vc, out = run_prefill(w)
