@@ -422,6 +422,8 @@ struct SimtState {
         }
     }
 
+    // PARTIAL: fewer than 16 valid tokens in the stage (see MmaState::stage).
+    template <bool PARTIAL>
     __device__ __forceinline__ void stage(uint32_t ktile, uint32_t vtile, int valid, int lane) {
         float v[16];
         // q.k partial sums v[r] of token r; tokens r and r+1 share one packed
@@ -472,7 +474,7 @@ struct SimtState {
             }
         }
         const int my_tok = lane >> 1;
-        const float score = (my_tok < valid) ? (KV8 ? v[0] * kscale : v[0]) : PKV_NEG_INF;
+        const float score = (!PARTIAL || my_tok < valid) ? (KV8 ? v[0] * kscale : v[0]) : PKV_NEG_INF;
         // stage max (one warp reduction), lazy rescale
         const float mx = warp_max_f32(score);
         if (mx > m + kRescaleSlack) {  // warp-uniform, rare after the first stage
@@ -490,7 +492,7 @@ struct SimtState {
         // row (packed fp32x2 FMA over element pairs)
 #pragma unroll
         for (int r = 0; r < 16; ++r) {
-            if (r < valid) {
+            if (!PARTIAL || r < valid) {
                 if constexpr (KV8) {
                     uint32_t v16[2];
                     load_row8(vtile, r, lane, v16);
@@ -599,6 +601,10 @@ struct MmaState {
         }
     }
 
+    // PARTIAL: the stage holds fewer than 16 valid tokens (a partition's last
+    // stage); only then are scores past `valid` masked and the V operand's
+    // rows of those tokens zeroed, so a full stage spends no instructions on it.
+    template <bool PARTIAL>
     __device__ __forceinline__ void stage(uint32_t ktile, uint32_t vtile, int valid, int lane, float scale_log2) {
         // S^T[token][head] = K . Q^T
         // two independent accumulator chains (even / odd k-steps), summed after
@@ -640,7 +646,8 @@ struct MmaState {
 #pragma unroll
             for (int c = 0; c < 4; ++c) s[nt][c] += s2[nt][c];
         const int t0 = lane >> 2;  // rows t0 and t0 + 8 (tokens, in perm16 order with H)
-        const bool ok0 = (H ? perm16(t0) : t0) < valid, ok1 = (H ? perm16(t0 + 8) : t0 + 8) < valid;
+        const bool ok0 = !PARTIAL || (H ? perm16(t0) : t0) < valid;
+        const bool ok1 = !PARTIAL || (H ? perm16(t0 + 8) : t0 + 8) < valid;
         uint32_t pb[NT][2];
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
@@ -682,7 +689,7 @@ struct MmaState {
         // token masks of this thread's V^T operand halves: k slots 2(l%4)+{0,1}
         // and +8, i.e. tokens 2(l%4)+{0,1} and +8 (with H: 4(l%4)+{0,1} and +{2,3})
         uint32_t mask01 = 0xffffffffu, mask23 = 0xffffffffu;
-        if (valid < 16) {
+        if constexpr (PARTIAL) {
             const int j0 = H ? 4 * (lane & 3) : 2 * (lane & 3);
             const int j2 = H ? j0 + 2 : j0 + 8;
             mask01 = (j0 < valid ? 0x0000ffffu : 0u) | (j0 + 1 < valid ? 0xffff0000u : 0u);
@@ -705,7 +712,7 @@ struct MmaState {
                 const int col = mt * 16 + 8 * (mi & 1);
                 ldmatrix_x4_trans(tile_addr(vtile, row, col), a0, a1, a2, a3);
             }
-            a0 &= mask01; a1 &= mask01; a2 &= mask23; a3 &= mask23;
+            if constexpr (PARTIAL) { a0 &= mask01; a1 &= mask01; a2 &= mask23; a3 &= mask23; }
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt) {
                 if constexpr (H)
@@ -746,10 +753,15 @@ struct MmaState {
 // PATH 0: CUDA cores, one query head per kv head (GSIMT = 1); PATH 1: tensor
 // cores with query heads padded to GPAD in {4, 8, 16} (n-tiles of 8: GPAD/8
 // rounded up).
+// CTAs per SM the register budget must allow: the FP8 tensor-core instances
+// with up to 8 padded heads take 44 KB of shared memory, so four CTAs fit
+// and the registers must not cut that to three.
+constexpr int decode_min_ctas(int PATH, int GPAD, bool KV8) { return (KV8 && PATH == 1 && GPAD <= 8) ? 4 : 1; }
+
 template <int D, int PATH, int GSIMT, int GPAD, int NS, bool KV8 = false>
-__global__ void __launch_bounds__(kDecodeThreads) paged_decode_kernel(const __grid_constant__ CUtensorMap tmap_k,
-                                                                      const __grid_constant__ CUtensorMap tmap_v,
-                                                                      const DecodeParams p) {
+__global__ void __launch_bounds__(kDecodeThreads, decode_min_ctas(PATH, GPAD, KV8))
+    paged_decode_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v,
+                        const DecodeParams p) {
     constexpr int W = kConsumerWarps;
     static_assert(PATH != 0 || GSIMT == 1, "the CUDA-core path serves one query head per kv head");
     constexpr int GP = PATH == 0 ? GSIMT : GPAD;
@@ -995,12 +1007,14 @@ __global__ void __launch_bounds__(kDecodeThreads) paged_decode_kernel(const __gr
             }
             if (si.valid > 0) {
                 const uint32_t kt = tiles + slot * L::kStage;
+                const bool partial = si.valid < kStageTok;  // warp-uniform
                 if constexpr (PATH == 0) {
-                    st0.stage(kt, kt + L::kTile, si.valid, lane);
-                } else if constexpr (KV8) {
-                    st1.stage(kt, kt + L::kTile, si.valid, lane, scale_log2 * __ldg(p.k_scale + si.h));
+                    if (partial) st0.template stage<true>(kt, kt + L::kTile, si.valid, lane);
+                    else st0.template stage<false>(kt, kt + L::kTile, si.valid, lane);
                 } else {
-                    st1.stage(kt, kt + L::kTile, si.valid, lane, scale_log2);
+                    const float sl = KV8 ? scale_log2 * __ldg(p.k_scale + si.h) : scale_log2;
+                    if (partial) st1.template stage<true>(kt, kt + L::kTile, si.valid, lane, sl);
+                    else st1.template stage<false>(kt, kt + L::kTile, si.valid, lane, sl);
                 }
             }
             __syncwarp();
