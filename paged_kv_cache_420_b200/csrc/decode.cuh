@@ -338,6 +338,15 @@ __device__ __forceinline__ uint32_t f16x2_from_e4m3x2(uint32_t pair16) {
     return r;
 }
 
+// The two code pairs of a word of four e4m3 codes as f16x2 words: lo from
+// bytes 0-1, hi from bytes 2-3 (the halves are taken from the register as
+// they are).
+__device__ __forceinline__ void f16x2_from_e4m3x4(uint32_t w, uint32_t &lo, uint32_t &hi) {
+    asm("{\n\t.reg .b16 l16, h16;\n\tmov.b32 {l16, h16}, %2;\n\t"
+        "cvt.rn.f16x2.e4m3x2 %0, l16;\n\tcvt.rn.f16x2.e4m3x2 %1, h16;\n\t}"
+        : "=r"(lo), "=r"(hi) : "r"(w));
+}
+
 __device__ __forceinline__ uint32_t f16x2_from_f32(float lo, float hi) {
     uint32_t r;
     asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
@@ -403,8 +412,7 @@ struct SimtState {
     __device__ __forceinline__ void load_row8(uint32_t tile, int r, int lane, uint32_t (&h)[2]) {
         uint32_t w;
         asm volatile("ld.shared.u32 %0, [%1];" : "=r"(w) : "r"(tile_addr8(tile, r, lane * EPL)));
-        h[0] = f16x2_from_e4m3x2(w & 0xffffu);
-        h[1] = f16x2_from_e4m3x2(w >> 16);
+        f16x2_from_e4m3x4(w, h[0], h[1]);
     }
 
     // Loads this lane's EPL elements of row r of a tile as fp32.
@@ -614,21 +622,21 @@ struct MmaState {
 #pragma unroll
             for (int c = 0; c < 4; ++c) { s[nt][c] = 0.f; s2[nt][c] = 0.f; }
         const int mi = lane >> 3, ri = lane & 7;
+        uint32_t kw[4];  // H: K codes of two k-steps
 #pragma unroll
         for (int kk = 0; kk < KS; ++kk) {
             // matrices: (rows 0-7, cols k0..+7), (rows 8-15, k0..), (rows 0-7, k0+8..), (rows 8-15, k0+8..)
             uint32_t a0, a1, a2, a3;
             if constexpr (H) {
-                uint32_t w0, w1;
-                const int c = kk * 16 + 4 * (lane & 3);
-                asm volatile("ld.shared.u32 %0, [%1];" : "=r"(w0) : "r"(tile_addr8(ktile, perm16(lane >> 2), c)));
-                asm volatile("ld.shared.u32 %0, [%1];"
-                             : "=r"(w1)
-                             : "r"(tile_addr8(ktile, perm16((lane >> 2) + 8), c)));
-                a0 = f16x2_from_e4m3x2(w0 & 0xffffu);
-                a1 = f16x2_from_e4m3x2(w1 & 0xffffu);
-                a2 = f16x2_from_e4m3x2(w0 >> 16);
-                a3 = f16x2_from_e4m3x2(w1 >> 16);
+                // one 8x8 matrix load per two k-steps: (rows perm16(0-7), bytes kk*16..+15),
+                // (rows perm16(8-15), same), then the same for k-step kk + 1; lane l
+                // receives codes 4(l%4) .. +3 of its rows, as one 32-bit load each would
+                if ((kk & 1) == 0)
+                    ldmatrix_x4(tile_addr8(ktile, perm16(ri + 8 * (mi & 1)), kk * 16 + 16 * (mi >> 1)), kw[0], kw[1],
+                                kw[2], kw[3]);
+                const uint32_t w0 = kw[2 * (kk & 1)], w1 = kw[2 * (kk & 1) + 1];
+                f16x2_from_e4m3x4(w0, a0, a2);
+                f16x2_from_e4m3x4(w1, a1, a3);
             } else {
                 const int row = ri + 8 * (mi & 1);
                 const int col = kk * 16 + 8 * (mi >> 1);
@@ -702,10 +710,8 @@ struct MmaState {
             if constexpr (H) {
                 uint32_t r0, r1;
                 ldmatrix_b8_trans(tile_addr8(vtile, lane & 15, mt * 16), r0, r1);
-                a0 = f16x2_from_e4m3x2(r0 & 0xffffu);  // d = l/4: tokens 4j, 4j+1
-                a1 = f16x2_from_e4m3x2(r1 & 0xffffu);  // d = l/4 + 8
-                a2 = f16x2_from_e4m3x2(r0 >> 16);      // d = l/4: tokens 4j+2, 4j+3
-                a3 = f16x2_from_e4m3x2(r1 >> 16);
+                f16x2_from_e4m3x4(r0, a0, a2);  // d = l/4: tokens 4j, 4j+1 and 4j+2, 4j+3
+                f16x2_from_e4m3x4(r1, a1, a3);  // d = l/4 + 8
             } else {
                 // matrices (stored rows = tokens): (tok 0-7, d0..+7), (tok 0-7, d0+8..), (tok 8-15, d0..), (tok 8-15, d0+8..)
                 const int row = ri + 8 * (mi >> 1);

@@ -212,6 +212,16 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     return *reinterpret_cast<uint32_t *>(&v);
 }
 
+// ------------------------------------------------------------------ e4m3 --
+
+// Two fp32 values rounded to e4m3 (nearest even, saturating to +-448),
+// packed with `lo` in the low byte.
+__device__ __forceinline__ uint32_t e4m3x2_from_f32(float lo, float hi) {
+    unsigned short r;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
 // ---------------------------------------------------------------- stores --
 
 // One 32-byte global store (a 256-bit vector store, sm_100 and later); `ptr`

@@ -70,13 +70,6 @@ struct WriteFp8Params {
     int vpr;               // vectors per row = D / 8
 };
 
-// Two fp32 values -> two e4m3 codes; lo lands in the low byte.
-__device__ __forceinline__ uint32_t e4m3x2_from_f32(float lo, float hi) {
-    uint16_t r;
-    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
-    return r;
-}
-
 __global__ void __launch_bounds__(256) kv_write_fp8_kernel(WriteFp8Params p) {
     const int per_token = 2 * p.num_kv_heads * p.vpr;
     const int per_kv = p.num_kv_heads * p.vpr;
