@@ -29,6 +29,7 @@
 // toward the head, in order.
 #pragma once
 
+#include <climits>
 #include <cstdint>
 
 #include "ptx.cuh"
@@ -86,8 +87,9 @@ __device__ __forceinline__ void bm_revive(const BmState &s, int32_t b) {
 // send a pop or push outside the stack).
 __device__ __forceinline__ int bm_top(const BmState &s, int nb) { return min(max(s.hdr[0], 0), nb); }
 
-// Block-wide exclusive scan of one int per thread (1024 threads); returns the
-// exclusive prefix and writes the block total to *total (all threads).
+// Block-wide exclusive scan of one int per thread (a block of any multiple of
+// 32 threads up to 1024); returns the exclusive prefix and writes the block
+// total to *total (all threads).
 __device__ __forceinline__ int block_scan_excl(int v, int *warp_sums, int *total) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     int x = v;
@@ -99,7 +101,7 @@ __device__ __forceinline__ int block_scan_excl(int v, int *warp_sums, int *total
     if (lane == 31) warp_sums[warp] = x;
     __syncthreads();
     if (warp == 0) {
-        int w = warp_sums[lane];
+        int w = lane < (int)(blockDim.x >> 5) ? warp_sums[lane] : 0;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
             const int y = __shfl_up_sync(0xffffffffu, w, o);
@@ -112,6 +114,46 @@ __device__ __forceinline__ int block_scan_excl(int v, int *warp_sums, int *total
     *total = warp_sums[31];
     __syncthreads();  // warp_sums reusable after return
     return before + x - v;
+}
+
+// N exclusive scans at once (one pass, three block barriers): v[k] becomes
+// its exclusive prefix and total[k] the block total.  warp_sums holds N * 32
+// ints.
+template <int N>
+__device__ __forceinline__ void block_scan_excl_n(int (&v)[N], int *warp_sums, int (&total)[N]) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    int x[N];
+#pragma unroll
+    for (int k = 0; k < N; ++k) {
+        x[k] = v[k];
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, x[k], o);
+            if (lane >= o) x[k] += y;
+        }
+        if (lane == 31) warp_sums[k * 32 + warp] = x[k];
+    }
+    __syncthreads();
+    if (warp == 0) {
+#pragma unroll
+        for (int k = 0; k < N; ++k) {
+            int w = lane < (int)(blockDim.x >> 5) ? warp_sums[k * 32 + lane] : 0;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int y = __shfl_up_sync(0xffffffffu, w, o);
+                if (lane >= o) w += y;
+            }
+            warp_sums[k * 32 + lane] = w;  // inclusive over warps
+        }
+    }
+    __syncthreads();
+#pragma unroll
+    for (int k = 0; k < N; ++k) {
+        const int before = warp == 0 ? 0 : warp_sums[k * 32 + warp - 1];
+        total[k] = warp_sums[k * 32 + 31];
+        v[k] = before + x[k] - v[k];
+    }
+    __syncthreads();  // warp_sums reusable after return
 }
 
 __global__ void __launch_bounds__(256) bm_init_kernel(BmState s, int nb) {
@@ -139,7 +181,7 @@ __device__ __forceinline__ int block_max(int v, int *warp_buf) {
     for (int o = 16; o > 0; o >>= 1) v = max(v, __shfl_xor_sync(0xffffffffu, v, o));
     if ((threadIdx.x & 31) == 0) warp_buf[threadIdx.x >> 5] = v;
     __syncthreads();
-    int w = warp_buf[threadIdx.x & 31];
+    int w = (threadIdx.x & 31) < (blockDim.x >> 5) ? warp_buf[threadIdx.x & 31] : INT_MIN;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) w = max(w, __shfl_xor_sync(0xffffffffu, w, o));
     __syncthreads();
@@ -157,7 +199,7 @@ __device__ int ring_collect(const BmState &s, int nb, int target, int collected,
     const uint32_t tail = ring_tail(s);
     uint32_t cur = *cursor;
     while (collected < target && cur != tail) {
-        const uint32_t span = min((uint32_t)kBmThreads, tail - cur);
+        const uint32_t span = min((uint32_t)blockDim.x, tail - cur);
         const int32_t b = threadIdx.x < span ? ring_live(s, nb, cur + threadIdx.x) : -1;
         int tot;
         const int excl = block_scan_excl(b >= 0 ? 1 : 0, warp_buf, &tot);
@@ -373,8 +415,11 @@ struct AppendParams {
 // the last sharer writes in place; a candidate's rank among earlier
 // candidates on the same block comes from __match_any_sync within its warp
 // and a per-block counter walked warp by warp.
+// Launched with one thread per sequence or per four output slots, whichever
+// is more, rounded up to a warp (at most kBmThreads): a decode batch of 128
+// takes four warps, and every block barrier waits for those alone.
 __global__ void __launch_bounds__(kBmThreads) bm_append_slots_kernel(const AppendParams p) {
-    __shared__ int warp_buf[32];
+    __shared__ int warp_buf[3 * 32];
     // per sequence of the chunk, for the cooperative slot pass: its first
     // slot index, and its first position (-1 unless it fits)
     __shared__ int sh_slot0[kBmThreads], sh_pos0[kBmThreads];
@@ -389,7 +434,8 @@ __global__ void __launch_bounds__(kBmThreads) bm_append_slots_kernel(const Appen
     int run_slots = 0;  // slot-mapping offset
     int run_pairs = 0;
     int handed = 0;     // blocks handed out
-    for (int base = 0; base < p.B; base += kBmThreads) {
+    const int nthr = blockDim.x;
+    for (int base = 0; base < p.B; base += nthr) {
         const int b = base + threadIdx.x;
         const bool live = b < p.B;
         int n = 0, pos0 = 0, first_new = 0, last = -1, need_new = 0;
@@ -415,13 +461,17 @@ __global__ void __launch_bounds__(kBmThreads) bm_append_slots_kernel(const Appen
         }
         // references of a candidate's block, after earlier chunks' copies
         const int R = cand ? s.refcount[cur] : 0;
-        const unsigned same = __match_any_sync(0xffffffffu, cand ? cur : -2 - (int)threadIdx.x);
+        // Only a block with more than one holder needs the ranking (its first
+        // R - 1 writers copy, the last keeps it); a block with one holder is
+        // written in place whatever its rank, and no other sequence holds it.
+        const bool shared = cand && R > 1;
+        const unsigned same = __match_any_sync(0xffffffffu, shared ? cur : -2 - (int)threadIdx.x);
         const int rank_in_warp = __popc(same & ((1u << lane) - 1u));
         int rank = 0;
-        if (__syncthreads_or(cand)) {  // only when some sequence writes into a block it may share
-            const int live_warps = (min(kBmThreads, p.B - base) + 31) / 32;
+        if (__syncthreads_or(shared)) {  // only when some sequence writes into a shared block
+            const int live_warps = (min(nthr, p.B - base) + 31) / 32;
             for (int w = 0; w < live_warps; ++w) {
-                if (warp == w && cand) {
+                if (warp == w && shared) {
                     rank = s.cow_rank[cur] + rank_in_warp;
                     __syncwarp(same);
                     if (rank_in_warp == 0) s.cow_rank[cur] += __popc(same);
@@ -429,18 +479,21 @@ __global__ void __launch_bounds__(kBmThreads) bm_append_slots_kernel(const Appen
                 __syncthreads();
             }
         }
-        const int cow = (cand && rank < R - 1) ? 1 : 0;
+        const int cow = (shared && rank < R - 1) ? 1 : 0;
         const int need = live ? need_new + cow : 0;
         const int flag = (bad_range || overflow) ? 1 : 0;
-        int tot_flags, tot_need, tot_n;
-        const int flags_before = run_flags + block_scan_excl(flag, warp_buf, &tot_flags);
-        const int excl_need = run_need + block_scan_excl(need, warp_buf, &tot_need);
-        const int excl_slots = run_slots + block_scan_excl(n, warp_buf, &tot_n);
+        int sc1[3] = {flag, need, n}, tot1[3];
+        block_scan_excl_n<3>(sc1, warp_buf, tot1);
+        const int tot_flags = tot1[0], tot_need = tot1[1], tot_n = tot1[2];
+        const int flags_before = run_flags + sc1[0];
+        const int excl_need = run_need + sc1[1];
+        const int excl_slots = run_slots + sc1[2];
         const bool earlier_ok = flags_before == 0 && excl_need <= avail0;
         const bool fits = live && earlier_ok && !flag && excl_need + need <= avail0;
-        int tot_pairs, tot_handed;
-        const int excl_pairs = run_pairs + block_scan_excl(fits ? cow : 0, warp_buf, &tot_pairs);
-        (void)block_scan_excl(fits ? need : 0, warp_buf, &tot_handed);
+        int sc2[2] = {fits ? cow : 0, fits ? need : 0}, tot2[2];
+        block_scan_excl_n<2>(sc2, warp_buf, tot2);
+        const int tot_pairs = tot2[0], tot_handed = tot2[1];
+        const int excl_pairs = run_pairs + sc2[0];
         // this chunk's pops beyond the free stack come from the eviction order
         collected = ring_collect(s, p.nb, max(0, handed + tot_handed - top0), collected, &cursor, warp_buf);
         if (live && bad_range) bm_error(s, kBmErrRange);
@@ -471,8 +524,8 @@ __global__ void __launch_bounds__(kBmThreads) bm_append_slots_kernel(const Appen
         // sequence without new tokens shares its first slot with the next one,
         // so the last such sequence is always one that owns entry j)
         const int chunk_first = sh_slot0[0];
-        const int nlive = min(kBmThreads, p.B - base);
-        for (int j = chunk_first + threadIdx.x; j < run_slots + tot_n; j += kBmThreads) {
+        const int nlive = min(nthr, p.B - base);
+        for (int j = chunk_first + threadIdx.x; j < run_slots + tot_n; j += nthr) {
             int lo = 0, hi = nlive - 1;
             while (lo < hi) {
                 const int mid = (lo + hi + 1) >> 1;
@@ -490,7 +543,7 @@ __global__ void __launch_bounds__(kBmThreads) bm_append_slots_kernel(const Appen
             }
         }
         if (live && (int64_t)excl_slots + n > p.slot_cap) bm_error(s, kBmErrNoSpace);  // output too short
-        if (cand) s.cow_rank[cur] = 0;  // scratch back to rest
+        if (shared) s.cow_rank[cur] = 0;  // scratch back to rest
         __syncthreads();
         run_need += tot_need;
         run_flags += tot_flags;

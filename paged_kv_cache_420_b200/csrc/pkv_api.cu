@@ -834,7 +834,12 @@ pkv_status pkv_bm_append_slots(void *state, int32_t num_blocks, int32_t *block_t
     p.mbs = max_blocks_per_seq;
     p.B = num_seqs;
     p.bs = block_size;
-    pkv::bm_append_slots_kernel<<<1, pkv::kBmThreads, 0, (cudaStream_t)stream>>>(p);
+    // One thread per sequence, and enough for the slot pass to write at most
+    // four slots per thread (the output capacity bounds the slots), rounded up
+    // to a warp: a 128-sequence decode step runs on four warps.
+    const int64_t want = std::max<int64_t>((int64_t)num_seqs, slot_capacity / 4);
+    const int threads = (int)std::min<int64_t>(pkv::kBmThreads, std::max<int64_t>(32, (want + 31) / 32 * 32));
+    pkv::bm_append_slots_kernel<<<1, threads, 0, (cudaStream_t)stream>>>(p);
     return launch_status();
 }
 
