@@ -332,12 +332,6 @@ __device__ __forceinline__ uint32_t tile_addr8(uint32_t tile, int r, int c) {
     return tile + r * 128 + ((((c >> 4) ^ (r & 7))) << 4) + (c & 15);
 }
 
-__device__ __forceinline__ uint32_t f16x2_from_e4m3x2(uint32_t pair16) {
-    uint32_t r;
-    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(r) : "h"((unsigned short)pair16));
-    return r;
-}
-
 // The two code pairs of a word of four e4m3 codes as f16x2 words: lo from
 // bytes 0-1, hi from bytes 2-3 (the halves are taken from the register as
 // they are).
